@@ -1,0 +1,487 @@
+#!/usr/bin/env python
+"""Benchmark of the quantized MoE expert matmul on B200.
+
+Metric: MoE-layer microseconds and achieved HBM GB/s (algorithmic bytes /
+time) against tokens-per-expert M.  Headline workload: a DeepSeek-V2-Lite-
+shaped decode MoE layer (H=2048, I=1408, 64 routed experts top-6 + 2 shared,
+INT4 FC1/FC2, block 64) with M tokens that share router logits, so each of
+the 8 selected experts receives exactly M tokens; the headline line is M=1.
+A step is one MoE-layer forward (route -> gather -> FC1+SwiGLU -> FC2 ->
+combine) through the C ABI.  8 copies of the layer's weights (2.4 GB) are
+rotated step by step, so consecutive steps never hit the 126 MB L2.
+
+Also reported: the M sweep 1..32 of the same layer and the single quantized
+linear K=5120 -> N=17408 (group 128, INT2 and INT4) at M = 1..32.
+
+`--impl reference` times the CPU fp64 oracle on the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from skinny_gemm_top_b200 import synth  # noqa: E402
+
+CFG = synth.V2LITE
+SEED = 1
+ROTATE = 8
+METRIC = "MoE-layer µs and HBM GB/s (% of B200 peak) vs tokens-per-expert M=1..32"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--sweep", default="1,2,4,8,16,32")
+    ap.add_argument("--linear-sweep", default="1,2,3,4,5,8,10,16,32")
+    ap.add_argument("--quick", action="store_true", help="skip the sweeps")
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------------ byte accounting
+
+def expert_bytes(fmt: str, rows: int, K: int, block: int) -> int:
+    code = rows * K * 13 // 64 if fmt == "ternary" else rows * K * {"int2": 2, "int4": 4}[fmt] // 8
+    return code + rows * (K // block) * 2
+
+
+FC1_BYTES = expert_bytes(CFG.fc1_fmt, 2 * CFG.I, CFG.H, CFG.block)
+FC2_BYTES = expert_bytes(CFG.fc2_fmt, CFG.H, CFG.I, CFG.block)
+
+
+def active_experts(logits_row: np.ndarray) -> list[int]:
+    order = np.argsort(-logits_row.astype(np.float64), kind="stable")
+    return sorted(int(e) for e in order[: CFG.k]) + [CFG.E + j for j in range(CFG.n_shared)]
+
+
+def layer_bytes(logits: np.ndarray) -> dict:
+    """Algorithmic bytes of one layer forward: weights of the active experts,
+    x, y and logits (each read or written once)."""
+    T = logits.shape[0]
+    act = set()
+    for t in range(T):
+        act.update(active_experts(logits[t]))
+    n = len(act)
+    io = T * CFG.H * 2 * 2 + T * CFG.E * 4
+    return {"total": n * (FC1_BYTES + FC2_BYTES) + io, "fc1": n * FC1_BYTES + T * CFG.H * 2, "experts": n}
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ------------------------------------------------------------------ GPU arm
+
+def _to_dev(torch, a):
+    a = np.ascontiguousarray(a)
+    if a.dtype == np.uint16:
+        a = a.view(np.int16)
+    return torch.from_numpy(a).cuda()
+
+
+def pack_moe(qmoe, torch, rotate: int):
+    """Pack the layer once on the host, then replicate it `rotate` times on the device."""
+    n = CFG.E + CFG.n_shared
+    f1, f2 = qmoe.FMT[CFG.fc1_fmt], qmoe.FMT[CFG.fc2_fmt]
+    c1, s1 = qmoe.pack_stack(f1, qmoe.ROWS_GATE_UP, (synth.expert_fc1(CFG, SEED, e) for e in range(n)), CFG.block)
+    c2, s2 = qmoe.pack_stack(f2, qmoe.ROWS_PLAIN, (synth.expert_fc2(CFG, SEED, e) for e in range(n)), CFG.block)
+    dev = [_to_dev(torch, a) for a in (c1, s1, c2, s2)]
+    layers, keep = [], []
+    for r in range(rotate):
+        copies = dev if r == 0 else [t.clone() for t in dev]
+        keep.append(copies)
+        w1 = qmoe.make_weights(f1, CFG.block, copies[0], copies[1])
+        w2 = qmoe.make_weights(f2, CFG.block, copies[2], copies[3])
+        layers.append(qmoe.make_layer(CFG.H, CFG.I, CFG.E, CFG.k, CFG.n_shared, w1, w2))
+    return layers, keep
+
+
+def graph_of(torch, fn, count: int):
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        fn(0, 1)  # one eager call on the capture stream (allocations, attributes)
+    torch.cuda.current_stream().wait_stream(s)
+    with torch.cuda.graph(g):
+        for i in range(count):
+            fn(i, count)
+    return g
+
+
+class Steps:
+    """K forward calls as graph replays: full graphs of `rotate` calls plus a tail graph."""
+
+    def __init__(self, torch, fn, rotate: int):
+        self.torch, self.fn, self.rotate = torch, fn, rotate
+        self.full = graph_of(torch, fn, rotate)
+        self.tails = {}
+
+    def prepare(self, *ks: int):
+        for k in ks:
+            rem = k % self.rotate
+            if rem and rem not in self.tails:
+                self.tails[rem] = graph_of(self.torch, self.fn, rem)
+
+    def run(self, k: int):
+        for _ in range(k // self.rotate):
+            self.full.replay()
+        rem = k % self.rotate
+        if rem:
+            if rem not in self.tails:
+                self.tails[rem] = graph_of(self.torch, self.fn, rem)
+            self.tails[rem].replay()
+
+
+def time_steps(torch, dist, steps: Steps, k: int) -> float:
+    """ms for k steps, device-timed with events, max over ranks."""
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    steps.run(k)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    if dist is not None:
+        t = torch.tensor([ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    return ms
+
+
+def moe_inputs(torch, M: int, rotate: int):
+    xs = [_to_dev(torch, synth.tokens(CFG.H, SEED, M, index=r)) for r in range(rotate)]
+    rows = synth.router_logits(CFG, SEED, rotate, index=7)
+    lgs_np = [np.repeat(rows[r:r + 1], M, axis=0) for r in range(rotate)]
+    lgs = [torch.from_numpy(l).cuda() for l in lgs_np]
+    return xs, lgs, lgs_np
+
+
+def run_ours(args):
+    import torch
+    from skinny_gemm_top_b200 import qmoe
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev_index = torch.cuda.current_device()
+    layers, keep = pack_moe(qmoe, torch, ROTATE)
+
+    def measure_moe(M: int, k: int, w: int, trace: bool = False, clocks: ClockSampler | None = None):
+        xs, lgs, lgs_np = moe_inputs(torch, M, ROTATE)
+        ws = torch.empty(qmoe.workspace_size(layers[0], M), dtype=torch.uint8, device="cuda")
+        ys = [torch.empty((M, CFG.H), dtype=torch.int16, device="cuda") for _ in range(ROTATE)]
+
+        def fn(i, n):
+            r = i % ROTATE
+            qmoe.forward(layers[r], xs[r], lgs[r], ys[r], ws)
+
+        if trace:  # the eager call of graph_of takes 5 records, the captured graph the next 5 * ROTATE
+            qmoe.trace_start(5 * (ROTATE + 1))
+        steps = Steps(torch, fn, ROTATE)
+        if trace:
+            qmoe.trace_stop()
+        steps.prepare(k, w)
+        if clocks is not None:  # settle clocks under this load before the timed region
+            t_end = time.time() + 1.5
+            while time.time() < t_end:
+                steps.run(ROTATE * 64)
+                torch.cuda.synchronize()
+        steps.run(w)
+        ms = time_steps(torch, dist, steps, k)
+        per = [layer_bytes(l) for l in lgs_np]
+        out = {"ms_per_step": ms / k, "bytes": statistics.mean(p["total"] for p in per),
+               "fc1_bytes": statistics.mean(p["fc1"] for p in per)}
+        if trace:
+            rec = qmoe.trace_read(5 * (ROTATE + 1))[5:]
+            out["fc1_ms"] = statistics.mean(t for n, t in rec if n == "fc1_small")
+            out["kernels"] = {n: statistics.mean(t for m, t in rec if m == n) for n in sorted({n for n, _ in rec})}
+        return out
+
+    sampler = ClockSampler(dev_index)
+    sampler.start()
+    head = measure_moe(1, args.steps, args.warmup, trace=True, clocks=sampler)
+    clocks = sampler.stop()
+
+    result_sweep = []
+    if not args.quick:
+        for M in [int(m) for m in args.sweep.split(",")]:
+            r = measure_moe(M, max(args.steps, 64), args.warmup)
+            result_sweep.append({"M": M, "us": round(r["ms_per_step"] * 1e3, 3),
+                                 "GBps": round(r["bytes"] / (r["ms_per_step"] * 1e6), 1),
+                                 "tokens_per_s": round(M / (r["ms_per_step"] * 1e-3), 1)})
+    linear = [] if args.quick else linear_sweep(qmoe, torch, dist, args)
+    e2e = measure_e2e(qmoe, torch, dist, layers[0], args.steps, args.warmup)
+
+    peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json"))) if os.path.exists(
+        os.path.join(ROOT, "MEASURED_PEAKS.json")) else {}
+    hbm_peak = peaks.get("hbm_gbs", 6650.0)
+    peak_src = "measured" if "hbm_gbs" in peaks else "fallback"
+    fc1_gbps = head["fc1_bytes"] / (head["fc1_ms"] * 1e6)
+    traffic = None
+    tpath = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(tpath):
+        traffic = json.load(open(tpath)).get("fc1_small_v2lite_M1_bytes_per_launch")
+
+    value = head["bytes"] / (head["ms_per_step"] * 1e6) * world
+    line = {
+        "metric": METRIC,
+        "value": round(value, 1),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(head["ms_per_step"], 6),
+        "us_per_layer": round(head["ms_per_step"] * 1e3, 3),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "int4-weights/bf16-act/fp32-acc",
+        "data": "synthetic",
+        "config": {
+            "workload": "v2lite-decode-moe-layer: H=2048 I=1408 E=64 top-6 + 2 shared, INT4 FC1/FC2 block 64, "
+                        "M=1 token per expert",
+            "tokens_per_expert": 1,
+            "global_batch": world,
+            "parallelism": f"replicas x{world} (independent decode batches, no data-path collective)",
+            "l2": "8 weight copies (2.4 GB) rotated step by step: inputs larger than L2",
+            "graph": "CUDA graphs of forward calls",
+            "bytes_per_step": int(head["bytes"]),
+            "pct_of_hbm_peak": round(100 * value / world / hbm_peak, 1),
+            "pct_of_nominal_8TBps": round(100 * value / world / 8000, 1),
+        },
+        "roofline": {"bound": "hbm", "kernel": "fc1_small (dequant + gate/up MMA + SwiGLU)",
+                     "achieved": round(fc1_gbps, 1), "peak": hbm_peak, "peak_source": peak_src,
+                     "unit": "GB/s", "frac": round(fc1_gbps / hbm_peak, 3), "traffic": traffic,
+                     "bytes_per_launch": int(head["fc1_bytes"]), "launch_us": round(head["fc1_ms"] * 1e3, 3),
+                     "kernels_us": {k: round(v * 1e3, 3) for k, v in head["kernels"].items()}},
+        "sweep_tokens_per_expert": result_sweep,
+        "linear_5120x17408_g128": linear,
+        "e2e": e2e,
+        "gpu_launches": 5 * args.steps,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1:
+        line["cpu_baseline"] = cpu_baseline(head["bytes"])
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    del keep
+    if dist is not None:
+        dist.destroy_process_group()
+
+
+def measure_e2e(qmoe, torch, dist, layer, k: int, w: int) -> dict:
+    """Through the public API with pinned host buffers: each step copies x and
+    logits host->device, runs the layer and reads y back."""
+    M = 1
+    x_h = torch.from_numpy(synth.tokens(CFG.H, SEED, M, index=99).view(np.int16)).pin_memory()
+    rows = synth.router_logits(CFG, SEED, 16, index=9)
+    lg_h = [torch.from_numpy(np.ascontiguousarray(rows[i:i + 1])).pin_memory() for i in range(16)]
+    y_h = torch.empty((M, CFG.H), dtype=torch.int16).pin_memory()
+    x_d = torch.empty((M, CFG.H), dtype=torch.int16, device="cuda")
+    lg_d = torch.empty((M, CFG.E), dtype=torch.float32, device="cuda")
+    y_d = torch.empty_like(x_d)
+    ws = torch.empty(qmoe.workspace_size(layer, M), dtype=torch.uint8, device="cuda")
+
+    def step(i):
+        x_d.copy_(x_h, non_blocking=True)
+        lg_d.copy_(lg_h[i % 16], non_blocking=True)
+        qmoe.forward(layer, x_d, lg_d, y_d, ws)
+        y_h.copy_(y_d, non_blocking=True)
+        torch.cuda.current_stream().synchronize()
+
+    for i in range(w):
+        step(i)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(k):
+        step(i)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / k
+    nbytes = statistics.mean(layer_bytes(rows[i:i + 1])["total"] for i in range(16))
+    return {"value": round(nbytes / (ms * 1e6), 1), "unit": "GB/s", "us_per_layer": round(ms * 1e3, 2),
+            "h2d_bytes_per_step": M * CFG.H * 2 + M * CFG.E * 4, "d2h_bytes_per_step": M * CFG.H * 2,
+            "note": "unfused single layer incl. launch latency (no graph) and a host sync per step"}
+
+
+def linear_sweep(qmoe, torch, dist, args) -> list:
+    N, K, block = 17408, 5120, 128
+    wb = synth.linear_weight(SEED, N, K)
+    out = []
+    for fmt in ("int2", "int4"):
+        c, s = qmoe.pack(qmoe.FMT[fmt], qmoe.ROWS_PLAIN, wb, block)
+        nbytes = c.nbytes + s.nbytes
+        rot = max(2, int(np.ceil(2 * 126e6 / nbytes)) + 1)
+        dc, ds = _to_dev(torch, c), _to_dev(torch, s)
+        copies = [(dc, ds)] + [(dc.clone(), ds.clone()) for _ in range(rot - 1)]
+        ws_list = [qmoe.make_weights(qmoe.FMT[fmt], block, a, b) for a, b in copies]
+        row = {"fmt": fmt, "bytes_M1": nbytes + K * 2 + N * 2, "copies_rotated": rot, "M": []}
+        for M in [int(m) for m in args.linear_sweep.split(",")]:
+            x = _to_dev(torch, synth.tokens(K, SEED, M))
+            y = torch.empty((M, N), dtype=torch.int16, device="cuda")
+            ws = torch.empty(qmoe.linear_workspace_size(N, K, M), dtype=torch.uint8, device="cuda")
+
+            def fn(i, n, M=M, x=x, y=y, ws=ws):
+                qmoe.linear(ws_list[i % rot], N, K, x, y, ws)
+
+            steps = Steps(torch, fn, rot)
+            k = max(args.steps, 64)
+            steps.prepare(k, args.warmup)
+            steps.run(args.warmup)
+            ms = time_steps(torch, dist, steps, k) / k
+            b = nbytes + M * K * 2 + M * N * 2
+            row["M"].append({"M": M, "us": round(ms * 1e3, 3), "GBps": round(b / (ms * 1e6), 1)})
+        out.append(row)
+    return out
+
+
+# ------------------------------------------------------------------ CPU oracle
+
+def _oracle_bank():
+    from oracle import qmoe_oracle as Q
+
+    def q(fmt, wbits):
+        w = Q.bf16_bits_to_f64(wbits)
+        return Q.quantize_ternary(w, CFG.block) if fmt == "ternary" else Q.quantize_sym(
+            w, 2 if fmt == "int2" else 4, CFG.block)
+
+    return Q, Q.QuantExpertBank(CFG.H, CFG.I, CFG.E, CFG.n_shared, CFG.block,
+                                lambda e: q(CFG.fc1_fmt, synth.expert_fc1(CFG, SEED, e)),
+                                lambda e: q(CFG.fc2_fmt, synth.expert_fc2(CFG, SEED, e)), cache=16)
+
+
+def _cores() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info()]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(gpu_bytes_per_step: float, budget_s: float = 12.0) -> dict:
+    """The oracle as it stands, one M=1 layer step at a time, for about budget_s seconds."""
+    Q, bank = _oracle_bank()
+    rows = synth.router_logits(CFG, SEED, 64, index=7)
+    x = Q.bf16_bits_to_f64(synth.tokens(CFG.H, SEED, 1))
+    t0 = time.perf_counter()
+    n = 0
+    nbytes = 0.0
+    while time.perf_counter() - t0 < budget_s or n == 0:
+        Q.moe_token(x[0], rows[n % 64], CFG.k, bank)
+        nbytes += layer_bytes(rows[n % 64:n % 64 + 1])["total"]
+        n += 1
+    dt = time.perf_counter() - t0
+    return {"value": round(nbytes / (dt * 1e9), 4), "unit": "GB/s", "cores": _cores(), "kind": "oracle",
+            "sample": f"{n} single-token layer steps (M=1, rotating router rows), {dt:.1f} s",
+            "us_per_layer": round(dt / n * 1e6, 1)}
+
+
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    Q, bank = _oracle_bank()
+    rows = synth.router_logits(CFG, SEED, 64, index=7)
+    x = Q.bf16_bits_to_f64(synth.tokens(CFG.H, SEED, 1))
+    for i in range(args.warmup):
+        Q.moe_token(x[0], rows[i % 64], CFG.k, bank)
+    t0 = time.perf_counter()
+    nbytes = 0.0
+    for i in range(args.steps):
+        r = (args.warmup + i) % 64
+        Q.moe_token(x[0], rows[r], CFG.k, bank)
+        nbytes += layer_bytes(rows[r:r + 1])["total"]
+    dt = time.perf_counter() - t0
+    value = nbytes / (dt * 1e9)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "v2lite-decode-moe-layer: H=2048 I=1408 E=64 top-6 + 2 shared, INT4 FC1/FC2 "
+                               "block 64, M=1 token per expert", "tokens_per_expert": 1},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": _cores(), "kind": "oracle",
+                         "sample": f"{args.steps} single-token layer steps after {args.warmup} warm-up steps"},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,191 @@
+/*
+ * qmoe.h - C ABI of the B200 (sm_100a) weight-only low-bit quantized MoE
+ * expert matmul.
+ *
+ * What it computes (sources by page and section):
+ *   - onnxruntime PR "Enable SM80+ FP16/BF16 mixed INT2/INT4 QMoE prefill by
+ *     default", Description / Current Scope: top-k routing, rows expanded by
+ *     expert, INT2 (or INT4) FC1 with interleaved fused SwiGLU and expert bias,
+ *     INT4 FC2, top-k weighted finalize with FC2 bias; symmetric block
+ *     quantization, block 64, no zero points; row tiling under a scratch
+ *     budget with an error when even one row does not fit.
+ *   - "The QMoE sub-1-bit expert kernel is a GEMV ..." note: the inner loop
+ *     over the tokens that share an expert (one pass over the weights serves
+ *     all of them).
+ *   - "Skip MoE channels ... top-k channel selection" explainer, ternary
+ *     sketch paragraph: ternary {-1,0,1} codes with one scale per block.
+ *   - MLX issue "2-bit quantized_matmul loses its size advantage over 4-bit
+ *     at M >= 3": the single quantized linear y = x W^T, group 128, M = 1..32.
+ *
+ * Conventions for every entry point:
+ *   - Return a qmoe_status; nothing aborts, no C++ exception crosses the ABI.
+ *   - Arguments are validated before any launch; a rejected call launches
+ *     nothing and writes nothing.
+ *   - Device entry points take device pointers and a cudaStream_t passed as
+ *     void* (NULL = legacy default stream); they enqueue work and return
+ *     without synchronising.  Host entry points (pack, unpack, sizes) are
+ *     synchronous and touch host memory only.
+ *   - All buffers are owned by the caller.  Device entry points allocate no
+ *     memory: scratch comes from the caller's workspace (ws, ws_bytes).
+ *   - Errors found on the device (a bounded wait that ran out) are recorded
+ *     in a device status word, read back by qmoe_get_stats().
+ *   - bf16 values are passed as uint16_t bit patterns.
+ */
+#ifndef QMOE_H
+#define QMOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  QMOE_OK = 0,
+  QMOE_ERR_INVALID_ARG = 1,   /* null pointer, bad size, bad enum value     */
+  QMOE_ERR_UNSUPPORTED = 2,   /* valid but outside what the kernels handle  */
+  QMOE_ERR_SCRATCH = 3,       /* workspace too small even for one token row */
+  QMOE_ERR_CUDA = 4,          /* a CUDA runtime call failed                 */
+  QMOE_ERR_TIMEOUT = 5        /* a device-side bounded wait ran out         */
+} qmoe_status;
+
+/* Weight code formats. */
+typedef enum {
+  QMOE_INT2 = 2,              /* symmetric, codes -2..1, 16 codes per u32          */
+  QMOE_TERNARY = 3,           /* codes -1, 0, 1, 5 trits per byte                   */
+  QMOE_INT4 = 4               /* symmetric, codes -8..7, 8 codes per u32            */
+} qmoe_fmt;
+
+/* Row order of a packed matrix.  GATE_UP is for FC1 whose logical rows
+ * interleave gate and up (row 2j = gate j, row 2j+1 = up j, the fused SwiGLU
+ * layout of the onnxruntime PR, Current Scope "swiglu_fusion=1"). */
+typedef enum { QMOE_ROWS_PLAIN = 0, QMOE_ROWS_GATE_UP = 1 } qmoe_row_order;
+
+/* Expert-compute path selection; AUTO picks per expert by its token count. */
+typedef enum { QMOE_PATH_AUTO = 0, QMOE_PATH_SMALL_M = 1, QMOE_PATH_GROUPED = 2 } qmoe_path;
+
+/* ------------------------------------------------------------------------
+ * Packed weight format (defined by this library).
+ *
+ * Quantization of a bf16 matrix W[rows, K] with block size B along K:
+ *   INT (bits b in {2,4}): s = bf16_rne(max|w| / 2^(b-1)) per (row, block);
+ *     c = clamp(rne(w / s), -2^(b-1), 2^(b-1)-1) computed in double; s == 0
+ *     gives c = 0.  Stored code u = c + 2^(b-1).
+ *   TERNARY (B = 64): delta = 0.7 * (sum|w| / 64) in double (sum in K order);
+ *     t = sign(w) if |w| > delta else 0; s = bf16_rne(mean |w| over the kept
+ *     weights), 0 if none.  Stored digit d = t + 1, base 3, 5 digits per byte.
+ *
+ * Physical layout (rows % 16 == 0).  Rows form tiles of 16 (NT = rows/16);
+ * tile row r of tile T is logical row 16T+r (PLAIN) or, for GATE_UP,
+ * 16T + 2r (r < 8, gate 8T+r) / 16T + 2(r-8) + 1 (r >= 8, up 8T+r-8).
+ * Each lane l (g = l/4, q = l%4) of a 32-lane warp owns the operand
+ * fragment of an m16n8k16 MMA: rows g and g+8, k = 16ks + 2q + {0,1} and
+ * 16ks + 2q + 8 + {0,1}.
+ *   INT2/INT4 codes: [K/64][NT][32 lanes][W u32], W = 2 (INT2) or 4 (INT4);
+ *     bytes = rows*K*bits/8.  Bit positions inside a lane's words follow the
+ *     register order of the kernels' unpack; qmoe_unpack_host() inverts it.
+ *   TERNARY codes: [K/128][NT][32 lanes][13 bytes]; bytes = rows*K*13/64 (1.625 bits per weight).
+ *   Scales: [K/B][NT][8 u32], u32 g = s(row g) | s(row g+8) << 16 (bf16 bits);
+ *     bytes = rows*(K/B)*2.
+ * A layer's experts are packed one after another with the same strides.
+ * ---------------------------------------------------------------------- */
+
+/* Sizes of one packed matrix.  Requires rows % 16 == 0, K % 64 == 0,
+ * block in {64, 128} (ternary: 64, K % 128 == 0; block 128: K % 128 == 0). */
+qmoe_status qmoe_pack_size(int fmt, int rows, int K, int block,
+                           size_t* codes_bytes, size_t* scales_bytes);
+
+/* Quantize and pack one bf16 matrix w[rows, K] (row-major, host memory) into
+ * codes / scales (host memory, sizes from qmoe_pack_size).  Deterministic. */
+qmoe_status qmoe_pack(int fmt, int row_order, const uint16_t* w, int rows, int K, int block,
+                      void* codes, void* scales);
+
+/* Inverse of the layout (host): logical signed codes [rows, K] (int8) and
+ * bf16 scales [rows, K/block].  Either output may be NULL. */
+qmoe_status qmoe_unpack_host(int fmt, int row_order, const void* codes, const void* scales,
+                             int rows, int K, int block, int8_t* codes_out, uint16_t* scales_out);
+
+/* One quantized weight set: n matrices of the same shape packed back to back
+ * (matrix e at codes + e*codes_bytes, scales + e*scales_bytes), optional bf16
+ * bias [n][rows] in logical row order (NULL = none).  Device pointers. */
+typedef struct {
+  int fmt;
+  int block;
+  const void* codes;
+  const void* scales;
+  const uint16_t* bias;
+} qmoe_weights;
+
+/* Dequantize n_mats packed matrices (device): out_f32[e][rows][K] = c*s
+ * (exact) and/or out_bf16 = bf16_rne(c*s), logical row order.  Debug and
+ * parity entry point; uses the hot kernels' unpack routines. */
+qmoe_status qmoe_dequant(const qmoe_weights* w, int row_order, int rows, int K, int n_mats,
+                         float* out_f32, uint16_t* out_bf16, void* stream);
+
+/* Routing (device): logits fp32 [T, E] -> ids int32 [T, k] (descending logit,
+ * ties to the lower index), weights fp32 [T, k] (softmax over the k selected
+ * logits), perm int32 [T*k] (flat index t*k+s at each expert-sorted
+ * position; stable), offsets int32 [E+1].  E <= 256, 1 <= k <= min(E, 32). */
+qmoe_status qmoe_route(const float* logits, int T, int E, int k, int32_t* ids, float* weights,
+                       int32_t* perm, int32_t* offsets, void* stream);
+
+/* One MoE layer.  fc1: E + n_shared matrices [2I, H] packed with
+ * QMOE_ROWS_GATE_UP (shared experts after the routed ones); bias [.][2I].
+ * fc2: E + n_shared matrices [H, I] packed with QMOE_ROWS_PLAIN; bias [.][H].
+ * H % 64 == 0, I % 64 == 0; E <= 256; shared experts get every token with
+ * weight 1.  max_row_tile bounds the tokens per row tile (0 = none). */
+typedef struct {
+  int H, I, E, k, n_shared;
+  qmoe_weights fc1;
+  qmoe_weights fc2;
+  int path;
+  int max_row_tile;
+} qmoe_layer;
+
+/* Workspace for qmoe_forward over T tokens without row tiling. */
+qmoe_status qmoe_workspace_size(const qmoe_layer* layer, int T, size_t* bytes);
+
+/* y[T, H] bf16 = MoE(x[T, H] bf16, logits[T, E] fp32).  With ws_bytes below
+ * qmoe_workspace_size(T), tokens are processed in row tiles (halved until the
+ * tile's workspace fits, explicit partial last tile); QMOE_ERR_SCRATCH when
+ * one row does not fit.  ws must be 256-byte aligned. */
+qmoe_status qmoe_forward(const qmoe_layer* layer, const uint16_t* x, const float* logits, int T,
+                         uint16_t* y, void* ws, size_t ws_bytes, void* stream);
+
+/* Single quantized linear y[M, N] bf16 = x[M, K] bf16 @ dequant(W)[N, K]^T,
+ * W packed PLAIN.  M >= 1. */
+qmoe_status qmoe_linear_workspace_size(int N, int K, int M, size_t* bytes);
+qmoe_status qmoe_linear(const qmoe_weights* w, int N, int K, const uint16_t* x, int M,
+                        uint16_t* y, void* ws, size_t ws_bytes, void* stream);
+
+/* Per-launch GPU timing (tracing).  After qmoe_trace_start(cap) every kernel
+ * the library launches - also while the stream is being captured into a CUDA
+ * graph - is bracketed by CUDA events, up to cap launches; qmoe_trace_stop()
+ * ends recording.  qmoe_trace_read() synchronizes the device and returns per
+ * recorded launch its kernel id (qmoe_kernel_name) and duration in ms; for a
+ * launch replayed from a graph, the duration of its latest execution. */
+qmoe_status qmoe_trace_start(int cap);
+qmoe_status qmoe_trace_stop(void);
+qmoe_status qmoe_trace_read(int cap, int* n, int* kernel_ids, float* ms);
+const char* qmoe_kernel_name(int kernel_id);
+
+typedef struct {
+  int last_path;          /* path the last qmoe_forward / qmoe_linear took  */
+  int row_tiles;          /* row tiles of the last qmoe_forward             */
+  int row_tile_tokens;    /* tokens per full row tile                       */
+  int small_launches;     /* small-M expert kernels launched by the last call */
+  int grouped_launches;   /* grouped (tcgen05) kernels launched by the last call */
+  uint32_t device_status; /* OR of device error flags since the last clear  */
+} qmoe_stats;
+
+/* Host-side stats of the last call plus the device status word (this call
+ * synchronises the current device to read it). */
+qmoe_status qmoe_get_stats(qmoe_stats* out);
+qmoe_status qmoe_clear_status(void);
+const char* qmoe_status_str(int status);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* QMOE_H */

@@ -1,0 +1,360 @@
+// Routing, activation gather, combine, single-linear setup and dequant kernels.
+#pragma once
+#include <cfloat>
+#include <climits>
+
+#include "device_common.cuh"
+#include "qmm_grouped.cuh"
+#include "qmm_small.cuh"
+#include "unpack.cuh"
+
+namespace qmoe {
+
+constexpr int kRouteThreads = 1024;
+constexpr int kMaxExperts = 256;
+
+struct RouteOut {
+  int* ids;          // [T*k]
+  float* w;          // [T*k]
+  int* perm;         // [T*k] position -> flat index
+  int* inv;          // [T*k] flat index -> position (may be null)
+  int* offsets;      // [E+1]
+  int* slot_token;   // [T*(k+n_shared)] (may be null)
+  int* nseg;         // segment count (may be null: no segment table)
+  Seg* segs;
+  int max_seg;
+  int* tickets;      // zeroed (may be null)
+  int n_tickets;
+  int thresh;        // experts with more tokens than this go to the grouped path
+  int* ngseg;        // grouped tile count (may be null: no grouped table)
+  GSeg* gsegs;
+  int max_gseg;
+  unsigned* status;
+};
+
+// One CTA: warp top-k per token, then a stable counting sort by expert (ranks
+// from warp match masks, offsets from a prefix over warps in warp order), then
+// the (expert, chunk of <= 16 tokens) segment table.  Deterministic.
+__global__ void __launch_bounds__(kRouteThreads, 1)
+    route_kernel(const float* __restrict__ logits, int T, int E, int k, int n_shared, RouteOut o) {
+  __shared__ int counts[kMaxExperts];
+  __shared__ int running[kMaxExperts];
+  __shared__ int warp_cnt[32][kMaxExperts];
+  __shared__ float selv[32][32];
+  __shared__ int seg_base[kMaxExperts + 64];
+  __shared__ int tg_base[kMaxExperts + 64];
+  __shared__ int gseg_base[kMaxExperts + 64];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int nwarps = blockDim.x >> 5;
+
+  for (int e = tid; e < kMaxExperts; e += blockDim.x) { counts[e] = 0; running[e] = 0; }
+
+  // ---- top-k per token (ties to the lower expert index) ----
+  for (int t = warp; t < T; t += nwarps) {
+    float v[kMaxExperts / 32];
+    unsigned taken = 0;
+#pragma unroll
+    for (int j = 0; j < kMaxExperts / 32; ++j) {
+      const int idx = lane + 32 * j;
+      v[j] = idx < E ? logits[(size_t)t * E + idx] : -FLT_MAX;
+    }
+    for (int s = 0; s < k; ++s) {
+      float bv = -FLT_MAX;
+      int bi = INT_MAX;
+#pragma unroll
+      for (int j = 0; j < kMaxExperts / 32; ++j) {
+        const int idx = lane + 32 * j;
+        if (idx < E && !((taken >> j) & 1u) && (bi == INT_MAX || v[j] > bv)) { bv = v[j]; bi = idx; }
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+        const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+        if (oi != INT_MAX && (bi == INT_MAX || ov > bv || (ov == bv && oi < bi))) { bv = ov; bi = oi; }
+      }
+      if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+      if (lane == 0) {
+        o.ids[(size_t)t * k + s] = bi;
+        selv[warp][s] = bv;
+      }
+    }
+    __syncwarp();
+    if (lane < k) {
+      const float lmax = selv[warp][0];
+      float sum = 0.f;
+      for (int s = 0; s < k; ++s) sum += expf(selv[warp][s] - lmax);
+      o.w[(size_t)t * k + lane] = expf(selv[warp][lane] - lmax) / sum;
+    }
+    __syncwarp();
+  }
+  __syncthreads();
+
+  // ---- counts and offsets ----
+  const int TK = T * k;
+  for (int i = tid; i < TK; i += blockDim.x) atomicAdd(&counts[o.ids[i]], 1);
+  __syncthreads();
+  if (tid == 0) {
+    int acc = 0;
+    for (int e = 0; e < E; ++e) { o.offsets[e] = acc; seg_base[e] = acc; acc += counts[e]; }
+    o.offsets[E] = acc;
+  }
+  __syncthreads();
+
+  // ---- stable scatter ----
+  const unsigned lt_mask = (1u << lane) - 1u;
+  for (int base = 0; base < TK; base += blockDim.x) {
+    for (int j = tid; j < 32 * kMaxExperts; j += blockDim.x) (&warp_cnt[0][0])[j] = 0;
+    __syncthreads();
+    const int i = base + tid;
+    const bool valid = i < TK;
+    const int e = valid ? o.ids[i] : -1;
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    const int rank = __popc(peers & lt_mask);
+    if (valid && rank == 0) warp_cnt[warp][e] = __popc(peers);
+    __syncthreads();
+    if (valid) {
+      int pre = running[e];
+      for (int w = 0; w < warp; ++w) pre += warp_cnt[w][e];
+      const int pos = seg_base[e] + pre + rank;
+      o.perm[pos] = i;
+      if (o.inv) o.inv[i] = pos;
+      if (o.slot_token) o.slot_token[pos] = i / k;
+    }
+    __syncthreads();
+    for (int ee = tid; ee < E; ee += blockDim.x) {
+      int sum = 0;
+      for (int w = 0; w < 32; ++w) sum += warp_cnt[w][ee];
+      running[ee] += sum;
+    }
+    __syncthreads();
+  }
+  if (o.slot_token)
+    for (int i = tid; i < n_shared * T; i += blockDim.x) o.slot_token[TK + i] = i % T;
+
+  // ---- segment tables: small-M chunks of <= 16 tokens, grouped tiles of <= 256 ----
+  if (o.nseg) {
+    const int EX = E + n_shared;
+    __syncthreads();
+    if (tid == 0) {
+      int sb = 0, tb = 0, gb = 0;
+      for (int e = 0; e < EX; ++e) {
+        const int cnt = e < E ? counts[e] : T;
+        const bool grouped = o.ngseg && cnt > o.thresh;
+        seg_base[e] = sb;
+        tg_base[e] = tb;
+        gseg_base[e] = gb;
+        if (grouped) {
+          gb += (cnt + kGTok - 1) / kGTok;
+        } else {
+          sb += (cnt + kChunkTokens - 1) / kChunkTokens;
+          tb += 2 * (cnt / kChunkTokens) + ((cnt % kChunkTokens) + 7) / 8;
+        }
+      }
+      if (sb > o.max_seg || (o.ngseg && gb > o.max_gseg)) {
+        atomicOr(o.status, kStatusBadSegment);
+        sb = 0;  // never index past the tables
+        gb = 0;
+      }
+      *o.nseg = sb;
+      if (o.ngseg) *o.ngseg = gb;
+    }
+    __syncthreads();
+    const bool ok = *o.nseg > 0 || (o.ngseg && *o.ngseg > 0);
+    for (int e = tid; e < EX && ok; e += blockDim.x) {
+      const int cnt = e < E ? counts[e] : T;
+      const int slot_base = e < E ? o.offsets[e] : TK + (e - E) * T;
+      if (o.ngseg && cnt > o.thresh) {
+        const int nch = (cnt + kGTok - 1) / kGTok;
+        for (int c = 0; c < nch; ++c) {
+          GSeg g;
+          g.expert = e;
+          g.slot0 = slot_base + kGTok * c;
+          g.ntok = min(kGTok, cnt - kGTok * c);
+          g.pad = 0;
+          o.gsegs[gseg_base[e] + c] = g;
+        }
+        continue;
+      }
+      const int nch = (cnt + kChunkTokens - 1) / kChunkTokens;
+      for (int c = 0; c < nch; ++c) {
+        Seg s;
+        s.expert = e;
+        s.m = min(kChunkTokens, cnt - kChunkTokens * c);
+        s.tg = (s.m + 7) / 8;
+        s.slot0 = slot_base + kChunkTokens * c;
+        s.xoff = tg_base[e] + 2 * c;
+        s.pad[0] = s.pad[1] = s.pad[2] = 0;
+        o.segs[seg_base[e] + c] = s;
+      }
+    }
+  }
+  if (o.tickets)
+    for (int i = tid; i < o.n_tickets; i += blockDim.x) o.tickets[i] = 0;
+}
+
+// Segment table of a single linear: chunks of <= 16 consecutive tokens.
+__global__ void linear_setup_kernel(int M, int* nseg, Seg* segs, int* tickets, int n_tickets) {
+  const int nchunks = (M + kChunkTokens - 1) / kChunkTokens;
+  for (int c = threadIdx.x; c < nchunks; c += blockDim.x) {
+    Seg s;
+    s.expert = 0;
+    s.m = min(kChunkTokens, M - kChunkTokens * c);
+    s.tg = (s.m + 7) / 8;
+    s.slot0 = kChunkTokens * c;
+    s.xoff = 2 * c;
+    s.pad[0] = s.pad[1] = s.pad[2] = 0;
+    segs[c] = s;
+  }
+  if (threadIdx.x == 0) *nseg = nchunks;
+  for (int i = threadIdx.x; i < n_tickets; i += blockDim.x) tickets[i] = 0;
+}
+
+// Activation operand fragments: for each segment, token group and 64-column
+// block, lane l = 4g + q stores x[token g][16ks + 2q + {0,1}] and
+// [16ks + 2q + 8 + {0,1}] for ks = 0..3 (the m16n8k16 B fragment), the second
+// pair divided by beta_hi (exact power-of-two scaling).  Padding tokens are 0.
+__global__ void gather_kernel(const uint16_t* __restrict__ x, int K, const int* __restrict__ slot_token,
+                              const int* __restrict__ nseg, const Seg* __restrict__ segs, uint8_t* frag,
+                              int beta_hi) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  const int g = lane >> 2, q = lane & 3;
+  const int KB = K / 64;
+  const int ns = *nseg;
+  for (int s = blockIdx.x; s < ns; s += gridDim.x) {
+    const Seg sg = segs[s];
+    const int items = KB * sg.tg;
+    uint8_t* base = frag + (size_t)sg.xoff * K * 16;
+    for (int it = warp; it < items; it += nw) {
+      const int kb = it / sg.tg, tg = it % sg.tg;
+      const int n = tg * 8 + g;
+      uint32_t r[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) r[j] = 0u;
+      if (n < sg.m) {
+        const int tok = slot_token ? slot_token[sg.slot0 + n] : sg.slot0 + n;
+        const uint32_t* row = reinterpret_cast<const uint32_t*>(x + (size_t)tok * K + kb * 64);
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+          r[2 * ks] = row[(16 * ks + 2 * q) >> 1];
+          uint32_t hi = row[(16 * ks + 2 * q + 8) >> 1];
+          if (beta_hi == 4) hi = fma_bf16x2(hi, kBf16Quarter, 0x80008000u);
+          r[2 * ks + 1] = hi;
+        }
+      }
+      uint4* dst = reinterpret_cast<uint4*>(base + ((size_t)(kb * sg.tg + tg) * 32 + lane) * 32);
+      dst[0] = make_uint4(r[0], r[1], r[2], r[3]);
+      dst[1] = make_uint4(r[4], r[5], r[6], r[7]);
+    }
+  }
+}
+
+// Token rows of the grouped tiles, in expert-sorted slot order: xrows[slot] = x[token(slot)].
+__global__ void gather_rows_kernel(const uint16_t* __restrict__ x, int K, const int* __restrict__ slot_token,
+                                   const int* __restrict__ ngseg, const GSeg* __restrict__ gsegs, uint16_t* xrows) {
+  const int ng = *ngseg;
+  const int vec = K / 8;  // uint4 per row
+  for (int gi = blockIdx.x; gi < ng; gi += gridDim.x) {
+    const GSeg g = gsegs[gi];
+    for (int i = threadIdx.x; i < g.ntok * vec; i += blockDim.x) {
+      const int r = i / vec, c = i % vec;
+      const int slot = g.slot0 + r;
+      const int tok = slot_token[slot];
+      reinterpret_cast<uint4*>(xrows + (size_t)slot * K)[c] = reinterpret_cast<const uint4*>(x + (size_t)tok * K)[c];
+    }
+  }
+}
+
+// y[t] = sum_s w[t,s] * yslot[inv[t*k+s]] + sum_j yslot[T*k + j*T + t], fixed order, bf16 out.
+__global__ void combine_kernel(const float* __restrict__ yslot, const float* __restrict__ w,
+                               const int* __restrict__ inv, int T, int k, int n_shared, int H,
+                               uint16_t* __restrict__ y) {
+  const int t = blockIdx.x;
+  for (int h = threadIdx.x * 4; h < H; h += blockDim.x * 4) {
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s = 0; s < k; ++s) {
+      const float ws = w[(size_t)t * k + s];
+      const float4 v = *reinterpret_cast<const float4*>(yslot + (size_t)inv[(size_t)t * k + s] * H + h);
+      acc.x = fmaf(ws, v.x, acc.x); acc.y = fmaf(ws, v.y, acc.y);
+      acc.z = fmaf(ws, v.z, acc.z); acc.w = fmaf(ws, v.w, acc.w);
+    }
+    for (int j = 0; j < n_shared; ++j) {
+      const float4 v = *reinterpret_cast<const float4*>(yslot + ((size_t)T * k + (size_t)j * T + t) * H + h);
+      acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+    }
+    uint2 out;
+    out.x = pack_bf16x2(acc.x, acc.y);
+    out.y = pack_bf16x2(acc.z, acc.w);
+    *reinterpret_cast<uint2*>(y + (size_t)t * H + h) = out;
+  }
+}
+
+// Dequantize through the hot kernels' unpack: one warp per (matrix, k-unit, tile).
+template <int FMT>
+__global__ void dequant_kernel(const uint8_t* __restrict__ codes, unsigned long long cstride,
+                               const uint8_t* __restrict__ scales, unsigned long long sstride, int NT, int K,
+                               int block, int row_order, int nmat, float* o32, uint16_t* o16) {
+  using Tr = FmtTraits<FMT>;
+  __shared__ uint32_t lut[243];
+  if constexpr (FMT == 3)
+    for (int i = threadIdx.x; i < 243; i += blockDim.x) lut[i] = tern_lut_entry(i);
+  __syncthreads();
+  const int lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
+  const int KU = K / Tr::kKUcols;
+  const long long items = (long long)nmat * KU * NT;
+  const long long wid = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const long long nwt = ((long long)gridDim.x * blockDim.x) >> 5;
+  const int bias = FMT == 3 ? 1 : (1 << (FMT - 1));
+  const int rows = NT * 16;
+  for (long long itm = wid; itm < items; itm += nwt) {
+    const int e = (int)(itm / ((long long)KU * NT));
+    const int r = (int)(itm % ((long long)KU * NT));
+    const int ku = r / NT, t = r % NT;
+    const uint8_t* cp = codes + (unsigned long long)e * cstride + ((unsigned long long)ku * NT + t) * Tr::kCodeBytes;
+    constexpr int NKS = Tr::kKUcols / 16;
+    uint32_t am[NKS][4];
+    if constexpr (FMT == 2) {
+      const uint2 w = *reinterpret_cast<const uint2*>(cp + lane * 8);
+      uint32_t (&a0)[4] = am[0]; uint32_t (&a1)[4] = am[1];
+      uint32_t (&a2)[4] = am[2 % NKS]; uint32_t (&a3)[4] = am[3 % NKS];
+      unpack_int2_word(w.x, a0, a1);
+      unpack_int2_word(w.y, a2, a3);
+    } else if constexpr (FMT == 4) {
+      const uint4 w = *reinterpret_cast<const uint4*>(cp + lane * 16);
+      unpack_int4_word(w.x, am[0]);
+      unpack_int4_word(w.y, am[1 % NKS]);
+      unpack_int4_word(w.z, am[2 % NKS]);
+      unpack_int4_word(w.w, am[3 % NKS]);
+    } else {
+      uint8_t rec[13];
+      for (int i = 0; i < 13; ++i) rec[i] = cp[lane * 13 + i];
+      uint32_t ta[8][4];
+      unpack_tern_record(rec, lut, ta);
+#pragma unroll
+      for (int ks = 0; ks < NKS; ++ks)
+#pragma unroll
+        for (int f = 0; f < 4; ++f) am[ks][f] = ta[ks % 8][f];
+    }
+    const uint8_t* sp = scales + (unsigned long long)e * sstride;
+#pragma unroll
+    for (int ks = 0; ks < NKS; ++ks)
+#pragma unroll
+      for (int f = 0; f < 4; ++f)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const float raw = h ? bf16_hi(am[ks][f]) : bf16_lo(am[ks][f]);
+          const float beta = (f >= 2) ? (float)Tr::kBetaHi : 1.0f;
+          const float c = (raw - 128.0f) / beta - (float)bias;
+          const int pr = g + 8 * (f & 1);
+          const int k = ku * Tr::kKUcols + 16 * ks + 2 * q + 8 * (f >> 1) + h;
+          const uint32_t sw = *reinterpret_cast<const uint32_t*>(sp + (((size_t)(k / block) * NT + t) * 8 + (pr & 7)) * 4);
+          const float s = pr < 8 ? bf16_lo(sw) : bf16_hi(sw);
+          const int lr = row_order == 1 ? 16 * t + (pr < 8 ? 2 * pr : 2 * (pr - 8) + 1) : 16 * t + pr;
+          const size_t o = ((size_t)e * rows + lr) * K + k;
+          const float val = c * s;
+          if (o32) o32[o] = val;
+          if (o16) o16[o] = __bfloat16_as_ushort(__float2bfloat16_rn(val));
+        }
+  }
+}
+
+}  // namespace qmoe

@@ -1,0 +1,292 @@
+// Host quantizer + packer and its inverse (C ABI: qmoe_pack_size, qmoe_pack,
+// qmoe_unpack_host).
+//
+// Quantization follows the onnxruntime PR "Enable SM80+ FP16/BF16 mixed
+// INT2/INT4 QMoE prefill by default", Current Scope (symmetric, no zero
+// points, block 64) and, for ternary, the channel-selection explainer's
+// ternary sketch (three values plus one scale per block); the exact scale and
+// threshold rules are stated in qmoe.h.
+#include <cmath>
+#include <cstring>
+#include <vector>
+
+#include "qmoe.h"
+#include "layout.h"
+
+namespace {
+
+double bf16_to_double(uint16_t b) {
+  uint32_t u = (uint32_t)b << 16;
+  float f;
+  std::memcpy(&f, &u, 4);
+  return (double)f;
+}
+
+// Nearest bf16 (8 significant bits, ties to even) of a finite double.
+uint16_t double_to_bf16(double v) {
+  if (v == 0.0) return std::signbit(v) ? 0x8000 : 0;
+  int e;
+  std::frexp(v, &e);                              // v = m * 2^e, 0.5 <= |m| < 1
+  int q = (e < -125 ? -125 : e) - 8;              // unit in the last place
+  double r = std::nearbyint(std::ldexp(v, -q));   // default rounding: half to even
+  double rv = std::ldexp(r, q);
+  float f = (float)rv;                            // exact: rv has <= 8 significant bits
+  uint32_t u;
+  std::memcpy(&u, &f, 4);
+  return (uint16_t)(u >> 16);
+}
+
+bool fmt_ok(int fmt) { return fmt == QMOE_INT2 || fmt == QMOE_INT4 || fmt == QMOE_TERNARY; }
+
+qmoe_status check_shape(int fmt, int rows, int K, int block) {
+  if (!fmt_ok(fmt)) return QMOE_ERR_INVALID_ARG;
+  if (rows <= 0 || K <= 0 || rows % 16 || K % 64) return QMOE_ERR_INVALID_ARG;
+  if (block != 64 && block != 128) return QMOE_ERR_UNSUPPORTED;
+  if (K % block) return QMOE_ERR_INVALID_ARG;
+  if (fmt == QMOE_TERNARY && (block != 64 || K % 128)) return QMOE_ERR_UNSUPPORTED;
+  return QMOE_OK;
+}
+
+size_t codes_bytes_of(int fmt, int rows, int K) {
+  if (fmt == QMOE_TERNARY) return (size_t)rows * (K / 128) * 26;  // 13 bytes per 64 weights
+  return (size_t)rows * K * fmt / 8;
+}
+
+// Quantize one row-block; writes signed codes c[0..B) and returns the bf16 scale bits.
+uint16_t quantize_block(int fmt, const uint16_t* w, int B, int8_t* c) {
+  if (fmt == QMOE_TERNARY) {
+    double sum_abs = 0.0;
+    for (int i = 0; i < B; ++i) sum_abs += std::fabs(bf16_to_double(w[i]));
+    double delta = 0.7 * (sum_abs / (double)B);
+    double sel = 0.0;
+    int cnt = 0;
+    for (int i = 0; i < B; ++i) {
+      double v = bf16_to_double(w[i]);
+      double a = std::fabs(v);
+      if (a > delta) {
+        c[i] = v > 0 ? 1 : -1;
+        sel += a;
+        ++cnt;
+      } else {
+        c[i] = 0;
+      }
+    }
+    return cnt ? double_to_bf16(sel / (double)cnt) : 0;
+  }
+  const int bits = fmt;
+  const int qmin = -(1 << (bits - 1)), qmax = (1 << (bits - 1)) - 1;
+  double amax = 0.0;
+  for (int i = 0; i < B; ++i) amax = std::fmax(amax, std::fabs(bf16_to_double(w[i])));
+  uint16_t sb = double_to_bf16(amax / (double)(1 << (bits - 1)));
+  double s = bf16_to_double(sb);
+  for (int i = 0; i < B; ++i) {
+    if (s > 0) {
+      double q = std::nearbyint(bf16_to_double(w[i]) / s);
+      if (q < qmin) q = qmin;
+      if (q > qmax) q = qmax;
+      c[i] = (int8_t)q;
+    } else {
+      c[i] = 0;
+    }
+  }
+  return sb;
+}
+
+// Physical position of logical element (tile row tr of tile t, column k) for INT formats:
+// returns (word index within the whole codes array, bit shift).
+inline void int_position(int fmt, int NT, int t, int tr, int k, size_t* word, int* shift) {
+  const int kb = k / 64, kk = k % 64;
+  const int ks = kk / 16, kc = kk % 16;
+  const int hi8 = kc >= 8;                  // f >> 1
+  const int q = (kc % 8) / 2, h = kc % 2;
+  const int g = tr % 8, rh = tr / 8;        // f & 1
+  const int f = rh | (hi8 << 1);
+  const int lane = 4 * g + q;
+  const int W = fmt == QMOE_INT2 ? 2 : 4;
+  int wi, slot;
+  if (fmt == QMOE_INT2) {
+    wi = ks / 2;
+    int m = -1;
+    for (int j = 0; j < 8; ++j)
+      if (qmoe::kInt2KsF[j][0] == ks % 2 && qmoe::kInt2KsF[j][1] == f) m = j;
+    slot = 2 * m + 16 * h;
+  } else {
+    wi = ks;
+    slot = 4 * f + 16 * h;
+  }
+  *word = (((size_t)kb * NT + t) * 32 + lane) * W + wi;
+  *shift = slot;
+}
+
+// Ternary: byte offset of the lane record and digit position for logical element.
+inline void tern_position(int NT, int t, int tr, int k, size_t* byte, int* pos) {
+  const int kp = k / 128, kk = k % 128;
+  const int ks = kk / 16, kc = kk % 16;
+  const int hi8 = kc >= 8;
+  const int q = (kc % 8) / 2, h = kc % 2;
+  const int g = tr % 8, rh = tr / 8;
+  const int f = rh | (hi8 << 1);
+  const int lane = 4 * g + q;
+  const int* list = hi8 ? qmoe::kTernHi : qmoe::kTernLo;
+  const int reg = list[2 * ks + rh];
+  (void)f;
+  const int* d = qmoe::kTernRegDigits[reg];
+  const int b = h ? d[2] : d[0];
+  *pos = h ? d[3] : d[1];
+  *byte = (((size_t)kp * NT + t) * 32 + lane) * 13 + b;
+}
+
+const int kPow3[5] = {1, 3, 9, 27, 81};
+
+// Per (tile row, column within the 64/128-column unit): word/byte offset inside
+// the unit's tile slab and the shift/digit position.
+struct PosTable {
+  int off[2][16][128];
+  int sh[2][16][128];
+  PosTable() {
+    for (int which = 0; which < 2; ++which)       // 0: INT2 (64 cols), 1: INT4 (64 cols)
+      for (int tr = 0; tr < 16; ++tr)
+        for (int k = 0; k < 64; ++k) {
+          size_t w;
+          int s;
+          int_position(which == 0 ? QMOE_INT2 : QMOE_INT4, 1, 0, tr, k, &w, &s);
+          off[which][tr][k] = (int)w;
+          sh[which][tr][k] = s;
+        }
+  }
+};
+struct TernTable {
+  int off[16][128];
+  int pos[16][128];
+  TernTable() {
+    for (int tr = 0; tr < 16; ++tr)
+      for (int k = 0; k < 128; ++k) {
+        size_t b;
+        int p;
+        tern_position(1, 0, tr, k, &b, &p);
+        off[tr][k] = (int)b;
+        pos[tr][k] = p;
+      }
+  }
+};
+const PosTable& pos_table() { static PosTable t; return t; }
+const TernTable& tern_table() { static TernTable t; return t; }
+
+}  // namespace
+
+extern "C" {
+
+qmoe_status qmoe_pack_size(int fmt, int rows, int K, int block, size_t* codes_bytes,
+                           size_t* scales_bytes) {
+  qmoe_status st = check_shape(fmt, rows, K, block);
+  if (st != QMOE_OK) return st;
+  if (codes_bytes) *codes_bytes = codes_bytes_of(fmt, rows, K);
+  if (scales_bytes) *scales_bytes = (size_t)rows * (K / block) * 2;
+  return QMOE_OK;
+}
+
+qmoe_status qmoe_pack(int fmt, int row_order, const uint16_t* w, int rows, int K, int block,
+                      void* codes, void* scales) {
+  qmoe_status st = check_shape(fmt, rows, K, block);
+  if (st != QMOE_OK) return st;
+  if (row_order != QMOE_ROWS_PLAIN && row_order != QMOE_ROWS_GATE_UP) return QMOE_ERR_INVALID_ARG;
+  if (!w || !codes || !scales) return QMOE_ERR_INVALID_ARG;
+  const int NT = rows / 16, SB = K / block;
+  const size_t cbytes = codes_bytes_of(fmt, rows, K);
+  uint8_t* cb = static_cast<uint8_t*>(codes);
+  uint32_t* sc = static_cast<uint32_t*>(scales);
+  if (fmt == QMOE_TERNARY) {
+    // every digit starts as 1 (t = 0), which also fills the padding digit
+    std::vector<uint8_t> digits(cbytes * 5, 1);
+    const TernTable& tt = tern_table();
+#pragma omp parallel for schedule(static)
+    for (int t = 0; t < NT; ++t) {
+      std::vector<int8_t> c(block);
+      for (int tr = 0; tr < 16; ++tr) {
+        const int lr = qmoe::logical_row(row_order, t, tr);
+        for (int b = 0; b < SB; ++b) {
+          uint16_t s = quantize_block(fmt, w + (size_t)lr * K + (size_t)b * block, block, c.data());
+          uint32_t& slot = sc[((size_t)b * NT + t) * 8 + (tr % 8)];
+          if (tr < 8) slot = (slot & 0xFFFF0000u) | s; else slot = (slot & 0xFFFFu) | ((uint32_t)s << 16);
+          for (int i = 0; i < block; ++i) {
+            const int k = b * block + i;
+            const size_t unit = ((size_t)(k / 128) * NT + t) * 32 * 13;
+            digits[(unit + tt.off[tr][k % 128]) * 5 + tt.pos[tr][k % 128]] = (uint8_t)(c[i] + 1);
+          }
+        }
+      }
+    }
+#pragma omp parallel for schedule(static)
+    for (size_t i = 0; i < cbytes; ++i) {
+      int v = 0;
+      for (int p = 0; p < 5; ++p) v += digits[i * 5 + p] * kPow3[p];
+      cb[i] = (uint8_t)v;
+    }
+    return QMOE_OK;
+  }
+  std::memset(codes, 0, cbytes);
+  uint32_t* cw = static_cast<uint32_t*>(codes);
+  const int bias = 1 << (fmt - 1);
+  const PosTable& pt = pos_table();
+  const int which = fmt == QMOE_INT2 ? 0 : 1;
+  const int W = fmt == QMOE_INT2 ? 2 : 4;
+#pragma omp parallel for schedule(static)
+  for (int t = 0; t < NT; ++t) {
+    std::vector<int8_t> c(block);
+    for (int tr = 0; tr < 16; ++tr) {
+      const int lr = qmoe::logical_row(row_order, t, tr);
+      for (int b = 0; b < SB; ++b) {
+        uint16_t s = quantize_block(fmt, w + (size_t)lr * K + (size_t)b * block, block, c.data());
+        uint32_t& slot = sc[((size_t)b * NT + t) * 8 + (tr % 8)];
+        if (tr < 8) slot = (slot & 0xFFFF0000u) | s; else slot = (slot & 0xFFFFu) | ((uint32_t)s << 16);
+        for (int i = 0; i < block; ++i) {
+          const int k = b * block + i;
+          const size_t unit = ((size_t)(k / 64) * NT + t) * 32 * W;
+          cw[unit + pt.off[which][tr][k % 64]] |= (uint32_t)(c[i] + bias) << pt.sh[which][tr][k % 64];
+        }
+      }
+    }
+  }
+  return QMOE_OK;
+}
+
+qmoe_status qmoe_unpack_host(int fmt, int row_order, const void* codes, const void* scales, int rows,
+                             int K, int block, int8_t* codes_out, uint16_t* scales_out) {
+  qmoe_status st = check_shape(fmt, rows, K, block);
+  if (st != QMOE_OK) return st;
+  if (row_order != QMOE_ROWS_PLAIN && row_order != QMOE_ROWS_GATE_UP) return QMOE_ERR_INVALID_ARG;
+  if ((codes_out && !codes) || (scales_out && !scales)) return QMOE_ERR_INVALID_ARG;
+  const int NT = rows / 16, SB = K / block;
+  for (int t = 0; t < NT; ++t)
+    for (int tr = 0; tr < 16; ++tr) {
+      const int lr = qmoe::logical_row(row_order, t, tr);
+      if (scales_out) {
+        const uint32_t* sc = static_cast<const uint32_t*>(scales);
+        for (int b = 0; b < SB; ++b) {
+          uint32_t v = sc[((size_t)b * NT + t) * 8 + (tr % 8)];
+          scales_out[(size_t)lr * SB + b] = (uint16_t)(tr < 8 ? (v & 0xFFFF) : (v >> 16));
+        }
+      }
+      if (!codes_out) continue;
+      for (int k = 0; k < K; ++k) {
+        int8_t c;
+        if (fmt == QMOE_TERNARY) {
+          size_t byte;
+          int pos;
+          tern_position(NT, t, tr, k, &byte, &pos);
+          int v = static_cast<const uint8_t*>(codes)[byte];
+          c = (int8_t)((v / kPow3[pos]) % 3 - 1);
+        } else {
+          size_t word;
+          int shift;
+          int_position(fmt, NT, t, tr, k, &word, &shift);
+          uint32_t v = static_cast<const uint32_t*>(codes)[word];
+          c = (int8_t)((int)((v >> shift) & ((1u << fmt) - 1)) - (1 << (fmt - 1)));
+        }
+        codes_out[(size_t)lr * K + k] = c;
+      }
+    }
+  return QMOE_OK;
+}
+
+}  // extern "C"

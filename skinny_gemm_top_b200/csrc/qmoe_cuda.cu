@@ -1,0 +1,632 @@
+// C ABI of the device entry points: qmoe_route, qmoe_forward, qmoe_linear,
+// qmoe_dequant, workspace sizing, stats.  One translation unit holds every
+// kernel so that the device status word is a single symbol.
+//
+// The MoE layer follows the onnxruntime PR "Enable SM80+ FP16/BF16 mixed
+// INT2/INT4 QMoE prefill by default" (Description; Current Scope): route,
+// expand rows by expert, FC1 with expert bias and interleaved SwiGLU, FC2,
+// top-k weighted finalize with FC2 bias, row tiling within a scratch budget.
+#include <algorithm>
+#include <climits>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "qmoe.h"
+#include "device_common.cuh"
+#include "unpack.cuh"
+#include "qmm_small.cuh"
+#include "qmm_grouped.cuh"
+#include "kernels_misc.cuh"
+
+#include <cudaTypedefs.h>
+
+namespace qmoe {
+
+__device__ unsigned g_status;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr size_t kAlign = 256;
+constexpr int kSmemLimit = 227 * 1024;
+
+struct DevInfo {
+  bool init = false;
+  int sms = 0;
+  unsigned* status = nullptr;
+};
+DevInfo g_dev[kMaxDevices];
+std::mutex g_mu;
+qmoe_stats g_stats = {};
+
+qmoe_status dev_info(DevInfo** out) {
+  int d = 0;
+  if (cudaGetDevice(&d) != cudaSuccess || d < 0 || d >= kMaxDevices) return QMOE_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_mu);
+  DevInfo& di = g_dev[d];
+  if (!di.init) {
+    if (cudaDeviceGetAttribute(&di.sms, cudaDevAttrMultiProcessorCount, d) != cudaSuccess) return QMOE_ERR_CUDA;
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_status) != cudaSuccess) return QMOE_ERR_CUDA;
+    di.status = static_cast<unsigned*>(p);
+    di.init = true;
+  }
+  *out = &di;
+  return QMOE_OK;
+}
+
+// ---- tracing: CUDA events around each kernel launch ----
+enum KernelId { K_ROUTE = 0, K_GATHER, K_FC1_SMALL, K_FC2_SMALL, K_COMBINE, K_LINEAR_SMALL, K_LINEAR_SETUP,
+                K_DEQUANT, K_FC1_GROUPED, K_FC2_GROUPED, K_COUNT };
+const char* const kKernelNames[K_COUNT] = {"route", "gather", "fc1_small", "fc2_small", "combine", "linear_small",
+                                           "linear_setup", "dequant", "fc1_grouped", "fc2_grouped"};
+struct Tracer {
+  bool on = false;
+  int cap = 0, n = 0;
+  std::vector<cudaEvent_t> ev;
+  std::vector<int> ids;
+} g_trace;
+
+void record_event(cudaEvent_t e, cudaStream_t st) {
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  cudaStreamIsCapturing(st, &cs);
+  if (cs == cudaStreamCaptureStatusActive) cudaEventRecordWithFlags(e, st, cudaEventRecordExternal);
+  else cudaEventRecord(e, st);
+}
+
+// Brackets one launch with events while tracing is on.
+struct TraceScope {
+  cudaStream_t st;
+  int id, slot = -1;
+  TraceScope(cudaStream_t s, int kid) : st(s), id(kid) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (g_trace.on && g_trace.n < g_trace.cap) {
+      slot = g_trace.n++;
+      g_trace.ids[slot] = id;
+      record_event(g_trace.ev[2 * slot], st);
+    }
+  }
+  ~TraceScope() {
+    if (slot >= 0) record_event(g_trace.ev[2 * slot + 1], st);
+  }
+};
+
+inline size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
+
+bool fmt_ok(int f) { return f == QMOE_INT2 || f == QMOE_INT4 || f == QMOE_TERNARY; }
+int ku_cols(int fmt) { return fmt == QMOE_TERNARY ? 128 : 64; }
+int beta_hi(int fmt) { return fmt == QMOE_INT4 ? 1 : 4; }
+size_t codes_bytes(int fmt, int rows, int K) {
+  return fmt == QMOE_TERNARY ? (size_t)rows * (K / 128) * 26 : (size_t)rows * K * fmt / 8;
+}
+size_t scales_bytes(int rows, int K, int block) { return (size_t)rows * (K / block) * 2; }
+
+qmoe_status check_weights(const qmoe_weights& w, int rows, int K) {
+  if (!fmt_ok(w.fmt) || !w.codes || !w.scales) return QMOE_ERR_INVALID_ARG;
+  if (w.block != 64 && w.block != 128) return QMOE_ERR_UNSUPPORTED;
+  if (rows % 16 || K % 64 || K % w.block) return QMOE_ERR_INVALID_ARG;
+  if (w.fmt == QMOE_TERNARY && (w.block != 64 || K % 128)) return QMOE_ERR_UNSUPPORTED;
+  if ((reinterpret_cast<uintptr_t>(w.codes) | reinterpret_cast<uintptr_t>(w.scales)) & 15) return QMOE_ERR_INVALID_ARG;
+  return QMOE_OK;
+}
+
+// Workspace plan of one row tile of T tokens.
+struct MoEPlan {
+  int T, S, TK, max_seg, max_tg, n_tickets, max_gseg;
+  bool grouped;
+  size_t ids, w, perm, inv, offsets, slot_token, nseg, segs, tickets, partials, xfrag, hfrag, yslot, ngseg, gsegs,
+      xrows, hrows, total;
+};
+
+constexpr int kGroupedThreshold = 32;  // AUTO: experts with more tokens take the tcgen05 path
+
+bool grouped_eligible(const qmoe_layer& L) {
+  return L.fc1.fmt != QMOE_TERNARY && L.fc2.fmt != QMOE_TERNARY && (2 * L.I) % kGRows == 0 && L.H % kGRows == 0;
+}
+
+// Token-count threshold above which an expert runs on the grouped path.
+int grouped_threshold(const qmoe_layer& L) {
+  if (L.path == QMOE_PATH_SMALL_M || !grouped_eligible(L)) return INT_MAX;
+  return L.path == QMOE_PATH_GROUPED ? 0 : kGroupedThreshold;
+}
+
+MoEPlan plan_moe(const qmoe_layer& L, int T, int grid) {
+  MoEPlan p{};
+  p.grouped = T > grouped_threshold(L);
+  p.T = T;
+  p.TK = T * L.k;
+  p.S = T * (L.k + L.n_shared);
+  p.max_seg = std::min(L.E, p.TK) + p.TK / kChunkTokens + L.n_shared * ((T + kChunkTokens - 1) / kChunkTokens);
+  p.max_tg = (p.S + 7) / 8 + p.max_seg;
+  const int nt = std::max(2 * L.I / 16, L.H / 16);
+  p.n_tickets = p.max_seg * nt;
+  size_t o = 0;
+  auto take = [&](size_t bytes) { size_t at = o; o = align_up(o + bytes); return at; };
+  p.ids = take((size_t)p.TK * 4);
+  p.w = take((size_t)p.TK * 4);
+  p.perm = take((size_t)p.TK * 4);
+  p.inv = take((size_t)p.TK * 4);
+  p.offsets = take((size_t)(L.E + 1) * 4);
+  p.slot_token = take((size_t)p.S * 4);
+  p.nseg = take(16);
+  p.segs = take((size_t)p.max_seg * sizeof(Seg));
+  p.tickets = take((size_t)p.n_tickets * 4);
+  p.partials = take((size_t)2 * grid * 2 * 32 * 16);
+  p.xfrag = take((size_t)p.max_tg * L.H * 16);
+  p.hfrag = take((size_t)p.max_tg * L.I * 16);
+  p.yslot = take((size_t)p.S * L.H * 4);
+  if (p.grouped) {
+    p.max_gseg = std::min(L.E, p.TK) + p.TK / kGTok + L.n_shared * ((T + kGTok - 1) / kGTok);
+    p.ngseg = take(16);
+    p.gsegs = take((size_t)p.max_gseg * sizeof(GSeg));
+    p.xrows = take((size_t)p.S * L.H * 2 + 16);
+    p.hrows = take((size_t)p.S * L.I * 2 + 16);
+  }
+  p.total = o;
+  return p;
+}
+
+// ---- TMA tensor maps (driver entry point through the runtime; no libcuda link) ----
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+qmoe_status encode_rows_map(CUtensorMap* map, const void* base, int K, int rows) {
+  if (!g_encode) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || !fn)
+      return QMOE_ERR_CUDA;
+    g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  }
+  const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+  const cuuint32_t box[2] = {64, (cuuint32_t)kGTmaRows};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? QMOE_OK : QMOE_ERR_CUDA;
+}
+
+// ---- small-M kernel launch ----
+template <int FMT, int TG, int EPI>
+qmoe_status launch_small_t(SmallParams prm, int grid, cudaStream_t st) {
+  using G = StageGeom<FMT, TG>;
+  const int fixed = 2048 + G::kRedBytes;
+  int nst = (kSmemLimit - fixed - 1024) / (kNW * G::kStageBytes);
+  nst = std::min(nst, 4);
+  if (nst < 2) return QMOE_ERR_UNSUPPORTED;
+  prm.nstages = nst;
+  const int smem = fixed + nst * kNW * G::kStageBytes;
+  static bool attr_set[kMaxDevices] = {};
+  int d = 0;
+  cudaGetDevice(&d);
+  if (!attr_set[d]) {
+    if (cudaFuncSetAttribute(qmm_small_kernel<FMT, TG, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+        cudaSuccess)
+      return QMOE_ERR_CUDA;
+    attr_set[d] = true;
+  }
+  TraceScope ts(st, EPI == EPI_SWIGLU ? K_FC1_SMALL : (EPI == EPI_FC2 ? K_FC2_SMALL : K_LINEAR_SMALL));
+  qmm_small_kernel<FMT, TG, EPI><<<grid, kNW * 32, smem, st>>>(prm);
+  return cudaGetLastError() == cudaSuccess ? QMOE_OK : QMOE_ERR_CUDA;
+}
+
+template <int EPI>
+qmoe_status launch_small(int fmt, int tg, const SmallParams& prm, int grid, cudaStream_t st) {
+  if (fmt == QMOE_INT2) return tg == 1 ? launch_small_t<2, 1, EPI>(prm, grid, st) : launch_small_t<2, 2, EPI>(prm, grid, st);
+  if (fmt == QMOE_INT4) return tg == 1 ? launch_small_t<4, 1, EPI>(prm, grid, st) : launch_small_t<4, 2, EPI>(prm, grid, st);
+  return tg == 1 ? launch_small_t<3, 1, EPI>(prm, grid, st) : launch_small_t<3, 2, EPI>(prm, grid, st);
+}
+
+template <int FMT, int EPI>
+qmoe_status launch_grouped_t(const CUtensorMap& map, const GroupedParams& prm, int grid, cudaStream_t st) {
+  constexpr int smem = GGeom<FMT>::kSmem;
+  static bool attr_set[kMaxDevices] = {};
+  int d = 0;
+  cudaGetDevice(&d);
+  if (!attr_set[d]) {
+    if (cudaFuncSetAttribute(qmm_grouped_kernel<FMT, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+        cudaSuccess)
+      return QMOE_ERR_CUDA;
+    attr_set[d] = true;
+  }
+  TraceScope ts(st, EPI == EPI_SWIGLU ? K_FC1_GROUPED : K_FC2_GROUPED);
+  qmm_grouped_kernel<FMT, EPI><<<grid, kGThreads, smem, st>>>(map, prm);
+  return cudaGetLastError() == cudaSuccess ? QMOE_OK : QMOE_ERR_CUDA;
+}
+
+template <int EPI>
+qmoe_status launch_grouped(int fmt, const CUtensorMap& map, const GroupedParams& prm, int grid, cudaStream_t st) {
+  if (fmt == QMOE_INT2) return launch_grouped_t<2, EPI>(map, prm, grid, st);
+  if (fmt == QMOE_INT4) return launch_grouped_t<4, EPI>(map, prm, grid, st);
+  return QMOE_ERR_UNSUPPORTED;
+}
+
+GroupedParams grouped_params(const qmoe_weights& w, int rows, int K, unsigned* status) {
+  GroupedParams p{};
+  p.codes = static_cast<const uint8_t*>(w.codes);
+  p.codes_stride = codes_bytes(w.fmt, rows, K);
+  p.scales = static_cast<const uint8_t*>(w.scales);
+  p.scales_stride = scales_bytes(rows, K, w.block);
+  p.NT = rows / 16;
+  p.K = K;
+  p.block = w.block;
+  p.rtiles = rows / kGRows;
+  p.status = status;
+  return p;
+}
+
+SmallParams small_params(const qmoe_weights& w, int rows, int K, unsigned* status) {
+  SmallParams p{};
+  p.codes = static_cast<const uint8_t*>(w.codes);
+  p.codes_stride = codes_bytes(w.fmt, rows, K);
+  p.scales = static_cast<const uint8_t*>(w.scales);
+  p.scales_stride = scales_bytes(rows, K, w.block);
+  p.NT = rows / 16;
+  p.K = K;
+  p.KU = K / ku_cols(w.fmt);
+  p.block = w.block;
+  p.status = status;
+  return p;
+}
+
+qmoe_status check_layer(const qmoe_layer* L) {
+  if (!L) return QMOE_ERR_INVALID_ARG;
+  if (L->H <= 0 || L->I <= 0 || L->E <= 0 || L->k <= 0 || L->n_shared < 0) return QMOE_ERR_INVALID_ARG;
+  if (L->E > kMaxExperts || L->k > 32 || L->k > L->E || L->n_shared > 64) return QMOE_ERR_UNSUPPORTED;
+  if (L->H % 64 || L->I % 64) return QMOE_ERR_INVALID_ARG;
+  if (L->path < QMOE_PATH_AUTO || L->path > QMOE_PATH_GROUPED) return QMOE_ERR_INVALID_ARG;
+  if (L->max_row_tile < 0) return QMOE_ERR_INVALID_ARG;
+  qmoe_status s = check_weights(L->fc1, 2 * L->I, L->H);
+  if (s != QMOE_OK) return s;
+  return check_weights(L->fc2, L->H, L->I);
+}
+
+}  // namespace
+}  // namespace qmoe
+
+using namespace qmoe;
+
+extern "C" {
+
+const char* qmoe_status_str(int s) {
+  switch (s) {
+    case QMOE_OK: return "ok";
+    case QMOE_ERR_INVALID_ARG: return "invalid argument";
+    case QMOE_ERR_UNSUPPORTED: return "unsupported configuration";
+    case QMOE_ERR_SCRATCH: return "workspace too small for one token row";
+    case QMOE_ERR_CUDA: return "CUDA runtime error";
+    case QMOE_ERR_TIMEOUT: return "device wait timed out";
+    default: return "unknown status";
+  }
+}
+
+const char* qmoe_kernel_name(int id) { return id >= 0 && id < K_COUNT ? kKernelNames[id] : "unknown"; }
+
+qmoe_status qmoe_trace_start(int cap) {
+  if (cap <= 0 || cap > (1 << 20)) return QMOE_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lk(g_mu);
+  for (cudaEvent_t e : g_trace.ev) cudaEventDestroy(e);
+  g_trace.ev.assign(2 * (size_t)cap, nullptr);
+  g_trace.ids.assign(cap, -1);
+  for (auto& e : g_trace.ev)
+    if (cudaEventCreate(&e) != cudaSuccess) {
+      g_trace.on = false;
+      return QMOE_ERR_CUDA;
+    }
+  g_trace.cap = cap;
+  g_trace.n = 0;
+  g_trace.on = true;
+  return QMOE_OK;
+}
+
+qmoe_status qmoe_trace_stop(void) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  g_trace.on = false;
+  return QMOE_OK;
+}
+
+qmoe_status qmoe_trace_read(int cap, int* n, int* kernel_ids, float* ms) {
+  if (!n || cap < 0 || (cap > 0 && (!kernel_ids || !ms))) return QMOE_ERR_INVALID_ARG;
+  if (cudaDeviceSynchronize() != cudaSuccess) return QMOE_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_mu);
+  const int m = std::min(cap, g_trace.n);
+  for (int i = 0; i < m; ++i) {
+    kernel_ids[i] = g_trace.ids[i];
+    float t = -1.f;
+    if (cudaEventElapsedTime(&t, g_trace.ev[2 * i], g_trace.ev[2 * i + 1]) != cudaSuccess) t = -1.f;
+    ms[i] = t;
+  }
+  *n = g_trace.n;
+  cudaGetLastError();  // an unrecorded event leaves a sticky-free error: clear it
+  return QMOE_OK;
+}
+
+qmoe_status qmoe_get_stats(qmoe_stats* out) {
+  if (!out) return QMOE_ERR_INVALID_ARG;
+  DevInfo* di;
+  qmoe_status s = dev_info(&di);
+  if (s != QMOE_OK) return s;
+  unsigned v = 0;
+  if (cudaMemcpy(&v, di->status, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return QMOE_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_mu);
+  *out = g_stats;
+  out->device_status = v;
+  return QMOE_OK;
+}
+
+qmoe_status qmoe_clear_status(void) {
+  DevInfo* di;
+  qmoe_status s = dev_info(&di);
+  if (s != QMOE_OK) return s;
+  return cudaMemset(di->status, 0, sizeof(unsigned)) == cudaSuccess ? QMOE_OK : QMOE_ERR_CUDA;
+}
+
+qmoe_status qmoe_route(const float* logits, int T, int E, int k, int32_t* ids, float* weights, int32_t* perm,
+                       int32_t* offsets, void* stream) {
+  if (!logits || !ids || !weights || !perm || !offsets || T <= 0 || E <= 0 || k <= 0) return QMOE_ERR_INVALID_ARG;
+  if (E > kMaxExperts || k > 32 || k > E) return QMOE_ERR_UNSUPPORTED;
+  DevInfo* di;
+  qmoe_status s = dev_info(&di);
+  if (s != QMOE_OK) return s;
+  RouteOut o{};
+  o.ids = ids;
+  o.w = weights;
+  o.perm = perm;
+  o.offsets = offsets;
+  o.status = di->status;
+  TraceScope ts(static_cast<cudaStream_t>(stream), K_ROUTE);
+  route_kernel<<<1, kRouteThreads, 0, static_cast<cudaStream_t>(stream)>>>(logits, T, E, k, 0, o);
+  return cudaGetLastError() == cudaSuccess ? QMOE_OK : QMOE_ERR_CUDA;
+}
+
+qmoe_status qmoe_workspace_size(const qmoe_layer* layer, int T, size_t* bytes) {
+  qmoe_status s = check_layer(layer);
+  if (s != QMOE_OK) return s;
+  if (T <= 0 || !bytes) return QMOE_ERR_INVALID_ARG;
+  DevInfo* di;
+  s = dev_info(&di);
+  if (s != QMOE_OK) return s;
+  int Tt = T;
+  if (layer->max_row_tile > 0) Tt = std::min(Tt, layer->max_row_tile);
+  *bytes = plan_moe(*layer, Tt, di->sms).total;
+  return QMOE_OK;
+}
+
+qmoe_status qmoe_forward(const qmoe_layer* layer, const uint16_t* x, const float* logits, int T, uint16_t* y,
+                         void* ws, size_t ws_bytes, void* stream) {
+  qmoe_status s = check_layer(layer);
+  if (s != QMOE_OK) return s;
+  if (!x || !logits || !y || !ws || T <= 0) return QMOE_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(ws) % kAlign) || (reinterpret_cast<uintptr_t>(x) & 3) ||
+      (reinterpret_cast<uintptr_t>(y) & 7))
+    return QMOE_ERR_INVALID_ARG;
+  if (layer->path == QMOE_PATH_GROUPED && !grouped_eligible(*layer)) return QMOE_ERR_UNSUPPORTED;
+  DevInfo* di;
+  s = dev_info(&di);
+  if (s != QMOE_OK) return s;
+  const qmoe_layer& L = *layer;
+  const int grid = di->sms;
+  // Row tile: the largest (<= T, <= max_row_tile) whose workspace fits; halve until it does.
+  int Tt = T;
+  if (L.max_row_tile > 0) Tt = std::min(Tt, L.max_row_tile);
+  while (plan_moe(L, Tt, grid).total > ws_bytes) {
+    if (Tt == 1) return QMOE_ERR_SCRATCH;
+    Tt = (Tt + 1) / 2;
+  }
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  int tiles = 0, small = 0, grouped = 0;
+  for (int t0 = 0; t0 < T; t0 += Tt) {
+    const int tt = std::min(Tt, T - t0);
+    const MoEPlan p = plan_moe(L, tt, grid);
+    RouteOut o{};
+    o.ids = reinterpret_cast<int*>(base + p.ids);
+    o.w = reinterpret_cast<float*>(base + p.w);
+    o.perm = reinterpret_cast<int*>(base + p.perm);
+    o.inv = reinterpret_cast<int*>(base + p.inv);
+    o.offsets = reinterpret_cast<int*>(base + p.offsets);
+    o.slot_token = reinterpret_cast<int*>(base + p.slot_token);
+    o.nseg = reinterpret_cast<int*>(base + p.nseg);
+    o.segs = reinterpret_cast<Seg*>(base + p.segs);
+    o.max_seg = p.max_seg;
+    o.tickets = reinterpret_cast<int*>(base + p.tickets);
+    o.n_tickets = p.n_tickets;
+    o.thresh = grouped_threshold(L);
+    if (p.grouped) {
+      o.ngseg = reinterpret_cast<int*>(base + p.ngseg);
+      o.gsegs = reinterpret_cast<GSeg*>(base + p.gsegs);
+      o.max_gseg = p.max_gseg;
+    }
+    o.status = di->status;
+    {
+      TraceScope ts(st, K_ROUTE);
+      route_kernel<<<1, kRouteThreads, 0, st>>>(logits + (size_t)t0 * L.E, tt, L.E, L.k, L.n_shared, o);
+    }
+    if (cudaGetLastError() != cudaSuccess) return QMOE_ERR_CUDA;
+    uint8_t* xfrag = base + p.xfrag;
+    uint8_t* hfrag = base + p.hfrag;
+    float* yslot = reinterpret_cast<float*>(base + p.yslot);
+    {
+      TraceScope ts(st, K_GATHER);
+      gather_kernel<<<std::min(p.max_seg, 4 * grid), 256, 0, st>>>(x + (size_t)t0 * L.H, L.H, o.slot_token,
+                                                                    o.nseg, o.segs, xfrag, beta_hi(L.fc1.fmt));
+    }
+    if (cudaGetLastError() != cudaSuccess) return QMOE_ERR_CUDA;
+    const int tg = tt <= 8 ? 1 : 2;
+    SmallParams p1 = small_params(L.fc1, 2 * L.I, L.H, di->status);
+    p1.nseg = o.nseg;
+    p1.segs = o.segs;
+    p1.xfrag = xfrag;
+    p1.bias = L.fc1.bias;
+    p1.bias_rows = 2 * L.I;
+    p1.hfrag = hfrag;
+    p1.I = L.I;
+    p1.h_beta_hi = beta_hi(L.fc2.fmt);
+    p1.partials = reinterpret_cast<float*>(base + p.partials);
+    p1.tickets = o.tickets;
+    s = launch_small<EPI_SWIGLU>(L.fc1.fmt, tg, p1, grid, st);
+    if (s != QMOE_OK) return s;
+    uint16_t* xrows = nullptr;
+    uint16_t* hrows = nullptr;
+    CUtensorMap map2;
+    GroupedParams g2{};
+    if (p.grouped) {
+      xrows = reinterpret_cast<uint16_t*>(base + p.xrows);
+      hrows = reinterpret_cast<uint16_t*>(base + p.hrows);
+      {
+        TraceScope ts(st, K_GATHER);
+        gather_rows_kernel<<<std::min(p.max_gseg, 4 * grid), 256, 0, st>>>(x + (size_t)t0 * L.H, L.H, o.slot_token,
+                                                                            o.ngseg, o.gsegs, xrows);
+        if (cudaGetLastError() != cudaSuccess) return QMOE_ERR_CUDA;
+      }
+      CUtensorMap map1;
+      s = encode_rows_map(&map1, xrows, L.H, p.S);
+      if (s != QMOE_OK) return s;
+      s = encode_rows_map(&map2, hrows, L.I, p.S);
+      if (s != QMOE_OK) return s;
+      GroupedParams g1 = grouped_params(L.fc1, 2 * L.I, L.H, di->status);
+      g1.ngseg = o.ngseg;
+      g1.gsegs = o.gsegs;
+      g1.bias = L.fc1.bias;
+      g1.bias_rows = 2 * L.I;
+      g1.hrows = hrows;
+      g1.I = L.I;
+      const int units1 = p.max_gseg * g1.rtiles;
+      s = launch_grouped<EPI_SWIGLU>(L.fc1.fmt, map1, g1, std::min(units1, grid), st);
+      if (s != QMOE_OK) return s;
+      g2 = grouped_params(L.fc2, L.H, L.I, di->status);
+      g2.ngseg = o.ngseg;
+      g2.gsegs = o.gsegs;
+      g2.bias = L.fc2.bias;
+      g2.bias_rows = L.H;
+      g2.yslot = yslot;
+      g2.H = L.H;
+    }
+    SmallParams p2 = small_params(L.fc2, L.H, L.I, di->status);
+    p2.nseg = o.nseg;
+    p2.segs = o.segs;
+    p2.xfrag = hfrag;
+    p2.bias = L.fc2.bias;
+    p2.bias_rows = L.H;
+    p2.yslot = yslot;
+    p2.H = L.H;
+    p2.partials = p1.partials;
+    p2.tickets = o.tickets;
+    s = launch_small<EPI_FC2>(L.fc2.fmt, tg, p2, grid, st);
+    if (s != QMOE_OK) return s;
+    if (p.grouped) {
+      s = launch_grouped<EPI_FC2>(L.fc2.fmt, map2, g2, std::min(p.max_gseg * g2.rtiles, grid), st);
+      if (s != QMOE_OK) return s;
+      ++grouped;
+    }
+    {
+      TraceScope ts(st, K_COMBINE);
+      combine_kernel<<<tt, 256, 0, st>>>(yslot, o.w, o.inv, tt, L.k, L.n_shared, L.H, y + (size_t)t0 * L.H);
+    }
+    if (cudaGetLastError() != cudaSuccess) return QMOE_ERR_CUDA;
+    ++tiles;
+    small += 2;
+  }
+  std::lock_guard<std::mutex> lk(g_mu);
+  g_stats.last_path = grouped ? (L.path == QMOE_PATH_GROUPED ? QMOE_PATH_GROUPED : QMOE_PATH_AUTO) : QMOE_PATH_SMALL_M;
+  g_stats.row_tiles = tiles;
+  g_stats.row_tile_tokens = Tt;
+  g_stats.small_launches = small;
+  g_stats.grouped_launches = 2 * grouped;
+  return QMOE_OK;
+}
+
+qmoe_status qmoe_linear_workspace_size(int N, int K, int M, size_t* bytes) {
+  if (N <= 0 || K <= 0 || M <= 0 || N % 16 || K % 64 || !bytes) return QMOE_ERR_INVALID_ARG;
+  DevInfo* di;
+  qmoe_status s = dev_info(&di);
+  if (s != QMOE_OK) return s;
+  const int nseg = (M + kChunkTokens - 1) / kChunkTokens;
+  size_t o = 0;
+  o = align_up(o + 16);                                   // nseg
+  o = align_up(o + (size_t)nseg * sizeof(Seg));           // segs
+  o = align_up(o + (size_t)nseg * (N / 16) * 4);          // tickets
+  o = align_up(o + (size_t)2 * di->sms * 2 * 32 * 16);    // partials
+  o = align_up(o + (size_t)2 * nseg * K * 16);            // activation fragments
+  *bytes = o;
+  return QMOE_OK;
+}
+
+qmoe_status qmoe_linear(const qmoe_weights* w, int N, int K, const uint16_t* x, int M, uint16_t* y, void* ws,
+                        size_t ws_bytes, void* stream) {
+  if (!w || !x || !y || !ws || M <= 0) return QMOE_ERR_INVALID_ARG;
+  qmoe_status s = check_weights(*w, N, K);
+  if (s != QMOE_OK) return s;
+  if ((reinterpret_cast<uintptr_t>(ws) % kAlign) || (reinterpret_cast<uintptr_t>(x) & 3)) return QMOE_ERR_INVALID_ARG;
+  size_t need = 0;
+  s = qmoe_linear_workspace_size(N, K, M, &need);
+  if (s != QMOE_OK) return s;
+  if (ws_bytes < need) return QMOE_ERR_SCRATCH;
+  DevInfo* di;
+  s = dev_info(&di);
+  if (s != QMOE_OK) return s;
+  const int nseg = (M + kChunkTokens - 1) / kChunkTokens;
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  size_t o = 0;
+  int* d_nseg = reinterpret_cast<int*>(base + o); o = align_up(o + 16);
+  Seg* segs = reinterpret_cast<Seg*>(base + o); o = align_up(o + (size_t)nseg * sizeof(Seg));
+  int* tickets = reinterpret_cast<int*>(base + o); o = align_up(o + (size_t)nseg * (N / 16) * 4);
+  float* partials = reinterpret_cast<float*>(base + o); o = align_up(o + (size_t)2 * di->sms * 2 * 32 * 16);
+  uint8_t* xfrag = base + o;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  {
+    TraceScope ts(st, K_LINEAR_SETUP);
+    linear_setup_kernel<<<1, 256, 0, st>>>(M, d_nseg, segs, tickets, nseg * (N / 16));
+  }
+  if (cudaGetLastError() != cudaSuccess) return QMOE_ERR_CUDA;
+  {
+    TraceScope ts(st, K_GATHER);
+    gather_kernel<<<nseg, 256, 0, st>>>(x, K, nullptr, d_nseg, segs, xfrag, beta_hi(w->fmt));
+  }
+  if (cudaGetLastError() != cudaSuccess) return QMOE_ERR_CUDA;
+  SmallParams p = small_params(*w, N, K, di->status);
+  p.nseg = d_nseg;
+  p.segs = segs;
+  p.xfrag = xfrag;
+  p.y = y;
+  p.N = N;
+  p.partials = partials;
+  p.tickets = tickets;
+  s = launch_small<EPI_LINEAR>(w->fmt, M <= 8 ? 1 : 2, p, di->sms, st);
+  if (s != QMOE_OK) return s;
+  std::lock_guard<std::mutex> lk(g_mu);
+  g_stats.last_path = QMOE_PATH_SMALL_M;
+  g_stats.row_tiles = 1;
+  g_stats.row_tile_tokens = M;
+  g_stats.small_launches = 1;
+  g_stats.grouped_launches = 0;
+  return QMOE_OK;
+}
+
+qmoe_status qmoe_dequant(const qmoe_weights* w, int row_order, int rows, int K, int n_mats, float* out_f32,
+                         uint16_t* out_bf16, void* stream) {
+  if (!w || n_mats <= 0 || (!out_f32 && !out_bf16)) return QMOE_ERR_INVALID_ARG;
+  if (row_order != QMOE_ROWS_PLAIN && row_order != QMOE_ROWS_GATE_UP) return QMOE_ERR_INVALID_ARG;
+  qmoe_status s = check_weights(*w, rows, K);
+  if (s != QMOE_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const unsigned long long cs = codes_bytes(w->fmt, rows, K), ss = scales_bytes(rows, K, w->block);
+  const uint8_t* c = static_cast<const uint8_t*>(w->codes);
+  const uint8_t* sc = static_cast<const uint8_t*>(w->scales);
+  const long long items = (long long)n_mats * (K / ku_cols(w->fmt)) * (rows / 16);
+  const int grid = (int)std::min<long long>((items + 7) / 8, 65535);
+  TraceScope ts(st, K_DEQUANT);
+  if (w->fmt == QMOE_INT2)
+    dequant_kernel<2><<<grid, 256, 0, st>>>(c, cs, sc, ss, rows / 16, K, w->block, row_order, n_mats, out_f32, out_bf16);
+  else if (w->fmt == QMOE_INT4)
+    dequant_kernel<4><<<grid, 256, 0, st>>>(c, cs, sc, ss, rows / 16, K, w->block, row_order, n_mats, out_f32, out_bf16);
+  else
+    dequant_kernel<3><<<grid, 256, 0, st>>>(c, cs, sc, ss, rows / 16, K, w->block, row_order, n_mats, out_f32, out_bf16);
+  return cudaGetLastError() == cudaSuccess ? QMOE_OK : QMOE_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -1,0 +1,87 @@
+"""Shared set-up for the GPU parity tests: synthetic weights packed by the
+library and, independently, quantized by the oracle from the same bf16
+weights.  The oracle side never sees anything the CUDA path produced."""
+from __future__ import annotations
+
+import dataclasses
+
+import numpy as np
+
+from oracle import qmoe_oracle as Q
+from skinny_gemm_top_b200 import synth
+
+FMTS = {"int2": 2, "int4": 4, "ternary": 3}
+
+# Tolerances: relative L2 error and max |err| / rms(ref) of the bf16 outputs.
+REL_L2 = 5e-3
+MAX_ERR_RMS = 3e-2
+
+
+def to_dev(a: np.ndarray):
+    import torch
+    a = np.ascontiguousarray(a)
+    if a.dtype == np.uint16:
+        a = a.view(np.int16)
+    return torch.from_numpy(a).cuda()
+
+
+def bf16_dev_to_f64(t) -> np.ndarray:
+    return Q.bf16_bits_to_f64(t.cpu().numpy().view(np.uint16))
+
+
+def oracle_quant(fmt: str, w_bits: np.ndarray, block: int):
+    w = Q.bf16_bits_to_f64(w_bits)
+    if fmt == "ternary":
+        return Q.quantize_ternary(w, block)
+    return Q.quantize_sym(w, FMTS[fmt], block)
+
+
+class MoECase:
+    """A MoE layer: packed on the device for the library, quantized lazily by
+    the oracle for reference values."""
+
+    def __init__(self, cfg: synth.MoEConfig, seed: int = 1):
+        from skinny_gemm_top_b200 import qmoe
+        self.cfg, self.seed = cfg, seed
+        n = cfg.E + cfg.n_shared
+        f1, f2 = FMTS[cfg.fc1_fmt], FMTS[cfg.fc2_fmt]
+        c1, s1 = qmoe.pack_stack(f1, qmoe.ROWS_GATE_UP, (synth.expert_fc1(cfg, seed, e) for e in range(n)), cfg.block)
+        c2, s2 = qmoe.pack_stack(f2, qmoe.ROWS_PLAIN, (synth.expert_fc2(cfg, seed, e) for e in range(n)), cfg.block)
+        self.dev = {"c1": to_dev(c1), "s1": to_dev(s1), "c2": to_dev(c2), "s2": to_dev(s2)}
+        self.b1 = self.b2 = None
+        if cfg.bias:
+            self.dev["b1"] = to_dev(np.stack([synth.expert_b1(cfg, seed, e) for e in range(n)]))
+            self.dev["b2"] = to_dev(np.stack([synth.expert_b2(cfg, seed, e) for e in range(n)]))
+        self.w1 = qmoe.make_weights(f1, cfg.block, self.dev["c1"], self.dev["s1"], self.dev.get("b1"))
+        self.w2 = qmoe.make_weights(f2, cfg.block, self.dev["c2"], self.dev["s2"], self.dev.get("b2"))
+        self.bank = Q.QuantExpertBank(
+            cfg.H, cfg.I, cfg.E, cfg.n_shared, cfg.block,
+            lambda e: oracle_quant(cfg.fc1_fmt, synth.expert_fc1(cfg, seed, e), cfg.block),
+            lambda e: oracle_quant(cfg.fc2_fmt, synth.expert_fc2(cfg, seed, e), cfg.block),
+            (lambda e: Q.bf16_bits_to_f64(synth.expert_b1(cfg, seed, e))) if cfg.bias else None,
+            (lambda e: Q.bf16_bits_to_f64(synth.expert_b2(cfg, seed, e))) if cfg.bias else None,
+            cache=16)
+
+    def layer(self, path=0, max_row_tile=0):
+        from skinny_gemm_top_b200 import qmoe
+        c = self.cfg
+        return qmoe.make_layer(c.H, c.I, c.E, c.k, c.n_shared, self.w1, self.w2, path, max_row_tile)
+
+    def run(self, x_bits: np.ndarray, logits: np.ndarray, ws_bytes: int | None = None, max_row_tile: int = 0,
+            path: int = 0):
+        import torch
+        from skinny_gemm_top_b200 import qmoe
+        T = x_bits.shape[0]
+        layer = self.layer(path=path, max_row_tile=max_row_tile)
+        need = qmoe.workspace_size(layer, T)
+        ws = torch.empty(need if ws_bytes is None else ws_bytes, dtype=torch.uint8, device="cuda")
+        x = to_dev(x_bits)
+        lg = torch.from_numpy(np.ascontiguousarray(logits, dtype=np.float32)).cuda()
+        y = torch.empty((T, self.cfg.H), dtype=torch.int16, device="cuda")
+        qmoe.forward(layer, x, lg, y, ws)
+        torch.cuda.synchronize()
+        return bf16_dev_to_f64(y)
+
+
+def small_cfg(base: synth.MoEConfig, **kw) -> synth.MoEConfig:
+    return dataclasses.replace(base, **kw)

@@ -1,0 +1,99 @@
+"""CPU tests of the C-ABI library: it loads, exports every declared symbol, and
+its host packer agrees bit for bit with the oracle's quantizer."""
+import os
+import re
+
+import numpy as np
+import pytest
+
+from oracle import qmoe_oracle as Q
+from skinny_gemm_top_b200 import qmoe, synth
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    src = open(os.path.join(ROOT, "include", "qmoe.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(qmoe_\w+)\s*\(", src)))
+
+
+def test_library_exports_every_declared_symbol():
+    names = _declared_functions()
+    assert len(names) >= 12
+    lib = qmoe.lib()
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(qmoe.EXPORTS), set(names) ^ set(qmoe.EXPORTS)
+
+
+def test_status_strings():
+    assert qmoe.status_str(qmoe.OK) == "ok"
+    assert "workspace" in qmoe.status_str(qmoe.ERR_SCRATCH)
+
+
+def _oracle_q(fmt, w_bits, block):
+    w = Q.bf16_bits_to_f64(w_bits)
+    if fmt == qmoe.TERNARY:
+        return Q.quantize_ternary(w, block)
+    return Q.quantize_sym(w, fmt, block)
+
+
+@pytest.mark.parametrize("fmt,block,order", [
+    (qmoe.INT2, 64, qmoe.ROWS_GATE_UP), (qmoe.INT4, 64, qmoe.ROWS_PLAIN), (qmoe.INT2, 128, qmoe.ROWS_PLAIN),
+    (qmoe.INT4, 128, qmoe.ROWS_PLAIN), (qmoe.TERNARY, 64, qmoe.ROWS_GATE_UP), (qmoe.TERNARY, 64, qmoe.ROWS_PLAIN)])
+def test_pack_matches_oracle_quantizer(fmt, block, order):
+    rows, K = 48, 256
+    w = synth.normal_bf16(9, 50, fmt * 10 + block, (rows, K), 0.02)
+    codes, scales = qmoe.pack(fmt, order, w, block)
+    cb, sb = qmoe.pack_size(fmt, rows, K, block)
+    assert codes.nbytes == cb and scales.nbytes == sb
+    c, s = qmoe.unpack_host(fmt, order, codes, scales, rows, K, block)
+    oc, os_ = _oracle_q(fmt, w, block)
+    assert np.array_equal(c, oc)
+    assert np.array_equal(Q.bf16_bits_to_f64(s), os_)
+
+
+def test_pack_sizes_are_the_format_densities():
+    assert qmoe.pack_size(qmoe.INT2, 16, 5120, 128) == (16 * 5120 // 4, 16 * 40 * 2)
+    assert qmoe.pack_size(qmoe.INT4, 16, 5120, 128) == (16 * 5120 // 2, 16 * 40 * 2)
+    assert qmoe.pack_size(qmoe.TERNARY, 16, 2048, 64) == (16 * 2048 * 13 // 64, 16 * 32 * 2)
+
+
+def test_pack_every_code_at_every_position():
+    """Weights that quantize to known codes (exact multiples of a power-of-two
+    scale) come back through the physical layout unchanged at every position."""
+    rows, K = 32, 128
+    g = np.random.default_rng(3)
+    for fmt in (qmoe.INT2, qmoe.INT4):
+        qmin, qmax = -(1 << (fmt - 1)), (1 << (fmt - 1)) - 1
+        c = g.integers(qmin, qmax + 1, size=(rows, K))
+        c[:, 0] = qmin
+        c[:, 64] = qmin
+        w = synth.f32_to_bf16_bits((c * 2.0 ** -7).astype(np.float32))
+        for order in (qmoe.ROWS_PLAIN, qmoe.ROWS_GATE_UP):
+            codes, scales = qmoe.pack(fmt, order, w, 64)
+            cc, ss = qmoe.unpack_host(fmt, order, codes, scales, rows, K, 64)
+            assert np.array_equal(cc, c)
+            assert np.all(Q.bf16_bits_to_f64(ss) == 2.0 ** -7)
+    t = g.integers(-1, 2, size=(rows, K))
+    w = synth.f32_to_bf16_bits((t * 0.25).astype(np.float32))
+    codes, scales = qmoe.pack(qmoe.TERNARY, qmoe.ROWS_PLAIN, w, 64)
+    cc, _ = qmoe.unpack_host(qmoe.TERNARY, qmoe.ROWS_PLAIN, codes, scales, rows, K, 64)
+    assert np.array_equal(cc, t)
+
+
+@pytest.mark.parametrize("args,status", [
+    ((qmoe.INT2, 0, 15, 64, 64), qmoe.ERR_INVALID_ARG),      # rows % 16
+    ((qmoe.INT2, 0, 16, 96, 64), qmoe.ERR_INVALID_ARG),      # K % 64
+    ((qmoe.INT2, 0, 16, 64, 32), qmoe.ERR_UNSUPPORTED),      # block
+    ((qmoe.TERNARY, 0, 16, 64, 64), qmoe.ERR_UNSUPPORTED),   # ternary needs K % 128
+    ((7, 0, 16, 64, 64), qmoe.ERR_INVALID_ARG),              # format
+    ((qmoe.INT4, 2, 16, 64, 64), qmoe.ERR_INVALID_ARG),      # row order
+])
+def test_pack_rejects_bad_arguments(args, status):
+    fmt, order, rows, K, block = args
+    w = np.zeros((max(rows, 1), K), dtype=np.uint16)
+    codes = np.zeros(1 << 16, dtype=np.uint8)
+    st = qmoe.lib().qmoe_pack(fmt, order, w.ctypes.data, rows, K, block, codes.ctypes.data, codes.ctypes.data)
+    assert st == status

@@ -1,0 +1,275 @@
+"""GPU parity of the CUDA path (through the C ABI) against the fp64 oracle.
+
+Bar: routing ids / permutation / offsets and dequantized weights bit-exact;
+outputs within rel-L2 5e-3 and max |err| 3e-2 * rms(ref)."""
+import numpy as np
+import pytest
+
+from oracle import qmoe_oracle as Q
+from skinny_gemm_top_b200 import synth
+
+from cases import FMTS, MAX_ERR_RMS, REL_L2, MoECase, bf16_dev_to_f64, oracle_quant, small_cfg, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def qm(cuda_ok):
+    from skinny_gemm_top_b200 import qmoe
+    qmoe.clear_status()
+    yield qmoe
+    assert qmoe.get_stats().device_status == 0
+
+
+def _close(got, ref, what=""):
+    r, m = Q.rel_l2(got, ref), Q.max_err_over_rms(got, ref)
+    assert r <= REL_L2 and m <= MAX_ERR_RMS, f"{what}: rel_l2={r:.3g} max_err/rms={m:.3g}"
+    return r, m
+
+
+# ------------------------------------------------------------------ dequant
+
+@pytest.mark.parametrize("fmt,block,order", [
+    ("int2", 64, 1), ("int2", 128, 0), ("int4", 64, 0), ("int4", 128, 1), ("ternary", 64, 1), ("ternary", 64, 0)])
+def test_dequant_bit_exact(qm, fmt, block, order):
+    import torch
+    rows, K, n = 48, 384, 2
+    mats = [synth.normal_bf16(21, 60, i, (rows, K), 0.02) for i in range(n)]
+    c, s = qm.pack_stack(FMTS[fmt], order, mats, block)
+    dc, ds = to_dev(c), to_dev(s)
+    w = qm.make_weights(FMTS[fmt], block, dc, ds)
+    o32 = torch.empty((n, rows, K), dtype=torch.float32, device="cuda")
+    o16 = torch.empty((n, rows, K), dtype=torch.int16, device="cuda")
+    qm.dequant(w, order, rows, K, n, o32, o16)
+    torch.cuda.synchronize()
+    for i in range(n):
+        codes, scales = oracle_quant(fmt, mats[i], block)
+        ref = Q.dequant(codes, scales, block)
+        assert np.array_equal(o32[i].cpu().numpy().astype(np.float64), ref)
+        ref16 = Q.dequant_bf16_operand(codes, scales, block)
+        assert np.array_equal(Q.bf16_bits_to_f64(o16[i].cpu().numpy().view(np.uint16)), ref16)
+
+
+# ------------------------------------------------------------------ routing
+
+@pytest.mark.parametrize("T,E,k,seed", [(1, 8, 2, 1), (37, 64, 6, 2), (300, 128, 8, 3), (129, 256, 1, 4),
+                                        (1100, 64, 6, 5)])
+def test_route_matches_oracle(qm, T, E, k, seed):
+    import torch
+    g = np.random.default_rng(seed)
+    lg = g.standard_normal((T, E)).astype(np.float32)
+    lg[::3, :: 5] = 0.5          # ties
+    d = torch.from_numpy(lg).cuda()
+    ids = torch.empty((T, k), dtype=torch.int32, device="cuda")
+    w = torch.empty((T, k), dtype=torch.float32, device="cuda")
+    perm = torch.empty(T * k, dtype=torch.int32, device="cuda")
+    off = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+    qm.route(d, k, ids, w, perm, off)
+    torch.cuda.synchronize()
+    rids, rw, rperm, roff = Q.route(lg, k)
+    assert np.array_equal(ids.cpu().numpy(), rids)
+    assert np.array_equal(perm.cpu().numpy(), rperm)
+    assert np.array_equal(off.cpu().numpy(), roff)
+    assert np.allclose(w.cpu().numpy(), rw, rtol=1e-6, atol=0)
+
+
+# ------------------------------------------------------------------ single linear
+
+def _linear_case(qm, fmt, block, N, K, M, seed):
+    import torch
+    wb = synth.linear_weight(seed, N, K)
+    c, s = qm.pack(FMTS[fmt], 0, wb, block)
+    dc, ds = to_dev(c), to_dev(s)
+    w = qm.make_weights(FMTS[fmt], block, dc, ds)
+    x = synth.tokens(K, seed, M)
+    y = torch.empty((M, N), dtype=torch.int16, device="cuda")
+    ws = torch.empty(qm.linear_workspace_size(N, K, M), dtype=torch.uint8, device="cuda")
+    qm.linear(w, N, K, to_dev(x), y, ws)
+    torch.cuda.synchronize()
+    return wb, x, bf16_dev_to_f64(y), (dc, ds)
+
+
+@pytest.mark.parametrize("fmt,block", [("int2", 128), ("int4", 128), ("int2", 64), ("int4", 64), ("ternary", 64)])
+@pytest.mark.parametrize("M", [1, 3, 8, 9, 16, 21])
+def test_linear_small_shapes(qm, fmt, block, M):
+    N, K = 272, 640      # 17 tiles, 10 (or 5 ternary) k-units: ragged against 8 warps and 148 CTAs
+    wb, x, y, _ = _linear_case(qm, fmt, block, N, K, M, seed=M)
+    codes, scales = oracle_quant(fmt, wb, block)
+    ref = Q.linear(Q.bf16_bits_to_f64(x), Q.dequant(codes, scales, block))
+    _close(y, ref, f"{fmt} M={M}")
+
+
+@pytest.mark.parametrize("fmt", ["int2", "int4", "ternary"])
+@pytest.mark.parametrize("M", [1, 16])
+def test_linear_medium_multi_tile_per_cta(qm, fmt, M):
+    """Enough tiles that every CTA streams several tiles per k-unit (sub-panels of 8)."""
+    N, K = 4096, 1024
+    wb, x, y, _ = _linear_case(qm, fmt, 64, N, K, M, seed=11)
+    codes, scales = oracle_quant(fmt, wb, 64)
+    ref = Q.linear(Q.bf16_bits_to_f64(x), Q.dequant(codes, scales, 64))
+    _close(y, ref, f"{fmt} M={M}")
+
+
+@pytest.mark.parametrize("fmt", ["int2", "int4"])
+@pytest.mark.parametrize("M", [1, 8])
+def test_linear_full_size_sampled_rows(qm, fmt, M):
+    """K=5120 -> N=17408, group 128, as benchmarked; the oracle computes 512 sampled rows."""
+    N, K = 17408, 5120
+    wb, x, y, _ = _linear_case(qm, fmt, 128, N, K, M, seed=7)
+    rows = np.random.default_rng(0).choice(N, 512, replace=False)
+    codes, scales = oracle_quant(fmt, wb[rows], 128)
+    ref = Q.linear(Q.bf16_bits_to_f64(x), Q.dequant(codes, scales, 128))
+    _close(y[:, rows], ref, f"{fmt} M={M}")
+
+
+# ------------------------------------------------------------------ MoE layer
+
+@pytest.mark.parametrize("T", [1, 3, 8, 13])
+def test_forward_tiny(qm, T):
+    case = MoECase(synth.TINY, seed=3)
+    x = synth.tokens(synth.TINY.H, 3, T)
+    lg = synth.router_logits(synth.TINY, 3, T)
+    y = case.run(x, lg)
+    ref = Q.moe_forward(Q.bf16_bits_to_f64(x), lg, synth.TINY.k, case.bank)
+    _close(y, ref, f"tiny T={T}")
+
+
+@pytest.fixture(scope="module")
+def v2lite(qm):
+    return MoECase(synth.V2LITE, seed=5)
+
+
+@pytest.mark.parametrize("T", [1, 2, 4, 8])
+def test_forward_v2lite_full_size(qm, v2lite, T):
+    cfg = synth.V2LITE
+    x = synth.tokens(cfg.H, 5, T)
+    lg = synth.router_logits(cfg, 5, T)
+    y = v2lite.run(x, lg)
+    ref = Q.moe_forward(Q.bf16_bits_to_f64(x), lg, cfg.k, v2lite.bank)
+    _close(y, ref, f"v2lite T={T}")
+
+
+@pytest.mark.parametrize("M", [1, 5, 16, 32])
+def test_forward_v2lite_tokens_per_expert(qm, v2lite, M):
+    """M tokens with identical router logits: every selected expert gets exactly M tokens."""
+    cfg = synth.V2LITE
+    x = synth.tokens(cfg.H, 6, M)
+    lg = synth.shared_logit_tokens(cfg, 6, M)
+    y = v2lite.run(x, lg)
+    pick = np.unique(np.linspace(0, M - 1, 4).astype(int))
+    ref = np.stack([Q.moe_token(Q.bf16_bits_to_f64(x[t]), lg[t], cfg.k, v2lite.bank) for t in pick])
+    _close(y[pick], ref, f"v2lite M={M}")
+
+
+def test_forward_ternary_reduced_experts(qm):
+    cfg = small_cfg(synth.TERNARY, E=6)
+    case = MoECase(cfg, seed=8)
+    T = 9
+    x = synth.tokens(cfg.H, 8, T)
+    lg = synth.router_logits(cfg, 8, T)
+    y = case.run(x, lg)
+    ref = Q.moe_forward(Q.bf16_bits_to_f64(x), lg, cfg.k, case.bank)
+    _close(y, ref, "ternary")
+
+
+def test_forward_prefill_bias_and_row_tiling(qm):
+    cfg = small_cfg(synth.PREFILL, E=16, k=4, H=256, I=192)
+    case = MoECase(cfg, seed=9)
+    T = 70
+    x = synth.tokens(cfg.H, 9, T)
+    lg = synth.router_logits(cfg, 9, T)
+    ref = Q.moe_forward(Q.bf16_bits_to_f64(x), lg, cfg.k, case.bank)
+    y = case.run(x, lg)
+    _close(y, ref, "prefill untiled")
+    # a workspace that only fits ~20 tokens: explicit partial last tile
+    from skinny_gemm_top_b200 import qmoe
+    small_ws = qmoe.workspace_size(case.layer(), 20)
+    y2 = case.run(x, lg, ws_bytes=small_ws)
+    st = qmoe.get_stats()
+    assert st.row_tiles > 1 and st.row_tile_tokens <= 20
+    _close(y2, ref, "prefill tiled")
+    y3 = case.run(x, lg, max_row_tile=32)
+    assert qmoe.get_stats().row_tiles == 3
+    _close(y3, ref, "prefill max_row_tile")
+
+
+def test_forward_scratch_error_and_invalid_args(qm):
+    import torch
+    from skinny_gemm_top_b200 import qmoe
+    case = MoECase(synth.TINY, seed=3)
+    x = to_dev(synth.tokens(synth.TINY.H, 3, 2))
+    lg = torch.from_numpy(synth.router_logits(synth.TINY, 3, 2)).cuda()
+    y = torch.empty((2, synth.TINY.H), dtype=torch.int16, device="cuda")
+    ws = torch.empty(4096, dtype=torch.uint8, device="cuda")
+    with pytest.raises(qmoe.QmoeError) as e:
+        qmoe.forward(case.layer(), x, lg, y, ws)
+    assert e.value.status == qmoe.ERR_SCRATCH
+    bad = case.layer()
+    bad.k = 0
+    with pytest.raises(qmoe.QmoeError) as e:
+        qmoe.forward(bad, x, lg, y, ws)
+    assert e.value.status == qmoe.ERR_INVALID_ARG
+    bad = case.layer()
+    bad.E = 300
+    with pytest.raises(qmoe.QmoeError) as e:
+        qmoe.forward(bad, x, lg, y, ws)
+    assert e.value.status == qmoe.ERR_UNSUPPORTED
+
+
+# ------------------------------------------------------------------ grouped (tcgen05) path
+
+@pytest.mark.parametrize("fc1,fc2", [("int2", "int4"), ("int4", "int4"), ("int2", "int2")])
+def test_forward_grouped_forced(qm, fc1, fc2):
+    """Every expert on the tcgen05 path (including experts with a single token)."""
+    from skinny_gemm_top_b200 import qmoe
+    cfg = small_cfg(synth.PREFILL, E=16, k=4, H=256, I=192, fc1_fmt=fc1, fc2_fmt=fc2)
+    case = MoECase(cfg, seed=12)
+    T = 90
+    x = synth.tokens(cfg.H, 12, T)
+    lg = synth.router_logits(cfg, 12, T)
+    y = case.run(x, lg, path=qmoe.PATH_GROUPED)
+    st = qmoe.get_stats()
+    assert st.grouped_launches == 2 and st.last_path == qmoe.PATH_GROUPED
+    ref = Q.moe_forward(Q.bf16_bits_to_f64(x), lg, cfg.k, case.bank)
+    _close(y, ref, f"grouped {fc1}/{fc2}")
+
+
+def test_forward_auto_mixes_paths(qm):
+    """Zipf-skewed routing: hot experts exceed the small-M chunk and take the
+    grouped path, cold ones stay on the small-M path; one token tile spans
+    more than 256 tokens."""
+    from skinny_gemm_top_b200 import qmoe
+    cfg = small_cfg(synth.PREFILL, E=8, k=2, H=384, I=256)
+    case = MoECase(cfg, seed=13)
+    T = 400
+    x = synth.tokens(cfg.H, 13, T)
+    lg = synth.router_logits(cfg, 13, T)
+    ids, _, _, _ = Q.route(lg, cfg.k)
+    counts = np.bincount(ids.ravel(), minlength=cfg.E)
+    assert counts.max() > 256 and counts.min() <= 32
+    y = case.run(x, lg)
+    st = qmoe.get_stats()
+    assert st.grouped_launches == 2 and st.small_launches == 2
+    ref = Q.moe_forward(Q.bf16_bits_to_f64(x), lg, cfg.k, case.bank)
+    _close(y, ref, "auto")
+    y2 = case.run(x, lg, path=qmoe.PATH_SMALL_M)
+    assert qmoe.get_stats().grouped_launches == 0
+    _close(y2, ref, "small-M forced")
+
+
+@pytest.mark.slow
+def test_forward_prefill_full_size_sampled(qm):
+    """Prefill layer at full size: T=4096, H=2048, I=768, 128 experts top-8,
+    expert biases, Zipf(1.1) router offsets, row-tiled within 256 MiB."""
+    from skinny_gemm_top_b200 import qmoe
+    cfg = synth.PREFILL
+    case = MoECase(cfg, seed=14)
+    T = 4096
+    x = synth.tokens(cfg.H, 14, T)
+    lg = synth.router_logits(cfg, 14, T)
+    y = case.run(x, lg, ws_bytes=256 << 20)
+    st = qmoe.get_stats()
+    assert st.row_tiles >= 2 and st.grouped_launches >= 2
+    pick = np.random.default_rng(1).choice(T, 6, replace=False)
+    ref = np.stack([Q.moe_token(Q.bf16_bits_to_f64(x[t]), lg[t], cfg.k, case.bank) for t in pick])
+    _close(y[pick], ref, "prefill full size")
