@@ -48,6 +48,8 @@ def parse():
     ap.add_argument("--sweep", default="1,2,4,8,16,32")
     ap.add_argument("--linear-sweep", default="1,2,3,4,5,8,10,16,32")
     ap.add_argument("--quick", action="store_true", help="skip the sweeps")
+    ap.add_argument("--profile", action="store_true",
+                    help="a few eager layer forwards and linears only (for an ncu launch list or capture)")
     return ap.parse_args()
 
 
@@ -188,6 +190,17 @@ class Steps:
             self.tails[rem].replay()
 
 
+def reduce_ranks(torch, dist, ms: float, nbytes: float, device: str = "cuda"):
+    """Whole-job aggregation: the slowest rank's time and the bytes all ranks moved."""
+    if dist is None:
+        return ms, nbytes
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    b = torch.tensor([nbytes], dtype=torch.float64, device=device)
+    dist.all_reduce(b, op=dist.ReduceOp.SUM)
+    return float(t.item()), float(b.item())
+
+
 def time_steps(torch, dist, steps: Steps, k: int) -> float:
     """ms for k steps, device-timed with events, max over ranks."""
     if dist is not None:
@@ -198,12 +211,7 @@ def time_steps(torch, dist, steps: Steps, k: int) -> float:
     steps.run(k)
     e1.record()
     torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1)
-    if dist is not None:
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
-    return ms
+    return e0.elapsed_time(e1)
 
 
 def moe_inputs(torch, M: int, rotate: int):
@@ -212,6 +220,31 @@ def moe_inputs(torch, M: int, rotate: int):
     lgs_np = [np.repeat(rows[r:r + 1], M, axis=0) for r in range(rotate)]
     lgs = [torch.from_numpy(l).cuda() for l in lgs_np]
     return xs, lgs, lgs_np
+
+
+def run_profile(args):
+    """A handful of eager forwards and linears on one GPU: small enough for ncu."""
+    import torch
+    from skinny_gemm_top_b200 import qmoe
+    layers, keep = pack_moe(qmoe, torch, 1)
+    for M in (1, 8):
+        xs, lgs, _ = moe_inputs(torch, M, 1)
+        ws = torch.empty(qmoe.workspace_size(layers[0], M), dtype=torch.uint8, device="cuda")
+        y = torch.empty((M, CFG.H), dtype=torch.int16, device="cuda")
+        for _ in range(args.steps):
+            qmoe.forward(layers[0], xs[0], lgs[0], y, ws)
+            torch.cuda.synchronize()
+    N, K = 17408, 5120
+    c, s = qmoe.pack(qmoe.INT2, qmoe.ROWS_PLAIN, synth.linear_weight(SEED, N, K), 128)
+    dc, ds = _to_dev(torch, c), _to_dev(torch, s)
+    w = qmoe.make_weights(qmoe.INT2, 128, dc, ds)
+    x = _to_dev(torch, synth.tokens(K, SEED, 1))
+    y = torch.empty((1, N), dtype=torch.int16, device="cuda")
+    ws = torch.empty(qmoe.linear_workspace_size(N, K, 1), dtype=torch.uint8, device="cuda")
+    for _ in range(args.steps):
+        qmoe.linear(w, N, K, x, y, ws)
+        torch.cuda.synchronize()
+    print("profile run done", flush=True)
 
 
 def run_ours(args):
@@ -239,11 +272,7 @@ def run_ours(args):
             r = i % ROTATE
             qmoe.forward(layers[r], xs[r], lgs[r], ys[r], ws)
 
-        if trace:  # the eager call of graph_of takes 5 records, the captured graph the next 5 * ROTATE
-            qmoe.trace_start(5 * (ROTATE + 1))
         steps = Steps(torch, fn, ROTATE)
-        if trace:
-            qmoe.trace_stop()
         steps.prepare(k, w)
         if clocks is not None:  # settle clocks under this load before the timed region
             t_end = time.time() + 1.5
@@ -253,12 +282,25 @@ def run_ours(args):
         steps.run(w)
         ms = time_steps(torch, dist, steps, k)
         per = [layer_bytes(l) for l in lgs_np]
-        out = {"ms_per_step": ms / k, "bytes": statistics.mean(p["total"] for p in per),
+        local_bytes = statistics.mean(p["total"] for p in per)
+        ms, job_bytes = reduce_ranks(torch, dist, ms, local_bytes)
+        out = {"ms_per_step": ms / k, "bytes": local_bytes, "job_bytes": job_bytes,
                "fc1_bytes": statistics.mean(p["fc1"] for p in per)}
         if trace:
+            # Per-kernel device time: a second graph of the same ROTATE calls with CUDA
+            # events around every launch (the eager call of graph_of takes 5 records).
+            qmoe.trace_start(5 * (ROTATE + 1))
+            traced = Steps(torch, fn, ROTATE)
+            qmoe.trace_stop()
+            traced.run(w)
+            t0 = time.time()
+            while time.time() - t0 < 0.2:  # the timed region of the trace: replays of the traced graph
+                traced.run(k)
+            torch.cuda.synchronize()
             rec = qmoe.trace_read(5 * (ROTATE + 1))[5:]
             out["fc1_ms"] = statistics.mean(t for n, t in rec if n == "fc1_small")
             out["kernels"] = {n: statistics.mean(t for m, t in rec if m == n) for n in sorted({n for n, _ in rec})}
+            del traced
         return out
 
     sampler = ClockSampler(dev_index)
@@ -286,7 +328,7 @@ def run_ours(args):
     if os.path.exists(tpath):
         traffic = json.load(open(tpath)).get("fc1_small_v2lite_M1_bytes_per_launch")
 
-    value = head["bytes"] / (head["ms_per_step"] * 1e6) * world
+    value = head["job_bytes"] / (head["ms_per_step"] * 1e6)
     line = {
         "metric": METRIC,
         "value": round(value, 1),
@@ -395,7 +437,7 @@ def linear_sweep(qmoe, torch, dist, args) -> list:
             k = max(args.steps, 64)
             steps.prepare(k, args.warmup)
             steps.run(args.warmup)
-            ms = time_steps(torch, dist, steps, k) / k
+            ms = reduce_ranks(torch, dist, time_steps(torch, dist, steps, k), 0.0)[0] / k
             b = nbytes + M * K * 2 + M * N * 2
             row["M"].append({"M": M, "us": round(ms * 1e3, 3), "GBps": round(b / (ms * 1e6), 1)})
         out.append(row)
@@ -479,6 +521,8 @@ def main():
     args = parse()
     if args.impl == "reference":
         run_reference(args)
+    elif args.profile:
+        run_profile(args)
     else:
         run_ours(args)
 
