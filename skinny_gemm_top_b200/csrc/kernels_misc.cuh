@@ -46,6 +46,9 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
   __shared__ int gseg_base[kMaxExperts + 64];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int nwarps = blockDim.x >> 5;
+  // Writes below may alias buffers the previous launch still reads.
+  pdl_wait();
+  pdl_trigger();
 
   for (int e = tid; e < kMaxExperts; e += blockDim.x) { counts[e] = 0; running[e] = 0; }
 
@@ -194,6 +197,8 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
 
 // Segment table of a single linear: chunks of <= 16 consecutive tokens.
 __global__ void linear_setup_kernel(int M, int* nseg, Seg* segs, int* tickets, int n_tickets) {
+  pdl_wait();
+  pdl_trigger();
   const int nchunks = (M + kChunkTokens - 1) / kChunkTokens;
   for (int c = threadIdx.x; c < nchunks; c += blockDim.x) {
     Seg s;
@@ -219,6 +224,8 @@ __global__ void gather_kernel(const uint16_t* __restrict__ x, int K, const int* 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
   const int g = lane >> 2, q = lane & 3;
   const int KB = K / 64;
+  pdl_wait();
+  pdl_trigger();
   const int ns = *nseg;
   for (int s = blockIdx.x; s < ns; s += gridDim.x) {
     const Seg sg = segs[s];
@@ -251,6 +258,8 @@ __global__ void gather_kernel(const uint16_t* __restrict__ x, int K, const int* 
 // Token rows of the grouped tiles, in expert-sorted slot order: xrows[slot] = x[token(slot)].
 __global__ void gather_rows_kernel(const uint16_t* __restrict__ x, int K, const int* __restrict__ slot_token,
                                    const int* __restrict__ ngseg, const GSeg* __restrict__ gsegs, uint16_t* xrows) {
+  pdl_wait();
+  pdl_trigger();
   const int ng = *ngseg;
   const int vec = K / 8;  // uint4 per row
   for (int gi = blockIdx.x; gi < ng; gi += gridDim.x) {
@@ -268,6 +277,8 @@ __global__ void gather_rows_kernel(const uint16_t* __restrict__ x, int K, const 
 __global__ void combine_kernel(const float* __restrict__ yslot, const float* __restrict__ w,
                                const int* __restrict__ inv, int T, int k, int n_shared, int H,
                                uint16_t* __restrict__ y) {
+  pdl_wait();
+  pdl_trigger();
   const int t = blockIdx.x;
   for (int h = threadIdx.x * 4; h < H; h += blockDim.x * 4) {
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);

@@ -93,6 +93,26 @@ struct TraceScope {
   }
 };
 
+// Launch with programmatic dependent launch: the kernel may start while its
+// predecessor in the stream finishes; every kernel calls griddepcontrol.wait
+// before touching its predecessor's outputs and only then allows its own
+// dependents to launch.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 inline size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 
 bool fmt_ok(int f) { return f == QMOE_INT2 || f == QMOE_INT4 || f == QMOE_TERNARY; }
@@ -210,8 +230,9 @@ qmoe_status launch_small_t(SmallParams prm, int grid, cudaStream_t st) {
     attr_set[d] = true;
   }
   TraceScope ts(st, EPI == EPI_SWIGLU ? K_FC1_SMALL : (EPI == EPI_FC2 ? K_FC2_SMALL : K_LINEAR_SMALL));
-  qmm_small_kernel<FMT, TG, EPI><<<grid, kNW * 32, smem, st>>>(prm);
-  return cudaGetLastError() == cudaSuccess ? QMOE_OK : QMOE_ERR_CUDA;
+  return launch_pdl(qmm_small_kernel<FMT, TG, EPI>, dim3(grid), dim3(kNW * 32), smem, st, prm) == cudaSuccess
+             ? QMOE_OK
+             : QMOE_ERR_CUDA;
 }
 
 template <int EPI>
@@ -444,18 +465,20 @@ qmoe_status qmoe_forward(const qmoe_layer* layer, const uint16_t* x, const float
     o.status = di->status;
     {
       TraceScope ts(st, K_ROUTE);
-      route_kernel<<<1, kRouteThreads, 0, st>>>(logits + (size_t)t0 * L.E, tt, L.E, L.k, L.n_shared, o);
+      if (launch_pdl(route_kernel, dim3(1), dim3(kRouteThreads), 0, st, logits + (size_t)t0 * L.E, tt, L.E, L.k,
+                     L.n_shared, o) != cudaSuccess)
+        return QMOE_ERR_CUDA;
     }
-    if (cudaGetLastError() != cudaSuccess) return QMOE_ERR_CUDA;
     uint8_t* xfrag = base + p.xfrag;
     uint8_t* hfrag = base + p.hfrag;
     float* yslot = reinterpret_cast<float*>(base + p.yslot);
     {
       TraceScope ts(st, K_GATHER);
-      gather_kernel<<<std::min(p.max_seg, 4 * grid), 256, 0, st>>>(x + (size_t)t0 * L.H, L.H, o.slot_token,
-                                                                    o.nseg, o.segs, xfrag, beta_hi(L.fc1.fmt));
+      if (launch_pdl(gather_kernel, dim3(std::min(p.max_seg, 4 * grid)), dim3(256), 0, st,
+                     x + (size_t)t0 * L.H, L.H, (const int*)o.slot_token, (const int*)o.nseg, (const Seg*)o.segs,
+                     xfrag, beta_hi(L.fc1.fmt)) != cudaSuccess)
+        return QMOE_ERR_CUDA;
     }
-    if (cudaGetLastError() != cudaSuccess) return QMOE_ERR_CUDA;
     const int tg = tt <= 8 ? 1 : 2;
     SmallParams p1 = small_params(L.fc1, 2 * L.I, L.H, di->status);
     p1.nseg = o.nseg;
@@ -525,9 +548,10 @@ qmoe_status qmoe_forward(const qmoe_layer* layer, const uint16_t* x, const float
     }
     {
       TraceScope ts(st, K_COMBINE);
-      combine_kernel<<<tt, 256, 0, st>>>(yslot, o.w, o.inv, tt, L.k, L.n_shared, L.H, y + (size_t)t0 * L.H);
+      if (launch_pdl(combine_kernel, dim3(tt), dim3(256), 0, st, (const float*)yslot, (const float*)o.w,
+                     (const int*)o.inv, tt, L.k, L.n_shared, L.H, y + (size_t)t0 * L.H) != cudaSuccess)
+        return QMOE_ERR_CUDA;
     }
-    if (cudaGetLastError() != cudaSuccess) return QMOE_ERR_CUDA;
     ++tiles;
     small += 2;
   }
@@ -580,14 +604,16 @@ qmoe_status qmoe_linear(const qmoe_weights* w, int N, int K, const uint16_t* x, 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   {
     TraceScope ts(st, K_LINEAR_SETUP);
-    linear_setup_kernel<<<1, 256, 0, st>>>(M, d_nseg, segs, tickets, nseg * (N / 16));
+    if (launch_pdl(linear_setup_kernel, dim3(1), dim3(256), 0, st, M, d_nseg, segs, tickets, nseg * (N / 16)) !=
+        cudaSuccess)
+      return QMOE_ERR_CUDA;
   }
-  if (cudaGetLastError() != cudaSuccess) return QMOE_ERR_CUDA;
   {
     TraceScope ts(st, K_GATHER);
-    gather_kernel<<<nseg, 256, 0, st>>>(x, K, nullptr, d_nseg, segs, xfrag, beta_hi(w->fmt));
+    if (launch_pdl(gather_kernel, dim3(nseg), dim3(256), 0, st, x, K, (const int*)nullptr, (const int*)d_nseg,
+                   (const Seg*)segs, xfrag, beta_hi(w->fmt)) != cudaSuccess)
+      return QMOE_ERR_CUDA;
   }
-  if (cudaGetLastError() != cudaSuccess) return QMOE_ERR_CUDA;
   SmallParams p = small_params(*w, N, K, di->status);
   p.nseg = d_nseg;
   p.segs = segs;
