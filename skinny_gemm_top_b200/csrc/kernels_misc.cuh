@@ -1,4 +1,4 @@
-// Routing, activation gather, combine, single-linear setup and dequant kernels.
+// Routing, grouped-path row gather, combine and dequant kernels.
 #pragma once
 #include <cfloat>
 #include <climits>
@@ -11,7 +11,6 @@
 namespace qmoe {
 
 constexpr int kRouteThreads = 1024;
-constexpr int kMaxExperts = 256;
 
 struct RouteOut {
   int* ids;          // [T*k]
@@ -42,7 +41,6 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
   __shared__ int warp_cnt[32][kMaxExperts];
   __shared__ float selv[32][32];
   __shared__ int seg_base[kMaxExperts + 64];
-  __shared__ int tg_base[kMaxExperts + 64];
   __shared__ int gseg_base[kMaxExperts + 64];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int nwarps = blockDim.x >> 5;
@@ -139,19 +137,14 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
     const int EX = E + n_shared;
     __syncthreads();
     if (tid == 0) {
-      int sb = 0, tb = 0, gb = 0;
+      int sb = 0, gb = 0;
       for (int e = 0; e < EX; ++e) {
         const int cnt = e < E ? counts[e] : T;
         const bool grouped = o.ngseg && cnt > o.thresh;
         seg_base[e] = sb;
-        tg_base[e] = tb;
         gseg_base[e] = gb;
-        if (grouped) {
-          gb += (cnt + kGTok - 1) / kGTok;
-        } else {
-          sb += (cnt + kChunkTokens - 1) / kChunkTokens;
-          tb += 2 * (cnt / kChunkTokens) + ((cnt % kChunkTokens) + 7) / 8;
-        }
+        if (grouped) gb += (cnt + kGTok - 1) / kGTok;
+        else sb += (cnt + kChunkTokens - 1) / kChunkTokens;
       }
       if (sb > o.max_seg || (o.ngseg && gb > o.max_gseg)) {
         atomicOr(o.status, kStatusBadSegment);
@@ -185,74 +178,12 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
         s.m = min(kChunkTokens, cnt - kChunkTokens * c);
         s.tg = (s.m + 7) / 8;
         s.slot0 = slot_base + kChunkTokens * c;
-        s.xoff = tg_base[e] + 2 * c;
-        s.pad[0] = s.pad[1] = s.pad[2] = 0;
         o.segs[seg_base[e] + c] = s;
       }
     }
   }
   if (o.tickets)
     for (int i = tid; i < o.n_tickets; i += blockDim.x) o.tickets[i] = 0;
-}
-
-// Segment table of a single linear: chunks of <= 16 consecutive tokens.
-__global__ void linear_setup_kernel(int M, int* nseg, Seg* segs, int* tickets, int n_tickets) {
-  pdl_wait();
-  pdl_trigger();
-  const int nchunks = (M + kChunkTokens - 1) / kChunkTokens;
-  for (int c = threadIdx.x; c < nchunks; c += blockDim.x) {
-    Seg s;
-    s.expert = 0;
-    s.m = min(kChunkTokens, M - kChunkTokens * c);
-    s.tg = (s.m + 7) / 8;
-    s.slot0 = kChunkTokens * c;
-    s.xoff = 2 * c;
-    s.pad[0] = s.pad[1] = s.pad[2] = 0;
-    segs[c] = s;
-  }
-  if (threadIdx.x == 0) *nseg = nchunks;
-  for (int i = threadIdx.x; i < n_tickets; i += blockDim.x) tickets[i] = 0;
-}
-
-// Activation operand fragments: for each segment, token group and 64-column
-// block, lane l = 4g + q stores x[token g][16ks + 2q + {0,1}] and
-// [16ks + 2q + 8 + {0,1}] for ks = 0..3 (the m16n8k16 B fragment), the second
-// pair divided by beta_hi (exact power-of-two scaling).  Padding tokens are 0.
-__global__ void gather_kernel(const uint16_t* __restrict__ x, int K, const int* __restrict__ slot_token,
-                              const int* __restrict__ nseg, const Seg* __restrict__ segs, uint8_t* frag,
-                              int beta_hi) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
-  const int g = lane >> 2, q = lane & 3;
-  const int KB = K / 64;
-  pdl_wait();
-  pdl_trigger();
-  const int ns = *nseg;
-  for (int s = blockIdx.x; s < ns; s += gridDim.x) {
-    const Seg sg = segs[s];
-    const int items = KB * sg.tg;
-    uint8_t* base = frag + (size_t)sg.xoff * K * 16;
-    for (int it = warp; it < items; it += nw) {
-      const int kb = it / sg.tg, tg = it % sg.tg;
-      const int n = tg * 8 + g;
-      uint32_t r[8];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) r[j] = 0u;
-      if (n < sg.m) {
-        const int tok = slot_token ? slot_token[sg.slot0 + n] : sg.slot0 + n;
-        const uint32_t* row = reinterpret_cast<const uint32_t*>(x + (size_t)tok * K + kb * 64);
-#pragma unroll
-        for (int ks = 0; ks < 4; ++ks) {
-          r[2 * ks] = row[(16 * ks + 2 * q) >> 1];
-          uint32_t hi = row[(16 * ks + 2 * q + 8) >> 1];
-          if (beta_hi == 4) hi = fma_bf16x2(hi, kBf16Quarter, 0x80008000u);
-          r[2 * ks + 1] = hi;
-        }
-      }
-      uint4* dst = reinterpret_cast<uint4*>(base + ((size_t)(kb * sg.tg + tg) * 32 + lane) * 32);
-      dst[0] = make_uint4(r[0], r[1], r[2], r[3]);
-      dst[1] = make_uint4(r[4], r[5], r[6], r[7]);
-    }
-  }
 }
 
 // Token rows of the grouped tiles, in expert-sorted slot order: xrows[slot] = x[token(slot)].

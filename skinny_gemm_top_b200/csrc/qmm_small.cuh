@@ -2,36 +2,44 @@
 //
 // For every (expert, chunk of <= 16 tokens) segment, y[rows, m] = dequant(W)
 // x[m, K] with fp32 accumulation, followed by one of three epilogues: plain
-// bf16 store (single linear), bias + interleaved SwiGLU into the FC2 operand
-// (FC1), bias into the expert-sorted slot buffer (FC2).
+// bf16 store (single linear), bias + interleaved SwiGLU into bf16 rows of h
+// (FC1), bias into the fp32 expert-sorted slot rows (FC2).
 //
 // Design (B200):
 //  * The weights are streamed from HBM once per segment: one pass over the
 //    codes serves all tokens routed to the expert, the remedy the QMoE note
 //    gives for the per-token GEMV relaunch ("inner loop over tokens").
 //  * Work = (segment, 16-row tile, k-unit of 64 columns; 128 for ternary).
-//    With at least as many tiles as CTAs, CTA c takes a balanced range of
-//    whole tiles; with fewer, a balanced range of units (stream-K), and tiles
-//    split between CTAs are finished by the last CTA to arrive (atomic ticket,
-//    no spin-wait), summing partials in CTA order: deterministic either way.
+//    CTA c takes a balanced range of whole tiles, so no tile is split
+//    between CTAs and every output is written once, deterministically.
 //  * Inside a CTA, up to 8 consecutive tiles form a sub-panel; its k-units go
 //    round-robin to 8 warps.  Each warp runs its own TMA bulk-copy pipeline
-//    (cp.async.bulk + mbarrier, no tensor map, no multicast) of stages holding
-//    the sub-panel's codes, scales and the activation fragments of that
-//    k-unit.  Each activation fragment is reused by every tile of the stage,
-//    and the MMAs of all tiles of a k-step are issued back to back so their
-//    latencies overlap.
+//    (cp.async.bulk + mbarrier, no tensor map, no multicast).  A stage holds
+//    the sub-panel's codes and scales at one k-unit plus that k-unit's slice
+//    of the segment's activation rows (one 128-byte copy per token, issued by
+//    one lane each).  B fragments come from those rows through ldmatrix and
+//    are reused by every tile of the stage; the MMAs of all tiles of a k-step
+//    issue back to back so their latencies overlap.
 //  * Codes become bf16 MMA operands with LOP3 magic numbers (unpack.cuh) and
 //    are multiplied on the tensor cores (mma.sync m16n8k16, tokens in N):
 //    the CUDA-core budget of sm_100a cannot afford an FMA per weight per
-//    token at HBM rate.  The per-block scale is applied to the fp32 partial
+//    token at HBM rate.  The per-block scale multiplies the fp32 partial
 //    product of each 64-column block, so the dequantized weight c*s is never
 //    rounded.
+//  * Segment sources: a table written by an earlier routing launch; routing
+//    computed in the kernel's prologue by every CTA for a decode batch of up
+//    to 8 tokens (identical, deterministic results in all CTAs; no routing
+//    launch); or fixed chunks of the rows of a single linear.
 //  * Programmatic dependent launch: the weights of the first stages are
-//    requested before griddepcontrol.wait (they depend only on the routing
-//    of an earlier launch), the activations after it.
-//  * Per-warp partial sums are reduced through shared memory in warp order.
+//    requested before griddepcontrol.wait (they depend only on the routing),
+//    the activations after it.
+//  * Decode FC2 fuses the router-weighted combine: the last CTA to finish a
+//    16-row output tile (atomic counter, no spin-wait) sums that tile's slot
+//    rows in slot order and writes y.
 #pragma once
+#include <cfloat>
+#include <climits>
+
 #include "device_common.cuh"
 #include "unpack.cuh"
 
@@ -42,16 +50,36 @@ constexpr int kMaxT = 8;          // tiles per sub-panel
 constexpr int kChunkTokens = 16;  // tokens per segment (<= 2 token groups of 8)
 
 enum Epi { EPI_LINEAR = 0, EPI_SWIGLU = 1, EPI_FC2 = 2 };
+enum SegSrc { SRC_TABLE = 0, SRC_DECODE = 1, SRC_LINEAR = 2 };
 
-// One (expert, token chunk) work item.  Fragments of its activation operand
-// live at token-group offset xoff of the fragment buffers.
+// Decode batches routed inside the kernels: up to 8 tokens, T*k <= 64,
+// at most 8 shared experts.
+constexpr int kDecMaxT = 8;
+constexpr int kDecMaxTK = 64;
+constexpr int kDecMaxShared = 8;
+constexpr int kDecMaxSegs = kDecMaxTK + kDecMaxShared;
+constexpr int kDecMaxSlots = kDecMaxTK + kDecMaxShared * kDecMaxT;
+constexpr int kMaxExperts = 256;
+
+// One (expert, token chunk) work item.
 struct Seg {
   int expert;  // weight matrix index
   int m;       // tokens in the chunk, 1..16
   int tg;      // token groups of 8 (1 or 2)
-  int slot0;   // first row of the chunk in the expert-sorted slot order (or token index)
-  int xoff;    // token-group offset into the fragment buffers
-  int pad[3];
+  int slot0;   // first row of the chunk in the slot order (or first token row)
+};
+
+// Routing of a decode batch, computed in shared memory.
+struct DecodeRoute {
+  int nseg;
+  Seg segs[kDecMaxSegs];
+  int slot_token[kDecMaxSlots];  // slot -> token
+  int pos[kDecMaxTK];            // flat index t*k+s -> slot
+  float w[kDecMaxTK];            // router weight of flat index
+  int ids[kDecMaxTK];
+  int counts[kMaxExperts];
+  int offs[kMaxExperts];
+  float selv[kDecMaxT][32];
 };
 
 struct SmallParams {
@@ -63,22 +91,27 @@ struct SmallParams {
   int K;
   int KU;                            // k-units per row
   int block;                         // scale block (64 or 128)
+  int nstages;
+  // segments (SRC_TABLE)
   const int* nseg;
   const Seg* segs;
-  const uint8_t* xfrag;              // activation fragments: segment at xoff * K * 16 bytes
-  int nstages;
+  // activation rows [*, K] bf16: row of slot s is act_index[s] (or s when null)
+  const uint16_t* act;
+  const int* act_index;
+  // routing inputs (SRC_DECODE) / row count (SRC_LINEAR)
+  const float* logits;
+  int T, E, k, n_shared;
   // epilogues
-  uint16_t* y;                       // LINEAR: y[token][N]
+  uint16_t* y;                       // LINEAR: y[token][N]; decode FC2: combined y[token][H]
   int N;
   const uint16_t* bias;              // SWIGLU/FC2: bias + expert * bias_rows (logical rows)
   int bias_rows;
-  uint8_t* hfrag;                    // SWIGLU: FC2 activation fragments (K = I)
+  uint16_t* hrows;                   // SWIGLU: h[slot][I] bf16
   int I;
-  int h_beta_hi;                     // 4: divide columns k%16 >= 8 by 4 (INT2 / ternary FC2)
   float* yslot;                      // FC2: yslot[slot][H]
   int H;
-  float* partials;                   // 2 slots per CTA of 2 token groups * 32 float4
-  int* tickets;                      // per (segment, tile), zero before the launch
+  int* ctick;                        // decode: per 16-row output tile counters (H/16)
+  int early;                         // 1: segments and weights may be read before griddepcontrol.wait
   unsigned* status;
 };
 
@@ -89,149 +122,156 @@ struct StageGeom {
   static constexpr int kBlocksPerKU = Tr::kKUcols / 64;                 // 64-col blocks per k-unit
   static constexpr int kCodeBytes = kMaxT * Tr::kCodeBytes;
   static constexpr int kScaleBytes = kBlocksPerKU * kMaxT * 32;
-  static constexpr int kXBytes = kBlocksPerKU * TG * 1024;
-  static constexpr int kStageBytes = ((kCodeBytes + kScaleBytes + kXBytes) + 127) / 128 * 128;
+  static constexpr int kActPitch = Tr::kKUcols * 2 + 16;               // padded: conflict-free ldmatrix
+  static constexpr int kActBytes = TG * 8 * kActPitch;
+  static constexpr int kStageBytes = ((kCodeBytes + kScaleBytes + kActBytes) + 127) / 128 * 128;
   static constexpr int kRedBytes = kNW * kMaxT * TG * 32 * 16;
 };
 
+template <int SRC>
+struct SmemHead {
+  static constexpr int kRouteBytes = SRC == SRC_DECODE ? ((int)sizeof(DecodeRoute) + 127) / 128 * 128 : 0;
+  static constexpr int kFixed = 2048 + kRouteBytes;  // barriers + ternary LUT + routing
+};
+
 // ---------------------------------------------------------------------------
-// Balanced split of n items over G CTAs (32-bit); item boundaries scaled by
-// `unit` units (KU for whole tiles, 1 for single k-units).
+// Balanced split of whole tiles over CTAs (32-bit).
 struct Part {
-  unsigned n, q, r, unit;
-  __device__ __forceinline__ void init(unsigned n_, unsigned G, unsigned unit_) {
-    n = n_;
-    q = n_ / G;
-    r = n_ - q * G;
+  unsigned q, r, unit;
+  __device__ __forceinline__ void init(unsigned n, unsigned G, unsigned unit_) {
+    q = n / G;
+    r = n - q * G;
     unit = unit_;
   }
   __device__ __forceinline__ unsigned begin(unsigned c) const { return (c * q + min(c, r)) * unit; }
-  // CTA whose range holds unit x (x < n * unit).
-  __device__ __forceinline__ unsigned owner(unsigned x) const {
-    const unsigned i = x / unit;
-    const unsigned big = r * (q + 1);
-    return i < big ? i / (q + 1) : r + (i - big) / q;
-  }
 };
 
-// Sub-panel: up to kMaxT consecutive tiles of one segment inside [pos, f1).
+// Sub-panel: up to kMaxT consecutive whole tiles of one segment inside [pos, f1).
 struct SubPanel {
   unsigned next;  // first unit after this sub-panel
   int seg, rt0, nt;
-  int kf;         // first k-unit of tile 0
-  int kl;         // end k-unit of tile nt-1
 };
 
 __device__ __forceinline__ void load_subpanel(SubPanel& sp, unsigned pos, unsigned f1, int NT, int KU) {
   const unsigned per_seg = (unsigned)NT * (unsigned)KU;
   const unsigned seg = pos / per_seg;
-  const unsigned r = pos - seg * per_seg;
-  const unsigned rt = r / (unsigned)KU;
-  const unsigned ku = r - rt * (unsigned)KU;
+  const unsigned rt = (pos - seg * per_seg) / (unsigned)KU;
   const unsigned tile_base = seg * per_seg + rt * (unsigned)KU;
   unsigned end = f1;
   const unsigned seg_end = (seg + 1) * per_seg;
   if (seg_end < end) end = seg_end;
   const unsigned cap = tile_base + (unsigned)(kMaxT * KU);
   if (cap < end) end = cap;
-  const int nt = (int)((end - tile_base + KU - 1) / (unsigned)KU);
   sp.next = end;
   sp.seg = (int)seg;
   sp.rt0 = (int)rt;
-  sp.nt = nt;
-  sp.kf = (int)ku;
-  sp.kl = (int)(end - (tile_base + (unsigned)(nt - 1) * KU));
+  sp.nt = (int)((end - tile_base) / (unsigned)KU);
 }
 
-// Tiles [a, b) of the sub-panel hold k-unit ku (a = 1 when the head tile starts after ku).
-__device__ __forceinline__ void active_tiles(const SubPanel& sp, int ku, int& a, int& b) {
-  a = ku >= sp.kf ? 0 : 1;
-  b = ku < sp.kl ? sp.nt : sp.nt - 1;
-}
+// Segments either come from a table (global or shared memory) or, for a
+// single linear, are fixed chunks of kChunkTokens rows.
+struct SegSource {
+  const Seg* table;
+  int rows;  // table == nullptr: number of rows
+  __device__ __forceinline__ Seg get(int c) const {
+    if (table) return table[c];
+    Seg sg;
+    sg.expert = 0;
+    sg.m = min(kChunkTokens, rows - kChunkTokens * c);
+    sg.tg = (sg.m + 7) / 8;
+    sg.slot0 = kChunkTokens * c;
+    return sg;
+  }
+};
 
-// Producer iterator over this warp's (sub-panel, k-unit) items; caches the
-// current segment so an item costs no global load.
+// Warp-uniform producer iterator over this warp's (sub-panel, k-unit) items.
+// Caches the segment and, per lane n < m, the row of token n.
 struct ItemIter {
   SubPanel sp;
   Seg sg;
   unsigned f1;
   int ku;
+  int row;     // this lane's activation row (lane < sg.m)
   bool valid;
 };
 
 template <int TG>
-__device__ __forceinline__ void iter_load_seg(ItemIter& it, const SmallParams& p, int prev_seg) {
-  if (it.sp.seg != prev_seg) {
-    it.sg = p.segs[it.sp.seg];
-    if (it.sg.tg > TG || it.sg.tg < 1) it.sg.tg = TG;  // never overrun the stage buffer (flagged by the consumer)
-  }
+__device__ __forceinline__ void iter_load_seg(ItemIter& it, const SmallParams& p, const SegSource& segs,
+                                              const int* act_index, int lane) {
+  it.sg = segs.get(it.sp.seg);
+  if (it.sg.tg > TG || it.sg.tg < 1) it.sg.tg = TG;  // never overrun the stage (flagged by the consumer)
+  if (it.sg.m > 8 * it.sg.tg) it.sg.m = 8 * it.sg.tg;
+  const int s = it.sg.slot0 + (lane < it.sg.m ? lane : 0);
+  it.row = act_index ? act_index[s] : s;
 }
 
 template <int TG>
-__device__ __forceinline__ void iter_advance(ItemIter& it, const SmallParams& p, int warp) {
+__device__ __forceinline__ void iter_advance(ItemIter& it, const SmallParams& p, const SegSource& segs,
+                                             const int* act_index, int warp, int lane) {
+  it.ku += kNW;
+  if (it.ku < p.KU) return;
   for (;;) {
-    it.ku += kNW;
-    if (it.ku >= p.KU) {
-      if (it.sp.next >= it.f1) { it.valid = false; return; }
-      const int prev = it.sp.seg;
-      load_subpanel(it.sp, it.sp.next, it.f1, p.NT, p.KU);
-      iter_load_seg<TG>(it, p, prev);
-      it.ku = warp;
-      if (it.ku >= p.KU) { it.ku = p.KU; continue; }  // this warp has no k-unit here
-    }
-    int a, b;
-    active_tiles(it.sp, it.ku, a, b);
-    if (a < b) return;
+    if (it.sp.next >= it.f1) { it.valid = false; return; }
+    const int prev = it.sp.seg;
+    load_subpanel(it.sp, it.sp.next, it.f1, p.NT, p.KU);
+    if (it.sp.seg != prev) iter_load_seg<TG>(it, p, segs, act_index, lane);
+    it.ku = warp;
+    if (it.ku < p.KU) return;
   }
 }
 
 template <int TG>
-__device__ __forceinline__ void iter_begin(ItemIter& it, const SmallParams& p, unsigned f0, unsigned f1, int warp) {
+__device__ __forceinline__ void iter_begin(ItemIter& it, const SmallParams& p, const SegSource& segs, const int* act_index,
+                                           unsigned f0, unsigned f1, int warp, int lane) {
   it.f1 = f1;
   it.valid = f0 < f1;
   if (!it.valid) return;
   load_subpanel(it.sp, f0, f1, p.NT, p.KU);
-  iter_load_seg<TG>(it, p, -1);
-  it.ku = warp - kNW;
-  iter_advance<TG>(it, p, warp);
+  iter_load_seg<TG>(it, p, segs, act_index, lane);
+  it.ku = warp;
+  if (it.ku >= p.KU) {
+    it.ku = p.KU - kNW;  // so that the advance moves to the next sub-panel
+    iter_advance<TG>(it, p, segs, act_index, warp, lane);
+  }
 }
 
-// Stage byte count of an item: codes/scales of tiles [0, b) plus the activations.
 template <int FMT, int TG>
 __device__ __forceinline__ uint32_t stage_bytes(const ItemIter& it) {
   using G = StageGeom<FMT, TG>;
-  int a, b;
-  active_tiles(it.sp, it.ku, a, b);
-  return (uint32_t)(b * FmtTraits<FMT>::kCodeBytes + G::kBlocksPerKU * b * 32 + G::kBlocksPerKU * it.sg.tg * 1024);
+  return (uint32_t)(it.sp.nt * (FmtTraits<FMT>::kCodeBytes + G::kBlocksPerKU * 32) +
+                    it.sg.m * FmtTraits<FMT>::kKUcols * 2);
 }
 
-// Weight part of a stage: codes and scales of tiles [0, b) of the sub-panel at k-unit ku.
+// Weight part of a stage (lane 0): expect the whole stage, copy codes and scales.
 template <int FMT, int TG>
 __device__ __forceinline__ void issue_weights(const SmallParams& p, const ItemIter& it, uint8_t* stage, uint64_t* bar) {
   using G = StageGeom<FMT, TG>;
   using Tr = FmtTraits<FMT>;
-  int a, b;
-  active_tiles(it.sp, it.ku, a, b);
-  const int tile = it.sp.rt0;
+  mbar_arrive_expect_tx(bar, stage_bytes<FMT, TG>(it));
+  const int tile = it.sp.rt0, n = it.sp.nt;
   const uint8_t* csrc = p.codes + (unsigned long long)it.sg.expert * p.codes_stride +
                         ((unsigned long long)it.ku * p.NT + tile) * Tr::kCodeBytes;
-  bulk_copy_g2s(stage, csrc, (uint32_t)(b * Tr::kCodeBytes), bar);
+  bulk_copy_g2s(stage, csrc, (uint32_t)(n * Tr::kCodeBytes), bar);
 #pragma unroll
   for (int bl = 0; bl < G::kBlocksPerKU; ++bl) {
     const int sb = (it.ku * Tr::kKUcols + bl * 64) / p.block;
     const uint8_t* ssrc = p.scales + (unsigned long long)it.sg.expert * p.scales_stride +
                           ((unsigned long long)sb * p.NT + tile) * 32;
-    bulk_copy_g2s(stage + G::kCodeBytes + bl * kMaxT * 32, ssrc, (uint32_t)(b * 32), bar);
+    bulk_copy_g2s(stage + G::kCodeBytes + bl * kMaxT * 32, ssrc, (uint32_t)(n * 32), bar);
   }
 }
 
-// Activation part of a stage.
+// Activation part of a stage: lane n < m copies its token's k-unit slice.
 template <int FMT, int TG>
-__device__ __forceinline__ void issue_acts(const SmallParams& p, const ItemIter& it, uint8_t* stage, uint64_t* bar) {
+__device__ __forceinline__ void issue_acts(const SmallParams& p, const ItemIter& it, uint8_t* stage, uint64_t* bar,
+                                           int lane) {
   using G = StageGeom<FMT, TG>;
-  const uint8_t* xsrc = p.xfrag + (unsigned long long)it.sg.xoff * p.K * 16 +
-                        (unsigned long long)it.ku * G::kBlocksPerKU * it.sg.tg * 1024;
-  bulk_copy_g2s(stage + G::kCodeBytes + G::kScaleBytes, xsrc, (uint32_t)(G::kBlocksPerKU * it.sg.tg * 1024), bar);
+  constexpr int kBytes = FmtTraits<FMT>::kKUcols * 2;
+  if (lane < it.sg.m) {
+    const uint8_t* src = reinterpret_cast<const uint8_t*>(p.act) + ((unsigned long long)it.row * p.K) * 2 +
+                         (unsigned long long)it.ku * kBytes;
+    bulk_copy_g2s(stage + G::kCodeBytes + G::kScaleBytes + lane * G::kActPitch, src, kBytes, bar);
+  }
 }
 
 __device__ __forceinline__ float silu_f(float g) { return g / (1.0f + __expf(-g)); }
@@ -239,10 +279,112 @@ __device__ __forceinline__ float silu_f(float g) { return g / (1.0f + __expf(-g)
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
+__device__ __forceinline__ void ldmatrix_x4(uint32_t (&r)[4], const void* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(smem_addr(p)));
+}
+
+// ---------------------------------------------------------------------------
+// Routing of a decode batch (T <= 8) in shared memory, identical in every CTA:
+// top-k with ties to the lower index, softmax over the selected logits, slot
+// order = stable sort of t*k+s by expert, shared experts after the routed
+// slots; one segment per active expert, experts in increasing order.
+__device__ void decode_route(const SmallParams& p, DecodeRoute& R) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int T = p.T, E = p.E, k = p.k, TK = T * k;
+  for (int e = tid; e < kMaxExperts; e += blockDim.x) R.counts[e] = 0;
+  if (warp < T) {
+    float v[kMaxExperts / 32];
+    unsigned taken = 0;
+#pragma unroll
+    for (int j = 0; j < kMaxExperts / 32; ++j) {
+      const int idx = lane + 32 * j;
+      v[j] = idx < E ? p.logits[(size_t)warp * E + idx] : -FLT_MAX;
+    }
+    for (int s = 0; s < k; ++s) {
+      float bv = -FLT_MAX;
+      int bi = INT_MAX;
+#pragma unroll
+      for (int j = 0; j < kMaxExperts / 32; ++j) {
+        const int idx = lane + 32 * j;
+        if (idx < E && !((taken >> j) & 1u) && (bi == INT_MAX || v[j] > bv)) { bv = v[j]; bi = idx; }
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+        const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+        if (oi != INT_MAX && (bi == INT_MAX || ov > bv || (ov == bv && oi < bi))) { bv = ov; bi = oi; }
+      }
+      if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+      if (lane == 0) {
+        R.ids[warp * k + s] = bi;
+        R.selv[warp][s] = bv;
+      }
+    }
+    __syncwarp();
+    if (lane < k) {
+      const float lmax = R.selv[warp][0];
+      float sum = 0.f;
+      for (int s = 0; s < k; ++s) sum += expf(R.selv[warp][s] - lmax);
+      R.w[warp * k + lane] = expf(R.selv[warp][lane] - lmax) / sum;
+    }
+  }
+  __syncthreads();
+  for (int i = tid; i < TK; i += blockDim.x) atomicAdd(&R.counts[R.ids[i]], 1);
+  __syncthreads();
+  if (warp == 0) {
+    // exclusive scan of counts -> offsets; compaction of active experts -> segments
+    int base = 0, sbase = 0;
+    const unsigned lt = (1u << lane) - 1u;
+    for (int c = 0; c < E; c += 32) {
+      const int e = c + lane;
+      const int cnt = e < E ? R.counts[e] : 0;
+      int incl = cnt;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int o = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += o;
+      }
+      if (e < E) R.offs[e] = base + incl - cnt;
+      const unsigned act = __ballot_sync(0xffffffffu, cnt > 0);
+      if (cnt > 0) {
+        Seg sg;
+        sg.expert = e;
+        sg.m = cnt;
+        sg.tg = (cnt + 7) / 8;
+        sg.slot0 = base + incl - cnt;
+        R.segs[sbase + __popc(act & lt)] = sg;
+      }
+      base += __shfl_sync(0xffffffffu, incl, 31);
+      sbase += __popc(act);
+    }
+    if (lane < p.n_shared) {
+      Seg sg;
+      sg.expert = E + lane;
+      sg.m = T;
+      sg.tg = (T + 7) / 8;
+      sg.slot0 = TK + lane * T;
+      R.segs[sbase + lane] = sg;
+    }
+    if (lane == 0) R.nseg = sbase + p.n_shared;
+  }
+  __syncthreads();
+  for (int i = tid; i < TK; i += blockDim.x) {
+    const int e = R.ids[i];
+    int rank = 0;
+    for (int j = 0; j < i; ++j) rank += R.ids[j] == e;
+    const int pos = R.offs[e] + rank;
+    R.pos[i] = pos;
+    R.slot_token[pos] = i / k;
+  }
+  for (int i = tid; i < p.n_shared * T; i += blockDim.x) R.slot_token[TK + i] = i % T;
+  __syncthreads();
+}
+
 // Epilogue of one reduced fragment: rows g / g+8 of tile rt, tokens n0, n0+1.
 template <int EPI>
-__device__ __forceinline__ void epilogue(const SmallParams& p, const Seg& sg, int rt, int tg, int lane,
-                                         float4 v) {
+__device__ __forceinline__ void epilogue(const SmallParams& p, const Seg& sg, int rt, int tg, int lane, float4 v) {
   const int g = lane >> 2, q = lane & 3;
   const int n0 = tg * 8 + 2 * q;
   if (EPI == EPI_LINEAR) {
@@ -283,37 +425,34 @@ __device__ __forceinline__ void epilogue(const SmallParams& p, const Seg& sg, in
       bg = bf16_to_f(bp[2 * j]);
       bu = bf16_to_f(bp[2 * j + 1]);
     }
-    const float h0 = n0 < sg.m ? silu_f(v.x + bg) * (v.z + bu) : 0.f;
-    const float h1 = n0 + 1 < sg.m ? silu_f(v.y + bg) * (v.w + bu) : 0.f;
-    // FC2 operand fragment position of (token, k = j).
-    const int kb = j >> 6, kk = j & 63, ks = kk >> 4, kc = kk & 15;
-    const float inv = (kc >= 8 && p.h_beta_hi == 4) ? 0.25f : 1.0f;
-    const int reg = ks * 2 + (kc >> 3), half = kc & 1;
-    uint16_t* base = reinterpret_cast<uint16_t*>(p.hfrag + (size_t)sg.xoff * p.I * 16);
-#pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      const int n = n0 + e;
-      const int ln = ((n & 7) << 2) | ((kc & 7) >> 1);
-      const size_t off = ((((size_t)kb * sg.tg + (n >> 3)) * 32 + ln) * 8 + reg) * 2 + half;
-      base[off] = __bfloat16_as_ushort(__float2bfloat16_rn((e ? h1 : h0) * inv));
-    }
+    if (n0 < sg.m)
+      p.hrows[(size_t)(sg.slot0 + n0) * p.I + j] =
+          __bfloat16_as_ushort(__float2bfloat16_rn(silu_f(v.x + bg) * (v.z + bu)));
+    if (n0 + 1 < sg.m)
+      p.hrows[(size_t)(sg.slot0 + n0 + 1) * p.I + j] =
+          __bfloat16_as_ushort(__float2bfloat16_rn(silu_f(v.y + bg) * (v.w + bu)));
   }
 }
 
 // ---------------------------------------------------------------------------
-// One item: tiles [0, NTL) of a stage (NTL = a power of two >= b).  Tiles
-// outside [mask_lo, b) contribute with scale 0 (their codes are stale but
-// finite), so all NTL tiles run the same straight-line code and the MMAs of a
-// k-step for every tile issue back to back.
+// One item: tiles [0, NTL) of a stage (NTL = a power of two >= nt).  Tiles
+// at or past nt contribute with scale 0 (their codes are stale but finite),
+// so all NTL tiles run the same straight-line code and the MMAs of a k-step
+// for every tile issue back to back.
 template <int FMT, int TG, int NTL>
-__device__ __forceinline__ void compute_item(const uint8_t* cbuf, const uint32_t* sbuf, const uint8_t* xbuf,
-                                             int sg_tg, bool tg2, int lane, int mask_lo, int b,
-                                             const uint32_t* lut, float (&acc)[kMaxT][TG][4]) {
+__device__ __forceinline__ void compute_item(const uint8_t* st, bool tg2, int lane, int nt, const uint32_t* lut,
+                                             float (&acc)[kMaxT][TG][4]) {
   using Tr = FmtTraits<FMT>;
+  using G = StageGeom<FMT, TG>;
   constexpr int BPK = Tr::kKUcols / 64;
+  const uint8_t* cbuf = st;
+  const uint32_t* sbuf = reinterpret_cast<const uint32_t*>(st + G::kCodeBytes);
+  const uint8_t* abuf = st + G::kCodeBytes + G::kScaleBytes;
   const uint32_t aconst[4] = {Tr::kConstLo, Tr::kConstLo, Tr::kConstHi, Tr::kConstHi};
   const int g = lane >> 2;
-  // activation fragments of each 64-column block and the constant-operand products
+  // B fragments from the token rows (ldmatrix: lanes 8j..8j+7 address the
+  // rows of matrix j = columns 8j..8j+7 of a 32-column half), columns
+  // k%16 >= 8 divided by the code multiplier, and the constant-operand products.
   uint32_t bfr[BPK][TG][4][2];
   float corr[BPK][TG][4];
 #pragma unroll
@@ -323,10 +462,19 @@ __device__ __forceinline__ void compute_item(const uint8_t* cbuf, const uint32_t
 #pragma unroll
       for (int e = 0; e < 4; ++e) corr[bl][t][e] = 0.f;
       if (t == 0 || tg2) {
-        const uint4* xp = reinterpret_cast<const uint4*>(xbuf + ((size_t)(bl * sg_tg + t) * 32 + lane) * 32);
-        const uint4 u0 = xp[0], u1 = xp[1];
-        bfr[bl][t][0][0] = u0.x; bfr[bl][t][0][1] = u0.y; bfr[bl][t][1][0] = u0.z; bfr[bl][t][1][1] = u0.w;
-        bfr[bl][t][2][0] = u1.x; bfr[bl][t][2][1] = u1.y; bfr[bl][t][3][0] = u1.z; bfr[bl][t][3][1] = u1.w;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t r[4];
+          ldmatrix_x4(r, abuf + (t * 8 + (lane & 7)) * G::kActPitch + (bl * 64 + h * 32 + (lane >> 3) * 8) * 2);
+          bfr[bl][t][2 * h][0] = r[0];
+          bfr[bl][t][2 * h][1] = r[1];
+          bfr[bl][t][2 * h + 1][0] = r[2];
+          bfr[bl][t][2 * h + 1][1] = r[3];
+        }
+        if (Tr::kBetaHi == 4) {
+#pragma unroll
+          for (int k2 = 0; k2 < 4; ++k2) bfr[bl][t][k2][1] = fma_bf16x2(bfr[bl][t][k2][1], kBf16Quarter, 0x80008000u);
+        }
 #pragma unroll
         for (int k2 = 0; k2 < 4; ++k2) mma_bf16_16816(corr[bl][t], aconst, bfr[bl][t][k2][0], bfr[bl][t][k2][1]);
       } else {
@@ -334,14 +482,14 @@ __device__ __forceinline__ void compute_item(const uint8_t* cbuf, const uint32_t
         for (int k2 = 0; k2 < 4; ++k2) bfr[bl][t][k2][0] = bfr[bl][t][k2][1] = 0u;
       }
     }
-  // per-tile scales (0 outside [mask_lo, b))
+  // per-tile scales (0 at or past nt)
   float s_lo[BPK][NTL], s_hi[BPK][NTL];
 #pragma unroll
   for (int bl = 0; bl < BPK; ++bl)
 #pragma unroll
     for (int i = 0; i < NTL; ++i) {
       const uint32_t sc = sbuf[bl * kMaxT * 8 + i * 8 + g];
-      const bool on = i >= mask_lo && i < b;
+      const bool on = i < nt;
       s_lo[bl][i] = on ? bf16_lo(sc) : 0.f;
       s_hi[bl][i] = on ? bf16_hi(sc) : 0.f;
     }
@@ -422,31 +570,66 @@ __device__ __forceinline__ void compute_item(const uint8_t* cbuf, const uint32_t
   }
 }
 
-template <int FMT, int TG, int EPI>
+// Decode FC2: router-weighted combine of output rows [16 rt, 16 rt + 16) over
+// all tokens, once every segment has written them.
+__device__ __forceinline__ void combine_tile(const SmallParams& p, const DecodeRoute& R, int rt) {
+  const int TK = p.T * p.k;
+  for (int e = threadIdx.x; e < p.T * 16; e += blockDim.x) {
+    const int t = e >> 4, r = rt * 16 + (e & 15);
+    float acc = 0.f;
+    for (int s = 0; s < p.k; ++s) acc = fmaf(R.w[t * p.k + s], __ldcg(p.yslot + (size_t)R.pos[t * p.k + s] * p.H + r), acc);
+    for (int j = 0; j < p.n_shared; ++j) acc += __ldcg(p.yslot + (size_t)(TK + j * p.T + t) * p.H + r);
+    p.y[(size_t)t * p.H + r] = __bfloat16_as_ushort(__float2bfloat16_rn(acc));
+  }
+}
+
+template <int FMT, int TG, int EPI, int SRC>
 __global__ void __launch_bounds__(kNW * 32, 1) qmm_small_kernel(const SmallParams p) {
   using G = StageGeom<FMT, TG>;
   extern __shared__ __align__(128) uint8_t smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int NST = p.nstages;
 
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem);                   // [kNW][NST]
-  uint32_t* lut = reinterpret_cast<uint32_t*>(smem + 1024);            // 243 entries (ternary)
-  float4* red = reinterpret_cast<float4*>(smem + 2048);                 // [kNW][kMaxT][TG][32]
-  uint8_t* stages = smem + 2048 + G::kRedBytes;                         // [kNW][NST][stage]
-  __shared__ int s_flag[2];
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem);                          // [kNW][NST]
+  uint32_t* lut = reinterpret_cast<uint32_t*>(smem + 1024);                   // 243 entries (ternary)
+  DecodeRoute& R = *reinterpret_cast<DecodeRoute*>(smem + 2048);               // SRC_DECODE only
+  float4* red = reinterpret_cast<float4*>(smem + SmemHead<SRC>::kFixed);      // [kNW][kMaxT][TG][32]
+  uint8_t* stages = smem + SmemHead<SRC>::kFixed + G::kRedBytes;               // [kNW][NST][stage]
   __shared__ int s_abort;
+  __shared__ int s_comb[kMaxT];
 
-  // The segment table comes from a launch at least two back in the stream.
-  const int nseg = *p.nseg;
+  // ---- segments ----
+  // With p.early the segment source was written at least two launches back
+  // (or is arithmetic), so segments and weights may be read before
+  // griddepcontrol.wait; otherwise wait first.
+  if (!p.early) pdl_wait();
+  int nseg;
+  SegSource segs;
+  segs.table = nullptr;
+  segs.rows = p.T;
+  const int* act_index = p.act_index;
+  if constexpr (SRC == SRC_DECODE) {
+    decode_route(p, R);
+    nseg = R.nseg;
+    segs.table = R.segs;
+    if (EPI == EPI_SWIGLU) act_index = R.slot_token;
+  } else if constexpr (SRC == SRC_LINEAR) {
+    nseg = (p.T + kChunkTokens - 1) / kChunkTokens;
+  } else {
+    nseg = *p.nseg;
+    segs.table = p.segs;
+  }
+
   const unsigned ntiles = (unsigned)nseg * (unsigned)p.NT;
-  const bool tile_mode = ntiles >= gridDim.x;
   Part part;
-  if (tile_mode) part.init(ntiles, gridDim.x, (unsigned)p.KU);
-  else part.init(ntiles * (unsigned)p.KU, gridDim.x, 1u);
+  part.init(ntiles, gridDim.x, (unsigned)p.KU);
   const unsigned f0 = part.begin(blockIdx.x), f1 = part.begin(blockIdx.x + 1);
+
   if (f0 >= f1) {  // whole CTA idle
     pdl_wait();
     pdl_trigger();
+    if (SRC == SRC_DECODE && EPI == EPI_SWIGLU && blockIdx.x == 0)
+      for (int i = tid; i < p.H / 16; i += blockDim.x) p.ctick[i] = 0;
     return;
   }
 
@@ -460,46 +643,44 @@ __global__ void __launch_bounds__(kNW * 32, 1) qmm_small_kernel(const SmallParam
   fence_mbar_init();
   __syncthreads();
 
-  // Producer (lane 0): the weights of the first NST items before the
-  // dependency wait, their activations after it.
+  // Producer: the weights of the first NST items before the dependency wait,
+  // their activation rows after it.
   ItemIter prod;
   int primed = 0;
-  if (lane == 0) {
-    iter_begin<TG>(prod, p, f0, f1, warp);
-    for (int s = 0; s < NST && prod.valid; ++s, ++primed) {
-      mbar_arrive_expect_tx(&wbar[s], stage_bytes<FMT, TG>(prod));
-      issue_weights<FMT, TG>(p, prod, wstage + s * G::kStageBytes, &wbar[s]);
-      iter_advance<TG>(prod, p, warp);
+  iter_begin<TG>(prod, p, segs, act_index, f0, f1, warp, lane);
+  {
+    ItemIter it = prod;
+    for (int s = 0; s < NST && it.valid; ++s, ++primed) {
+      if (lane == 0) issue_weights<FMT, TG>(p, it, wstage + s * G::kStageBytes, &wbar[s]);
+      iter_advance<TG>(it, p, segs, act_index, warp, lane);
     }
   }
   pdl_wait();
   pdl_trigger();
-  if (lane == 0) {
-    ItemIter again;
-    iter_begin<TG>(again, p, f0, f1, warp);
-    for (int s = 0; s < primed; ++s) {
-      issue_acts<FMT, TG>(p, again, wstage + s * G::kStageBytes, &wbar[s]);
-      iter_advance<TG>(again, p, warp);
-    }
-  }
+  if (SRC == SRC_DECODE && EPI == EPI_SWIGLU && blockIdx.x == 0)
+    for (int i = tid; i < p.H / 16; i += blockDim.x) p.ctick[i] = 0;  // for the FC2 launch that follows
   __syncwarp();
+  for (int s = 0; s < primed; ++s) {
+    issue_acts<FMT, TG>(p, prod, wstage + s * G::kStageBytes, &wbar[s], lane);
+    iter_advance<TG>(prod, p, segs, act_index, warp, lane);
+  }
 
   int item = 0;           // this warp's consumed items
   bool aborted = false;   // this warp gave up waiting
 
   SubPanel sp;
   unsigned pos = f0;
-  const int head_tile_glob = (int)(f0 / (unsigned)p.KU);
   int cur_seg = -1;
   Seg sg;
   while (pos < f1) {
     load_subpanel(sp, pos, f1, p.NT, p.KU);
     if (sp.seg != cur_seg) {
       cur_seg = sp.seg;
-      sg = p.segs[sp.seg];
-      if (sg.tg > TG || sg.tg < 1) {
+      sg = segs.get(sp.seg);
+      if (sg.tg > TG || sg.tg < 1 || sg.m > 8 * sg.tg) {
         if (tid == 0) atomicOr(p.status, kStatusBadSegment);
         sg.tg = TG;
+        sg.m = min(sg.m, 8 * TG);
       }
     }
     const bool tg2 = TG == 2 && sg.tg == 2;
@@ -512,9 +693,6 @@ __global__ void __launch_bounds__(kNW * 32, 1) qmm_small_kernel(const SmallParam
         for (int e = 0; e < 4; ++e) acc[i][t][e] = 0.f;
 
     for (int ku = warp; ku < p.KU; ku += kNW) {
-      int a, b;
-      active_tiles(sp, ku, a, b);
-      if (a >= b) continue;
       const int s = item % NST;
       const uint32_t par = (uint32_t)(item / NST) & 1u;
       ++item;
@@ -524,26 +702,25 @@ __global__ void __launch_bounds__(kNW * 32, 1) qmm_small_kernel(const SmallParam
       }
       uint8_t* st = wstage + s * G::kStageBytes;
       if (!aborted) {
-        const uint8_t* cbuf = st;
-        const uint32_t* sbuf = reinterpret_cast<const uint32_t*>(st + G::kCodeBytes);
-        const uint8_t* xbuf = st + G::kCodeBytes + G::kScaleBytes;
-        if (b > 4) compute_item<FMT, TG, 8>(cbuf, sbuf, xbuf, sg.tg, tg2, lane, a, b, lut, acc);
-        else if (b > 2) compute_item<FMT, TG, 4>(cbuf, sbuf, xbuf, sg.tg, tg2, lane, a, b, lut, acc);
-        else if (b > 1) compute_item<FMT, TG, 2>(cbuf, sbuf, xbuf, sg.tg, tg2, lane, a, b, lut, acc);
-        else compute_item<FMT, TG, 1>(cbuf, sbuf, xbuf, sg.tg, tg2, lane, a, b, lut, acc);
+        if (sp.nt > 4) compute_item<FMT, TG, 8>(st, tg2, lane, sp.nt, lut, acc);
+        else if (sp.nt > 2) compute_item<FMT, TG, 4>(st, tg2, lane, sp.nt, lut, acc);
+        else if (sp.nt > 1) compute_item<FMT, TG, 2>(st, tg2, lane, sp.nt, lut, acc);
+        else compute_item<FMT, TG, 1>(st, tg2, lane, sp.nt, lut, acc);
       }
       __syncwarp();
-      if (lane == 0 && prod.valid && !aborted) {
-        fence_proxy_async_smem();
-        mbar_arrive_expect_tx(&wbar[s], stage_bytes<FMT, TG>(prod));
-        issue_weights<FMT, TG>(p, prod, st, &wbar[s]);
-        issue_acts<FMT, TG>(p, prod, st, &wbar[s]);
-        iter_advance<TG>(prod, p, warp);
+      if (prod.valid && !aborted) {
+        if (lane == 0) {
+          fence_proxy_async_smem();
+          issue_weights<FMT, TG>(p, prod, st, &wbar[s]);
+        }
+        __syncwarp();
+        issue_acts<FMT, TG>(p, prod, st, &wbar[s], lane);
+        iter_advance<TG>(prod, p, segs, act_index, warp, lane);
       }
       __syncwarp();
     }
 
-    // ---- CTA reduction of the sub-panel -------------------------------------
+    // ---- CTA reduction of the sub-panel, epilogue ----------------------------
 #pragma unroll
     for (int i = 0; i < kMaxT; ++i) {
       if (i >= sp.nt) continue;
@@ -555,13 +732,10 @@ __global__ void __launch_bounds__(kNW * 32, 1) qmm_small_kernel(const SmallParam
     __syncthreads();
     const bool ab = s_abort != 0;
     const int nel = sp.nt * TG * 32;
-    const int last_tile = sp.nt - 1;
-    const bool head_partial = sp.kf > 0 || (sp.nt == 1 && sp.kl < p.KU);
-    const bool tail_partial = sp.kl < p.KU && sp.nt > 1;
 #pragma unroll
     for (int r = 0; r < (kMaxT * TG * 32 + kNW * 32 - 1) / (kNW * 32); ++r) {
       const int e = tid + r * kNW * 32;
-      if (e >= nel) continue;
+      if (e >= nel || ab) continue;
       float4 v = red[e];
       for (int w = 1; w < kNW; ++w) {
         const float4 u = red[w * kMaxT * TG * 32 + e];
@@ -569,62 +743,23 @@ __global__ void __launch_bounds__(kNW * 32, 1) qmm_small_kernel(const SmallParam
       }
       const int i = e / (TG * 32), t = (e / 32) % TG, ln = e % 32;
       if (t == 1 && !tg2) continue;
-      const bool partial = (i == 0 && head_partial) || (i == last_tile && tail_partial);
-      if (ab) continue;
-      if (!partial) {
-        epilogue<EPI>(p, sg, sp.rt0 + i, t, ln, v);
-      } else {
-        const int tglob = sp.seg * p.NT + sp.rt0 + i;
-        const int slot = 2 * blockIdx.x + (tglob == head_tile_glob ? 0 : 1);
-        reinterpret_cast<float4*>(p.partials)[((size_t)slot * 2 + t) * 32 + ln] = v;
-      }
+      epilogue<EPI>(p, sg, sp.rt0 + i, t, ln, v);
     }
-    if (head_partial || tail_partial) {  // only in unit mode
+    if constexpr (SRC == SRC_DECODE && EPI == EPI_FC2) {
+      // fused combine: the last segment to finish an output tile combines it
       __threadfence();
       __syncthreads();
-      if (tid < 2) {
-        s_flag[tid] = 0;
-        const bool want = tid == 0 ? head_partial : tail_partial;
-        if (want && !ab) {
-          const int i = tid == 0 ? 0 : last_tile;
-          const int tglob = sp.seg * p.NT + sp.rt0 + i;
-          const unsigned T0 = (unsigned)tglob * (unsigned)p.KU;
-          const unsigned clo = part.owner(T0), chi = part.owner(T0 + p.KU - 1);
-          int ncontrib = 0;
-          for (unsigned c = clo; c <= chi; ++c)
-            if (part.begin(c + 1) > part.begin(c)) ++ncontrib;
-          const int old = atomicAdd(&p.tickets[tglob], 1);
-          if (old == ncontrib - 1) {
-            s_flag[tid] = 1;
-            p.tickets[tglob] = 0;  // leave the ticket clean for the next launch
-          }
-        }
+      if (tid < sp.nt) {
+        const int old = ab ? -1 : atomicAdd(&p.ctick[sp.rt0 + tid], 1);
+        s_comb[tid] = old == nseg - 1;
+        if (old == nseg - 1) p.ctick[sp.rt0 + tid] = 0;
       }
       __syncthreads();
-      if (s_flag[0] || s_flag[1]) {
-        __threadfence();
-#pragma unroll
-        for (int r = 0; r < (kMaxT * TG * 32 + kNW * 32 - 1) / (kNW * 32); ++r) {
-          const int e = tid + r * kNW * 32;
-          if (e >= nel) continue;
-          const int i = e / (TG * 32), t = (e / 32) % TG, ln = e % 32;
-          if (t == 1 && !tg2) continue;
-          const int which = (i == 0 && head_partial) ? 0 : ((i == last_tile && tail_partial) ? 1 : -1);
-          if (which < 0 || !s_flag[which]) continue;
-          const int tglob = sp.seg * p.NT + sp.rt0 + i;
-          const unsigned T0 = (unsigned)tglob * (unsigned)p.KU;
-          const unsigned clo = part.owner(T0), chi = part.owner(T0 + p.KU - 1);
-          float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-          for (unsigned c = clo; c <= chi; ++c) {
-            const unsigned b0 = part.begin(c), b1 = part.begin(c + 1);
-            if (b1 <= b0) continue;
-            const int slot = 2 * (int)c + ((int)(b0 / (unsigned)p.KU) == tglob ? 0 : 1);
-            const float4 u = __ldcg(reinterpret_cast<const float4*>(p.partials) + ((size_t)slot * 2 + t) * 32 + ln);
-            v.x += u.x; v.y += u.y; v.z += u.z; v.w += u.w;
-          }
-          epilogue<EPI>(p, sg, sp.rt0 + i, t, ln, v);
+      for (int i = 0; i < sp.nt; ++i)
+        if (s_comb[i]) {
+          __threadfence();
+          combine_tile(p, R, sp.rt0 + i);
         }
-      }
     }
     __syncthreads();
     pos = sp.next;

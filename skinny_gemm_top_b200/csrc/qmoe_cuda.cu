@@ -134,10 +134,9 @@ qmoe_status check_weights(const qmoe_weights& w, int rows, int K) {
 
 // Workspace plan of one row tile of T tokens.
 struct MoEPlan {
-  int T, S, TK, max_seg, max_tg, n_tickets, max_gseg;
-  bool grouped;
-  size_t ids, w, perm, inv, offsets, slot_token, nseg, segs, tickets, partials, xfrag, hfrag, yslot, ngseg, gsegs,
-      xrows, hrows, total;
+  int T, S, TK, max_seg, n_tickets, max_gseg;
+  bool grouped, decode;
+  size_t ids, w, perm, inv, offsets, slot_token, nseg, segs, yslot, hrows, ctick, ngseg, gsegs, xrows, total;
 };
 
 constexpr int kGroupedThreshold = 32;  // AUTO: experts with more tokens take the tcgen05 path
@@ -152,37 +151,40 @@ int grouped_threshold(const qmoe_layer& L) {
   return L.path == QMOE_PATH_GROUPED ? 0 : kGroupedThreshold;
 }
 
+// Decode batches route inside the expert kernels (two launches per layer).
+bool decode_eligible(const qmoe_layer& L, int T) {
+  return T <= kDecMaxT && T * L.k <= kDecMaxTK && L.n_shared <= kDecMaxShared && T <= grouped_threshold(L);
+}
+
 MoEPlan plan_moe(const qmoe_layer& L, int T, int grid) {
+  (void)grid;
   MoEPlan p{};
-  p.grouped = T > grouped_threshold(L);
   p.T = T;
   p.TK = T * L.k;
   p.S = T * (L.k + L.n_shared);
+  p.decode = decode_eligible(L, T);
+  p.grouped = !p.decode && T > grouped_threshold(L);
   p.max_seg = std::min(L.E, p.TK) + p.TK / kChunkTokens + L.n_shared * ((T + kChunkTokens - 1) / kChunkTokens);
-  p.max_tg = (p.S + 7) / 8 + p.max_seg;
-  const int nt = std::max(2 * L.I / 16, L.H / 16);
-  p.n_tickets = p.max_seg * nt;
   size_t o = 0;
   auto take = [&](size_t bytes) { size_t at = o; o = align_up(o + bytes); return at; };
-  p.ids = take((size_t)p.TK * 4);
-  p.w = take((size_t)p.TK * 4);
-  p.perm = take((size_t)p.TK * 4);
-  p.inv = take((size_t)p.TK * 4);
-  p.offsets = take((size_t)(L.E + 1) * 4);
-  p.slot_token = take((size_t)p.S * 4);
-  p.nseg = take(16);
-  p.segs = take((size_t)p.max_seg * sizeof(Seg));
-  p.tickets = take((size_t)p.n_tickets * 4);
-  p.partials = take((size_t)2 * grid * 2 * 32 * 16);
-  p.xfrag = take((size_t)p.max_tg * L.H * 16);
-  p.hfrag = take((size_t)p.max_tg * L.I * 16);
   p.yslot = take((size_t)p.S * L.H * 4);
+  p.hrows = take((size_t)p.S * L.I * 2 + 16);
+  p.ctick = take((size_t)(L.H / 16) * 4);
+  if (!p.decode) {
+    p.ids = take((size_t)p.TK * 4);
+    p.w = take((size_t)p.TK * 4);
+    p.perm = take((size_t)p.TK * 4);
+    p.inv = take((size_t)p.TK * 4);
+    p.offsets = take((size_t)(L.E + 1) * 4);
+    p.slot_token = take((size_t)p.S * 4);
+    p.nseg = take(16);
+    p.segs = take((size_t)p.max_seg * sizeof(Seg));
+  }
   if (p.grouped) {
     p.max_gseg = std::min(L.E, p.TK) + p.TK / kGTok + L.n_shared * ((T + kGTok - 1) / kGTok);
     p.ngseg = take(16);
     p.gsegs = take((size_t)p.max_gseg * sizeof(GSeg));
     p.xrows = take((size_t)p.S * L.H * 2 + 16);
-    p.hrows = take((size_t)p.S * L.I * 2 + 16);
   }
   p.total = o;
   return p;
@@ -211,10 +213,10 @@ qmoe_status encode_rows_map(CUtensorMap* map, const void* base, int K, int rows)
 }
 
 // ---- small-M kernel launch ----
-template <int FMT, int TG, int EPI>
+template <int FMT, int TG, int EPI, int SRC>
 qmoe_status launch_small_t(SmallParams prm, int grid, cudaStream_t st) {
   using G = StageGeom<FMT, TG>;
-  const int fixed = 2048 + G::kRedBytes;
+  const int fixed = SmemHead<SRC>::kFixed + G::kRedBytes;
   int nst = (kSmemLimit - fixed - 1024) / (kNW * G::kStageBytes);
   nst = std::min(nst, 4);
   if (nst < 2) return QMOE_ERR_UNSUPPORTED;
@@ -224,22 +226,29 @@ qmoe_status launch_small_t(SmallParams prm, int grid, cudaStream_t st) {
   int d = 0;
   cudaGetDevice(&d);
   if (!attr_set[d]) {
-    if (cudaFuncSetAttribute(qmm_small_kernel<FMT, TG, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
-        cudaSuccess)
+    if (cudaFuncSetAttribute(qmm_small_kernel<FMT, TG, EPI, SRC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             smem) != cudaSuccess)
       return QMOE_ERR_CUDA;
     attr_set[d] = true;
   }
   TraceScope ts(st, EPI == EPI_SWIGLU ? K_FC1_SMALL : (EPI == EPI_FC2 ? K_FC2_SMALL : K_LINEAR_SMALL));
-  return launch_pdl(qmm_small_kernel<FMT, TG, EPI>, dim3(grid), dim3(kNW * 32), smem, st, prm) == cudaSuccess
+  return launch_pdl(qmm_small_kernel<FMT, TG, EPI, SRC>, dim3(grid), dim3(kNW * 32), smem, st, prm) == cudaSuccess
              ? QMOE_OK
              : QMOE_ERR_CUDA;
 }
 
-template <int EPI>
+template <int EPI, int SRC>
 qmoe_status launch_small(int fmt, int tg, const SmallParams& prm, int grid, cudaStream_t st) {
-  if (fmt == QMOE_INT2) return tg == 1 ? launch_small_t<2, 1, EPI>(prm, grid, st) : launch_small_t<2, 2, EPI>(prm, grid, st);
-  if (fmt == QMOE_INT4) return tg == 1 ? launch_small_t<4, 1, EPI>(prm, grid, st) : launch_small_t<4, 2, EPI>(prm, grid, st);
-  return tg == 1 ? launch_small_t<3, 1, EPI>(prm, grid, st) : launch_small_t<3, 2, EPI>(prm, grid, st);
+  if (SRC == SRC_DECODE) {  // decode batches have at most 8 tokens: one token group
+    if (fmt == QMOE_INT2) return launch_small_t<2, 1, EPI, SRC>(prm, grid, st);
+    if (fmt == QMOE_INT4) return launch_small_t<4, 1, EPI, SRC>(prm, grid, st);
+    return launch_small_t<3, 1, EPI, SRC>(prm, grid, st);
+  }
+  if (fmt == QMOE_INT2)
+    return tg == 1 ? launch_small_t<2, 1, EPI, SRC>(prm, grid, st) : launch_small_t<2, 2, EPI, SRC>(prm, grid, st);
+  if (fmt == QMOE_INT4)
+    return tg == 1 ? launch_small_t<4, 1, EPI, SRC>(prm, grid, st) : launch_small_t<4, 2, EPI, SRC>(prm, grid, st);
+  return tg == 1 ? launch_small_t<3, 1, EPI, SRC>(prm, grid, st) : launch_small_t<3, 2, EPI, SRC>(prm, grid, st);
 }
 
 template <int FMT, int EPI>
@@ -422,7 +431,7 @@ qmoe_status qmoe_forward(const qmoe_layer* layer, const uint16_t* x, const float
   qmoe_status s = check_layer(layer);
   if (s != QMOE_OK) return s;
   if (!x || !logits || !y || !ws || T <= 0) return QMOE_ERR_INVALID_ARG;
-  if ((reinterpret_cast<uintptr_t>(ws) % kAlign) || (reinterpret_cast<uintptr_t>(x) & 3) ||
+  if ((reinterpret_cast<uintptr_t>(ws) % kAlign) || (reinterpret_cast<uintptr_t>(x) & 15) ||
       (reinterpret_cast<uintptr_t>(y) & 7))
     return QMOE_ERR_INVALID_ARG;
   if (layer->path == QMOE_PATH_GROUPED && !grouped_eligible(*layer)) return QMOE_ERR_UNSUPPORTED;
@@ -440,10 +449,52 @@ qmoe_status qmoe_forward(const qmoe_layer* layer, const uint16_t* x, const float
   }
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   uint8_t* base = static_cast<uint8_t*>(ws);
-  int tiles = 0, small = 0, grouped = 0;
+  int tiles = 0, small = 0, grouped = 0, decode = 0;
   for (int t0 = 0; t0 < T; t0 += Tt) {
     const int tt = std::min(Tt, T - t0);
     const MoEPlan p = plan_moe(L, tt, grid);
+    const uint16_t* xt = x + (size_t)t0 * L.H;
+    const float* lt = logits + (size_t)t0 * L.E;
+    uint16_t* yt = y + (size_t)t0 * L.H;
+    float* yslot = reinterpret_cast<float*>(base + p.yslot);
+    uint16_t* hrows = reinterpret_cast<uint16_t*>(base + p.hrows);
+    SmallParams p1 = small_params(L.fc1, 2 * L.I, L.H, di->status);
+    p1.act = xt;
+    p1.bias = L.fc1.bias;
+    p1.bias_rows = 2 * L.I;
+    p1.hrows = hrows;
+    p1.I = L.I;
+    p1.H = L.H;
+    SmallParams p2 = small_params(L.fc2, L.H, L.I, di->status);
+    p2.act = hrows;
+    p2.act_index = nullptr;
+    p2.bias = L.fc2.bias;
+    p2.bias_rows = L.H;
+    p2.yslot = yslot;
+    p2.H = L.H;
+    p2.I = L.I;
+    if (p.decode) {
+      // Decode batch: both expert kernels route in their prologue; FC2 fuses the combine.
+      for (SmallParams* q : {&p1, &p2}) {
+        q->logits = lt;
+        q->T = tt;
+        q->E = L.E;
+        q->k = L.k;
+        q->n_shared = L.n_shared;
+        q->ctick = reinterpret_cast<int*>(base + p.ctick);
+      }
+      p1.early = 0;  // the logits may come from the previous launch
+      p2.early = 1;  // routing inputs were consumed by FC1 after its wait
+      p2.y = yt;
+      s = launch_small<EPI_SWIGLU, SRC_DECODE>(L.fc1.fmt, 1, p1, grid, st);
+      if (s != QMOE_OK) return s;
+      s = launch_small<EPI_FC2, SRC_DECODE>(L.fc2.fmt, 1, p2, grid, st);
+      if (s != QMOE_OK) return s;
+      ++tiles;
+      small += 2;
+      ++decode;
+      continue;
+    }
     RouteOut o{};
     o.ids = reinterpret_cast<int*>(base + p.ids);
     o.w = reinterpret_cast<float*>(base + p.w);
@@ -454,8 +505,6 @@ qmoe_status qmoe_forward(const qmoe_layer* layer, const uint16_t* x, const float
     o.nseg = reinterpret_cast<int*>(base + p.nseg);
     o.segs = reinterpret_cast<Seg*>(base + p.segs);
     o.max_seg = p.max_seg;
-    o.tickets = reinterpret_cast<int*>(base + p.tickets);
-    o.n_tickets = p.n_tickets;
     o.thresh = grouped_threshold(L);
     if (p.grouped) {
       o.ngseg = reinterpret_cast<int*>(base + p.ngseg);
@@ -465,45 +514,28 @@ qmoe_status qmoe_forward(const qmoe_layer* layer, const uint16_t* x, const float
     o.status = di->status;
     {
       TraceScope ts(st, K_ROUTE);
-      if (launch_pdl(route_kernel, dim3(1), dim3(kRouteThreads), 0, st, logits + (size_t)t0 * L.E, tt, L.E, L.k,
-                     L.n_shared, o) != cudaSuccess)
-        return QMOE_ERR_CUDA;
-    }
-    uint8_t* xfrag = base + p.xfrag;
-    uint8_t* hfrag = base + p.hfrag;
-    float* yslot = reinterpret_cast<float*>(base + p.yslot);
-    {
-      TraceScope ts(st, K_GATHER);
-      if (launch_pdl(gather_kernel, dim3(std::min(p.max_seg, 4 * grid)), dim3(256), 0, st,
-                     x + (size_t)t0 * L.H, L.H, (const int*)o.slot_token, (const int*)o.nseg, (const Seg*)o.segs,
-                     xfrag, beta_hi(L.fc1.fmt)) != cudaSuccess)
+      if (launch_pdl(route_kernel, dim3(1), dim3(kRouteThreads), 0, st, lt, tt, L.E, L.k, L.n_shared, o) !=
+          cudaSuccess)
         return QMOE_ERR_CUDA;
     }
     const int tg = tt <= 8 ? 1 : 2;
-    SmallParams p1 = small_params(L.fc1, 2 * L.I, L.H, di->status);
     p1.nseg = o.nseg;
     p1.segs = o.segs;
-    p1.xfrag = xfrag;
-    p1.bias = L.fc1.bias;
-    p1.bias_rows = 2 * L.I;
-    p1.hfrag = hfrag;
-    p1.I = L.I;
-    p1.h_beta_hi = beta_hi(L.fc2.fmt);
-    p1.partials = reinterpret_cast<float*>(base + p.partials);
-    p1.tickets = o.tickets;
-    s = launch_small<EPI_SWIGLU>(L.fc1.fmt, tg, p1, grid, st);
+    p1.act_index = o.slot_token;
+    p1.early = 0;  // the segment table comes from the routing launch just before
+    p2.nseg = o.nseg;
+    p2.segs = o.segs;
+    p2.early = 1;
+    s = launch_small<EPI_SWIGLU, SRC_TABLE>(L.fc1.fmt, tg, p1, grid, st);
     if (s != QMOE_OK) return s;
-    uint16_t* xrows = nullptr;
-    uint16_t* hrows = nullptr;
     CUtensorMap map2;
     GroupedParams g2{};
     if (p.grouped) {
-      xrows = reinterpret_cast<uint16_t*>(base + p.xrows);
-      hrows = reinterpret_cast<uint16_t*>(base + p.hrows);
+      uint16_t* xrows = reinterpret_cast<uint16_t*>(base + p.xrows);
       {
         TraceScope ts(st, K_GATHER);
-        gather_rows_kernel<<<std::min(p.max_gseg, 4 * grid), 256, 0, st>>>(x + (size_t)t0 * L.H, L.H, o.slot_token,
-                                                                            o.ngseg, o.gsegs, xrows);
+        gather_rows_kernel<<<std::min(p.max_gseg, 4 * grid), 256, 0, st>>>(xt, L.H, o.slot_token, o.ngseg, o.gsegs,
+                                                                            xrows);
         if (cudaGetLastError() != cudaSuccess) return QMOE_ERR_CUDA;
       }
       CUtensorMap map1;
@@ -518,8 +550,7 @@ qmoe_status qmoe_forward(const qmoe_layer* layer, const uint16_t* x, const float
       g1.bias_rows = 2 * L.I;
       g1.hrows = hrows;
       g1.I = L.I;
-      const int units1 = p.max_gseg * g1.rtiles;
-      s = launch_grouped<EPI_SWIGLU>(L.fc1.fmt, map1, g1, std::min(units1, grid), st);
+      s = launch_grouped<EPI_SWIGLU>(L.fc1.fmt, map1, g1, std::min(p.max_gseg * g1.rtiles, grid), st);
       if (s != QMOE_OK) return s;
       g2 = grouped_params(L.fc2, L.H, L.I, di->status);
       g2.ngseg = o.ngseg;
@@ -529,17 +560,7 @@ qmoe_status qmoe_forward(const qmoe_layer* layer, const uint16_t* x, const float
       g2.yslot = yslot;
       g2.H = L.H;
     }
-    SmallParams p2 = small_params(L.fc2, L.H, L.I, di->status);
-    p2.nseg = o.nseg;
-    p2.segs = o.segs;
-    p2.xfrag = hfrag;
-    p2.bias = L.fc2.bias;
-    p2.bias_rows = L.H;
-    p2.yslot = yslot;
-    p2.H = L.H;
-    p2.partials = p1.partials;
-    p2.tickets = o.tickets;
-    s = launch_small<EPI_FC2>(L.fc2.fmt, tg, p2, grid, st);
+    s = launch_small<EPI_FC2, SRC_TABLE>(L.fc2.fmt, tg, p2, grid, st);
     if (s != QMOE_OK) return s;
     if (p.grouped) {
       s = launch_grouped<EPI_FC2>(L.fc2.fmt, map2, g2, std::min(p.max_gseg * g2.rtiles, grid), st);
@@ -549,7 +570,7 @@ qmoe_status qmoe_forward(const qmoe_layer* layer, const uint16_t* x, const float
     {
       TraceScope ts(st, K_COMBINE);
       if (launch_pdl(combine_kernel, dim3(tt), dim3(256), 0, st, (const float*)yslot, (const float*)o.w,
-                     (const int*)o.inv, tt, L.k, L.n_shared, L.H, y + (size_t)t0 * L.H) != cudaSuccess)
+                     (const int*)o.inv, tt, L.k, L.n_shared, L.H, yt) != cudaSuccess)
         return QMOE_ERR_CUDA;
     }
     ++tiles;
@@ -566,63 +587,29 @@ qmoe_status qmoe_forward(const qmoe_layer* layer, const uint16_t* x, const float
 
 qmoe_status qmoe_linear_workspace_size(int N, int K, int M, size_t* bytes) {
   if (N <= 0 || K <= 0 || M <= 0 || N % 16 || K % 64 || !bytes) return QMOE_ERR_INVALID_ARG;
-  DevInfo* di;
-  qmoe_status s = dev_info(&di);
-  if (s != QMOE_OK) return s;
-  const int nseg = (M + kChunkTokens - 1) / kChunkTokens;
-  size_t o = 0;
-  o = align_up(o + 16);                                   // nseg
-  o = align_up(o + (size_t)nseg * sizeof(Seg));           // segs
-  o = align_up(o + (size_t)nseg * (N / 16) * 4);          // tickets
-  o = align_up(o + (size_t)2 * di->sms * 2 * 32 * 16);    // partials
-  o = align_up(o + (size_t)2 * nseg * K * 16);            // activation fragments
-  *bytes = o;
+  *bytes = kAlign;  // the single linear needs no scratch; a minimal workspace keeps the ABI stable
   return QMOE_OK;
 }
 
 qmoe_status qmoe_linear(const qmoe_weights* w, int N, int K, const uint16_t* x, int M, uint16_t* y, void* ws,
                         size_t ws_bytes, void* stream) {
-  if (!w || !x || !y || !ws || M <= 0) return QMOE_ERR_INVALID_ARG;
+  if (!w || !x || !y || M <= 0) return QMOE_ERR_INVALID_ARG;
   qmoe_status s = check_weights(*w, N, K);
   if (s != QMOE_OK) return s;
-  if ((reinterpret_cast<uintptr_t>(ws) % kAlign) || (reinterpret_cast<uintptr_t>(x) & 3)) return QMOE_ERR_INVALID_ARG;
-  size_t need = 0;
-  s = qmoe_linear_workspace_size(N, K, M, &need);
-  if (s != QMOE_OK) return s;
-  if (ws_bytes < need) return QMOE_ERR_SCRATCH;
+  (void)ws;
+  (void)ws_bytes;
+  if (reinterpret_cast<uintptr_t>(x) & 15) return QMOE_ERR_INVALID_ARG;
   DevInfo* di;
   s = dev_info(&di);
   if (s != QMOE_OK) return s;
-  const int nseg = (M + kChunkTokens - 1) / kChunkTokens;
-  uint8_t* base = static_cast<uint8_t*>(ws);
-  size_t o = 0;
-  int* d_nseg = reinterpret_cast<int*>(base + o); o = align_up(o + 16);
-  Seg* segs = reinterpret_cast<Seg*>(base + o); o = align_up(o + (size_t)nseg * sizeof(Seg));
-  int* tickets = reinterpret_cast<int*>(base + o); o = align_up(o + (size_t)nseg * (N / 16) * 4);
-  float* partials = reinterpret_cast<float*>(base + o); o = align_up(o + (size_t)2 * di->sms * 2 * 32 * 16);
-  uint8_t* xfrag = base + o;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  {
-    TraceScope ts(st, K_LINEAR_SETUP);
-    if (launch_pdl(linear_setup_kernel, dim3(1), dim3(256), 0, st, M, d_nseg, segs, tickets, nseg * (N / 16)) !=
-        cudaSuccess)
-      return QMOE_ERR_CUDA;
-  }
-  {
-    TraceScope ts(st, K_GATHER);
-    if (launch_pdl(gather_kernel, dim3(nseg), dim3(256), 0, st, x, K, (const int*)nullptr, (const int*)d_nseg,
-                   (const Seg*)segs, xfrag, beta_hi(w->fmt)) != cudaSuccess)
-      return QMOE_ERR_CUDA;
-  }
   SmallParams p = small_params(*w, N, K, di->status);
-  p.nseg = d_nseg;
-  p.segs = segs;
-  p.xfrag = xfrag;
+  p.act = x;
+  p.T = M;
   p.y = y;
   p.N = N;
-  p.partials = partials;
-  p.tickets = tickets;
-  s = launch_small<EPI_LINEAR>(w->fmt, M <= 8 ? 1 : 2, p, di->sms, st);
+  p.early = 1;  // static weights, arithmetic segments
+  s = launch_small<EPI_LINEAR, SRC_LINEAR>(w->fmt, M <= 8 ? 1 : 2, p, di->sms, st);
   if (s != QMOE_OK) return s;
   std::lock_guard<std::mutex> lk(g_mu);
   g_stats.last_path = QMOE_PATH_SMALL_M;
