@@ -88,10 +88,6 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
       : "memory");
 }
 
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
-}
-
 // K-major operand with 128-byte swizzle: 8-row atoms of 1024 bytes.
 __device__ __forceinline__ uint64_t umma_desc_sw128(const void* p) {
   const uint64_t a = smem_addr(p);

@@ -47,6 +47,7 @@ namespace qmoe {
 
 constexpr int kNW = 8;            // warps per CTA
 constexpr int kMaxT = 8;          // tiles per sub-panel
+constexpr int kMaxStages = 6;     // stages per consumer warp (barriers: 1024 bytes of shared memory)
 constexpr int kChunkTokens = 16;  // tokens per segment (<= 2 token groups of 8)
 
 enum Epi { EPI_LINEAR = 0, EPI_SWIGLU = 1, EPI_FC2 = 2 };
@@ -76,10 +77,11 @@ struct DecodeRoute {
   int slot_token[kDecMaxSlots];  // slot -> token
   int pos[kDecMaxTK];            // flat index t*k+s -> slot
   float w[kDecMaxTK];            // router weight of flat index
-  int ids[kDecMaxTK];
-  int counts[kMaxExperts];
-  int offs[kMaxExperts];
-  float selv[kDecMaxT][32];
+  int ids[kDecMaxTK];            // expert of flat index
+  int less[kDecMaxTK];           // entries routed to a lower expert
+  int cnt[kDecMaxTK];            // entries routed to the same expert
+  int first[kDecMaxTK];          // entry is its expert's first in flat order
+  float selv[kDecMaxT][32];      // selected logits in selection order
 };
 
 struct SmallParams {
@@ -184,8 +186,9 @@ struct SegSource {
   }
 };
 
-// Warp-uniform producer iterator over this warp's (sub-panel, k-unit) items.
-// Caches the segment and, per lane n < m, the row of token n.
+// Warp-uniform iterator over one warp's (sub-panel, k-unit) items: in every
+// sub-panel, warp w takes k-units w, w + kNW, ...  Caches the segment and,
+// per lane n < m, the row of token n.
 struct ItemIter {
   SubPanel sp;
   Seg sg;
@@ -235,42 +238,54 @@ __device__ __forceinline__ void iter_begin(ItemIter& it, const SmallParams& p, c
   }
 }
 
-template <int FMT, int TG>
-__device__ __forceinline__ uint32_t stage_bytes(const ItemIter& it) {
-  using G = StageGeom<FMT, TG>;
-  return (uint32_t)(it.sp.nt * (FmtTraits<FMT>::kCodeBytes + G::kBlocksPerKU * 32) +
-                    it.sg.m * FmtTraits<FMT>::kKUcols * 2);
-}
+// Stage fills (issued by the consuming warp itself).  The codes of an item are one contiguous run
+// (nt x 256..512 bytes): one TMA bulk copy by lane 0, completing as
+// transaction bytes on the stage's full barrier.  Scales and activation rows
+// are several pieces of 16..256 bytes: per-lane 16-byte cp.async, each lane
+// arriving on the barrier once its copies landed.  Full barrier count: 33
+// (lane 0's expect-tx arrival and 32 cp.async arrivals).
 
-// Weight part of a stage (lane 0): expect the whole stage, copy codes and scales.
+// Codes (TMA) and scales (cp.async) of the sub-panel's nt tiles at k-unit ku.
 template <int FMT, int TG>
-__device__ __forceinline__ void issue_weights(const SmallParams& p, const ItemIter& it, uint8_t* stage, uint64_t* bar) {
+__device__ __forceinline__ void issue_weights(const SmallParams& p, const ItemIter& it, uint8_t* stage, uint64_t* bar,
+                                              int lane) {
   using G = StageGeom<FMT, TG>;
   using Tr = FmtTraits<FMT>;
-  mbar_arrive_expect_tx(bar, stage_bytes<FMT, TG>(it));
   const int tile = it.sp.rt0, n = it.sp.nt;
-  const uint8_t* csrc = p.codes + (unsigned long long)it.sg.expert * p.codes_stride +
-                        ((unsigned long long)it.ku * p.NT + tile) * Tr::kCodeBytes;
-  bulk_copy_g2s(stage, csrc, (uint32_t)(n * Tr::kCodeBytes), bar);
+  if (lane == 0) {
+    const uint8_t* csrc = p.codes + (unsigned long long)it.sg.expert * p.codes_stride +
+                          ((unsigned long long)it.ku * p.NT + tile) * Tr::kCodeBytes;
+    const uint32_t bytes = (uint32_t)(n * Tr::kCodeBytes);
+    // No proxy fence: the warp's reads of this stage were consumed by its MMAs
+    // before the refill is issued.
+    mbar_arrive_expect_tx(bar, bytes);
+    bulk_copy_g2s(stage, csrc, bytes, bar);
+  }
 #pragma unroll
   for (int bl = 0; bl < G::kBlocksPerKU; ++bl) {
-    const int sb = (it.ku * Tr::kKUcols + bl * 64) / p.block;
+    const int sb = (it.ku * Tr::kKUcols + bl * 64) >> (p.block == 128 ? 7 : 6);  // block is 64 or 128
     const uint8_t* ssrc = p.scales + (unsigned long long)it.sg.expert * p.scales_stride +
                           ((unsigned long long)sb * p.NT + tile) * 32;
-    bulk_copy_g2s(stage + G::kCodeBytes + bl * kMaxT * 32, ssrc, (uint32_t)(n * 32), bar);
+    if (lane < 2 * n) cp_async16(stage + G::kCodeBytes + bl * kMaxT * 32 + 16 * lane, ssrc + 16 * lane);
   }
 }
 
-// Activation part of a stage: lane n < m copies its token's k-unit slice.
+// Activation part of a stage: the k-unit slice of each of the segment's m
+// token rows (the row of token n is held by lane n of the iterator).
 template <int FMT, int TG>
-__device__ __forceinline__ void issue_acts(const SmallParams& p, const ItemIter& it, uint8_t* stage, uint64_t* bar,
-                                           int lane) {
+__device__ __forceinline__ void issue_acts(const SmallParams& p, const ItemIter& it, uint8_t* stage, int lane) {
   using G = StageGeom<FMT, TG>;
-  constexpr int kBytes = FmtTraits<FMT>::kKUcols * 2;
-  if (lane < it.sg.m) {
-    const uint8_t* src = reinterpret_cast<const uint8_t*>(p.act) + ((unsigned long long)it.row * p.K) * 2 +
-                         (unsigned long long)it.ku * kBytes;
-    bulk_copy_g2s(stage + G::kCodeBytes + G::kScaleBytes + lane * G::kActPitch, src, kBytes, bar);
+  constexpr int kChunks = FmtTraits<FMT>::kKUcols * 2 / 16;  // 16-byte pieces per row slice
+  const int total = it.sg.m * kChunks;
+  for (int base = 0; base < total; base += 32) {
+    const int c = base + lane;
+    const int n = c / kChunks, j = c % kChunks;
+    const int row = __shfl_sync(0xffffffffu, it.row, n < 32 ? n : 0);
+    if (c < total) {
+      const uint8_t* src = reinterpret_cast<const uint8_t*>(p.act) + ((unsigned long long)row * p.K) * 2 +
+                           (unsigned long long)it.ku * kChunks * 16 + 16 * j;
+      cp_async16(stage + G::kCodeBytes + G::kScaleBytes + n * G::kActPitch + 16 * j, src);
+    }
   }
 }
 
@@ -290,36 +305,52 @@ __device__ __forceinline__ void ldmatrix_x4(uint32_t (&r)[4], const void* p) {
 // top-k with ties to the lower index, softmax over the selected logits, slot
 // order = stable sort of t*k+s by expert, shared experts after the routed
 // slots; one segment per active expert, experts in increasing order.
+
+// Order-preserving key of a logit: a larger key is a larger value; -0 and +0
+// are equal; NaN is below every number.
+__device__ __forceinline__ uint32_t logit_key(float v) {
+  if (v != v) return 0u;
+  if (v == 0.f) v = 0.f;
+  const uint32_t b = __float_as_uint(v);
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
 __device__ void decode_route(const SmallParams& p, DecodeRoute& R) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int T = p.T, E = p.E, k = p.k, TK = T * k;
-  for (int e = tid; e < kMaxExperts; e += blockDim.x) R.counts[e] = 0;
+  constexpr int V = kMaxExperts / 32;
   if (warp < T) {
-    float v[kMaxExperts / 32];
-    unsigned taken = 0;
+    // warp t selects token t's experts: k rounds of a warp arg-max over
+    // (key desc, index asc); lane holds experts lane + 32j.
+    float v[V];
+    uint32_t key[V];
+    unsigned live = 0;
 #pragma unroll
-    for (int j = 0; j < kMaxExperts / 32; ++j) {
+    for (int j = 0; j < V; ++j) {
       const int idx = lane + 32 * j;
-      v[j] = idx < E ? p.logits[(size_t)warp * E + idx] : -FLT_MAX;
+      v[j] = idx < E ? p.logits[(size_t)warp * E + idx] : 0.f;
+    }
+#pragma unroll
+    for (int j = 0; j < V; ++j) {
+      key[j] = logit_key(v[j]);
+      if (lane + 32 * j < E) live |= 1u << j;
     }
     for (int s = 0; s < k; ++s) {
-      float bv = -FLT_MAX;
-      int bi = INT_MAX;
+      uint32_t bk = 0;
+      int bj = -1;
 #pragma unroll
-      for (int j = 0; j < kMaxExperts / 32; ++j) {
-        const int idx = lane + 32 * j;
-        if (idx < E && !((taken >> j) & 1u) && (bi == INT_MAX || v[j] > bv)) { bv = v[j]; bi = idx; }
-      }
+      for (int j = 0; j < V; ++j)
+        if (((live >> j) & 1u) && (bj < 0 || key[j] > bk)) { bk = key[j]; bj = j; }
+      const uint32_t mk = __reduce_max_sync(0xffffffffu, bj >= 0 ? bk : 0u);
+      const int win = __reduce_min_sync(0xffffffffu, (bj >= 0 && bk == mk) ? lane + 32 * bj : INT_MAX);
+      if ((win & 31) == lane) {
+        live &= ~(1u << (win >> 5));
+        float wv = 0.f;
 #pragma unroll
-      for (int off = 16; off > 0; off >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-        const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
-        if (oi != INT_MAX && (bi == INT_MAX || ov > bv || (ov == bv && oi < bi))) { bv = ov; bi = oi; }
-      }
-      if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
-      if (lane == 0) {
-        R.ids[warp * k + s] = bi;
-        R.selv[warp][s] = bv;
+        for (int j = 0; j < V; ++j)
+          if (j == (win >> 5)) wv = v[j];
+        R.ids[warp * k + s] = win;
+        R.selv[warp][s] = wv;
       }
     }
     __syncwarp();
@@ -331,54 +362,49 @@ __device__ void decode_route(const SmallParams& p, DecodeRoute& R) {
     }
   }
   __syncthreads();
-  for (int i = tid; i < TK; i += blockDim.x) atomicAdd(&R.counts[R.ids[i]], 1);
-  __syncthreads();
-  if (warp == 0) {
-    // exclusive scan of counts -> offsets; compaction of active experts -> segments
-    int base = 0, sbase = 0;
-    const unsigned lt = (1u << lane) - 1u;
-    for (int c = 0; c < E; c += 32) {
-      const int e = c + lane;
-      const int cnt = e < E ? R.counts[e] : 0;
-      int incl = cnt;
-#pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const int o = __shfl_up_sync(0xffffffffu, incl, off);
-        if (lane >= off) incl += o;
-      }
-      if (e < E) R.offs[e] = base + incl - cnt;
-      const unsigned act = __ballot_sync(0xffffffffu, cnt > 0);
-      if (cnt > 0) {
-        Seg sg;
-        sg.expert = e;
-        sg.m = cnt;
-        sg.tg = (cnt + 7) / 8;
-        sg.slot0 = base + incl - cnt;
-        R.segs[sbase + __popc(act & lt)] = sg;
-      }
-      base += __shfl_sync(0xffffffffu, incl, 31);
-      sbase += __popc(act);
-    }
-    if (lane < p.n_shared) {
-      Seg sg;
-      sg.expert = E + lane;
-      sg.m = T;
-      sg.tg = (T + 7) / 8;
-      sg.slot0 = TK + lane * T;
-      R.segs[sbase + lane] = sg;
-    }
-    if (lane == 0) R.nseg = sbase + p.n_shared;
-  }
-  __syncthreads();
+  // slot of entry i = entries with a lower expert + earlier entries with the same expert
+  int nfirst_local = 0;
   for (int i = tid; i < TK; i += blockDim.x) {
     const int e = R.ids[i];
-    int rank = 0;
-    for (int j = 0; j < i; ++j) rank += R.ids[j] == e;
-    const int pos = R.offs[e] + rank;
+    int less = 0, before = 0, cnt = 0;
+    for (int j = 0; j < TK; ++j) {
+      const int f = R.ids[j];
+      less += f < e;
+      cnt += f == e;
+      before += (f == e) & (j < i);
+    }
+    const int pos = less + before;
     R.pos[i] = pos;
     R.slot_token[pos] = i / k;
+    R.less[i] = less;
+    R.cnt[i] = cnt;
+    R.first[i] = before == 0;
+    nfirst_local += before == 0;
   }
   for (int i = tid; i < p.n_shared * T; i += blockDim.x) R.slot_token[TK + i] = i % T;
+  // one segment per distinct expert, at the rank of its expert among them
+  const int nfirst = __syncthreads_count(nfirst_local);  // a thread holds at most one entry (TK < blockDim)
+  for (int i = tid; i < TK; i += blockDim.x) {
+    if (!R.first[i]) continue;
+    const int e = R.ids[i];
+    int idx = 0;
+    for (int j = 0; j < TK; ++j) idx += R.first[j] & (R.ids[j] < e);
+    Seg sg;
+    sg.expert = e;
+    sg.m = R.cnt[i];
+    sg.tg = (sg.m + 7) / 8;
+    sg.slot0 = R.less[i];
+    R.segs[idx] = sg;
+  }
+  if (tid < p.n_shared) {
+    Seg sg;
+    sg.expert = E + tid;
+    sg.m = T;
+    sg.tg = (T + 7) / 8;
+    sg.slot0 = TK + tid * T;
+    R.segs[nfirst + tid] = sg;
+  }
+  if (tid == 0) R.nseg = nfirst + p.n_shared;
   __syncthreads();
 }
 
@@ -572,13 +598,36 @@ __device__ __forceinline__ void compute_item(const uint8_t* st, bool tg2, int la
 
 // Decode FC2: router-weighted combine of output rows [16 rt, 16 rt + 16) over
 // all tokens, once every segment has written them.
-__device__ __forceinline__ void combine_tile(const SmallParams& p, const DecodeRoute& R, int rt) {
-  const int TK = p.T * p.k;
-  for (int e = threadIdx.x; e < p.T * 16; e += blockDim.x) {
-    const int t = e >> 4, r = rt * 16 + (e & 15);
+// Router-weighted combine of the output tiles flagged in comb[0..nt) (tiles
+// rt0 + i): y[t][r] = sum_s w[t][s] * yslot[pos(t,s)][r] + sum_j yslot[shared j, t][r].
+// Slot rows are read in batches of 8 so that the loads overlap.
+template <int NTHR>
+__device__ __forceinline__ void combine_tiles(const SmallParams& p, const DecodeRoute& R, int rt0, int nt,
+                                              const int* comb) {
+  const int TK = p.T * p.k, per = p.T * 16;
+  for (int e = threadIdx.x; e < nt * per; e += NTHR) {
+    const int i = e / per;
+    if (!comb[i]) continue;
+    const int t = (e - i * per) >> 4, r = (rt0 + i) * 16 + (e & 15);
     float acc = 0.f;
-    for (int s = 0; s < p.k; ++s) acc = fmaf(R.w[t * p.k + s], __ldcg(p.yslot + (size_t)R.pos[t * p.k + s] * p.H + r), acc);
-    for (int j = 0; j < p.n_shared; ++j) acc += __ldcg(p.yslot + (size_t)(TK + j * p.T + t) * p.H + r);
+    for (int s0 = 0; s0 < p.k; s0 += 8) {
+      float v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        v[u] = s0 + u < p.k ? __ldcg(p.yslot + (size_t)R.pos[t * p.k + s0 + u] * p.H + r) : 0.f;
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        if (s0 + u < p.k) acc = fmaf(R.w[t * p.k + s0 + u], v[u], acc);
+    }
+    for (int j0 = 0; j0 < p.n_shared; j0 += 8) {
+      float v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        v[u] = j0 + u < p.n_shared ? __ldcg(p.yslot + (size_t)(TK + (j0 + u) * p.T + t) * p.H + r) : 0.f;
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        if (j0 + u < p.n_shared) acc += v[u];
+    }
     p.y[(size_t)t * p.H + r] = __bfloat16_as_ushort(__float2bfloat16_rn(acc));
   }
 }
@@ -636,22 +685,22 @@ __global__ void __launch_bounds__(kNW * 32, 1) qmm_small_kernel(const SmallParam
   if (tid == 0) s_abort = 0;
   if constexpr (FMT == 3)
     for (int i = tid; i < 243; i += blockDim.x) lut[i] = tern_lut_entry(i);
-  uint64_t* wbar = bars + warp * NST;
+  uint64_t* wfull = bars + warp * NST;  // [kNW][NST]: the stage's copies landed
   uint8_t* wstage = stages + (size_t)warp * NST * G::kStageBytes;
   if (lane == 0)
-    for (int s = 0; s < NST; ++s) mbar_init(&wbar[s], 1);
+    for (int s = 0; s < NST; ++s) mbar_init(&wfull[s], 33);
   fence_mbar_init();
   __syncthreads();
 
-  // Producer: the weights of the first NST items before the dependency wait,
-  // their activation rows after it.
+  // Every warp fills its own NST-stage ring: the weights of its first NST
+  // items before the dependency wait, their activation rows after it.
   ItemIter prod;
   int primed = 0;
   iter_begin<TG>(prod, p, segs, act_index, f0, f1, warp, lane);
   {
     ItemIter it = prod;
     for (int s = 0; s < NST && it.valid; ++s, ++primed) {
-      if (lane == 0) issue_weights<FMT, TG>(p, it, wstage + s * G::kStageBytes, &wbar[s]);
+      issue_weights<FMT, TG>(p, it, wstage + s * G::kStageBytes, &wfull[s], lane);
       iter_advance<TG>(it, p, segs, act_index, warp, lane);
     }
   }
@@ -661,12 +710,18 @@ __global__ void __launch_bounds__(kNW * 32, 1) qmm_small_kernel(const SmallParam
     for (int i = tid; i < p.H / 16; i += blockDim.x) p.ctick[i] = 0;  // for the FC2 launch that follows
   __syncwarp();
   for (int s = 0; s < primed; ++s) {
-    issue_acts<FMT, TG>(p, prod, wstage + s * G::kStageBytes, &wbar[s], lane);
+    issue_acts<FMT, TG>(p, prod, wstage + s * G::kStageBytes, lane);
+    cp_async_arrive(&wfull[s]);
     iter_advance<TG>(prod, p, segs, act_index, warp, lane);
   }
+  constexpr int kCT = kNW * 32;
 
-  int item = 0;           // this warp's consumed items
-  bool aborted = false;   // this warp gave up waiting
+  int item = 0;          // this warp's consumed items
+  int stage = 0;         // item % NST
+  uint32_t phase = 0;    // (item / NST) & 1
+  int issued = primed;   // this warp's issued items
+  int fail_at = 0;       // first item whose wait gave up
+  bool aborted = false;  // this warp gave up waiting
 
   SubPanel sp;
   unsigned pos = f0;
@@ -693,15 +748,20 @@ __global__ void __launch_bounds__(kNW * 32, 1) qmm_small_kernel(const SmallParam
         for (int e = 0; e < 4; ++e) acc[i][t][e] = 0.f;
 
     for (int ku = warp; ku < p.KU; ku += kNW) {
-      const int s = item % NST;
-      const uint32_t par = (uint32_t)(item / NST) & 1u;
+      const int s = stage;
+      const uint32_t par = phase;
       ++item;
-      if (!aborted && !mbar_wait_bounded(&wbar[s], par, p.status)) {
+      if (++stage == NST) {
+        stage = 0;
+        phase ^= 1u;
+      }
+      if (!aborted && __any_sync(0xffffffffu, !mbar_wait_bounded(&wfull[s], par, p.status))) {
         aborted = true;
+        fail_at = item - 1;
         s_abort = 1;
       }
-      uint8_t* st = wstage + s * G::kStageBytes;
       if (!aborted) {
+        const uint8_t* st = wstage + s * G::kStageBytes;
         if (sp.nt > 4) compute_item<FMT, TG, 8>(st, tg2, lane, sp.nt, lut, acc);
         else if (sp.nt > 2) compute_item<FMT, TG, 4>(st, tg2, lane, sp.nt, lut, acc);
         else if (sp.nt > 1) compute_item<FMT, TG, 2>(st, tg2, lane, sp.nt, lut, acc);
@@ -709,12 +769,11 @@ __global__ void __launch_bounds__(kNW * 32, 1) qmm_small_kernel(const SmallParam
       }
       __syncwarp();
       if (prod.valid && !aborted) {
-        if (lane == 0) {
-          fence_proxy_async_smem();
-          issue_weights<FMT, TG>(p, prod, st, &wbar[s]);
-        }
-        __syncwarp();
-        issue_acts<FMT, TG>(p, prod, st, &wbar[s], lane);
+        uint8_t* st = wstage + s * G::kStageBytes;
+        issue_weights<FMT, TG>(p, prod, st, &wfull[s], lane);
+        issue_acts<FMT, TG>(p, prod, st, lane);
+        cp_async_arrive(&wfull[s]);
+        ++issued;
         iter_advance<TG>(prod, p, segs, act_index, warp, lane);
       }
       __syncwarp();
@@ -733,8 +792,8 @@ __global__ void __launch_bounds__(kNW * 32, 1) qmm_small_kernel(const SmallParam
     const bool ab = s_abort != 0;
     const int nel = sp.nt * TG * 32;
 #pragma unroll
-    for (int r = 0; r < (kMaxT * TG * 32 + kNW * 32 - 1) / (kNW * 32); ++r) {
-      const int e = tid + r * kNW * 32;
+    for (int r = 0; r < (kMaxT * TG * 32 + kCT - 1) / kCT; ++r) {
+      const int e = tid + r * kCT;
       if (e >= nel || ab) continue;
       float4 v = red[e];
       for (int w = 1; w < kNW; ++w) {
@@ -746,28 +805,27 @@ __global__ void __launch_bounds__(kNW * 32, 1) qmm_small_kernel(const SmallParam
       epilogue<EPI>(p, sg, sp.rt0 + i, t, ln, v);
     }
     if constexpr (SRC == SRC_DECODE && EPI == EPI_FC2) {
-      // fused combine: the last segment to finish an output tile combines it
-      __threadfence();
+      // fused combine: the CTA that adds an output tile's last segment combines
+      // it.  After the barrier, one acquire-release ticket per tile publishes
+      // this CTA's slot rows and acquires the other CTAs' ones.
       __syncthreads();
       if (tid < sp.nt) {
-        const int old = ab ? -1 : atomicAdd(&p.ctick[sp.rt0 + tid], 1);
+        const int old = ab ? -1 : atomic_add_acq_rel_gpu(&p.ctick[sp.rt0 + tid], 1);
         s_comb[tid] = old == nseg - 1;
-        if (old == nseg - 1) p.ctick[sp.rt0 + tid] = 0;
+        if (old == nseg - 1) p.ctick[sp.rt0 + tid] = 0;  // ready for the next launch
       }
       __syncthreads();
-      for (int i = 0; i < sp.nt; ++i)
-        if (s_comb[i]) {
-          __threadfence();
-          combine_tile(p, R, sp.rt0 + i);
-        }
+      combine_tiles<kCT>(p, R, sp.rt0, sp.nt, s_comb);
     }
     __syncthreads();
     pos = sp.next;
   }
-
-  // Drain: if this warp gave up waiting, let its copies in flight land (bounded).
-  if (aborted && lane == 0) {
-    for (int s = 0; s < NST; ++s) mbar_wait_bounded(&wbar[s], (uint32_t)((item + s) / NST) & 1u, nullptr);
+  // Drain: if this warp gave up waiting, let its copies in flight land.
+  if (aborted) {
+    cp_async_wait_all();
+    if (lane == 0)
+      for (int j = fail_at; j < issued; ++j)  // issued, unconsumed items: their bulk copies (bounded)
+        mbar_wait_bounded(&wfull[j % NST], (uint32_t)(j / NST) & 1u, nullptr);
   }
 }
 

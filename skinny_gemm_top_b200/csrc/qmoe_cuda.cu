@@ -218,7 +218,7 @@ qmoe_status launch_small_t(SmallParams prm, int grid, cudaStream_t st) {
   using G = StageGeom<FMT, TG>;
   const int fixed = SmemHead<SRC>::kFixed + G::kRedBytes;
   int nst = (kSmemLimit - fixed - 1024) / (kNW * G::kStageBytes);
-  nst = std::min(nst, 4);
+  nst = std::min(nst, kMaxStages);
   if (nst < 2) return QMOE_ERR_UNSUPPORTED;
   prm.nstages = nst;
   const int smem = fixed + nst * kNW * G::kStageBytes;
