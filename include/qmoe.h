@@ -47,7 +47,8 @@ typedef enum {
   QMOE_ERR_UNSUPPORTED = 2,   /* valid but outside what the kernels handle  */
   QMOE_ERR_SCRATCH = 3,       /* workspace too small even for one token row */
   QMOE_ERR_CUDA = 4,          /* a CUDA runtime call failed                 */
-  QMOE_ERR_TIMEOUT = 5        /* a device-side bounded wait ran out         */
+  QMOE_ERR_TIMEOUT = 5,       /* a device-side bounded wait ran out         */
+  QMOE_ERR_STATIC_SCRATCH = 6 /* needs more than QMOE_STATIC_SCRATCH_BYTES  */
 } qmoe_status;
 
 /* Weight code formats. */
@@ -152,6 +153,24 @@ qmoe_status qmoe_workspace_size(const qmoe_layer* layer, int T, size_t* bytes);
  * one row does not fit.  ws must be 256-byte aligned. */
 qmoe_status qmoe_forward(const qmoe_layer* layer, const uint16_t* x, const float* logits, int T,
                          uint16_t* y, void* ws, size_t ws_bytes, void* stream);
+
+/* qmoe_forward without a caller workspace, allocating nothing.  The pages
+ * describe no counterpart: this is a deployment entry point for callers that
+ * own no device allocator or must not call cudaMalloc/cudaFree inside a step
+ * (they synchronise the device and can fail under memory pressure).
+ * Scratch: a fixed device array of QMOE_STATIC_SCRATCH_BYTES inside the
+ * library, one per device.  Arguments and results as qmoe_forward (x, logits,
+ * y device pointers; stream a cudaStream_t or NULL).  Errors: those of
+ * qmoe_forward, and QMOE_ERR_STATIC_SCRATCH when qmoe_workspace_size(T)
+ * exceeds the array (no row tiling; nothing is launched).  The first call on
+ * a device resolves the array's address (cudaGetSymbolAddress with that
+ * device current) and can load the library's device code: make it before any
+ * stream capture.  No scratch value must start at zero (the per-tile tickets
+ * are cleared inside each call).  Calls that overlap in time on one device
+ * share the array and race: serialise them. */
+#define QMOE_STATIC_SCRATCH_BYTES (8u << 20)
+qmoe_status qmoe_forward_static(const qmoe_layer* layer, const uint16_t* x, const float* logits, int T,
+                                uint16_t* y, void* stream);
 
 /* Single quantized linear y[M, N] bf16 = x[M, K] bf16 @ dequant(W)[N, K]^T,
  * W packed PLAIN.  M >= 1. */

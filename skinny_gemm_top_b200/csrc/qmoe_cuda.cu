@@ -330,6 +330,7 @@ const char* qmoe_status_str(int s) {
     case QMOE_ERR_SCRATCH: return "workspace too small for one token row";
     case QMOE_ERR_CUDA: return "CUDA runtime error";
     case QMOE_ERR_TIMEOUT: return "device wait timed out";
+    case QMOE_ERR_STATIC_SCRATCH: return "request needs more than the static scratch (QMOE_STATIC_SCRATCH_BYTES)";
     default: return "unknown status";
   }
 }

@@ -18,7 +18,8 @@ INT2, TERNARY, INT4 = 2, 3, 4
 FMT = {"int2": INT2, "int4": INT4, "ternary": TERNARY}
 ROWS_PLAIN, ROWS_GATE_UP = 0, 1
 PATH_AUTO, PATH_SMALL_M, PATH_GROUPED = 0, 1, 2
-OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_SCRATCH, ERR_CUDA, ERR_TIMEOUT = range(6)
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_SCRATCH, ERR_CUDA, ERR_TIMEOUT, ERR_STATIC_SCRATCH = range(7)
+STATIC_SCRATCH_BYTES = 8 << 20  # QMOE_STATIC_SCRATCH_BYTES
 
 
 class QmoeError(RuntimeError):
@@ -53,6 +54,7 @@ EXPORTS = {
     "qmoe_workspace_size": [C.POINTER(Layer), C.c_int, C.POINTER(C.c_size_t)],
     "qmoe_forward": [C.POINTER(Layer), C.c_void_p, C.c_void_p, C.c_int, C.c_void_p, C.c_void_p, C.c_size_t,
                      C.c_void_p],
+    "qmoe_forward_static": [C.POINTER(Layer), C.c_void_p, C.c_void_p, C.c_int, C.c_void_p, C.c_void_p],
     "qmoe_linear_workspace_size": [C.c_int, C.c_int, C.c_int, C.POINTER(C.c_size_t)],
     "qmoe_linear": [C.POINTER(Weights), C.c_int, C.c_int, C.c_void_p, C.c_int, C.c_void_p, C.c_void_p,
                     C.c_size_t, C.c_void_p],
@@ -176,6 +178,12 @@ def forward(layer: Layer, x, logits, y, ws, ws_bytes: int | None = None, stream=
     nbytes = ws.numel() * ws.element_size() if ws_bytes is None else ws_bytes
     _check(_lib.qmoe_forward(C.byref(layer), _ptr(x), _ptr(logits), T, _ptr(y), _ptr(ws), nbytes,
                              _stream(stream)), "qmoe_forward")
+
+
+def forward_static(layer: Layer, x, logits, y, stream=None):
+    """qmoe_forward with the library's fixed device scratch (no workspace, no allocation)."""
+    _check(_lib.qmoe_forward_static(C.byref(layer), _ptr(x), _ptr(logits), x.shape[0], _ptr(y), _stream(stream)),
+           "qmoe_forward_static")
 
 
 def linear_workspace_size(N: int, K: int, M: int) -> int:
