@@ -45,7 +45,11 @@
 
 namespace qmoe {
 
-constexpr int kNW = 8;            // warps per CTA
+// Warps per CTA: 12 for one token group (three warps per SM sub-partition
+// hide the unpack/MMA latency better than two), 8 for two token groups, whose
+// accumulators need more than the 168 registers a 12-warp CTA leaves.
+template <int TG>
+constexpr int kWarps = TG == 1 ? 12 : 8;
 constexpr int kMaxT = 8;          // tiles per sub-panel
 constexpr int kMaxStages = 6;     // stages per consumer warp (barriers: 1024 bytes of shared memory)
 constexpr int kChunkTokens = 16;  // tokens per segment (<= 2 token groups of 8)
@@ -113,6 +117,7 @@ struct SmallParams {
   float* yslot;                      // FC2: yslot[slot][H]
   int H;
   int* ctick;                        // decode: per 16-row output tile counters (H/16)
+  DecodeRoute* route_tab;            // decode: routing tables, written by FC1's CTA 0, read by FC2
   int early;                         // 1: segments and weights may be read before griddepcontrol.wait
   unsigned* status;
 };
@@ -127,6 +132,7 @@ struct StageGeom {
   static constexpr int kActPitch = Tr::kKUcols * 2 + 16;               // padded: conflict-free ldmatrix
   static constexpr int kActBytes = TG * 8 * kActPitch;
   static constexpr int kStageBytes = ((kCodeBytes + kScaleBytes + kActBytes) + 127) / 128 * 128;
+  static constexpr int kNW = kWarps<TG>;
   static constexpr int kRedBytes = kNW * kMaxT * TG * 32 * 16;
 };
 
@@ -187,7 +193,7 @@ struct SegSource {
 };
 
 // Warp-uniform iterator over one warp's (sub-panel, k-unit) items: in every
-// sub-panel, warp w takes k-units w, w + kNW, ...  Caches the segment and,
+// sub-panel, warp w takes k-units w, w + kWarps, ...  Caches the segment and,
 // per lane n < m, the row of token n.
 struct ItemIter {
   SubPanel sp;
@@ -211,7 +217,7 @@ __device__ __forceinline__ void iter_load_seg(ItemIter& it, const SmallParams& p
 template <int TG>
 __device__ __forceinline__ void iter_advance(ItemIter& it, const SmallParams& p, const SegSource& segs,
                                              const int* act_index, int warp, int lane) {
-  it.ku += kNW;
+  it.ku += kWarps<TG>;
   if (it.ku < p.KU) return;
   for (;;) {
     if (it.sp.next >= it.f1) { it.valid = false; return; }
@@ -233,7 +239,7 @@ __device__ __forceinline__ void iter_begin(ItemIter& it, const SmallParams& p, c
   iter_load_seg<TG>(it, p, segs, act_index, lane);
   it.ku = warp;
   if (it.ku >= p.KU) {
-    it.ku = p.KU - kNW;  // so that the advance moves to the next sub-panel
+    it.ku = p.KU - kWarps<TG>;  // so that the advance moves to the next sub-panel
     iter_advance<TG>(it, p, segs, act_index, warp, lane);
   }
 }
@@ -633,8 +639,9 @@ __device__ __forceinline__ void combine_tiles(const SmallParams& p, const Decode
 }
 
 template <int FMT, int TG, int EPI, int SRC>
-__global__ void __launch_bounds__(kNW * 32, 1) qmm_small_kernel(const SmallParams p) {
+__global__ void __launch_bounds__(kWarps<TG> * 32, 1) qmm_small_kernel(const SmallParams p) {
   using G = StageGeom<FMT, TG>;
+  constexpr int kNW = kWarps<TG>;
   extern __shared__ __align__(128) uint8_t smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int NST = p.nstages;
@@ -658,7 +665,20 @@ __global__ void __launch_bounds__(kNW * 32, 1) qmm_small_kernel(const SmallParam
   segs.rows = p.T;
   const int* act_index = p.act_index;
   if constexpr (SRC == SRC_DECODE) {
-    decode_route(p, R);
+    if constexpr (EPI == EPI_FC2) {
+      // the routing of this call, from the FC1 launch just before (after the wait)
+      const uint32_t* src = reinterpret_cast<const uint32_t*>(p.route_tab);
+      uint32_t* dst = reinterpret_cast<uint32_t*>(&R);
+      for (int i = tid; i < (int)(sizeof(DecodeRoute) / 4); i += blockDim.x) dst[i] = __ldcg(src + i);
+      __syncthreads();
+    } else {
+      decode_route(p, R);
+      if (blockIdx.x == 0) {  // for the FC2 launch of this call
+        const uint32_t* src = reinterpret_cast<const uint32_t*>(&R);
+        uint32_t* dst = reinterpret_cast<uint32_t*>(p.route_tab);
+        for (int i = tid; i < (int)(sizeof(DecodeRoute) / 4); i += blockDim.x) dst[i] = src[i];
+      }
+    }
     nseg = R.nseg;
     segs.table = R.segs;
     if (EPI == EPI_SWIGLU) act_index = R.slot_token;

@@ -136,7 +136,7 @@ qmoe_status check_weights(const qmoe_weights& w, int rows, int K) {
 struct MoEPlan {
   int T, S, TK, max_seg, n_tickets, max_gseg;
   bool grouped, decode;
-  size_t ids, w, perm, inv, offsets, slot_token, nseg, segs, yslot, hrows, ctick, ngseg, gsegs, xrows, total;
+  size_t ids, w, perm, inv, offsets, slot_token, nseg, segs, yslot, hrows, ctick, route, ngseg, gsegs, xrows, total;
 };
 
 constexpr int kGroupedThreshold = 32;  // AUTO: experts with more tokens take the tcgen05 path
@@ -170,6 +170,7 @@ MoEPlan plan_moe(const qmoe_layer& L, int T, int grid) {
   p.yslot = take((size_t)p.S * L.H * 4);
   p.hrows = take((size_t)p.S * L.I * 2 + 16);
   p.ctick = take((size_t)(L.H / 16) * 4);
+  if (p.decode) p.route = take(sizeof(DecodeRoute));
   if (!p.decode) {
     p.ids = take((size_t)p.TK * 4);
     p.w = take((size_t)p.TK * 4);
@@ -216,6 +217,7 @@ qmoe_status encode_rows_map(CUtensorMap* map, const void* base, int K, int rows)
 template <int FMT, int TG, int EPI, int SRC>
 qmoe_status launch_small_t(SmallParams prm, int grid, cudaStream_t st) {
   using G = StageGeom<FMT, TG>;
+  constexpr int kNW = kWarps<TG>;
   const int fixed = SmemHead<SRC>::kFixed + G::kRedBytes;
   int nst = (kSmemLimit - fixed - 1024) / (kNW * G::kStageBytes);
   nst = std::min(nst, kMaxStages);
@@ -239,16 +241,17 @@ qmoe_status launch_small_t(SmallParams prm, int grid, cudaStream_t st) {
 
 template <int EPI, int SRC>
 qmoe_status launch_small(int fmt, int tg, const SmallParams& prm, int grid, cudaStream_t st) {
-  if (SRC == SRC_DECODE) {  // decode batches have at most 8 tokens: one token group
+  if constexpr (SRC == SRC_DECODE) {  // decode batches have at most 8 tokens: one token group
     if (fmt == QMOE_INT2) return launch_small_t<2, 1, EPI, SRC>(prm, grid, st);
     if (fmt == QMOE_INT4) return launch_small_t<4, 1, EPI, SRC>(prm, grid, st);
     return launch_small_t<3, 1, EPI, SRC>(prm, grid, st);
+  } else {
+    if (fmt == QMOE_INT2)
+      return tg == 1 ? launch_small_t<2, 1, EPI, SRC>(prm, grid, st) : launch_small_t<2, 2, EPI, SRC>(prm, grid, st);
+    if (fmt == QMOE_INT4)
+      return tg == 1 ? launch_small_t<4, 1, EPI, SRC>(prm, grid, st) : launch_small_t<4, 2, EPI, SRC>(prm, grid, st);
+    return tg == 1 ? launch_small_t<3, 1, EPI, SRC>(prm, grid, st) : launch_small_t<3, 2, EPI, SRC>(prm, grid, st);
   }
-  if (fmt == QMOE_INT2)
-    return tg == 1 ? launch_small_t<2, 1, EPI, SRC>(prm, grid, st) : launch_small_t<2, 2, EPI, SRC>(prm, grid, st);
-  if (fmt == QMOE_INT4)
-    return tg == 1 ? launch_small_t<4, 1, EPI, SRC>(prm, grid, st) : launch_small_t<4, 2, EPI, SRC>(prm, grid, st);
-  return tg == 1 ? launch_small_t<3, 1, EPI, SRC>(prm, grid, st) : launch_small_t<3, 2, EPI, SRC>(prm, grid, st);
 }
 
 template <int FMT, int EPI>
@@ -483,9 +486,10 @@ qmoe_status qmoe_forward(const qmoe_layer* layer, const uint16_t* x, const float
         q->k = L.k;
         q->n_shared = L.n_shared;
         q->ctick = reinterpret_cast<int*>(base + p.ctick);
+        q->route_tab = reinterpret_cast<DecodeRoute*>(base + p.route);
       }
       p1.early = 0;  // the logits may come from the previous launch
-      p2.early = 1;  // routing inputs were consumed by FC1 after its wait
+      p2.early = 0;  // FC2 reads FC1's routing tables after its wait
       p2.y = yt;
       s = launch_small<EPI_SWIGLU, SRC_DECODE>(L.fc1.fmt, 1, p1, grid, st);
       if (s != QMOE_OK) return s;
