@@ -272,6 +272,11 @@ def run_ours(args):
             r = i % ROTATE
             qmoe.forward(layers[r], xs[r], lgs[r], ys[r], ws)
 
+        # launches of one forward call (traced eager call)
+        qmoe.trace_start(64)
+        fn(0, 1)
+        qmoe.trace_stop()
+        per_call = len(qmoe.trace_read(64))
         steps = Steps(torch, fn, ROTATE)
         steps.prepare(k, w)
         if clocks is not None:  # settle clocks under this load before the timed region
@@ -285,11 +290,11 @@ def run_ours(args):
         local_bytes = statistics.mean(p["total"] for p in per)
         ms, job_bytes = reduce_ranks(torch, dist, ms, local_bytes)
         out = {"ms_per_step": ms / k, "bytes": local_bytes, "job_bytes": job_bytes,
-               "fc1_bytes": statistics.mean(p["fc1"] for p in per)}
+               "fc1_bytes": statistics.mean(p["fc1"] for p in per), "launches_per_step": per_call}
         if trace:
             # Per-kernel device time: a second graph of the same ROTATE calls with CUDA
-            # events around every launch (the eager call of graph_of takes 5 records).
-            qmoe.trace_start(5 * (ROTATE + 1))
+            # events around every launch (the eager call of graph_of takes per_call records).
+            qmoe.trace_start(per_call * (ROTATE + 1))
             traced = Steps(torch, fn, ROTATE)
             qmoe.trace_stop()
             traced.run(w)
@@ -297,7 +302,7 @@ def run_ours(args):
             while time.time() - t0 < 0.2:  # the timed region of the trace: replays of the traced graph
                 traced.run(k)
             torch.cuda.synchronize()
-            rec = qmoe.trace_read(5 * (ROTATE + 1))[5:]
+            rec = qmoe.trace_read(per_call * (ROTATE + 1))[per_call:]
             out["fc1_ms"] = statistics.mean(t for n, t in rec if n == "fc1_small")
             out["kernels"] = {n: statistics.mean(t for m, t in rec if m == n) for n in sorted({n for n, _ in rec})}
             del traced
@@ -363,7 +368,7 @@ def run_ours(args):
         "sweep_tokens_per_expert": result_sweep,
         "linear_5120x17408_g128": linear,
         "e2e": e2e,
-        "gpu_launches": 5 * args.steps,
+        "gpu_launches": head["launches_per_step"] * args.steps,
         "clocks": clocks,
     }
     if rank == 0 and world == 1:
