@@ -18,6 +18,7 @@ linear K=5120 -> N=17408 (group 128, INT2 and INT4) at M = 1..32.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import os
 import statistics
@@ -321,6 +322,13 @@ def run_ours(args):
                                  "GBps": round(r["bytes"] / (r["ms_per_step"] * 1e6), 1),
                                  "tokens_per_s": round(M / (r["ms_per_step"] * 1e-3), 1)})
     linear = [] if args.quick else linear_sweep(qmoe, torch, dist, args)
+    lmhead = [] if args.quick else lmhead_sweep(qmoe, torch, dist, args)
+    # ternary layer (C4 per-expert shapes, 32 experts: one top-1 expert per token) and the
+    # prefill layer (C5, T = 4096, tcgen05 grouped path, 256 MiB workspace with row tiling)
+    ternary = [] if args.quick else cfg_sweep(qmoe, torch, dist, args,
+                                              dataclasses.replace(synth.TERNARY, E=32), (1, 8, 32), rotate=32)
+    prefill = [] if args.quick else cfg_sweep(qmoe, torch, dist, args, synth.PREFILL, (4096,), rotate=1,
+                                              ws_cap=256 << 20)
     e2e = measure_e2e(qmoe, torch, dist, layers[0], args.steps, args.warmup)
 
     peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json"))) if os.path.exists(
@@ -367,6 +375,9 @@ def run_ours(args):
                      "kernels_us": {k: round(v * 1e3, 3) for k, v in head["kernels"].items()}},
         "sweep_tokens_per_expert": result_sweep,
         "linear_5120x17408_g128": linear,
+        "linear_5120x248320_g128": lmhead,
+        "ternary_layer": ternary,
+        "prefill_layer": prefill,
         "e2e": e2e,
         "gpu_launches": head["launches_per_step"] * args.steps,
         "clocks": clocks,
@@ -446,6 +457,100 @@ def linear_sweep(qmoe, torch, dist, args) -> list:
             b = nbytes + M * K * 2 + M * N * 2
             row["M"].append({"M": M, "us": round(ms * 1e3, 3), "GBps": round(b / (ms * 1e6), 1)})
         out.append(row)
+    return out
+
+
+def cfg_layer_bytes(cfg, logits: np.ndarray) -> tuple[int, int]:
+    """(algorithmic bytes, active experts) of one forward of `cfg` on these logits."""
+    f1 = expert_bytes(cfg.fc1_fmt, 2 * cfg.I, cfg.H, cfg.block) + (2 * cfg.I * 2 if cfg.bias else 0)
+    f2 = expert_bytes(cfg.fc2_fmt, cfg.H, cfg.I, cfg.block) + (cfg.H * 2 if cfg.bias else 0)
+    T = logits.shape[0]
+    top = np.argsort(-logits.astype(np.float64), axis=1, kind="stable")[:, : cfg.k]
+    n = len(set(top.ravel().tolist())) + cfg.n_shared
+    return n * (f1 + f2) + T * cfg.H * 2 * 2 + T * cfg.E * 4, n
+
+
+def pack_cfg(qmoe, torch, cfg):
+    n = cfg.E + cfg.n_shared
+    f1, f2 = qmoe.FMT[cfg.fc1_fmt], qmoe.FMT[cfg.fc2_fmt]
+    c1, s1 = qmoe.pack_stack(f1, qmoe.ROWS_GATE_UP, (synth.expert_fc1(cfg, SEED, e) for e in range(n)), cfg.block)
+    c2, s2 = qmoe.pack_stack(f2, qmoe.ROWS_PLAIN, (synth.expert_fc2(cfg, SEED, e) for e in range(n)), cfg.block)
+    keep = [_to_dev(torch, a) for a in (c1, s1, c2, s2)]
+    b1 = b2 = None
+    if cfg.bias:
+        b1 = _to_dev(torch, np.stack([synth.expert_b1(cfg, SEED, e) for e in range(n)]))
+        b2 = _to_dev(torch, np.stack([synth.expert_b2(cfg, SEED, e) for e in range(n)]))
+        keep += [b1, b2]
+    w1 = qmoe.make_weights(f1, cfg.block, keep[0], keep[1], b1)
+    w2 = qmoe.make_weights(f2, cfg.block, keep[2], keep[3], b2)
+    return qmoe.make_layer(cfg.H, cfg.I, cfg.E, cfg.k, cfg.n_shared, w1, w2), keep
+
+
+def cfg_sweep(qmoe, torch, dist, args, cfg, Ts, rotate: int, ws_cap: int | None = None) -> dict:
+    """One layer forward per step on `cfg` for each T; router rows rotate over
+    `rotate` seeded draws so that consecutive steps touch different experts."""
+    layer, keep = pack_cfg(qmoe, torch, cfg)
+    out = {"config": f"{cfg.name}: H={cfg.H} I={cfg.I} E={cfg.E} top-{cfg.k}"
+                     f"{' + %d shared' % cfg.n_shared if cfg.n_shared else ''}, "
+                     f"FC1 {cfg.fc1_fmt} / FC2 {cfg.fc2_fmt}, block {cfg.block}", "T": []}
+    for T in Ts:
+        xs = [_to_dev(torch, synth.tokens(cfg.H, SEED, T, index=r)) for r in range(rotate)]
+        lgs_np = [synth.router_logits(cfg, SEED, T, index=100 + r) for r in range(rotate)]
+        lgs = [torch.from_numpy(np.ascontiguousarray(l)).cuda() for l in lgs_np]
+        need = qmoe.workspace_size(layer, T)
+        ws = torch.empty(min(need, ws_cap) if ws_cap else need, dtype=torch.uint8, device="cuda")
+        ys = [torch.empty((T, cfg.H), dtype=torch.int16, device="cuda") for _ in range(rotate)]
+
+        def fn(i, n, xs=xs, lgs=lgs, ys=ys, ws=ws):
+            r = i % rotate
+            qmoe.forward(layer, xs[r], lgs[r], ys[r], ws)
+
+        steps = Steps(torch, fn, rotate)
+        k = max(rotate, (args.steps // rotate) * rotate) if T <= 64 else rotate * 2
+        steps.prepare(k, args.warmup)
+        steps.run(max(args.warmup, 3))
+        ms = reduce_ranks(torch, dist, time_steps(torch, dist, steps, k), 0.0)[0] / k
+        per = [cfg_layer_bytes(cfg, l) for l in lgs_np]
+        nbytes = statistics.mean(b for b, _ in per)
+        flops = 2.0 * T * cfg.k * (2 * cfg.I * cfg.H + cfg.H * cfg.I) + 2.0 * T * cfg.n_shared * 3 * cfg.I * cfg.H
+        out["T"].append({"T": T, "us": round(ms * 1e3, 3), "tokens_per_s": round(T / (ms * 1e-3), 1),
+                         "active_experts": round(statistics.mean(a for _, a in per), 1),
+                         "GBps": round(nbytes / (ms * 1e6), 1), "TFLOPs": round(flops / (ms * 1e9), 2),
+                         "workspace_bytes": ws.numel(), "row_tiles": qmoe.get_stats().row_tiles})
+    del keep
+    return out
+
+
+def lmhead_sweep(qmoe, torch, dist, args) -> list:
+    """Single quantized linear 5120 -> 248320, g128: one copy is > 2x L2."""
+    N, K, block = 248320, 5120, 128
+    wb = synth.linear_weight(SEED, N, K)
+    out = []
+    for fmt in ("int2", "int4"):
+        c, s = qmoe.pack(qmoe.FMT[fmt], qmoe.ROWS_PLAIN, wb, block)
+        nbytes = c.nbytes + s.nbytes
+        dc, ds = _to_dev(torch, c), _to_dev(torch, s)
+        del c, s
+        w = qmoe.make_weights(qmoe.FMT[fmt], block, dc, ds)
+        row = {"fmt": fmt, "bytes_M1": nbytes + K * 2 + N * 2, "M": []}
+        for M in (1, 2, 4, 8):
+            x = _to_dev(torch, synth.tokens(K, SEED, M))
+            y = torch.empty((M, N), dtype=torch.int16, device="cuda")
+            ws = torch.empty(qmoe.linear_workspace_size(N, K, M), dtype=torch.uint8, device="cuda")
+
+            def fn(i, n, x=x, y=y, ws=ws):
+                qmoe.linear(w, N, K, x, y, ws)
+
+            steps = Steps(torch, fn, 4)
+            k = 40
+            steps.prepare(k, args.warmup)
+            steps.run(args.warmup)
+            ms = reduce_ranks(torch, dist, time_steps(torch, dist, steps, k), 0.0)[0] / k
+            b = nbytes + M * K * 2 + M * N * 2
+            row["M"].append({"M": M, "us": round(ms * 1e3, 3), "GBps": round(b / (ms * 1e6), 1)})
+        out.append(row)
+        del dc, ds, w
+    del wb
     return out
 
 

@@ -29,6 +29,7 @@ struct RouteOut {
   GSeg* gsegs;
   int max_gseg;
   unsigned* status;
+  int* chunk_counts; // [nchunks][E] (two-kernel routing)
 };
 
 // One CTA: warp top-k per token, then a stable counting sort by expert (ranks
@@ -184,6 +185,210 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
   }
   if (o.tickets)
     for (int i = tid; i < o.n_tickets; i += blockDim.x) o.tickets[i] = 0;
+}
+
+// ---- Two-kernel routing of the general path (any T) ------------------------
+// route_topk_kernel: one CTA per chunk of kRouteChunk tokens; warp top-k per
+// token (ties to the lower expert index), softmax over the k selected logits,
+// and the chunk's per-expert counts.  route_scatter_kernel: one CTA per chunk;
+// expert offsets from all chunks' counts, the chunk's base per expert from the
+// chunks before it, then a stable scatter of its flat entries t*k+s in flat
+// order (ranks from warp match masks and warp counts in warp order).  CTA 0
+// also writes the offsets, the shared-expert slots and the segment tables.
+// Deterministic: no result depends on atomics' order.
+constexpr int kRouteChunk = 64;
+constexpr int kRouteWarps = 8;
+
+__device__ __forceinline__ void warp_topk(const float* __restrict__ row, int E, int k, int lane, float* selv,
+                                          int* ids_out) {
+  float v[kMaxExperts / 32];
+  unsigned taken = 0;
+  const int nv = (E + 31) >> 5;
+#pragma unroll
+  for (int j = 0; j < kMaxExperts / 32; ++j) {
+    const int idx = lane + 32 * j;
+    v[j] = (j < nv && idx < E) ? row[idx] : -FLT_MAX;
+  }
+  for (int s = 0; s < k; ++s) {
+    float bv = -FLT_MAX;
+    int bi = INT_MAX;
+#pragma unroll
+    for (int j = 0; j < kMaxExperts / 32; ++j) {
+      const int idx = lane + 32 * j;
+      if (j < nv && idx < E && !((taken >> j) & 1u) && (bi == INT_MAX || v[j] > bv)) { bv = v[j]; bi = idx; }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+      if (oi != INT_MAX && (bi == INT_MAX || ov > bv || (ov == bv && oi < bi))) { bv = ov; bi = oi; }
+    }
+    if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+    if (lane == 0) {
+      ids_out[s] = bi;
+      selv[s] = bv;
+    }
+  }
+  __syncwarp();
+}
+
+__global__ void __launch_bounds__(kRouteWarps * 32)
+    route_topk_kernel(const float* __restrict__ logits, int T, int E, int k, RouteOut o) {
+  __shared__ int cnt[kMaxExperts];
+  __shared__ int sid[kRouteWarps][32];
+  __shared__ float selv[kRouteWarps][32];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  // Writes below may alias buffers the previous launch still reads.
+  pdl_wait();
+  pdl_trigger();
+  const int t0 = blockIdx.x * kRouteChunk, t1 = min(T, t0 + kRouteChunk);
+  for (int e = tid; e < E; e += blockDim.x) cnt[e] = 0;
+  __syncthreads();
+  for (int t = t0 + warp; t < t1; t += kRouteWarps) {
+    warp_topk(logits + (size_t)t * E, E, k, lane, selv[warp], sid[warp]);
+    if (lane < k) {
+      const float lmax = selv[warp][0];
+      float sum = 0.f;
+      for (int s = 0; s < k; ++s) sum += expf(selv[warp][s] - lmax);
+      o.w[(size_t)t * k + lane] = expf(selv[warp][lane] - lmax) / sum;
+      o.ids[(size_t)t * k + lane] = sid[warp][lane];
+      atomicAdd(&cnt[sid[warp][lane]], 1);  // order-independent count
+    }
+    __syncwarp();
+  }
+  __syncthreads();
+  for (int e = tid; e < E; e += blockDim.x) o.chunk_counts[(size_t)blockIdx.x * E + e] = cnt[e];
+}
+
+__global__ void __launch_bounds__(kRouteWarps * 32)
+    route_scatter_kernel(int T, int E, int k, int n_shared, RouteOut o) {
+  __shared__ int base[kMaxExperts];   // this chunk's first position per expert (running)
+  __shared__ int tot[kMaxExperts];    // all chunks' count per expert
+  __shared__ int offs[kMaxExperts + 1];
+  __shared__ int wtot[kRouteWarps];
+  __shared__ int wcnt[kRouteWarps][kMaxExperts];
+  __shared__ int seg_base[kMaxExperts + 64];
+  __shared__ int gseg_base[kMaxExperts + 64];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  pdl_wait();
+  pdl_trigger();
+  const int chunk = blockIdx.x, nchunks = gridDim.x;
+  for (int e = tid; e < E; e += blockDim.x) {
+    int before = 0, all = 0;
+    for (int c = 0; c < nchunks; ++c) {
+      const int v = o.chunk_counts[(size_t)c * E + e];
+      all += v;
+      before += c < chunk ? v : 0;
+    }
+    tot[e] = all;
+    base[e] = before;
+  }
+  __syncthreads();
+  // exclusive scan of tot over experts (E <= 256 = blockDim.x)
+  {
+    const int v = tid < E ? tot[tid] : 0;
+    int inc = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int u = __shfl_up_sync(0xffffffffu, inc, off);
+      if (lane >= off) inc += u;
+    }
+    if (lane == 31) wtot[warp] = inc;
+    __syncthreads();
+    int pre = 0;
+    for (int w = 0; w < warp; ++w) pre += wtot[w];
+    if (tid < E) {
+      offs[tid] = pre + inc - v;
+      base[tid] += pre + inc - v;
+    }
+    if (tid == E - 1) offs[E] = pre + inc;
+  }
+  __syncthreads();
+  if (chunk == 0)
+    for (int e = tid; e <= E; e += blockDim.x) o.offsets[e] = offs[e];
+  // stable scatter of flat entries [i0, i1) of this chunk, in rounds of blockDim entries
+  const int TK = T * k;
+  const int i0 = chunk * kRouteChunk * k, i1 = min(T, (chunk + 1) * kRouteChunk) * k;
+  const unsigned lt_mask = (1u << lane) - 1u;
+  for (int r0 = i0; r0 < i1; r0 += blockDim.x) {
+    for (int j = tid; j < kRouteWarps * kMaxExperts; j += blockDim.x) (&wcnt[0][0])[j] = 0;
+    __syncthreads();
+    const int i = r0 + tid;
+    const bool valid = i < i1;
+    const int e = valid ? o.ids[i] : -1;
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    const int rank = __popc(peers & lt_mask);
+    if (valid && rank == 0) wcnt[warp][e] = __popc(peers);
+    __syncthreads();
+    if (valid) {
+      int pre = base[e];
+      for (int w = 0; w < warp; ++w) pre += wcnt[w][e];
+      const int pos = pre + rank;
+      o.perm[pos] = i;
+      if (o.inv) o.inv[i] = pos;
+      if (o.slot_token) o.slot_token[pos] = i / k;
+    }
+    __syncthreads();
+    for (int ee = tid; ee < E; ee += blockDim.x) {
+      int sum = 0;
+      for (int w = 0; w < kRouteWarps; ++w) sum += wcnt[w][ee];
+      base[ee] += sum;
+    }
+    __syncthreads();
+  }
+  if (chunk != 0) return;
+  if (o.slot_token)
+    for (int i = tid; i < n_shared * T; i += blockDim.x) o.slot_token[TK + i] = i % T;
+  // ---- segment tables: small-M chunks of <= 16 tokens, grouped tiles of <= 256 ----
+  if (o.nseg) {
+    const int EX = E + n_shared;
+    if (tid == 0) {
+      int sb = 0, gb = 0;
+      for (int e = 0; e < EX; ++e) {
+        const int cnt = e < E ? tot[e] : T;
+        const bool grouped = o.ngseg && cnt > o.thresh;
+        seg_base[e] = sb;
+        gseg_base[e] = gb;
+        if (grouped) gb += (cnt + kGTok - 1) / kGTok;
+        else sb += (cnt + kChunkTokens - 1) / kChunkTokens;
+      }
+      if (sb > o.max_seg || (o.ngseg && gb > o.max_gseg)) {
+        atomicOr(o.status, kStatusBadSegment);
+        sb = 0;  // never index past the tables
+        gb = 0;
+      }
+      *o.nseg = sb;
+      if (o.ngseg) *o.ngseg = gb;
+      wtot[0] = sb > 0 || gb > 0;
+    }
+    __syncthreads();
+    const bool ok = wtot[0] != 0;
+    for (int e = tid; e < EX && ok; e += blockDim.x) {
+      const int cnt = e < E ? tot[e] : T;
+      const int slot_base = e < E ? offs[e] : TK + (e - E) * T;
+      if (o.ngseg && cnt > o.thresh) {
+        const int nch = (cnt + kGTok - 1) / kGTok;
+        for (int c = 0; c < nch; ++c) {
+          GSeg g;
+          g.expert = e;
+          g.slot0 = slot_base + kGTok * c;
+          g.ntok = min(kGTok, cnt - kGTok * c);
+          g.pad = 0;
+          o.gsegs[gseg_base[e] + c] = g;
+        }
+        continue;
+      }
+      const int nch = (cnt + kChunkTokens - 1) / kChunkTokens;
+      for (int c = 0; c < nch; ++c) {
+        Seg sg;
+        sg.expert = e;
+        sg.m = min(kChunkTokens, cnt - kChunkTokens * c);
+        sg.tg = (sg.m + 7) / 8;
+        sg.slot0 = slot_base + kChunkTokens * c;
+        o.segs[seg_base[e] + c] = sg;
+      }
+    }
+  }
 }
 
 // Token rows of the grouped tiles, in expert-sorted slot order: xrows[slot] = x[token(slot)].

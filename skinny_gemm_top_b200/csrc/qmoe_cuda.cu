@@ -136,7 +136,8 @@ qmoe_status check_weights(const qmoe_weights& w, int rows, int K) {
 struct MoEPlan {
   int T, S, TK, max_seg, n_tickets, max_gseg;
   bool grouped, decode;
-  size_t ids, w, perm, inv, offsets, slot_token, nseg, segs, yslot, hrows, ctick, route, ngseg, gsegs, xrows, total;
+  size_t ids, w, perm, inv, offsets, slot_token, nseg, segs, chunk_counts, yslot, hrows, ctick, route, ngseg, gsegs,
+      xrows, total;
 };
 
 constexpr int kGroupedThreshold = 32;  // AUTO: experts with more tokens take the tcgen05 path
@@ -180,6 +181,7 @@ MoEPlan plan_moe(const qmoe_layer& L, int T, int grid) {
     p.slot_token = take((size_t)p.S * 4);
     p.nseg = take(16);
     p.segs = take((size_t)p.max_seg * sizeof(Seg));
+    p.chunk_counts = take((size_t)((T + kRouteChunk - 1) / kRouteChunk) * L.E * 4);
   }
   if (p.grouped) {
     p.max_gseg = std::min(L.E, p.TK) + p.TK / kGTok + L.n_shared * ((T + kGTok - 1) / kGTok);
@@ -517,10 +519,14 @@ qmoe_status qmoe_forward(const qmoe_layer* layer, const uint16_t* x, const float
       o.max_gseg = p.max_gseg;
     }
     o.status = di->status;
+    o.chunk_counts = reinterpret_cast<int*>(base + p.chunk_counts);
     {
+      const int nchunks = (tt + kRouteChunk - 1) / kRouteChunk;
       TraceScope ts(st, K_ROUTE);
-      if (launch_pdl(route_kernel, dim3(1), dim3(kRouteThreads), 0, st, lt, tt, L.E, L.k, L.n_shared, o) !=
-          cudaSuccess)
+      if (launch_pdl(route_topk_kernel, dim3(nchunks), dim3(kRouteWarps * 32), 0, st, lt, tt, L.E, L.k, o) !=
+              cudaSuccess ||
+          launch_pdl(route_scatter_kernel, dim3(nchunks), dim3(kRouteWarps * 32), 0, st, tt, L.E, L.k, L.n_shared,
+                     o) != cudaSuccess)
         return QMOE_ERR_CUDA;
     }
     const int tg = tt <= 8 ? 1 : 2;
