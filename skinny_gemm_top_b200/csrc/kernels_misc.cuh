@@ -391,20 +391,37 @@ __global__ void __launch_bounds__(kRouteWarps * 32)
   }
 }
 
-// Token rows of the grouped tiles, in expert-sorted slot order: xrows[slot] = x[token(slot)].
+// Token rows of the grouped tiles, in expert-sorted slot order: xrows[slot] =
+// x[token(slot)].  One warp per row (grid-stride over gseg x 256 row slots):
+// each lane moves K/256 16-byte pieces with its loads issued before its stores.
 __global__ void gather_rows_kernel(const uint16_t* __restrict__ x, int K, const int* __restrict__ slot_token,
                                    const int* __restrict__ ngseg, const GSeg* __restrict__ gsegs, uint16_t* xrows) {
   pdl_wait();
   pdl_trigger();
   const int ng = *ngseg;
   const int vec = K / 8;  // uint4 per row
-  for (int gi = blockIdx.x; gi < ng; gi += gridDim.x) {
-    const GSeg g = gsegs[gi];
-    for (int i = threadIdx.x; i < g.ntok * vec; i += blockDim.x) {
-      const int r = i / vec, c = i % vec;
-      const int slot = g.slot0 + r;
-      const int tok = slot_token[slot];
-      reinterpret_cast<uint4*>(xrows + (size_t)slot * K)[c] = reinterpret_cast<const uint4*>(x + (size_t)tok * K)[c];
+  const int lane = threadIdx.x & 31;
+  const long long nw = ((long long)gridDim.x * blockDim.x) >> 5;
+  for (long long w = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5; w < (long long)ng * kGTok; w += nw) {
+    const GSeg g = gsegs[w / kGTok];
+    const int r = (int)(w % kGTok);
+    if (r >= g.ntok) continue;
+    const int slot = g.slot0 + r;
+    const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)slot_token[slot] * K);
+    uint4* dst = reinterpret_cast<uint4*>(xrows + (size_t)slot * K);
+    constexpr int kU = 8;
+    for (int c0 = 0; c0 < vec; c0 += 32 * kU) {
+      uint4 v[kU];
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int c = c0 + u * 32 + lane;
+        if (c < vec) v[u] = __ldg(src + c);
+      }
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int c = c0 + u * 32 + lane;
+        if (c < vec) dst[c] = v[u];
+      }
     }
   }
 }

@@ -8,15 +8,16 @@
 // never materialized (the onnxruntime PR's Description: "Avoid full A16
 // expert-weight materialization").
 //
-// One persistent CTA per SM, 10 warps, all waits bounded:
+// One persistent CTA per SM, 18 warps, all waits bounded:
 //   warp 0      TMA producer: packed codes + scales (cp.async.bulk) and the
 //               token tile (cp.async.bulk.tensor 2-D, 128-byte swizzle, no
 //               multicast) for every 64-column k-stage;
 //   warp 1      TMEM allocator and single-thread MMA issuer
 //               (tcgen05.mma.cta_group::1.kind::f16, M=128, N<=256, bf16);
-//   warps 2-5   dequantize: codes -> bf16(c*s) written in the UMMA K-major
+//   warps 2-9   dequantize (one 16-row tile each): codes -> bf16(c*s) in the UMMA K-major
 //               128-byte-swizzle layout;
-//   warps 6-9   epilogue: tcgen05.ld the fp32 accumulators, bias + SwiGLU
+//   warps 10-17 epilogue (two per TMEM lane quarter, alternate 32-column chunks):
+//               tcgen05.ld the fp32 accumulators, bias + SwiGLU
 //               (FC1) or bias (FC2), store.
 // Two TMEM accumulators (2 x 256 columns) let the epilogue of one unit overlap
 // the main loop of the next.
@@ -36,7 +37,10 @@ namespace qmoe {
 constexpr int kGRows = 128;        // UMMA M: weight rows per unit
 constexpr int kGTok = 256;         // UMMA N upper bound: tokens per unit
 constexpr int kGStages = 4;
-constexpr int kGWarps = 10;
+constexpr int kGDeqWarps = 8;     // one 16-row tile of the 128-row unit each
+constexpr int kGDeqTiles = 8 / kGDeqWarps;
+constexpr int kGEpiWarps = 8;     // two per TMEM lane quarter
+constexpr int kGWarps = 2 + kGDeqWarps + kGEpiWarps;
 constexpr int kGThreads = kGWarps * 32;
 constexpr int kGABytes = kGRows * 64 * 2;      // 16 KB bf16 weight tile per k-stage
 constexpr int kGBBytes = kGTok * 64 * 2;       // 32 KB token tile per k-stage
@@ -176,13 +180,13 @@ __global__ void __launch_bounds__(kGThreads, 1)
   if (tid == 0) {
     for (int s = 0; s < kGStages; ++s) {
       mbar_init(&full_c[s], 1);
-      mbar_init(&empty_c[s], 4);
-      mbar_init(&full_ab[s], 1 + 4);
+      mbar_init(&empty_c[s], kGDeqWarps);
+      mbar_init(&full_ab[s], 1 + kGDeqWarps);
       mbar_init(&empty_ab[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tm_full[a], 1);
-      mbar_init(&tm_empty[a], 4);
+      mbar_init(&tm_empty[a], kGEpiWarps);
     }
     mbar_init(mma_done, 1);
     *abort_flag = 0;
@@ -201,31 +205,41 @@ __global__ void __launch_bounds__(kGThreads, 1)
 
   if (warp == 0) {
     // ---------------- producer ----------------
-    if (lane == 0) {
-      uint32_t it = 0;
-      for (int u = blockIdx.x; u < n_units && !*abort_flag; u += gridDim.x) {
-        const GSeg sg = p.gsegs[u / p.rtiles];
-        const int rt = u % p.rtiles;
-        const int nsub = (sg.ntok + kGTmaRows - 1) / kGTmaRows;
-        for (int ks = 0; ks < KS; ++ks, ++it) {
-          const int s = it % kGStages;
-          const uint32_t ph = (it / kGStages) & 1u;
-          if (!gwait(&empty_c[s], ph ^ 1u, p.status, abort_flag)) break;
-          uint8_t* cdst = sC + s * GG::kCStage;
-          mbar_arrive_expect_tx(&full_c[s], GG::kCStage);
+    // The copies of a stage are issued by different lanes in one step (codes:
+    // lane 0, scales: lane 1, token boxes: lanes 2..): a bulk copy costs ~117
+    // cycles to issue from one lane, while the SM accepts one every ~56.
+    uint32_t it = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < n_units && ok && !*abort_flag; u += gridDim.x) {
+      const GSeg sg = p.gsegs[u / p.rtiles];
+      const int rt = u % p.rtiles;
+      const int nsub = (sg.ntok + kGTmaRows - 1) / kGTmaRows;
+      for (int ks = 0; ks < KS; ++ks, ++it) {
+        const int s = it % kGStages;
+        const uint32_t ph = (it / kGStages) & 1u;
+        int w_ok = lane == 0 ? (int)gwait(&empty_c[s], ph ^ 1u, p.status, abort_flag) : 0;
+        if (!__shfl_sync(0xffffffffu, w_ok, 0)) { ok = false; break; }
+        uint8_t* cdst = sC + s * GG::kCStage;
+        if (lane == 0) mbar_arrive_expect_tx(&full_c[s], GG::kCStage);
+        __syncwarp();
+        if (lane == 0)
           bulk_copy_g2s(cdst, p.codes + (unsigned long long)sg.expert * p.codes_stride +
                                   ((unsigned long long)ks * p.NT + rt * 8) * Tr::kCodeBytes,
                         GG::kCodeBytes, &full_c[s]);
+        if (lane == 1) {
           const int sb = ks * 64 / p.block;
           bulk_copy_g2s(cdst + GG::kCodeBytes, p.scales + (unsigned long long)sg.expert * p.scales_stride +
                                                    ((unsigned long long)sb * p.NT + rt * 8) * 32,
                         8 * 32, &full_c[s]);
-          if (!gwait(&empty_ab[s], ph ^ 1u, p.status, abort_flag)) break;
-          mbar_arrive_expect_tx(&full_ab[s], (uint32_t)(nsub * kGTmaRows * 128));
-          for (int sub = 0; sub < nsub; ++sub)
-            tma_load_2d(sB + s * kGBBytes + sub * kGTmaRows * 128, &tmap, ks * 64, sg.slot0 + sub * kGTmaRows,
-                        &full_ab[s]);
         }
+        w_ok = lane == 0 ? (int)gwait(&empty_ab[s], ph ^ 1u, p.status, abort_flag) : 0;
+        if (!__shfl_sync(0xffffffffu, w_ok, 0)) { ok = false; break; }
+        if (lane == 0) mbar_arrive_expect_tx(&full_ab[s], (uint32_t)(nsub * kGTmaRows * 128));
+        __syncwarp();
+        const int sub = lane - 2;
+        if (sub >= 0 && sub < nsub)
+          tma_load_2d(sB + s * kGBBytes + sub * kGTmaRows * 128, &tmap, ks * 64, sg.slot0 + sub * kGTmaRows,
+                      &full_ab[s]);
       }
     }
   } else if (warp == 1) {
@@ -261,7 +275,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
       gwait(mma_done, 0, p.status, abort_flag);
       if (*abort_flag) mbar_wait_bounded(mma_done, 0, nullptr);
     }
-  } else if (warp < 6) {
+  } else if (warp < 2 + kGDeqWarps) {
     // ---------------- dequantize ----------------
     const int d = warp - 2, g = lane >> 2, q = lane & 3;
     uint32_t it = 0;
@@ -271,11 +285,11 @@ __global__ void __launch_bounds__(kGThreads, 1)
         const uint32_t ph = (it / kGStages) & 1u;
         if (!gwait(&full_c[s], ph, p.status, abort_flag)) break;
         const uint8_t* cs = sC + s * GG::kCStage;
-        uint32_t am[2][4][4];
-        uint32_t sw[2];
+        uint32_t am[kGDeqTiles][4][4];
+        uint32_t sw[kGDeqTiles];
 #pragma unroll
-        for (int tt = 0; tt < 2; ++tt) {
-          const int tile = 2 * d + tt;
+        for (int tt = 0; tt < kGDeqTiles; ++tt) {
+          const int tile = kGDeqTiles * d + tt;
           if constexpr (FMT == 2) {
             const uint2 w = *reinterpret_cast<const uint2*>(cs + tile * Tr::kCodeBytes + lane * 8);
             unpack_int2_word(w.x, am[tt][0], am[tt][1]);
@@ -294,8 +308,8 @@ __global__ void __launch_bounds__(kGThreads, 1)
         if (!gwait(&empty_ab[s], ph ^ 1u, p.status, abort_flag)) break;
         uint8_t* as = sA + s * kGABytes;
 #pragma unroll
-        for (int tt = 0; tt < 2; ++tt) {
-          const int tile = 2 * d + tt;
+        for (int tt = 0; tt < kGDeqTiles; ++tt) {
+          const int tile = kGDeqTiles * d + tt;
           const float s_row[2] = {bf16_lo(sw[tt]), bf16_hi(sw[tt])};
 #pragma unroll
           for (int f = 0; f < 4; ++f) {
@@ -321,6 +335,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
   } else {
     // ---------------- epilogue ----------------
     const int quarter = warp & 3;
+    const int half = (warp - 2 - kGDeqWarps) >> 2;  // which alternate 32-column chunks
     const int r = quarter * 32 + lane;  // accumulator lane = tile row
     uint32_t acc_it = 0;
     for (int u = blockIdx.x; u < n_units && !*abort_flag; u += gridDim.x, ++acc_it) {
@@ -346,7 +361,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
       } else if (p.bias) {
         bias_v = bf16_to_f(p.bias[(size_t)sg.expert * p.bias_rows + prow]);
       }
-      for (int c0 = 0; c0 < sg.ntok; c0 += 32) {
+      for (int c0 = 32 * half; c0 < sg.ntok; c0 += 64) {
         uint32_t v[32];
         tmem_ld32(tbase + c0, v);
 #pragma unroll

@@ -545,7 +545,7 @@ qmoe_status qmoe_forward(const qmoe_layer* layer, const uint16_t* x, const float
       uint16_t* xrows = reinterpret_cast<uint16_t*>(base + p.xrows);
       {
         TraceScope ts(st, K_GATHER);
-        gather_rows_kernel<<<std::min(p.max_gseg, 4 * grid), 256, 0, st>>>(xt, L.H, o.slot_token, o.ngseg, o.gsegs,
+        gather_rows_kernel<<<8 * grid, 256, 0, st>>>(xt, L.H, o.slot_token, o.ngseg, o.gsegs,
                                                                             xrows);
         if (cudaGetLastError() != cudaSuccess) return QMOE_ERR_CUDA;
       }
