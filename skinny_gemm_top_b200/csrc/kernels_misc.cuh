@@ -427,23 +427,41 @@ __global__ void gather_rows_kernel(const uint16_t* __restrict__ x, int K, const 
 }
 
 // y[t] = sum_s w[t,s] * yslot[inv[t*k+s]] + sum_j yslot[T*k + j*T + t], fixed order, bf16 out.
+// The token's slot indices and weights are staged in shared memory; slot rows
+// are read 4 at a time so that the loads overlap.
 __global__ void combine_kernel(const float* __restrict__ yslot, const float* __restrict__ w,
                                const int* __restrict__ inv, int T, int k, int n_shared, int H,
                                uint16_t* __restrict__ y) {
+  __shared__ int s_row[32 + 64];
+  __shared__ float s_w[32];
   pdl_wait();
   pdl_trigger();
   const int t = blockIdx.x;
+  for (int i = threadIdx.x; i < k + n_shared; i += blockDim.x) {
+    s_row[i] = i < k ? inv[(size_t)t * k + i] : T * k + (i - k) * T + t;
+    if (i < k) s_w[i] = w[(size_t)t * k + i];
+  }
+  __syncthreads();
+  const int ns = k + n_shared;
   for (int h = threadIdx.x * 4; h < H; h += blockDim.x * 4) {
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int s = 0; s < k; ++s) {
-      const float ws = w[(size_t)t * k + s];
-      const float4 v = *reinterpret_cast<const float4*>(yslot + (size_t)inv[(size_t)t * k + s] * H + h);
-      acc.x = fmaf(ws, v.x, acc.x); acc.y = fmaf(ws, v.y, acc.y);
-      acc.z = fmaf(ws, v.z, acc.z); acc.w = fmaf(ws, v.w, acc.w);
-    }
-    for (int j = 0; j < n_shared; ++j) {
-      const float4 v = *reinterpret_cast<const float4*>(yslot + ((size_t)T * k + (size_t)j * T + t) * H + h);
-      acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+    for (int s0 = 0; s0 < ns; s0 += 4) {
+      float4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (s0 + u < ns) v[u] = *reinterpret_cast<const float4*>(yslot + (size_t)s_row[s0 + u] * H + h);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int s = s0 + u;
+        if (s >= ns) break;
+        if (s < k) {
+          const float ws = s_w[s];
+          acc.x = fmaf(ws, v[u].x, acc.x); acc.y = fmaf(ws, v[u].y, acc.y);
+          acc.z = fmaf(ws, v[u].z, acc.z); acc.w = fmaf(ws, v[u].w, acc.w);
+        } else {
+          acc.x += v[u].x; acc.y += v[u].y; acc.z += v[u].z; acc.w += v[u].w;
+        }
+      }
     }
     uint2 out;
     out.x = pack_bf16x2(acc.x, acc.y);
