@@ -154,6 +154,39 @@ struct Part {
   __device__ __forceinline__ unsigned begin(unsigned c) const { return (c * q + min(c, r)) * unit; }
 };
 
+// This CTA's unit range [f0, f1) (units = tile x k-unit, segment-major).
+// With no more segments than CTAs, every segment gets its own group of
+// CTAs (sizes differ by at most one) and its tiles are split within the
+// group, so no CTA straddles a segment boundary: a CTA range that did would
+// run two sub-panel k-loops.  Otherwise whole tiles are split evenly over
+// the CTAs in segment-major order.
+__device__ __forceinline__ void cta_range(int nseg, int NT, int KU, unsigned& f0, unsigned& f1) {
+  const unsigned G = gridDim.x, c = blockIdx.x;
+  if (nseg > 0 && (unsigned)nseg <= G) {
+    const unsigned cps = G / (unsigned)nseg, rem = G % (unsigned)nseg;
+    // segments [0, rem) have cps + 1 CTAs, the others cps
+    const unsigned big = rem * (cps + 1);
+    unsigned seg, j, n;
+    if (c < big) {
+      seg = c / (cps + 1);
+      j = c - seg * (cps + 1);
+      n = cps + 1;
+    } else {
+      seg = rem + (c - big) / cps;
+      j = (c - big) - (seg - rem) * cps;
+      n = cps;
+    }
+    const unsigned t0 = (unsigned)NT * j / n, t1 = (unsigned)NT * (j + 1) / n;
+    f0 = (seg * (unsigned)NT + t0) * (unsigned)KU;
+    f1 = (seg * (unsigned)NT + t1) * (unsigned)KU;
+    return;
+  }
+  Part part;
+  part.init((unsigned)nseg * (unsigned)NT, G, (unsigned)KU);
+  f0 = part.begin(c);
+  f1 = part.begin(c + 1);
+}
+
 // Sub-panel: up to kMaxT consecutive whole tiles of one segment inside [pos, f1).
 struct SubPanel {
   unsigned next;  // first unit after this sub-panel
@@ -638,10 +671,183 @@ __device__ __forceinline__ void combine_tiles(const SmallParams& p, const Decode
   }
 }
 
+// ---------------------------------------------------------------------------
+// One matmul phase of a small-M kernel on the warps' stage rings.  The rings
+// (barriers, stage buffers, item counters) are kept in a context that could
+// persist across phases of one kernel.
+struct PhaseCtx {
+  uint64_t* wfull;  // this warp's full barriers [NST]
+  uint8_t* wstage;  // this warp's first stage
+  int stride;       // bytes per stage
+  int NST;
+  int item;         // this warp's consumed items
+  int stage;        // item % NST
+  uint32_t phase;   // (item / NST) & 1
+  int issued;       // this warp's issued items
+  int fail_at;      // first item whose wait gave up
+  bool aborted;     // this warp gave up waiting
+  float4* red;
+  const uint32_t* lut;
+  DecodeRoute* R;
+  int* s_abort;
+  int* s_comb;
+};
+
+// Partition, prime (weights, then hook(), then activation rows), stream the
+// items, reduce and run the epilogue.  hook() is called by every thread of
+// the CTA exactly once (also by CTAs without work): the dependency wait, or a
+// grid barrier.
+template <int FMT, int TG, int EPI, int SRC, class Hook>
+__device__ __forceinline__ void run_phase(const SmallParams& p, const SegSource& segs, int nseg, const int* act_index,
+                                          PhaseCtx& cx, Hook&& hook) {
+  using G = StageGeom<FMT, TG>;
+  constexpr int kNW = kWarps<TG>;
+  constexpr int kCT = kNW * 32;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int NST = cx.NST;
+
+  unsigned f0, f1;
+  cta_range(nseg, p.NT, p.KU, f0, f1);
+  if (f0 >= f1) {  // whole CTA idle in this phase
+    hook();
+    return;
+  }
+
+  // Every warp fills its own ring: the weights of its next NST items before
+  // hook(), their activation rows after it.
+  ItemIter prod;
+  int primed = 0;
+  iter_begin<TG>(prod, p, segs, act_index, f0, f1, warp, lane);
+  {
+    ItemIter it = prod;
+    for (int i = 0; i < NST && it.valid; ++i, ++primed) {
+      const int s = (cx.issued + i) % NST;
+      issue_weights<FMT, TG>(p, it, cx.wstage + s * cx.stride, &cx.wfull[s], lane);
+      iter_advance<TG>(it, p, segs, act_index, warp, lane);
+    }
+  }
+  hook();
+  __syncwarp();
+  for (int i = 0; i < primed; ++i) {
+    const int s = (cx.issued + i) % NST;
+    issue_acts<FMT, TG>(p, prod, cx.wstage + s * cx.stride, lane);
+    cp_async_arrive(&cx.wfull[s]);
+    iter_advance<TG>(prod, p, segs, act_index, warp, lane);
+  }
+  cx.issued += primed;
+
+  SubPanel sp;
+  unsigned pos = f0;
+  int cur_seg = -1;
+  Seg sg;
+  while (pos < f1) {
+    load_subpanel(sp, pos, f1, p.NT, p.KU);
+    if (sp.seg != cur_seg) {
+      cur_seg = sp.seg;
+      sg = segs.get(sp.seg);
+      if (sg.tg > TG || sg.tg < 1 || sg.m > 8 * sg.tg) {
+        if (tid == 0) atomicOr(p.status, kStatusBadSegment);
+        sg.tg = TG;
+        sg.m = min(sg.m, 8 * TG);
+      }
+    }
+    const bool tg2 = TG == 2 && sg.tg == 2;
+    float acc[kMaxT][TG][4];
+#pragma unroll
+    for (int i = 0; i < kMaxT; ++i)
+#pragma unroll
+      for (int t = 0; t < TG; ++t)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[i][t][e] = 0.f;
+
+    for (int ku = warp; ku < p.KU; ku += kNW) {
+      const int s = cx.stage;
+      const uint32_t par = cx.phase;
+      ++cx.item;
+      if (++cx.stage == NST) {
+        cx.stage = 0;
+        cx.phase ^= 1u;
+      }
+      if (!cx.aborted && __any_sync(0xffffffffu, !mbar_wait_bounded(&cx.wfull[s], par, p.status))) {
+        cx.aborted = true;
+        cx.fail_at = cx.item - 1;
+        *cx.s_abort = 1;
+      }
+      if (!cx.aborted) {
+        const uint8_t* st = cx.wstage + s * cx.stride;
+        if (sp.nt > 4) compute_item<FMT, TG, 8>(st, tg2, lane, sp.nt, cx.lut, acc);
+        else if (sp.nt > 2) compute_item<FMT, TG, 4>(st, tg2, lane, sp.nt, cx.lut, acc);
+        else if (sp.nt > 1) compute_item<FMT, TG, 2>(st, tg2, lane, sp.nt, cx.lut, acc);
+        else compute_item<FMT, TG, 1>(st, tg2, lane, sp.nt, cx.lut, acc);
+      }
+      __syncwarp();
+      if (prod.valid && !cx.aborted) {
+        uint8_t* st = cx.wstage + s * cx.stride;
+        issue_weights<FMT, TG>(p, prod, st, &cx.wfull[s], lane);
+        issue_acts<FMT, TG>(p, prod, st, lane);
+        cp_async_arrive(&cx.wfull[s]);
+        ++cx.issued;
+        iter_advance<TG>(prod, p, segs, act_index, warp, lane);
+      }
+      __syncwarp();
+    }
+
+    // ---- CTA reduction of the sub-panel, epilogue ----------------------------
+    float4* red = cx.red;
+#pragma unroll
+    for (int i = 0; i < kMaxT; ++i) {
+      if (i >= sp.nt) continue;
+#pragma unroll
+      for (int t = 0; t < TG; ++t)
+        red[((warp * kMaxT + i) * TG + t) * 32 + lane] =
+            make_float4(acc[i][t][0], acc[i][t][1], acc[i][t][2], acc[i][t][3]);
+    }
+    __syncthreads();
+    const bool ab = *cx.s_abort != 0;
+    const int nel = sp.nt * TG * 32;
+#pragma unroll
+    for (int r = 0; r < (kMaxT * TG * 32 + kCT - 1) / kCT; ++r) {
+      const int e = tid + r * kCT;
+      if (e >= nel || ab) continue;
+      float4 v = red[e];
+      for (int w = 1; w < kNW; ++w) {
+        const float4 u = red[w * kMaxT * TG * 32 + e];
+        v.x += u.x; v.y += u.y; v.z += u.z; v.w += u.w;
+      }
+      const int i = e / (TG * 32), t = (e / 32) % TG, ln = e % 32;
+      if (t == 1 && !tg2) continue;
+      epilogue<EPI>(p, sg, sp.rt0 + i, t, ln, v);
+    }
+    if constexpr (SRC == SRC_DECODE && EPI == EPI_FC2) {
+      // fused combine: the CTA that adds an output tile's last segment combines
+      // it.  After the barrier, one acquire-release ticket per tile publishes
+      // this CTA's slot rows and acquires the other CTAs' ones.
+      __syncthreads();
+      if (tid < sp.nt) {
+        const int old = ab ? -1 : atomic_add_acq_rel_gpu(&p.ctick[sp.rt0 + tid], 1);
+        cx.s_comb[tid] = old == nseg - 1;
+        if (old == nseg - 1) p.ctick[sp.rt0 + tid] = 0;  // ready for the next launch
+      }
+      __syncthreads();
+      combine_tiles<kCT>(p, *cx.R, sp.rt0, sp.nt, cx.s_comb);
+    }
+    __syncthreads();
+    pos = sp.next;
+  }
+}
+
+// Drain: if this warp gave up waiting, let its copies in flight land.
+__device__ __forceinline__ void drain_ring(const PhaseCtx& cx, int lane) {
+  if (!cx.aborted) return;
+  cp_async_wait_all();
+  if (lane == 0)
+    for (int j = cx.fail_at; j < cx.issued; ++j)  // issued, unconsumed items: their bulk copies (bounded)
+      mbar_wait_bounded(&cx.wfull[j % cx.NST], (uint32_t)(j / cx.NST) & 1u, nullptr);
+}
+
 template <int FMT, int TG, int EPI, int SRC>
 __global__ void __launch_bounds__(kWarps<TG> * 32, 1) qmm_small_kernel(const SmallParams p) {
   using G = StageGeom<FMT, TG>;
-  constexpr int kNW = kWarps<TG>;
   extern __shared__ __align__(128) uint8_t smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int NST = p.nstages;
@@ -689,164 +895,31 @@ __global__ void __launch_bounds__(kWarps<TG> * 32, 1) qmm_small_kernel(const Sma
     segs.table = p.segs;
   }
 
-  const unsigned ntiles = (unsigned)nseg * (unsigned)p.NT;
-  Part part;
-  part.init(ntiles, gridDim.x, (unsigned)p.KU);
-  const unsigned f0 = part.begin(blockIdx.x), f1 = part.begin(blockIdx.x + 1);
-
-  if (f0 >= f1) {  // whole CTA idle
-    pdl_wait();
-    pdl_trigger();
-    if (SRC == SRC_DECODE && EPI == EPI_SWIGLU && blockIdx.x == 0)
-      for (int i = tid; i < p.H / 16; i += blockDim.x) p.ctick[i] = 0;
-    return;
-  }
-
   if (tid == 0) s_abort = 0;
   if constexpr (FMT == 3)
     for (int i = tid; i < 243; i += blockDim.x) lut[i] = tern_lut_entry(i);
-  uint64_t* wfull = bars + warp * NST;  // [kNW][NST]: the stage's copies landed
-  uint8_t* wstage = stages + (size_t)warp * NST * G::kStageBytes;
+  PhaseCtx cx{};
+  cx.wfull = bars + warp * NST;
+  cx.wstage = stages + (size_t)warp * NST * G::kStageBytes;
+  cx.stride = G::kStageBytes;
+  cx.NST = NST;
+  cx.red = red;
+  cx.lut = lut;
+  cx.R = &R;
+  cx.s_abort = &s_abort;
+  cx.s_comb = s_comb;
   if (lane == 0)
-    for (int s = 0; s < NST; ++s) mbar_init(&wfull[s], 33);
+    for (int s = 0; s < NST; ++s) mbar_init(&cx.wfull[s], 33);
   fence_mbar_init();
   __syncthreads();
 
-  // Every warp fills its own NST-stage ring: the weights of its first NST
-  // items before the dependency wait, their activation rows after it.
-  ItemIter prod;
-  int primed = 0;
-  iter_begin<TG>(prod, p, segs, act_index, f0, f1, warp, lane);
-  {
-    ItemIter it = prod;
-    for (int s = 0; s < NST && it.valid; ++s, ++primed) {
-      issue_weights<FMT, TG>(p, it, wstage + s * G::kStageBytes, &wfull[s], lane);
-      iter_advance<TG>(it, p, segs, act_index, warp, lane);
-    }
-  }
-  pdl_wait();
-  pdl_trigger();
-  if (SRC == SRC_DECODE && EPI == EPI_SWIGLU && blockIdx.x == 0)
-    for (int i = tid; i < p.H / 16; i += blockDim.x) p.ctick[i] = 0;  // for the FC2 launch that follows
-  __syncwarp();
-  for (int s = 0; s < primed; ++s) {
-    issue_acts<FMT, TG>(p, prod, wstage + s * G::kStageBytes, lane);
-    cp_async_arrive(&wfull[s]);
-    iter_advance<TG>(prod, p, segs, act_index, warp, lane);
-  }
-  constexpr int kCT = kNW * 32;
-
-  int item = 0;          // this warp's consumed items
-  int stage = 0;         // item % NST
-  uint32_t phase = 0;    // (item / NST) & 1
-  int issued = primed;   // this warp's issued items
-  int fail_at = 0;       // first item whose wait gave up
-  bool aborted = false;  // this warp gave up waiting
-
-  SubPanel sp;
-  unsigned pos = f0;
-  int cur_seg = -1;
-  Seg sg;
-  while (pos < f1) {
-    load_subpanel(sp, pos, f1, p.NT, p.KU);
-    if (sp.seg != cur_seg) {
-      cur_seg = sp.seg;
-      sg = segs.get(sp.seg);
-      if (sg.tg > TG || sg.tg < 1 || sg.m > 8 * sg.tg) {
-        if (tid == 0) atomicOr(p.status, kStatusBadSegment);
-        sg.tg = TG;
-        sg.m = min(sg.m, 8 * TG);
-      }
-    }
-    const bool tg2 = TG == 2 && sg.tg == 2;
-    float acc[kMaxT][TG][4];
-#pragma unroll
-    for (int i = 0; i < kMaxT; ++i)
-#pragma unroll
-      for (int t = 0; t < TG; ++t)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) acc[i][t][e] = 0.f;
-
-    for (int ku = warp; ku < p.KU; ku += kNW) {
-      const int s = stage;
-      const uint32_t par = phase;
-      ++item;
-      if (++stage == NST) {
-        stage = 0;
-        phase ^= 1u;
-      }
-      if (!aborted && __any_sync(0xffffffffu, !mbar_wait_bounded(&wfull[s], par, p.status))) {
-        aborted = true;
-        fail_at = item - 1;
-        s_abort = 1;
-      }
-      if (!aborted) {
-        const uint8_t* st = wstage + s * G::kStageBytes;
-        if (sp.nt > 4) compute_item<FMT, TG, 8>(st, tg2, lane, sp.nt, lut, acc);
-        else if (sp.nt > 2) compute_item<FMT, TG, 4>(st, tg2, lane, sp.nt, lut, acc);
-        else if (sp.nt > 1) compute_item<FMT, TG, 2>(st, tg2, lane, sp.nt, lut, acc);
-        else compute_item<FMT, TG, 1>(st, tg2, lane, sp.nt, lut, acc);
-      }
-      __syncwarp();
-      if (prod.valid && !aborted) {
-        uint8_t* st = wstage + s * G::kStageBytes;
-        issue_weights<FMT, TG>(p, prod, st, &wfull[s], lane);
-        issue_acts<FMT, TG>(p, prod, st, lane);
-        cp_async_arrive(&wfull[s]);
-        ++issued;
-        iter_advance<TG>(prod, p, segs, act_index, warp, lane);
-      }
-      __syncwarp();
-    }
-
-    // ---- CTA reduction of the sub-panel, epilogue ----------------------------
-#pragma unroll
-    for (int i = 0; i < kMaxT; ++i) {
-      if (i >= sp.nt) continue;
-#pragma unroll
-      for (int t = 0; t < TG; ++t)
-        red[((warp * kMaxT + i) * TG + t) * 32 + lane] =
-            make_float4(acc[i][t][0], acc[i][t][1], acc[i][t][2], acc[i][t][3]);
-    }
-    __syncthreads();
-    const bool ab = s_abort != 0;
-    const int nel = sp.nt * TG * 32;
-#pragma unroll
-    for (int r = 0; r < (kMaxT * TG * 32 + kCT - 1) / kCT; ++r) {
-      const int e = tid + r * kCT;
-      if (e >= nel || ab) continue;
-      float4 v = red[e];
-      for (int w = 1; w < kNW; ++w) {
-        const float4 u = red[w * kMaxT * TG * 32 + e];
-        v.x += u.x; v.y += u.y; v.z += u.z; v.w += u.w;
-      }
-      const int i = e / (TG * 32), t = (e / 32) % TG, ln = e % 32;
-      if (t == 1 && !tg2) continue;
-      epilogue<EPI>(p, sg, sp.rt0 + i, t, ln, v);
-    }
-    if constexpr (SRC == SRC_DECODE && EPI == EPI_FC2) {
-      // fused combine: the CTA that adds an output tile's last segment combines
-      // it.  After the barrier, one acquire-release ticket per tile publishes
-      // this CTA's slot rows and acquires the other CTAs' ones.
-      __syncthreads();
-      if (tid < sp.nt) {
-        const int old = ab ? -1 : atomic_add_acq_rel_gpu(&p.ctick[sp.rt0 + tid], 1);
-        s_comb[tid] = old == nseg - 1;
-        if (old == nseg - 1) p.ctick[sp.rt0 + tid] = 0;  // ready for the next launch
-      }
-      __syncthreads();
-      combine_tiles<kCT>(p, R, sp.rt0, sp.nt, s_comb);
-    }
-    __syncthreads();
-    pos = sp.next;
-  }
-  // Drain: if this warp gave up waiting, let its copies in flight land.
-  if (aborted) {
-    cp_async_wait_all();
-    if (lane == 0)
-      for (int j = fail_at; j < issued; ++j)  // issued, unconsumed items: their bulk copies (bounded)
-        mbar_wait_bounded(&wfull[j % NST], (uint32_t)(j / NST) & 1u, nullptr);
-  }
+  run_phase<FMT, TG, EPI, SRC>(p, segs, nseg, act_index, cx, [&] {
+    pdl_wait();
+    pdl_trigger();
+    if (SRC == SRC_DECODE && EPI == EPI_SWIGLU && blockIdx.x == 0)
+      for (int i = tid; i < p.H / 16; i += blockDim.x) p.ctick[i] = 0;  // for the FC2 launch that follows
+  });
+  drain_ring(cx, lane);
 }
 
 }  // namespace qmoe

@@ -149,6 +149,18 @@ def test_forward_v2lite_full_size(qm, v2lite, T):
     _close(y, ref, f"v2lite T={T}")
 
 
+def test_decode_mixed_formats_and_ternary(qm):
+    """Decode batches with INT2 FC1 / INT4 FC2 (tiny) and with ternary experts,
+    including a segment partition where CTA groups own whole experts."""
+    for cfg, T in ((synth.TINY, 5), (small_cfg(synth.TERNARY, E=16, H=512, I=768), 4)):
+        case = MoECase(cfg, seed=16)
+        x = synth.tokens(cfg.H, 16, T)
+        lg = synth.router_logits(cfg, 16, T)
+        y = case.run(x, lg)
+        ref = Q.moe_forward(Q.bf16_bits_to_f64(x), lg, cfg.k, case.bank)
+        _close(y, ref, f"{cfg.name} decode T={T}")
+
+
 @pytest.mark.parametrize("M", [1, 5, 16, 32])
 def test_forward_v2lite_tokens_per_expert(qm, v2lite, M):
     """M tokens with identical router logits: every selected expert gets exactly M tokens."""
