@@ -45,17 +45,24 @@
 
 namespace qmoe {
 
+enum Epi { EPI_LINEAR = 0, EPI_SWIGLU = 1, EPI_FC2 = 2 };
+enum SegSrc { SRC_TABLE = 0, SRC_DECODE = 1, SRC_LINEAR = 2 };
+
 // Warps per CTA: 12 for one token group (three warps per SM sub-partition
 // hide the unpack/MMA latency better than two), 8 for two token groups, whose
 // accumulators need more than the 168 registers a 12-warp CTA leaves.
 template <int TG>
 constexpr int kWarps = TG == 1 ? 12 : 8;
-constexpr int kMaxT = 8;          // tiles per sub-panel
+constexpr int kMaxT = 10;         // largest sub-panel (tiles)
+// Tiles per sub-panel: 10 for the INT2/INT4 decode and linear kernels (a
+// decode layer's FC1 gives a CTA 9-10 tiles: one k-loop instead of 8 + 1..2;
+// larger items also help the long linears), 8 otherwise (registers, and the
+// larger reduction buffer would cost the general path pipeline stages).
+template <int FMT, int TG, int SRC>
+constexpr int kTiles = (FMT != 3 && TG == 1 && SRC != SRC_TABLE) ? 10 : 8;
 constexpr int kMaxStages = 6;     // stages per consumer warp (barriers: 1024 bytes of shared memory)
 constexpr int kChunkTokens = 16;  // tokens per segment (<= 2 token groups of 8)
 
-enum Epi { EPI_LINEAR = 0, EPI_SWIGLU = 1, EPI_FC2 = 2 };
-enum SegSrc { SRC_TABLE = 0, SRC_DECODE = 1, SRC_LINEAR = 2 };
 
 // Decode batches routed inside the kernels: up to 8 tokens, T*k <= 64,
 // at most 8 shared experts.
@@ -123,17 +130,18 @@ struct SmallParams {
 };
 
 // Stage geometry for a format and token-group count.
-template <int FMT, int TG>
+template <int FMT, int TG, int SRC>
 struct StageGeom {
   using Tr = FmtTraits<FMT>;
   static constexpr int kBlocksPerKU = Tr::kKUcols / 64;                 // 64-col blocks per k-unit
-  static constexpr int kCodeBytes = kMaxT * Tr::kCodeBytes;
-  static constexpr int kScaleBytes = kBlocksPerKU * kMaxT * 32;
+  static constexpr int kMT = kTiles<FMT, TG, SRC>;
+  static constexpr int kCodeBytes = kMT * Tr::kCodeBytes;
+  static constexpr int kScaleBytes = kBlocksPerKU * kMT * 32;
   static constexpr int kActPitch = Tr::kKUcols * 2 + 16;               // padded: conflict-free ldmatrix
   static constexpr int kActBytes = TG * 8 * kActPitch;
   static constexpr int kStageBytes = ((kCodeBytes + kScaleBytes + kActBytes) + 127) / 128 * 128;
   static constexpr int kNW = kWarps<TG>;
-  static constexpr int kRedBytes = kNW * kMaxT * TG * 32 * 16;
+  static constexpr int kRedBytes = kNW * kMT * TG * 32 * 16;
 };
 
 template <int SRC>
@@ -155,14 +163,15 @@ struct Part {
 };
 
 // This CTA's unit range [f0, f1) (units = tile x k-unit, segment-major).
-// With no more segments than CTAs, every segment gets its own group of
+// With at least two CTAs per segment, every segment gets its own group of
 // CTAs (sizes differ by at most one) and its tiles are split within the
 // group, so no CTA straddles a segment boundary: a CTA range that did would
-// run two sub-panel k-loops.  Otherwise whole tiles are split evenly over
-// the CTAs in segment-major order.
+// run two sub-panel k-loops.  With fewer, groups of one or two CTAs would be
+// unbalanced, and whole tiles are split evenly over the CTAs in
+// segment-major order.
 __device__ __forceinline__ void cta_range(int nseg, int NT, int KU, unsigned& f0, unsigned& f1) {
   const unsigned G = gridDim.x, c = blockIdx.x;
-  if (nseg > 0 && (unsigned)nseg <= G) {
+  if (nseg > 0 && 2u * (unsigned)nseg <= G) {
     const unsigned cps = G / (unsigned)nseg, rem = G % (unsigned)nseg;
     // segments [0, rem) have cps + 1 CTAs, the others cps
     const unsigned big = rem * (cps + 1);
@@ -187,13 +196,13 @@ __device__ __forceinline__ void cta_range(int nseg, int NT, int KU, unsigned& f0
   f1 = part.begin(c + 1);
 }
 
-// Sub-panel: up to kMaxT consecutive whole tiles of one segment inside [pos, f1).
+// Sub-panel: up to cap_tiles consecutive whole tiles of one segment inside [pos, f1).
 struct SubPanel {
   unsigned next;  // first unit after this sub-panel
   int seg, rt0, nt;
 };
 
-__device__ __forceinline__ void load_subpanel(SubPanel& sp, unsigned pos, unsigned f1, int NT, int KU) {
+__device__ __forceinline__ void load_subpanel(SubPanel& sp, unsigned pos, unsigned f1, int NT, int KU, int cap_tiles) {
   const unsigned per_seg = (unsigned)NT * (unsigned)KU;
   const unsigned seg = pos / per_seg;
   const unsigned rt = (pos - seg * per_seg) / (unsigned)KU;
@@ -201,7 +210,7 @@ __device__ __forceinline__ void load_subpanel(SubPanel& sp, unsigned pos, unsign
   unsigned end = f1;
   const unsigned seg_end = (seg + 1) * per_seg;
   if (seg_end < end) end = seg_end;
-  const unsigned cap = tile_base + (unsigned)(kMaxT * KU);
+  const unsigned cap = tile_base + (unsigned)(cap_tiles * KU);
   if (cap < end) end = cap;
   sp.next = end;
   sp.seg = (int)seg;
@@ -234,6 +243,7 @@ struct ItemIter {
   unsigned f1;
   int ku;
   int row;     // this lane's activation row (lane < sg.m)
+  int cap;     // tiles per sub-panel
   bool valid;
 };
 
@@ -255,7 +265,7 @@ __device__ __forceinline__ void iter_advance(ItemIter& it, const SmallParams& p,
   for (;;) {
     if (it.sp.next >= it.f1) { it.valid = false; return; }
     const int prev = it.sp.seg;
-    load_subpanel(it.sp, it.sp.next, it.f1, p.NT, p.KU);
+    load_subpanel(it.sp, it.sp.next, it.f1, p.NT, p.KU, it.cap);
     if (it.sp.seg != prev) iter_load_seg<TG>(it, p, segs, act_index, lane);
     it.ku = warp;
     if (it.ku < p.KU) return;
@@ -264,11 +274,12 @@ __device__ __forceinline__ void iter_advance(ItemIter& it, const SmallParams& p,
 
 template <int TG>
 __device__ __forceinline__ void iter_begin(ItemIter& it, const SmallParams& p, const SegSource& segs, const int* act_index,
-                                           unsigned f0, unsigned f1, int warp, int lane) {
+                                           unsigned f0, unsigned f1, int cap, int warp, int lane) {
   it.f1 = f1;
+  it.cap = cap;
   it.valid = f0 < f1;
   if (!it.valid) return;
-  load_subpanel(it.sp, f0, f1, p.NT, p.KU);
+  load_subpanel(it.sp, f0, f1, p.NT, p.KU, cap);
   iter_load_seg<TG>(it, p, segs, act_index, lane);
   it.ku = warp;
   if (it.ku >= p.KU) {
@@ -285,10 +296,10 @@ __device__ __forceinline__ void iter_begin(ItemIter& it, const SmallParams& p, c
 // (lane 0's expect-tx arrival and 32 cp.async arrivals).
 
 // Codes (TMA) and scales (cp.async) of the sub-panel's nt tiles at k-unit ku.
-template <int FMT, int TG>
+template <int FMT, int TG, int SRC>
 __device__ __forceinline__ void issue_weights(const SmallParams& p, const ItemIter& it, uint8_t* stage, uint64_t* bar,
                                               int lane) {
-  using G = StageGeom<FMT, TG>;
+  using G = StageGeom<FMT, TG, SRC>;
   using Tr = FmtTraits<FMT>;
   const int tile = it.sp.rt0, n = it.sp.nt;
   if (lane == 0) {
@@ -305,15 +316,15 @@ __device__ __forceinline__ void issue_weights(const SmallParams& p, const ItemIt
     const int sb = (it.ku * Tr::kKUcols + bl * 64) >> (p.block == 128 ? 7 : 6);  // block is 64 or 128
     const uint8_t* ssrc = p.scales + (unsigned long long)it.sg.expert * p.scales_stride +
                           ((unsigned long long)sb * p.NT + tile) * 32;
-    if (lane < 2 * n) cp_async16(stage + G::kCodeBytes + bl * kMaxT * 32 + 16 * lane, ssrc + 16 * lane);
+    if (lane < 2 * n) cp_async16(stage + G::kCodeBytes + bl * G::kMT * 32 + 16 * lane, ssrc + 16 * lane);
   }
 }
 
 // Activation part of a stage: the k-unit slice of each of the segment's m
 // token rows (the row of token n is held by lane n of the iterator).
-template <int FMT, int TG>
+template <int FMT, int TG, int SRC>
 __device__ __forceinline__ void issue_acts(const SmallParams& p, const ItemIter& it, uint8_t* stage, int lane) {
-  using G = StageGeom<FMT, TG>;
+  using G = StageGeom<FMT, TG, SRC>;
   constexpr int kChunks = FmtTraits<FMT>::kKUcols * 2 / 16;  // 16-byte pieces per row slice
   const int total = it.sg.m * kChunks;
   for (int base = 0; base < total; base += 32) {
@@ -504,11 +515,11 @@ __device__ __forceinline__ void epilogue(const SmallParams& p, const Seg& sg, in
 // at or past nt contribute with scale 0 (their codes are stale but finite),
 // so all NTL tiles run the same straight-line code and the MMAs of a k-step
 // for every tile issue back to back.
-template <int FMT, int TG, int NTL>
+template <int FMT, int TG, int SRC, int NTL>
 __device__ __forceinline__ void compute_item(const uint8_t* st, bool tg2, int lane, int nt, const uint32_t* lut,
-                                             float (&acc)[kMaxT][TG][4]) {
+                                             float (&acc)[kTiles<FMT, TG, SRC>][TG][4]) {
   using Tr = FmtTraits<FMT>;
-  using G = StageGeom<FMT, TG>;
+  using G = StageGeom<FMT, TG, SRC>;
   constexpr int BPK = Tr::kKUcols / 64;
   const uint8_t* cbuf = st;
   const uint32_t* sbuf = reinterpret_cast<const uint32_t*>(st + G::kCodeBytes);
@@ -553,7 +564,7 @@ __device__ __forceinline__ void compute_item(const uint8_t* st, bool tg2, int la
   for (int bl = 0; bl < BPK; ++bl)
 #pragma unroll
     for (int i = 0; i < NTL; ++i) {
-      const uint32_t sc = sbuf[bl * kMaxT * 8 + i * 8 + g];
+      const uint32_t sc = sbuf[bl * G::kMT * 8 + i * 8 + g];
       const bool on = i < nt;
       s_lo[bl][i] = on ? bf16_lo(sc) : 0.f;
       s_hi[bl][i] = on ? bf16_hi(sc) : 0.f;
@@ -700,7 +711,7 @@ struct PhaseCtx {
 template <int FMT, int TG, int EPI, int SRC, class Hook>
 __device__ __forceinline__ void run_phase(const SmallParams& p, const SegSource& segs, int nseg, const int* act_index,
                                           PhaseCtx& cx, Hook&& hook) {
-  using G = StageGeom<FMT, TG>;
+  using G = StageGeom<FMT, TG, SRC>;
   constexpr int kNW = kWarps<TG>;
   constexpr int kCT = kNW * 32;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -717,12 +728,12 @@ __device__ __forceinline__ void run_phase(const SmallParams& p, const SegSource&
   // hook(), their activation rows after it.
   ItemIter prod;
   int primed = 0;
-  iter_begin<TG>(prod, p, segs, act_index, f0, f1, warp, lane);
+  iter_begin<TG>(prod, p, segs, act_index, f0, f1, G::kMT, warp, lane);
   {
     ItemIter it = prod;
     for (int i = 0; i < NST && it.valid; ++i, ++primed) {
       const int s = (cx.issued + i) % NST;
-      issue_weights<FMT, TG>(p, it, cx.wstage + s * cx.stride, &cx.wfull[s], lane);
+      issue_weights<FMT, TG, SRC>(p, it, cx.wstage + s * cx.stride, &cx.wfull[s], lane);
       iter_advance<TG>(it, p, segs, act_index, warp, lane);
     }
   }
@@ -730,7 +741,7 @@ __device__ __forceinline__ void run_phase(const SmallParams& p, const SegSource&
   __syncwarp();
   for (int i = 0; i < primed; ++i) {
     const int s = (cx.issued + i) % NST;
-    issue_acts<FMT, TG>(p, prod, cx.wstage + s * cx.stride, lane);
+    issue_acts<FMT, TG, SRC>(p, prod, cx.wstage + s * cx.stride, lane);
     cp_async_arrive(&cx.wfull[s]);
     iter_advance<TG>(prod, p, segs, act_index, warp, lane);
   }
@@ -741,7 +752,7 @@ __device__ __forceinline__ void run_phase(const SmallParams& p, const SegSource&
   int cur_seg = -1;
   Seg sg;
   while (pos < f1) {
-    load_subpanel(sp, pos, f1, p.NT, p.KU);
+    load_subpanel(sp, pos, f1, p.NT, p.KU, G::kMT);
     if (sp.seg != cur_seg) {
       cur_seg = sp.seg;
       sg = segs.get(sp.seg);
@@ -752,9 +763,9 @@ __device__ __forceinline__ void run_phase(const SmallParams& p, const SegSource&
       }
     }
     const bool tg2 = TG == 2 && sg.tg == 2;
-    float acc[kMaxT][TG][4];
+    float acc[G::kMT][TG][4];
 #pragma unroll
-    for (int i = 0; i < kMaxT; ++i)
+    for (int i = 0; i < G::kMT; ++i)
 #pragma unroll
       for (int t = 0; t < TG; ++t)
 #pragma unroll
@@ -775,16 +786,17 @@ __device__ __forceinline__ void run_phase(const SmallParams& p, const SegSource&
       }
       if (!cx.aborted) {
         const uint8_t* st = cx.wstage + s * cx.stride;
-        if (sp.nt > 4) compute_item<FMT, TG, 8>(st, tg2, lane, sp.nt, cx.lut, acc);
-        else if (sp.nt > 2) compute_item<FMT, TG, 4>(st, tg2, lane, sp.nt, cx.lut, acc);
-        else if (sp.nt > 1) compute_item<FMT, TG, 2>(st, tg2, lane, sp.nt, cx.lut, acc);
-        else compute_item<FMT, TG, 1>(st, tg2, lane, sp.nt, cx.lut, acc);
+        if (G::kMT > 8 && sp.nt > 8) compute_item<FMT, TG, SRC, G::kMT>(st, tg2, lane, sp.nt, cx.lut, acc);
+        else if (sp.nt > 4) compute_item<FMT, TG, SRC, 8>(st, tg2, lane, sp.nt, cx.lut, acc);
+        else if (sp.nt > 2) compute_item<FMT, TG, SRC, 4>(st, tg2, lane, sp.nt, cx.lut, acc);
+        else if (sp.nt > 1) compute_item<FMT, TG, SRC, 2>(st, tg2, lane, sp.nt, cx.lut, acc);
+        else compute_item<FMT, TG, SRC, 1>(st, tg2, lane, sp.nt, cx.lut, acc);
       }
       __syncwarp();
       if (prod.valid && !cx.aborted) {
         uint8_t* st = cx.wstage + s * cx.stride;
-        issue_weights<FMT, TG>(p, prod, st, &cx.wfull[s], lane);
-        issue_acts<FMT, TG>(p, prod, st, lane);
+        issue_weights<FMT, TG, SRC>(p, prod, st, &cx.wfull[s], lane);
+        issue_acts<FMT, TG, SRC>(p, prod, st, lane);
         cp_async_arrive(&cx.wfull[s]);
         ++cx.issued;
         iter_advance<TG>(prod, p, segs, act_index, warp, lane);
@@ -795,23 +807,23 @@ __device__ __forceinline__ void run_phase(const SmallParams& p, const SegSource&
     // ---- CTA reduction of the sub-panel, epilogue ----------------------------
     float4* red = cx.red;
 #pragma unroll
-    for (int i = 0; i < kMaxT; ++i) {
+    for (int i = 0; i < G::kMT; ++i) {
       if (i >= sp.nt) continue;
 #pragma unroll
       for (int t = 0; t < TG; ++t)
-        red[((warp * kMaxT + i) * TG + t) * 32 + lane] =
+        red[((warp * G::kMT + i) * TG + t) * 32 + lane] =
             make_float4(acc[i][t][0], acc[i][t][1], acc[i][t][2], acc[i][t][3]);
     }
     __syncthreads();
     const bool ab = *cx.s_abort != 0;
     const int nel = sp.nt * TG * 32;
 #pragma unroll
-    for (int r = 0; r < (kMaxT * TG * 32 + kCT - 1) / kCT; ++r) {
+    for (int r = 0; r < (G::kMT * TG * 32 + kCT - 1) / kCT; ++r) {
       const int e = tid + r * kCT;
       if (e >= nel || ab) continue;
       float4 v = red[e];
       for (int w = 1; w < kNW; ++w) {
-        const float4 u = red[w * kMaxT * TG * 32 + e];
+        const float4 u = red[w * G::kMT * TG * 32 + e];
         v.x += u.x; v.y += u.y; v.z += u.z; v.w += u.w;
       }
       const int i = e / (TG * 32), t = (e / 32) % TG, ln = e % 32;
@@ -847,7 +859,7 @@ __device__ __forceinline__ void drain_ring(const PhaseCtx& cx, int lane) {
 
 template <int FMT, int TG, int EPI, int SRC>
 __global__ void __launch_bounds__(kWarps<TG> * 32, 1) qmm_small_kernel(const SmallParams p) {
-  using G = StageGeom<FMT, TG>;
+  using G = StageGeom<FMT, TG, SRC>;
   extern __shared__ __align__(128) uint8_t smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int NST = p.nstages;
@@ -855,7 +867,7 @@ __global__ void __launch_bounds__(kWarps<TG> * 32, 1) qmm_small_kernel(const Sma
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem);                          // [kNW][NST]
   uint32_t* lut = reinterpret_cast<uint32_t*>(smem + 1024);                   // 243 entries (ternary)
   DecodeRoute& R = *reinterpret_cast<DecodeRoute*>(smem + 2048);               // SRC_DECODE only
-  float4* red = reinterpret_cast<float4*>(smem + SmemHead<SRC>::kFixed);      // [kNW][kMaxT][TG][32]
+  float4* red = reinterpret_cast<float4*>(smem + SmemHead<SRC>::kFixed);      // [kNW][kMT][TG][32]
   uint8_t* stages = smem + SmemHead<SRC>::kFixed + G::kRedBytes;               // [kNW][NST][stage]
   __shared__ int s_abort;
   __shared__ int s_comb[kMaxT];

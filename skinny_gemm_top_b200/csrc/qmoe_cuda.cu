@@ -218,7 +218,7 @@ qmoe_status encode_rows_map(CUtensorMap* map, const void* base, int K, int rows)
 // ---- small-M kernel launch ----
 template <int FMT, int TG, int EPI, int SRC>
 qmoe_status launch_small_t(SmallParams prm, int grid, cudaStream_t st) {
-  using G = StageGeom<FMT, TG>;
+  using G = StageGeom<FMT, TG, SRC>;
   constexpr int kNW = kWarps<TG>;
   const int fixed = SmemHead<SRC>::kFixed + G::kRedBytes;
   int nst = (kSmemLimit - fixed - 1024) / (kNW * G::kStageBytes);
