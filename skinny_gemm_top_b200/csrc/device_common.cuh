@@ -103,6 +103,49 @@ __device__ __forceinline__ int atomic_add_acq_rel_gpu(int* p, int v) {
   return old;
 }
 
+__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void red_add_release_gpu(int* p, int v) {
+  asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Split barrier over all CTAs of a launch whose CTAs are all resident at once
+// (one per SM).  *count starts the launch at 0 (cleared by the launch before)
+// and is used once.  grid_arrive (every thread, after a CTA barrier that
+// follows the CTA's writes) publishes them; grid_wait (every thread) returns
+// once every CTA has arrived, with all arrived CTAs' writes visible.  Work
+// that needs no other CTA's writes goes between the two.  grid_wait gives up
+// after kWaitLimitNs (status flag) and returns false then, in every thread.
+__device__ __forceinline__ void grid_arrive(int* count) {
+  if (threadIdx.x == 0) red_add_release_gpu(count, 1);  // cumulative: covers the writes the CTA barrier ordered
+}
+
+__device__ __forceinline__ bool grid_wait(const int* count, unsigned* status, int* s_ok) {
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int ok = 1;
+    const int n = (int)gridDim.x;
+    if (ld_acquire_gpu(count) < n) {
+      const unsigned long long t0 = global_timer_ns();
+      for (uint32_t it = 1;; ++it) {
+        if (ld_acquire_gpu(count) >= n) break;
+        if ((it & 63) == 0 && global_timer_ns() - t0 > kWaitLimitNs) {
+          atomicOr(status, kStatusTimeout);
+          ok = 0;
+          break;
+        }
+      }
+    }
+    *s_ok = ok;
+  }
+  __syncthreads();
+  return *s_ok != 0;
+}
+
 // D (+)= A * B, m16n8k16, bf16 inputs, fp32 accumulators.
 __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
   asm volatile(

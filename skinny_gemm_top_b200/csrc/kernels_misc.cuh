@@ -394,6 +394,17 @@ __global__ void __launch_bounds__(kRouteWarps * 32)
 // Token rows of the grouped tiles, in expert-sorted slot order: xrows[slot] =
 // x[token(slot)].  One warp per row (grid-stride over gseg x 256 row slots):
 // each lane moves K/256 16-byte pieces with its loads issued before its stores.
+// Clears the grid-barrier count and the combine tickets of the fused decode
+// launch that follows.  It lets that launch start at once (its CTAs wait for
+// this kernel's completion at their first instruction, so they see the
+// cleared words), then waits for the launch before, which may still use them.
+__global__ void decode_reset_kernel(int* gbar, int* ctick, int n) {
+  pdl_trigger();
+  pdl_wait();
+  for (int i = threadIdx.x; i < n; i += blockDim.x) ctick[i] = 0;
+  if (threadIdx.x == 0) *gbar = 0;
+}
+
 __global__ void gather_rows_kernel(const uint16_t* __restrict__ x, int K, const int* __restrict__ slot_token,
                                    const int* __restrict__ ngseg, const GSeg* __restrict__ gsegs, uint16_t* xrows) {
   pdl_wait();

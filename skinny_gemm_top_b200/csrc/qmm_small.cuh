@@ -89,11 +89,10 @@ struct DecodeRoute {
   int pos[kDecMaxTK];            // flat index t*k+s -> slot
   float w[kDecMaxTK];            // router weight of flat index
   int ids[kDecMaxTK];            // expert of flat index
-  int less[kDecMaxTK];           // entries routed to a lower expert
-  int cnt[kDecMaxTK];            // entries routed to the same expert
-  int first[kDecMaxTK];          // entry is its expert's first in flat order
-  float selv[kDecMaxT][32];      // selected logits in selection order
+  int hist[kMaxExperts];         // scratch: entries per expert, then their exclusive prefix
 };
+// The part of DecodeRoute that FC2 reads (the scratch at the end is not copied).
+constexpr int kDecodeRouteWords = (int)(offsetof(DecodeRoute, hist) / 4);
 
 struct SmallParams {
   const uint8_t* codes;
@@ -295,17 +294,26 @@ __device__ __forceinline__ void iter_begin(ItemIter& it, const SmallParams& p, c
 // arriving on the barrier once its copies landed.  Full barrier count: 33
 // (lane 0's expect-tx arrival and 32 cp.async arrivals).
 
-// Codes (TMA) and scales (cp.async) of the sub-panel's nt tiles at k-unit ku.
+// Codes and scales (cp.async) of the sub-panel's nt tiles at k-unit ku.  The
+// codes go through the TMA engine (one bulk copy by lane 0), or, with lsu,
+// through the load/store unit as 16-byte cp.async by every lane: a CTA's
+// first stages are requested by all warps at once, and the TMA engine takes
+// them one copy at a time (tens of cycles each), while the load/store units
+// of the four sub-partitions take them in parallel.  Either way lane 0
+// arrives once on the barrier (with the expected bytes of the bulk copy).
 template <int FMT, int TG, int SRC>
 __device__ __forceinline__ void issue_weights(const SmallParams& p, const ItemIter& it, uint8_t* stage, uint64_t* bar,
-                                              int lane) {
+                                              int lane, bool lsu = false) {
   using G = StageGeom<FMT, TG, SRC>;
   using Tr = FmtTraits<FMT>;
   const int tile = it.sp.rt0, n = it.sp.nt;
-  if (lane == 0) {
-    const uint8_t* csrc = p.codes + (unsigned long long)it.sg.expert * p.codes_stride +
-                          ((unsigned long long)it.ku * p.NT + tile) * Tr::kCodeBytes;
-    const uint32_t bytes = (uint32_t)(n * Tr::kCodeBytes);
+  const uint8_t* csrc = p.codes + (unsigned long long)it.sg.expert * p.codes_stride +
+                        ((unsigned long long)it.ku * p.NT + tile) * Tr::kCodeBytes;
+  const uint32_t bytes = (uint32_t)(n * Tr::kCodeBytes);
+  if (lsu) {
+    for (uint32_t o = 16u * lane; o < bytes; o += 512u) cp_async16(stage + o, csrc + o);
+    if (lane == 0) mbar_arrive(bar);
+  } else if (lane == 0) {
     // No proxy fence: the warp's reads of this stage were consumed by its MMAs
     // before the refill is issued.
     mbar_arrive_expect_tx(bar, bytes);
@@ -365,27 +373,41 @@ __device__ __forceinline__ uint32_t logit_key(float v) {
   return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
 }
 
+// The logit of a key (inverse of logit_key up to the sign of zero; NaN stays NaN).
+__device__ __forceinline__ float logit_of_key(uint32_t key) {
+  return __uint_as_float((key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key);
+}
+
+// Routing in warp-level steps, every one a register, shuffle or
+// shared-memory operation, so that the dependency chain stays short:
+//  1. warp t < T: k rounds of a warp arg-max over token t's logits; lane s
+//     keeps selection s; softmax over the selected logits in selection order.
+//  2. T = 1 (warp 0 goes on without a CTA barrier): the k experts are
+//     distinct; the slot and the segment of selection s are the rank of its
+//     expert among them.
+//     T > 1 (warp 0, after a CTA barrier): per expert, the mask of the tokens
+//     that selected it (shared-memory atomic OR: the same result in every CTA
+//     whatever the order); an entry's rank within its expert is the count of
+//     earlier tokens in the mask; a warp scan over the experts gives each
+//     entry the entries at lower experts (its slot base) and its expert's
+//     rank among the selected ones (its segment).
 __device__ void decode_route(const SmallParams& p, DecodeRoute& R) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int T = p.T, E = p.E, k = p.k, TK = T * k;
   constexpr int V = kMaxExperts / 32;
+  int nsel = k;  // selected experts (warp 0)
   if (warp < T) {
-    // warp t selects token t's experts: k rounds of a warp arg-max over
-    // (key desc, index asc); lane holds experts lane + 32j.
-    float v[V];
-    uint32_t key[V];
+    uint32_t key[V];  // lane holds experts lane + 32j
     unsigned live = 0;
 #pragma unroll
     for (int j = 0; j < V; ++j) {
       const int idx = lane + 32 * j;
-      v[j] = idx < E ? p.logits[(size_t)warp * E + idx] : 0.f;
+      key[j] = idx < E ? logit_key(p.logits[(size_t)warp * E + idx]) : 0u;
+      if (idx < E) live |= 1u << j;
     }
-#pragma unroll
-    for (int j = 0; j < V; ++j) {
-      key[j] = logit_key(v[j]);
-      if (lane + 32 * j < E) live |= 1u << j;
-    }
-    for (int s = 0; s < k; ++s) {
+    int my_id = 0;
+    float my_v = 0.f;
+    for (int s = 0; s < k; ++s) {  // (key desc, index asc)
       uint32_t bk = 0;
       int bj = -1;
 #pragma unroll
@@ -393,68 +415,106 @@ __device__ void decode_route(const SmallParams& p, DecodeRoute& R) {
         if (((live >> j) & 1u) && (bj < 0 || key[j] > bk)) { bk = key[j]; bj = j; }
       const uint32_t mk = __reduce_max_sync(0xffffffffu, bj >= 0 ? bk : 0u);
       const int win = __reduce_min_sync(0xffffffffu, (bj >= 0 && bk == mk) ? lane + 32 * bj : INT_MAX);
-      if ((win & 31) == lane) {
-        live &= ~(1u << (win >> 5));
-        float wv = 0.f;
-#pragma unroll
-        for (int j = 0; j < V; ++j)
-          if (j == (win >> 5)) wv = v[j];
-        R.ids[warp * k + s] = win;
-        R.selv[warp][s] = wv;
+      if ((win & 31) == lane) live &= ~(1u << (win >> 5));
+      if (lane == s) {
+        my_id = win;
+        my_v = logit_of_key(mk);
       }
     }
-    __syncwarp();
+    const float ex = expf(my_v - __shfl_sync(0xffffffffu, my_v, 0));
+    float sum = 0.f;
+    for (int s = 0; s < k; ++s) sum += __shfl_sync(0xffffffffu, ex, s);
     if (lane < k) {
-      const float lmax = R.selv[warp][0];
-      float sum = 0.f;
-      for (int s = 0; s < k; ++s) sum += expf(R.selv[warp][s] - lmax);
-      R.w[warp * k + lane] = expf(R.selv[warp][lane] - lmax) / sum;
+      R.ids[warp * k + lane] = my_id;
+      R.w[warp * k + lane] = ex / sum;
+    }
+    if (T == 1) {
+      int rank = 0;
+      for (int j = 0; j < k; ++j) rank += __shfl_sync(0xffffffffu, my_id, j) < my_id;
+      if (lane < k) {
+        R.pos[lane] = rank;
+        R.slot_token[rank] = 0;
+        Seg sg;
+        sg.expert = my_id;
+        sg.m = 1;
+        sg.tg = 1;
+        sg.slot0 = rank;
+        R.segs[rank] = sg;
+      }
     }
   }
-  __syncthreads();
-  // slot of entry i = entries with a lower expert + earlier entries with the same expert
-  int nfirst_local = 0;
-  for (int i = tid; i < TK; i += blockDim.x) {
-    const int e = R.ids[i];
-    int less = 0, before = 0, cnt = 0;
-    for (int j = 0; j < TK; ++j) {
-      const int f = R.ids[j];
-      less += f < e;
-      cnt += f == e;
-      before += (f == e) & (j < i);
+  if (T > 1) {
+    __syncthreads();
+    if (warp == 0) {
+      int* hist = R.hist;  // per expert: the mask of the tokens that selected it
+      const int nb = (E + 31) / 32;  // experts per lane in the scan
+      for (int b = lane; b < E; b += 32) hist[b] = 0;
+      __syncwarp();
+      const int i0 = lane, i1 = lane + 32;
+      const int e0 = i0 < TK ? R.ids[i0] : -1, e1 = i1 < TK ? R.ids[i1] : -1;
+      const int t0 = i0 / k, t1 = i1 / k;
+      if (e0 >= 0) atomicOr(&hist[e0], 1 << t0);
+      if (e1 >= 0) atomicOr(&hist[e1], 1 << t1);
+      __syncwarp();
+      const int mk0 = e0 >= 0 ? hist[e0] : 0, mk1 = e1 >= 0 ? hist[e1] : 0;
+      const int before0 = __popc(mk0 & ((1 << t0) - 1)), before1 = __popc(mk1 & ((1 << t1) - 1));
+      const int cnt0 = __popc(mk0), cnt1 = __popc(mk1);
+      int loc[V];
+      int run = 0;  // (entries) | (selected experts) << 16 over this lane's experts
+#pragma unroll
+      for (int q = 0; q < V; ++q) {
+        const int b = lane * nb + q;
+        loc[q] = (q < nb && b < E) ? __popc(hist[b]) : 0;
+        run += loc[q] | ((loc[q] > 0) << 16);
+      }
+      __syncwarp();
+      int inc = run;
+#pragma unroll
+      for (int d = 1; d < 32; d <<= 1) {
+        const int u = __shfl_up_sync(0xffffffffu, inc, d);
+        if (lane >= d) inc += u;
+      }
+      __syncwarp();
+      int ex = inc - run;
+#pragma unroll
+      for (int q = 0; q < V; ++q) {
+        const int b = lane * nb + q;
+        if (q < nb && b < E) hist[b] = ex;
+        ex += loc[q] | ((loc[q] > 0) << 16);
+      }
+      __syncwarp();
+      const int is[2] = {i0, i1}, es[2] = {e0, e1}, bs[2] = {before0, before1}, cs[2] = {cnt0, cnt1};
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        if (is[h] >= TK) continue;
+        const int pre = hist[es[h]], less = pre & 0xFFFF;
+        const int pos = less + bs[h];
+        R.pos[is[h]] = pos;
+        R.slot_token[pos] = is[h] / k;
+        if (bs[h] == 0) {
+          Seg sg;
+          sg.expert = es[h];
+          sg.m = cs[h];
+          sg.tg = (sg.m + 7) / 8;
+          sg.slot0 = less;
+          R.segs[pre >> 16] = sg;
+        }
+      }
+      nsel = __shfl_sync(0xffffffffu, inc, 31) >> 16;
     }
-    const int pos = less + before;
-    R.pos[i] = pos;
-    R.slot_token[pos] = i / k;
-    R.less[i] = less;
-    R.cnt[i] = cnt;
-    R.first[i] = before == 0;
-    nfirst_local += before == 0;
   }
-  for (int i = tid; i < p.n_shared * T; i += blockDim.x) R.slot_token[TK + i] = i % T;
-  // one segment per distinct expert, at the rank of its expert among them
-  const int nfirst = __syncthreads_count(nfirst_local);  // a thread holds at most one entry (TK < blockDim)
-  for (int i = tid; i < TK; i += blockDim.x) {
-    if (!R.first[i]) continue;
-    const int e = R.ids[i];
-    int idx = 0;
-    for (int j = 0; j < TK; ++j) idx += R.first[j] & (R.ids[j] < e);
-    Seg sg;
-    sg.expert = e;
-    sg.m = R.cnt[i];
-    sg.tg = (sg.m + 7) / 8;
-    sg.slot0 = R.less[i];
-    R.segs[idx] = sg;
+  if (warp == 0) {  // shared experts: one segment each (all T tokens), after the routed slots
+    if (lane < p.n_shared) {
+      Seg sg;
+      sg.expert = E + lane;
+      sg.m = T;
+      sg.tg = (T + 7) / 8;
+      sg.slot0 = TK + lane * T;
+      R.segs[nsel + lane] = sg;
+    }
+    for (int i = lane; i < p.n_shared * T; i += 32) R.slot_token[TK + i] = i % T;
+    if (lane == 0) R.nseg = nsel + p.n_shared;
   }
-  if (tid < p.n_shared) {
-    Seg sg;
-    sg.expert = E + tid;
-    sg.m = T;
-    sg.tg = (T + 7) / 8;
-    sg.slot0 = TK + tid * T;
-    R.segs[nfirst + tid] = sg;
-  }
-  if (tid == 0) R.nseg = nfirst + p.n_shared;
   __syncthreads();
 }
 
@@ -646,37 +706,34 @@ __device__ __forceinline__ void compute_item(const uint8_t* st, bool tg2, int la
   }
 }
 
-// Decode FC2: router-weighted combine of output rows [16 rt, 16 rt + 16) over
-// all tokens, once every segment has written them.
 // Router-weighted combine of the output tiles flagged in comb[0..nt) (tiles
-// rt0 + i): y[t][r] = sum_s w[t][s] * yslot[pos(t,s)][r] + sum_j yslot[shared j, t][r].
-// Slot rows are read in batches of 8 so that the loads overlap.
+// rt0 + i): y[t][r] = sum_s w[t][s] * yslot[pos(t,s)][r] + sum_j yslot[shared j, t][r],
+// routed slots first, in slot order.  The k + n_shared slot rows of an output
+// are read in batches of 8 (one batch for k + n_shared <= 8), so that the
+// loads overlap.
 template <int NTHR>
 __device__ __forceinline__ void combine_tiles(const SmallParams& p, const DecodeRoute& R, int rt0, int nt,
                                               const int* comb) {
-  const int TK = p.T * p.k, per = p.T * 16;
+  const int k = p.k, TK = p.T * k, per = p.T * 16, ns = k + p.n_shared;
   for (int e = threadIdx.x; e < nt * per; e += NTHR) {
     const int i = e / per;
     if (!comb[i]) continue;
     const int t = (e - i * per) >> 4, r = (rt0 + i) * 16 + (e & 15);
     float acc = 0.f;
-    for (int s0 = 0; s0 < p.k; s0 += 8) {
+    for (int s0 = 0; s0 < ns; s0 += 8) {
       float v[8];
 #pragma unroll
-      for (int u = 0; u < 8; ++u)
-        v[u] = s0 + u < p.k ? __ldcg(p.yslot + (size_t)R.pos[t * p.k + s0 + u] * p.H + r) : 0.f;
+      for (int u = 0; u < 8; ++u) {
+        const int sl = s0 + u;
+        const int row = sl < k ? R.pos[t * k + sl] : TK + (sl - k) * p.T + t;
+        v[u] = sl < ns ? __ldcg(p.yslot + (size_t)row * p.H + r) : 0.f;
+      }
 #pragma unroll
-      for (int u = 0; u < 8; ++u)
-        if (s0 + u < p.k) acc = fmaf(R.w[t * p.k + s0 + u], v[u], acc);
-    }
-    for (int j0 = 0; j0 < p.n_shared; j0 += 8) {
-      float v[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u)
-        v[u] = j0 + u < p.n_shared ? __ldcg(p.yslot + (size_t)(TK + (j0 + u) * p.T + t) * p.H + r) : 0.f;
-#pragma unroll
-      for (int u = 0; u < 8; ++u)
-        if (j0 + u < p.n_shared) acc += v[u];
+      for (int u = 0; u < 8; ++u) {
+        const int sl = s0 + u;
+        if (sl < k) acc = fmaf(R.w[t * k + sl], v[u], acc);
+        else if (sl < ns) acc += v[u];
+      }
     }
     p.y[(size_t)t * p.H + r] = __bfloat16_as_ushort(__float2bfloat16_rn(acc));
   }
@@ -731,7 +788,7 @@ __device__ __forceinline__ void run_phase(const SmallParams& p, const SegSource&
   iter_begin<TG>(prod, p, segs, act_index, f0, f1, G::kMT, warp, lane);
   {
     ItemIter it = prod;
-    for (int i = 0; i < NST && it.valid; ++i, ++primed) {
+    for (int i = 0; i < NST && it.valid && !cx.aborted; ++i, ++primed) {  // (a warp that gave up issues nothing)
       const int s = (cx.issued + i) % NST;
       issue_weights<FMT, TG, SRC>(p, it, cx.wstage + s * cx.stride, &cx.wfull[s], lane);
       iter_advance<TG>(it, p, segs, act_index, warp, lane);
@@ -857,18 +914,54 @@ __device__ __forceinline__ void drain_ring(const PhaseCtx& cx, int lane) {
       mbar_wait_bounded(&cx.wfull[j % cx.NST], (uint32_t)(j / cx.NST) & 1u, nullptr);
 }
 
+// Shared-memory layout of a small-M kernel and the rings' context.
+template <int FMT, int TG, int SRC>
+struct SmallSmem {
+  uint64_t* bars;  // [kNW][NST] full barriers
+  uint32_t* lut;   // 243 entries (ternary)
+  DecodeRoute* R;  // SRC_DECODE only
+  float4* red;     // [kNW][kMT][TG][32]
+  uint8_t* stages; // [kNW][NST][stage]
+  __device__ __forceinline__ explicit SmallSmem(uint8_t* smem) {
+    bars = reinterpret_cast<uint64_t*>(smem);
+    lut = reinterpret_cast<uint32_t*>(smem + 1024);
+    R = reinterpret_cast<DecodeRoute*>(smem + 2048);
+    red = reinterpret_cast<float4*>(smem + SmemHead<SRC>::kFixed);
+    stages = smem + SmemHead<SRC>::kFixed + StageGeom<FMT, TG, SRC>::kRedBytes;
+  }
+};
+
+// Ternary table, ring barriers and the phase context (ends with a CTA barrier).
+template <int FMT, int TG, int SRC>
+__device__ __forceinline__ void init_rings(const SmallSmem<FMT, TG, SRC>& sm, int NST, int* s_abort, int* s_comb,
+                                           PhaseCtx& cx) {
+  using G = StageGeom<FMT, TG, SRC>;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (tid == 0) *s_abort = 0;
+  if constexpr (FMT == 3)
+    for (int i = tid; i < 243; i += blockDim.x) sm.lut[i] = tern_lut_entry(i);
+  cx = PhaseCtx{};
+  cx.wfull = sm.bars + warp * NST;
+  cx.wstage = sm.stages + (size_t)warp * NST * G::kStageBytes;
+  cx.stride = G::kStageBytes;
+  cx.NST = NST;
+  cx.red = sm.red;
+  cx.lut = sm.lut;
+  cx.R = sm.R;
+  cx.s_abort = s_abort;
+  cx.s_comb = s_comb;
+  if (lane == 0)
+    for (int s = 0; s < NST; ++s) mbar_init(&cx.wfull[s], 33);
+  fence_mbar_init();
+  __syncthreads();
+}
+
 template <int FMT, int TG, int EPI, int SRC>
 __global__ void __launch_bounds__(kWarps<TG> * 32, 1) qmm_small_kernel(const SmallParams p) {
-  using G = StageGeom<FMT, TG, SRC>;
   extern __shared__ __align__(128) uint8_t smem[];
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int NST = p.nstages;
-
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem);                          // [kNW][NST]
-  uint32_t* lut = reinterpret_cast<uint32_t*>(smem + 1024);                   // 243 entries (ternary)
-  DecodeRoute& R = *reinterpret_cast<DecodeRoute*>(smem + 2048);               // SRC_DECODE only
-  float4* red = reinterpret_cast<float4*>(smem + SmemHead<SRC>::kFixed);      // [kNW][kMT][TG][32]
-  uint8_t* stages = smem + SmemHead<SRC>::kFixed + G::kRedBytes;               // [kNW][NST][stage]
+  const int tid = threadIdx.x, lane = tid & 31;
+  const SmallSmem<FMT, TG, SRC> sm(smem);
+  DecodeRoute& R = *sm.R;
   __shared__ int s_abort;
   __shared__ int s_comb[kMaxT];
 
@@ -887,14 +980,14 @@ __global__ void __launch_bounds__(kWarps<TG> * 32, 1) qmm_small_kernel(const Sma
       // the routing of this call, from the FC1 launch just before (after the wait)
       const uint32_t* src = reinterpret_cast<const uint32_t*>(p.route_tab);
       uint32_t* dst = reinterpret_cast<uint32_t*>(&R);
-      for (int i = tid; i < (int)(sizeof(DecodeRoute) / 4); i += blockDim.x) dst[i] = __ldcg(src + i);
+      for (int i = tid; i < kDecodeRouteWords; i += blockDim.x) dst[i] = __ldcg(src + i);
       __syncthreads();
     } else {
       decode_route(p, R);
       if (blockIdx.x == 0) {  // for the FC2 launch of this call
         const uint32_t* src = reinterpret_cast<const uint32_t*>(&R);
         uint32_t* dst = reinterpret_cast<uint32_t*>(p.route_tab);
-        for (int i = tid; i < (int)(sizeof(DecodeRoute) / 4); i += blockDim.x) dst[i] = src[i];
+        for (int i = tid; i < kDecodeRouteWords; i += blockDim.x) dst[i] = src[i];
       }
     }
     nseg = R.nseg;
@@ -907,29 +1000,50 @@ __global__ void __launch_bounds__(kWarps<TG> * 32, 1) qmm_small_kernel(const Sma
     segs.table = p.segs;
   }
 
-  if (tid == 0) s_abort = 0;
-  if constexpr (FMT == 3)
-    for (int i = tid; i < 243; i += blockDim.x) lut[i] = tern_lut_entry(i);
-  PhaseCtx cx{};
-  cx.wfull = bars + warp * NST;
-  cx.wstage = stages + (size_t)warp * NST * G::kStageBytes;
-  cx.stride = G::kStageBytes;
-  cx.NST = NST;
-  cx.red = red;
-  cx.lut = lut;
-  cx.R = &R;
-  cx.s_abort = &s_abort;
-  cx.s_comb = s_comb;
-  if (lane == 0)
-    for (int s = 0; s < NST; ++s) mbar_init(&cx.wfull[s], 33);
-  fence_mbar_init();
-  __syncthreads();
+  PhaseCtx cx;
+  init_rings<FMT, TG, SRC>(sm, p.nstages, &s_abort, s_comb, cx);
 
   run_phase<FMT, TG, EPI, SRC>(p, segs, nseg, act_index, cx, [&] {
     pdl_wait();
     pdl_trigger();
     if (SRC == SRC_DECODE && EPI == EPI_SWIGLU && blockIdx.x == 0)
       for (int i = tid; i < p.H / 16; i += blockDim.x) p.ctick[i] = 0;  // for the FC2 launch that follows
+  });
+  drain_ring(cx, lane);
+}
+
+// ---------------------------------------------------------------------------
+// A whole decode layer (T <= 8, FC1 and FC2 in one format) in one launch of
+// one CTA per SM: routing in the prologue, the FC1 phase, then the FC2 phase
+// on the same rings with the fused combine.  A split grid barrier (every CTA
+// resident) orders all of h before FC2's activation copies: a CTA arrives as
+// soon as its rows of h are written, requests FC2's first stages of weights,
+// and only then waits.  The launch before (decode_reset_kernel) cleared the
+// barrier count and the combine tickets.
+template <int FMT>
+__global__ void __launch_bounds__(kWarps<1> * 32, 1)
+    qmm_decode_kernel(const SmallParams p1, const SmallParams p2, int* gbar) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int lane = threadIdx.x & 31;
+  const SmallSmem<FMT, 1, SRC_DECODE> sm(smem);
+  DecodeRoute& R = *sm.R;
+  __shared__ int s_abort;
+  __shared__ int s_comb[kMaxT];
+  __shared__ int s_bar_ok;
+
+  pdl_wait();  // logits and x from the launches before; cleared barrier and tickets
+  decode_route(p1, R);
+  const int nseg = R.nseg;
+  SegSource segs;
+  segs.table = R.segs;
+  segs.rows = p1.T;
+  PhaseCtx cx;
+  init_rings<FMT, 1, SRC_DECODE>(sm, p1.nstages, &s_abort, s_comb, cx);
+
+  run_phase<FMT, 1, EPI_SWIGLU, SRC_DECODE>(p1, segs, nseg, R.slot_token, cx, [] { pdl_trigger(); });
+  grid_arrive(gbar);  // this CTA's rows of h are written (run_phase ends with a CTA barrier)
+  run_phase<FMT, 1, EPI_FC2, SRC_DECODE>(p2, segs, nseg, nullptr, cx, [&] {
+    if (!grid_wait(gbar, p2.status, &s_bar_ok) && threadIdx.x == 0) s_abort = 1;  // h incomplete: no epilogue
   });
   drain_ring(cx, lane);
 }

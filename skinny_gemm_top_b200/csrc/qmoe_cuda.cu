@@ -59,9 +59,10 @@ qmoe_status dev_info(DevInfo** out) {
 
 // ---- tracing: CUDA events around each kernel launch ----
 enum KernelId { K_ROUTE = 0, K_GATHER, K_FC1_SMALL, K_FC2_SMALL, K_COMBINE, K_LINEAR_SMALL, K_LINEAR_SETUP,
-                K_DEQUANT, K_FC1_GROUPED, K_FC2_GROUPED, K_COUNT };
-const char* const kKernelNames[K_COUNT] = {"route", "gather", "fc1_small", "fc2_small", "combine", "linear_small",
-                                           "linear_setup", "dequant", "fc1_grouped", "fc2_grouped"};
+                K_DEQUANT, K_FC1_GROUPED, K_FC2_GROUPED, K_DECODE_RESET, K_DECODE_LAYER, K_COUNT };
+const char* const kKernelNames[K_COUNT] = {"route",        "gather",      "fc1_small",   "fc2_small",
+                                           "combine",      "linear_small", "linear_setup", "dequant",
+                                           "fc1_grouped",  "fc2_grouped", "decode_reset", "decode_layer"};
 struct Tracer {
   bool on = false;
   int cap = 0, n = 0;
@@ -136,8 +137,8 @@ qmoe_status check_weights(const qmoe_weights& w, int rows, int K) {
 struct MoEPlan {
   int T, S, TK, max_seg, n_tickets, max_gseg;
   bool grouped, decode;
-  size_t ids, w, perm, inv, offsets, slot_token, nseg, segs, chunk_counts, yslot, hrows, ctick, route, ngseg, gsegs,
-      xrows, total;
+  size_t ids, w, perm, inv, offsets, slot_token, nseg, segs, chunk_counts, yslot, hrows, ctick, route, gbar, ngseg,
+      gsegs, xrows, total;
 };
 
 constexpr int kGroupedThreshold = 32;  // AUTO: experts with more tokens take the tcgen05 path
@@ -152,7 +153,9 @@ int grouped_threshold(const qmoe_layer& L) {
   return L.path == QMOE_PATH_GROUPED ? 0 : kGroupedThreshold;
 }
 
-// Decode batches route inside the expert kernels (two launches per layer).
+// Decode batches route inside the expert kernels: one fused launch per layer
+// (after a tiny reset launch), or two expert launches when FC1 and FC2 differ
+// in format.
 bool decode_eligible(const qmoe_layer& L, int T) {
   return T <= kDecMaxT && T * L.k <= kDecMaxTK && L.n_shared <= kDecMaxShared && T <= grouped_threshold(L);
 }
@@ -171,7 +174,10 @@ MoEPlan plan_moe(const qmoe_layer& L, int T, int grid) {
   p.yslot = take((size_t)p.S * L.H * 4);
   p.hrows = take((size_t)p.S * L.I * 2 + 16);
   p.ctick = take((size_t)(L.H / 16) * 4);
-  if (p.decode) p.route = take(sizeof(DecodeRoute));
+  if (p.decode) {
+    p.route = take(sizeof(DecodeRoute));
+    p.gbar = take(16);
+  }
   if (!p.decode) {
     p.ids = take((size_t)p.TK * 4);
     p.w = take((size_t)p.TK * 4);
@@ -216,16 +222,25 @@ qmoe_status encode_rows_map(CUtensorMap* map, const void* base, int K, int rows)
 }
 
 // ---- small-M kernel launch ----
-template <int FMT, int TG, int EPI, int SRC>
-qmoe_status launch_small_t(SmallParams prm, int grid, cudaStream_t st) {
+// Dynamic shared memory of a small-M kernel: fixed head, reduction buffer and
+// as many ring stages per warp as fit (at most kMaxStages, at least 2).
+template <int FMT, int TG, int SRC>
+int small_smem(int* nstages) {
   using G = StageGeom<FMT, TG, SRC>;
   constexpr int kNW = kWarps<TG>;
   const int fixed = SmemHead<SRC>::kFixed + G::kRedBytes;
-  int nst = (kSmemLimit - fixed - 1024) / (kNW * G::kStageBytes);
-  nst = std::min(nst, kMaxStages);
-  if (nst < 2) return QMOE_ERR_UNSUPPORTED;
+  const int nst = std::min((kSmemLimit - fixed - 1024) / (kNW * G::kStageBytes), kMaxStages);
+  *nstages = nst;
+  return nst < 2 ? -1 : fixed + nst * kNW * G::kStageBytes;
+}
+
+template <int FMT, int TG, int EPI, int SRC>
+qmoe_status launch_small_t(SmallParams prm, int grid, cudaStream_t st) {
+  constexpr int kNW = kWarps<TG>;
+  int nst = 0;
+  const int smem = small_smem<FMT, TG, SRC>(&nst);
+  if (smem < 0) return QMOE_ERR_UNSUPPORTED;
   prm.nstages = nst;
-  const int smem = fixed + nst * kNW * G::kStageBytes;
   static bool attr_set[kMaxDevices] = {};
   int d = 0;
   cudaGetDevice(&d);
@@ -239,6 +254,45 @@ qmoe_status launch_small_t(SmallParams prm, int grid, cudaStream_t st) {
   return launch_pdl(qmm_small_kernel<FMT, TG, EPI, SRC>, dim3(grid), dim3(kNW * 32), smem, st, prm) == cudaSuccess
              ? QMOE_OK
              : QMOE_ERR_CUDA;
+}
+
+// Fused decode layer: decode_reset_kernel, then qmm_decode_kernel (one CTA per SM).
+template <int FMT>
+qmoe_status launch_decode_t(SmallParams p1, SmallParams p2, int* gbar, int grid, cudaStream_t st) {
+  int nst = 0;
+  const int smem = small_smem<FMT, 1, SRC_DECODE>(&nst);
+  if (smem < 0) return QMOE_ERR_UNSUPPORTED;
+  p1.nstages = p2.nstages = nst;
+  // 0: not checked, 1: one CTA fits per SM (the grid barrier needs all CTAs resident), -1: it does not
+  static int resident[kMaxDevices] = {};
+  int d = 0;
+  cudaGetDevice(&d);
+  if (!resident[d]) {
+    int per_sm = 0;
+    if (cudaFuncSetAttribute(qmm_decode_kernel<FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+            cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, qmm_decode_kernel<FMT>, kWarps<1> * 32, smem) !=
+            cudaSuccess)
+      return QMOE_ERR_CUDA;
+    resident[d] = per_sm >= 1 ? 1 : -1;
+  }
+  if (resident[d] < 0) return QMOE_ERR_UNSUPPORTED;
+  {
+    TraceScope ts(st, K_DECODE_RESET);
+    if (launch_pdl(decode_reset_kernel, dim3(1), dim3(128), 0, st, gbar, p2.ctick, p2.H / 16) != cudaSuccess)
+      return QMOE_ERR_CUDA;
+  }
+  TraceScope ts(st, K_DECODE_LAYER);
+  return launch_pdl(qmm_decode_kernel<FMT>, dim3(grid), dim3(kWarps<1> * 32), smem, st, p1, p2, gbar) == cudaSuccess
+             ? QMOE_OK
+             : QMOE_ERR_CUDA;
+}
+
+qmoe_status launch_decode(int fmt, const SmallParams& p1, const SmallParams& p2, int* gbar, int grid,
+                          cudaStream_t st) {
+  if (fmt == QMOE_INT2) return launch_decode_t<2>(p1, p2, gbar, grid, st);
+  if (fmt == QMOE_INT4) return launch_decode_t<4>(p1, p2, gbar, grid, st);
+  return launch_decode_t<3>(p1, p2, gbar, grid, st);
 }
 
 template <int EPI, int SRC>
@@ -493,12 +547,19 @@ qmoe_status qmoe_forward(const qmoe_layer* layer, const uint16_t* x, const float
       p1.early = 0;  // the logits may come from the previous launch
       p2.early = 0;  // FC2 reads FC1's routing tables after its wait
       p2.y = yt;
-      s = launch_small<EPI_SWIGLU, SRC_DECODE>(L.fc1.fmt, 1, p1, grid, st);
-      if (s != QMOE_OK) return s;
-      s = launch_small<EPI_FC2, SRC_DECODE>(L.fc2.fmt, 1, p2, grid, st);
-      if (s != QMOE_OK) return s;
+      s = QMOE_ERR_UNSUPPORTED;
+      if (L.fc1.fmt == L.fc2.fmt)  // one launch for the layer (after the reset launch)
+        s = launch_decode(L.fc1.fmt, p1, p2, reinterpret_cast<int*>(base + p.gbar), grid, st);
+      if (s != QMOE_OK && s != QMOE_ERR_UNSUPPORTED) return s;
+      const bool fused = s == QMOE_OK;
+      if (!fused) {
+        s = launch_small<EPI_SWIGLU, SRC_DECODE>(L.fc1.fmt, 1, p1, grid, st);
+        if (s != QMOE_OK) return s;
+        s = launch_small<EPI_FC2, SRC_DECODE>(L.fc2.fmt, 1, p2, grid, st);
+        if (s != QMOE_OK) return s;
+      }
       ++tiles;
-      small += 2;
+      small += fused ? 1 : 2;
       ++decode;
       continue;
     }

@@ -161,6 +161,21 @@ def test_decode_mixed_formats_and_ternary(qm):
         _close(y, ref, f"{cfg.name} decode T={T}")
 
 
+@pytest.mark.parametrize("T", [1, 5, 8])
+def test_decode_routing_ties(qm, T):
+    """Decode batches whose logits tie (a few distinct values, both signs of
+    zero): top-k takes the lower expert index among equal logits."""
+    cfg = synth.TINY
+    case = MoECase(cfg, seed=17)
+    x = synth.tokens(cfg.H, 17, T)
+    lg = np.round(synth.router_logits(cfg, 17, T) * 2.0).astype(np.float32) / 2.0
+    lg[:, 1::4] = -0.0
+    lg[:, 3::4] = 0.0
+    y = case.run(x, lg)
+    ref = Q.moe_forward(Q.bf16_bits_to_f64(x), lg, cfg.k, case.bank)
+    _close(y, ref, f"tiny ties T={T}")
+
+
 @pytest.mark.parametrize("M", [1, 5, 16, 32])
 def test_forward_v2lite_tokens_per_expert(qm, v2lite, M):
     """M tokens with identical router logits: every selected expert gets exactly M tokens."""
