@@ -8,19 +8,24 @@
 // never materialized (the onnxruntime PR's Description: "Avoid full A16
 // expert-weight materialization").
 //
-// One persistent CTA per SM, 18 warps, all waits bounded:
-//   warp 0      TMA producer: packed codes + scales (cp.async.bulk) and the
-//               token tile (cp.async.bulk.tensor 2-D, 128-byte swizzle, no
-//               multicast) for every 64-column k-stage;
+// One persistent CTA per SM, 19 warps, all waits bounded:
+//   warp 0      weight producer: packed codes + scales (cp.async.bulk) of every
+//               64-column k-stage, into a ring of CS stages;
+//   warp 18     token producer: the token tile of every k-stage
+//               (cp.async.bulk.tensor 2-D, 128-byte swizzle, no multicast),
+//               into a ring of kGStages stages;
 //   warp 1      TMEM allocator and single-thread MMA issuer
 //               (tcgen05.mma.cta_group::1.kind::f16, M=128, N<=256, bf16);
 //   warps 2-9   dequantize (one 16-row tile each): codes -> bf16(c*s) in the UMMA K-major
 //               128-byte-swizzle layout;
 //   warps 10-17 epilogue (two per TMEM lane quarter, alternate 32-column chunks):
 //               tcgen05.ld the fp32 accumulators, bias + SwiGLU
-//               (FC1) or bias (FC2), store.
+//               (FC1), bias (FC2) or nothing (single linear), store.
 // Two TMEM accumulators (2 x 256 columns) let the epilogue of one unit overlap
-// the main loop of the next.
+// the main loop of the next.  Template parameters: BT = token rows per unit (256
+// for expert tiles, 128 for the single linear), CS = weight-ring depth.  A
+// k-stage of packed weights is only 2-4 KB, so with few tokens (the single
+// linear) the ring must hold many of them to keep enough bytes in flight.
 //
 // The weight operand is bf16_rne(c*s): the tensor-core product needs one bf16
 // operand per weight, so this path rounds the dequantized weight once (the
@@ -40,11 +45,12 @@ constexpr int kGStages = 4;
 constexpr int kGDeqWarps = 8;     // one 16-row tile of the 128-row unit each
 constexpr int kGDeqTiles = 8 / kGDeqWarps;
 constexpr int kGEpiWarps = 8;     // two per TMEM lane quarter
-constexpr int kGWarps = 2 + kGDeqWarps + kGEpiWarps;
+constexpr int kGWarps = 3 + kGDeqWarps + kGEpiWarps;
+constexpr int kGTokWarp = 2 + kGDeqWarps + kGEpiWarps;  // the token producer
 constexpr int kGThreads = kGWarps * 32;
 constexpr int kGABytes = kGRows * 64 * 2;      // 16 KB bf16 weight tile per k-stage
-constexpr int kGBBytes = kGTok * 64 * 2;       // 32 KB token tile per k-stage
 constexpr int kGTmaRows = 64;                  // rows per 2-D TMA box
+constexpr int kLinBT = 128;                    // single linear: token rows per unit
 constexpr int kGAccCols = 256;
 
 struct GSeg {
@@ -71,15 +77,36 @@ struct GroupedParams {
   int I;
   float* yslot;     // FC2 output [slot][H]
   int H;
+  uint16_t* y;      // single linear output [token][N] bf16 (EPI_LINEAR)
+  int N;
+  int ntok;         // ngseg == nullptr: segments are chunks of BT of ntok token rows of matrix 0
   unsigned* status;
 };
 
-template <int FMT>
+template <int BT>
+__device__ __forceinline__ int g_nseg(const GroupedParams& p) {
+  return p.ngseg ? *p.ngseg : (p.ntok + BT - 1) / BT;
+}
+
+template <int BT>
+__device__ __forceinline__ GSeg g_seg(const GroupedParams& p, int i) {
+  if (p.gsegs) return p.gsegs[i];
+  GSeg sg;
+  sg.expert = 0;
+  sg.slot0 = i * BT;
+  sg.ntok = min(BT, p.ntok - i * BT);
+  sg.pad = 0;
+  return sg;
+}
+
+template <int FMT, int BT, int CS>
 struct GGeom {
   static constexpr int kCodeBytes = 8 * FmtTraits<FMT>::kCodeBytes;  // 8 tiles of 16 rows, 64 columns
   static constexpr int kCStage = kCodeBytes + 8 * 32;
-  static constexpr int kSmem = 1024 /*align slack*/ + kGStages * (kGABytes + kGBBytes) +
-                               ((kGStages * kCStage + 127) / 128) * 128 + 256;
+  static constexpr int kBBytes = BT * 64 * 2;                         // token tile per k-stage
+  static constexpr int kCRing = ((CS * kCStage + 127) / 128) * 128;
+  static constexpr int kBars = (((2 * CS + 4 * kGStages + 5) * 8 + 16 + 127) / 128) * 128;
+  static constexpr int kSmem = 1024 /*align slack*/ + kGStages * (kGABytes + kBBytes) + kCRing + kBars;
 };
 
 // ---- tcgen05 / TMA helpers ----------------------------------------------------
@@ -151,36 +178,38 @@ __device__ __forceinline__ bool gwait(uint64_t* bar, uint32_t parity, unsigned* 
   }
 }
 
-template <int FMT, int EPI>
+template <int FMT, int EPI, int BT, int CS>
 __global__ void __launch_bounds__(kGThreads, 1)
     qmm_grouped_kernel(const __grid_constant__ CUtensorMap tmap, const GroupedParams p) {
   using Tr = FmtTraits<FMT>;
-  using GG = GGeom<FMT>;
+  using GG = GGeom<FMT, BT, CS>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024 - (smem_addr(smem_raw) & 1023)) & 1023);
-  uint8_t* sA = smem;                                        // [stage][16 KB]
-  uint8_t* sB = sA + kGStages * kGABytes;                    // [stage][32 KB]
-  uint8_t* sC = sB + kGStages * kGBBytes;                    // [stage][codes | scales]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sC + ((kGStages * GG::kCStage + 127) / 128) * 128);
-  uint64_t* full_c = bars;
-  uint64_t* empty_c = bars + kGStages;
-  uint64_t* full_ab = bars + 2 * kGStages;
-  uint64_t* empty_ab = bars + 3 * kGStages;
-  uint64_t* tm_full = bars + 4 * kGStages;
+  uint8_t* sA = smem;                                        // [kGStages][16 KB]
+  uint8_t* sB = sA + kGStages * kGABytes;                    // [kGStages][BT rows x 128 B]
+  uint8_t* sC = sB + kGStages * GG::kBBytes;                 // [CS][codes | scales]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sC + GG::kCRing);
+  uint64_t* full_c = bars;                                   // [CS]
+  uint64_t* empty_c = bars + CS;                             // [CS]
+  uint64_t* full_ab = bars + 2 * CS;                         // [kGStages]
+  uint64_t* empty_ab = bars + 2 * CS + kGStages;             // [kGStages]
+  uint64_t* tm_full = bars + 2 * CS + 2 * kGStages;
   uint64_t* tm_empty = tm_full + 2;
   uint64_t* mma_done = tm_empty + 2;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mma_done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int n_units = *p.ngseg * p.rtiles;
+  const int n_units = g_nseg<BT>(p) * p.rtiles;
   if ((int)blockIdx.x >= n_units) return;
   const int KS = p.K / 64;
 
   if (tid == 0) {
-    for (int s = 0; s < kGStages; ++s) {
+    for (int s = 0; s < CS; ++s) {
       mbar_init(&full_c[s], 1);
       mbar_init(&empty_c[s], kGDeqWarps);
+    }
+    for (int s = 0; s < kGStages; ++s) {
       mbar_init(&full_ab[s], 1 + kGDeqWarps);
       mbar_init(&empty_ab[s], 1);
     }
@@ -204,20 +233,19 @@ __global__ void __launch_bounds__(kGThreads, 1)
   const uint32_t tmem_base = *tmem_holder;
 
   if (warp == 0) {
-    // ---------------- producer ----------------
-    // The copies of a stage are issued by different lanes in one step (codes:
-    // lane 0, scales: lane 1, token boxes: lanes 2..): a bulk copy costs ~117
-    // cycles to issue from one lane, while the SM accepts one every ~56.
+    // ---------------- weight producer ----------------
+    // The two copies of a stage are issued by different lanes in one step: a
+    // bulk copy costs ~117 cycles to issue from one lane, while the SM accepts
+    // one every ~56.
     uint32_t it = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < n_units && ok && !*abort_flag; u += gridDim.x) {
-      const GSeg sg = p.gsegs[u / p.rtiles];
+      const GSeg sg = g_seg<BT>(p, u / p.rtiles);
       const int rt = u % p.rtiles;
-      const int nsub = (sg.ntok + kGTmaRows - 1) / kGTmaRows;
       for (int ks = 0; ks < KS; ++ks, ++it) {
-        const int s = it % kGStages;
-        const uint32_t ph = (it / kGStages) & 1u;
-        int w_ok = lane == 0 ? (int)gwait(&empty_c[s], ph ^ 1u, p.status, abort_flag) : 0;
+        const int s = it % CS;
+        const uint32_t ph = (it / CS) & 1u;
+        const int w_ok = lane == 0 ? (int)gwait(&empty_c[s], ph ^ 1u, p.status, abort_flag) : 0;
         if (!__shfl_sync(0xffffffffu, w_ok, 0)) { ok = false; break; }
         uint8_t* cdst = sC + s * GG::kCStage;
         if (lane == 0) mbar_arrive_expect_tx(&full_c[s], GG::kCStage);
@@ -232,13 +260,24 @@ __global__ void __launch_bounds__(kGThreads, 1)
                                                    ((unsigned long long)sb * p.NT + rt * 8) * 32,
                         8 * 32, &full_c[s]);
         }
-        w_ok = lane == 0 ? (int)gwait(&empty_ab[s], ph ^ 1u, p.status, abort_flag) : 0;
+      }
+    }
+  } else if (warp == kGTokWarp) {
+    // ---------------- token producer ----------------
+    uint32_t it = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < n_units && ok && !*abort_flag; u += gridDim.x) {
+      const GSeg sg = g_seg<BT>(p, u / p.rtiles);
+      const int nsub = (sg.ntok + kGTmaRows - 1) / kGTmaRows;
+      for (int ks = 0; ks < KS; ++ks, ++it) {
+        const int s = it % kGStages;
+        const uint32_t ph = (it / kGStages) & 1u;
+        const int w_ok = lane == 0 ? (int)gwait(&empty_ab[s], ph ^ 1u, p.status, abort_flag) : 0;
         if (!__shfl_sync(0xffffffffu, w_ok, 0)) { ok = false; break; }
         if (lane == 0) mbar_arrive_expect_tx(&full_ab[s], (uint32_t)(nsub * kGTmaRows * 128));
         __syncwarp();
-        const int sub = lane - 2;
-        if (sub >= 0 && sub < nsub)
-          tma_load_2d(sB + s * kGBBytes + sub * kGTmaRows * 128, &tmap, ks * 64, sg.slot0 + sub * kGTmaRows,
+        if (lane < nsub)
+          tma_load_2d(sB + s * GG::kBBytes + lane * kGTmaRows * 128, &tmap, ks * 64, sg.slot0 + lane * kGTmaRows,
                       &full_ab[s]);
       }
     }
@@ -247,7 +286,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
     if (lane == 0) {
       uint32_t it = 0, acc_it = 0;
       for (int u = blockIdx.x; u < n_units && !*abort_flag; u += gridDim.x, ++acc_it) {
-        const GSeg sg = p.gsegs[u / p.rtiles];
+        const GSeg sg = g_seg<BT>(p, u / p.rtiles);
         const int n = (sg.ntok + 15) / 16 * 16;
         const uint32_t idesc = umma_idesc_bf16(n);
         const uint32_t a = acc_it & 1u;
@@ -261,7 +300,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
           if (!gwait(&full_ab[s], ph, p.status, abort_flag)) { ok = false; break; }
           tc_fence_after();
           const uint64_t ad = umma_desc_sw128(sA + s * kGABytes);
-          const uint64_t bd = umma_desc_sw128(sB + s * kGBBytes);
+          const uint64_t bd = umma_desc_sw128(sB + s * GG::kBBytes);
 #pragma unroll
           for (int j = 0; j < 4; ++j)  // 16 bf16 = 32 bytes per k-step: +2 in the 16-byte address field
             umma_bf16(d_tmem, ad + 2 * j, bd + 2 * j, idesc, (ks > 0 || j > 0) ? 1u : 0u);
@@ -281,10 +320,12 @@ __global__ void __launch_bounds__(kGThreads, 1)
     uint32_t it = 0;
     for (int u = blockIdx.x; u < n_units && !*abort_flag; u += gridDim.x) {
       for (int ks = 0; ks < KS; ++ks, ++it) {
+        const int sc = it % CS;
+        const uint32_t phc = (it / CS) & 1u;
         const int s = it % kGStages;
         const uint32_t ph = (it / kGStages) & 1u;
-        if (!gwait(&full_c[s], ph, p.status, abort_flag)) break;
-        const uint8_t* cs = sC + s * GG::kCStage;
+        if (!gwait(&full_c[sc], phc, p.status, abort_flag)) break;
+        const uint8_t* cs = sC + sc * GG::kCStage;
         uint32_t am[kGDeqTiles][4][4];
         uint32_t sw[kGDeqTiles];
 #pragma unroll
@@ -304,7 +345,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
           sw[tt] = *reinterpret_cast<const uint32_t*>(cs + GG::kCodeBytes + tile * 32 + g * 4);
         }
         __syncwarp();
-        if (lane == 0) mbar_arrive(&empty_c[s]);
+        if (lane == 0) mbar_arrive(&empty_c[sc]);
         if (!gwait(&empty_ab[s], ph ^ 1u, p.status, abort_flag)) break;
         uint8_t* as = sA + s * kGABytes;
 #pragma unroll
@@ -332,14 +373,14 @@ __global__ void __launch_bounds__(kGThreads, 1)
         if (lane == 0) mbar_arrive(&full_ab[s]);
       }
     }
-  } else {
+  } else if (warp < 2 + kGDeqWarps + kGEpiWarps) {
     // ---------------- epilogue ----------------
     const int quarter = warp & 3;
     const int half = (warp - 2 - kGDeqWarps) >> 2;  // which alternate 32-column chunks
     const int r = quarter * 32 + lane;  // accumulator lane = tile row
     uint32_t acc_it = 0;
     for (int u = blockIdx.x; u < n_units && !*abort_flag; u += gridDim.x, ++acc_it) {
-      const GSeg sg = p.gsegs[u / p.rtiles];
+      const GSeg sg = g_seg<BT>(p, u / p.rtiles);
       const int rt = u % p.rtiles;
       const uint32_t a = acc_it & 1u;
       if (!gwait(&tm_full[a], (acc_it >> 1) & 1u, p.status, abort_flag)) break;
@@ -374,6 +415,8 @@ __global__ void __launch_bounds__(kGThreads, 1)
               const float h = silu_f(x + bias_v) * (up + bias_u);
               p.hrows[(size_t)(sg.slot0 + n) * p.I + j] = __bfloat16_as_ushort(__float2bfloat16_rn(h));
             }
+          } else if (EPI == EPI_LINEAR) {
+            if (n < sg.ntok) p.y[(size_t)(sg.slot0 + n) * p.N + prow] = __bfloat16_as_ushort(__float2bfloat16_rn(x));
           } else {
             if (n < sg.ntok) p.yslot[(size_t)(sg.slot0 + n) * p.H + prow] = x + bias_v;
           }

@@ -294,26 +294,17 @@ __device__ __forceinline__ void iter_begin(ItemIter& it, const SmallParams& p, c
 // arriving on the barrier once its copies landed.  Full barrier count: 33
 // (lane 0's expect-tx arrival and 32 cp.async arrivals).
 
-// Codes and scales (cp.async) of the sub-panel's nt tiles at k-unit ku.  The
-// codes go through the TMA engine (one bulk copy by lane 0), or, with lsu,
-// through the load/store unit as 16-byte cp.async by every lane: a CTA's
-// first stages are requested by all warps at once, and the TMA engine takes
-// them one copy at a time (tens of cycles each), while the load/store units
-// of the four sub-partitions take them in parallel.  Either way lane 0
-// arrives once on the barrier (with the expected bytes of the bulk copy).
+// Codes (TMA) and scales (cp.async) of the sub-panel's nt tiles at k-unit ku.
 template <int FMT, int TG, int SRC>
 __device__ __forceinline__ void issue_weights(const SmallParams& p, const ItemIter& it, uint8_t* stage, uint64_t* bar,
-                                              int lane, bool lsu = false) {
+                                              int lane) {
   using G = StageGeom<FMT, TG, SRC>;
   using Tr = FmtTraits<FMT>;
   const int tile = it.sp.rt0, n = it.sp.nt;
-  const uint8_t* csrc = p.codes + (unsigned long long)it.sg.expert * p.codes_stride +
-                        ((unsigned long long)it.ku * p.NT + tile) * Tr::kCodeBytes;
-  const uint32_t bytes = (uint32_t)(n * Tr::kCodeBytes);
-  if (lsu) {
-    for (uint32_t o = 16u * lane; o < bytes; o += 512u) cp_async16(stage + o, csrc + o);
-    if (lane == 0) mbar_arrive(bar);
-  } else if (lane == 0) {
+  if (lane == 0) {
+    const uint8_t* csrc = p.codes + (unsigned long long)it.sg.expert * p.codes_stride +
+                          ((unsigned long long)it.ku * p.NT + tile) * Tr::kCodeBytes;
+    const uint32_t bytes = (uint32_t)(n * Tr::kCodeBytes);
     // No proxy fence: the warp's reads of this stage were consumed by its MMAs
     // before the refill is issued.
     mbar_arrive_expect_tx(bar, bytes);

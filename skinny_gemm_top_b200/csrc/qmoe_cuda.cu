@@ -59,10 +59,11 @@ qmoe_status dev_info(DevInfo** out) {
 
 // ---- tracing: CUDA events around each kernel launch ----
 enum KernelId { K_ROUTE = 0, K_GATHER, K_FC1_SMALL, K_FC2_SMALL, K_COMBINE, K_LINEAR_SMALL, K_LINEAR_SETUP,
-                K_DEQUANT, K_FC1_GROUPED, K_FC2_GROUPED, K_DECODE_RESET, K_DECODE_LAYER, K_COUNT };
-const char* const kKernelNames[K_COUNT] = {"route",        "gather",      "fc1_small",   "fc2_small",
+                K_DEQUANT, K_FC1_GROUPED, K_FC2_GROUPED, K_DECODE_RESET, K_DECODE_LAYER, K_LINEAR_GROUPED, K_COUNT };
+const char* const kKernelNames[K_COUNT] = {"route",        "gather",      "fc1_small",    "fc2_small",
                                            "combine",      "linear_small", "linear_setup", "dequant",
-                                           "fc1_grouped",  "fc2_grouped", "decode_reset", "decode_layer"};
+                                           "fc1_grouped",  "fc2_grouped", "decode_reset", "decode_layer",
+                                           "linear_grouped"};
 struct Tracer {
   bool on = false;
   int cap = 0, n = 0;
@@ -142,6 +143,7 @@ struct MoEPlan {
 };
 
 constexpr int kGroupedThreshold = 32;  // AUTO: experts with more tokens take the tcgen05 path
+constexpr int kLinearGroupedMinM = 48;  // single linear: from this many rows on, the tcgen05 path
 
 bool grouped_eligible(const qmoe_layer& L) {
   return L.fc1.fmt != QMOE_TERNARY && L.fc2.fmt != QMOE_TERNARY && (2 * L.I) % kGRows == 0 && L.H % kGRows == 0;
@@ -310,27 +312,38 @@ qmoe_status launch_small(int fmt, int tg, const SmallParams& prm, int grid, cuda
   }
 }
 
-template <int FMT, int EPI>
+template <int FMT, int EPI, int BT, int CS>
 qmoe_status launch_grouped_t(const CUtensorMap& map, const GroupedParams& prm, int grid, cudaStream_t st) {
-  constexpr int smem = GGeom<FMT>::kSmem;
+  constexpr int smem = GGeom<FMT, BT, CS>::kSmem;
+  static_assert(smem <= kSmemLimit, "grouped kernel shared memory");
   static bool attr_set[kMaxDevices] = {};
   int d = 0;
   cudaGetDevice(&d);
   if (!attr_set[d]) {
-    if (cudaFuncSetAttribute(qmm_grouped_kernel<FMT, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
-        cudaSuccess)
+    if (cudaFuncSetAttribute(qmm_grouped_kernel<FMT, EPI, BT, CS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             smem) != cudaSuccess)
       return QMOE_ERR_CUDA;
     attr_set[d] = true;
   }
-  TraceScope ts(st, EPI == EPI_SWIGLU ? K_FC1_GROUPED : K_FC2_GROUPED);
-  qmm_grouped_kernel<FMT, EPI><<<grid, kGThreads, smem, st>>>(map, prm);
+  TraceScope ts(st, EPI == EPI_SWIGLU ? K_FC1_GROUPED : (EPI == EPI_FC2 ? K_FC2_GROUPED : K_LINEAR_GROUPED));
+  qmm_grouped_kernel<FMT, EPI, BT, CS><<<grid, kGThreads, smem, st>>>(map, prm);
   return cudaGetLastError() == cudaSuccess ? QMOE_OK : QMOE_ERR_CUDA;
 }
 
+// Expert tiles: units of up to 256 tokens, a weight ring as deep as the token ring.
 template <int EPI>
 qmoe_status launch_grouped(int fmt, const CUtensorMap& map, const GroupedParams& prm, int grid, cudaStream_t st) {
-  if (fmt == QMOE_INT2) return launch_grouped_t<2, EPI>(map, prm, grid, st);
-  if (fmt == QMOE_INT4) return launch_grouped_t<4, EPI>(map, prm, grid, st);
+  if (fmt == QMOE_INT2) return launch_grouped_t<2, EPI, kGTok, kGStages>(map, prm, grid, st);
+  if (fmt == QMOE_INT4) return launch_grouped_t<4, EPI, kGTok, kGStages>(map, prm, grid, st);
+  return QMOE_ERR_UNSUPPORTED;
+}
+
+// Single linear: units of up to 128 tokens; a weight ring of about 64 KB (28
+// INT2 or 16 INT4 stages), the bytes in flight an SM needs for its HBM share.
+qmoe_status launch_grouped_linear(int fmt, const CUtensorMap& map, const GroupedParams& prm, int grid,
+                                  cudaStream_t st) {
+  if (fmt == QMOE_INT2) return launch_grouped_t<2, EPI_LINEAR, kLinBT, 28>(map, prm, grid, st);
+  if (fmt == QMOE_INT4) return launch_grouped_t<4, EPI_LINEAR, kLinBT, 16>(map, prm, grid, st);
   return QMOE_ERR_UNSUPPORTED;
 }
 
@@ -681,14 +694,30 @@ qmoe_status qmoe_linear(const qmoe_weights* w, int N, int K, const uint16_t* x, 
   p.y = y;
   p.N = N;
   p.early = 1;  // static weights, arithmetic segments
-  s = launch_small<EPI_LINEAR, SRC_LINEAR>(w->fmt, M <= 8 ? 1 : 2, p, di->sms, st);
+  // More than one token group: the tcgen05 path, whose cost barely depends on
+  // M (the dequantized tile serves up to 256 tokens; the small-M kernel's
+  // mma.sync work grows with every group of 8 tokens).
+  const bool grouped = M >= kLinearGroupedMinM && N % kGRows == 0 && w->fmt != QMOE_TERNARY;
+  if (grouped) {
+    CUtensorMap map;
+    s = encode_rows_map(&map, x, K, M);
+    if (s != QMOE_OK) return s;
+    GroupedParams g = grouped_params(*w, N, K, di->status);
+    g.y = y;
+    g.N = N;
+    g.ntok = M;
+    const int units = (M + kLinBT - 1) / kLinBT * g.rtiles;
+    s = launch_grouped_linear(w->fmt, map, g, std::min(units, di->sms), st);
+  } else {
+    s = launch_small<EPI_LINEAR, SRC_LINEAR>(w->fmt, M <= 8 ? 1 : 2, p, di->sms, st);
+  }
   if (s != QMOE_OK) return s;
   std::lock_guard<std::mutex> lk(g_mu);
-  g_stats.last_path = QMOE_PATH_SMALL_M;
+  g_stats.last_path = grouped ? QMOE_PATH_GROUPED : QMOE_PATH_SMALL_M;
   g_stats.row_tiles = 1;
   g_stats.row_tile_tokens = M;
-  g_stats.small_launches = 1;
-  g_stats.grouped_launches = 0;
+  g_stats.small_launches = grouped ? 0 : 1;
+  g_stats.grouped_launches = grouped ? 1 : 0;
   return QMOE_OK;
 }
 

@@ -110,8 +110,22 @@ def test_linear_medium_multi_tile_per_cta(qm, fmt, M):
     _close(y, ref, f"{fmt} M={M}")
 
 
+@pytest.mark.parametrize("fmt,block", [("int2", 128), ("int4", 64)])
+@pytest.mark.parametrize("M", [48, 64, 300])
+def test_linear_grouped_path(qm, fmt, block, M):
+    """48 rows or more with N a multiple of 128: the tcgen05 path (weights rounded
+    once to bf16 there), including further 128-token chunks with a ragged tail."""
+    N, K = 1024, 768
+    wb, x, y, _ = _linear_case(qm, fmt, block, N, K, M, seed=40 + M)
+    st = qm.get_stats()
+    assert st.last_path == qm.PATH_GROUPED and st.grouped_launches == 1
+    codes, scales = oracle_quant(fmt, wb, block)
+    ref = Q.linear(Q.bf16_bits_to_f64(x), Q.dequant(codes, scales, block))
+    _close(y, ref, f"{fmt} M={M}")
+
+
 @pytest.mark.parametrize("fmt", ["int2", "int4"])
-@pytest.mark.parametrize("M", [1, 8])
+@pytest.mark.parametrize("M", [1, 8, 32])
 def test_linear_full_size_sampled_rows(qm, fmt, M):
     """K=5120 -> N=17408, group 128, as benchmarked; the oracle computes 512 sampled rows."""
     N, K = 17408, 5120
