@@ -12,13 +12,13 @@
 //  * Work = (segment, 16-row tile, k-unit of 64 columns; 128 for ternary).
 //    CTA c takes a balanced range of whole tiles, so no tile is split
 //    between CTAs and every output is written once, deterministically.
-//  * Inside a CTA, up to 8 consecutive tiles form a sub-panel; its k-units go
-//    round-robin to 8 warps.  Each warp runs its own TMA bulk-copy pipeline
-//    (cp.async.bulk + mbarrier, no tensor map, no multicast).  A stage holds
-//    the sub-panel's codes and scales at one k-unit plus that k-unit's slice
-//    of the segment's activation rows (one 128-byte copy per token, issued by
-//    one lane each).  B fragments come from those rows through ldmatrix and
-//    are reused by every tile of the stage; the MMAs of all tiles of a k-step
+//  * Inside a CTA, up to 10 consecutive tiles (kTiles) form a sub-panel; its
+//    k-units go round-robin to the CTA's warps (12, or 8 for two token
+//    groups).  Each warp runs its own stage ring: the codes by one bulk copy
+//    (cp.async.bulk + mbarrier, no tensor map, no multicast), the scales and
+//    the k-unit's slice of the segment's activation rows by 16-byte
+//    cp.async.  B fragments come from those rows through ldmatrix and are
+//    reused by every tile of the stage; the MMAs of all tiles of a k-step
 //    issue back to back so their latencies overlap.
 //  * Codes become bf16 MMA operands with LOP3 magic numbers (unpack.cuh) and
 //    are multiplied on the tensor cores (mma.sync m16n8k16, tokens in N):
@@ -36,6 +36,9 @@
 //  * Decode FC2 fuses the router-weighted combine: the last CTA to finish a
 //    16-row output tile (atomic counter, no spin-wait) sums that tile's slot
 //    rows in slot order and writes y.
+//  * A decode layer whose FC1 and FC2 share a format runs as one launch
+//    (qmm_decode_kernel): routing, the FC1 phase, a split grid barrier and the
+//    FC2 phase with the combine, on the same stage rings.
 #pragma once
 #include <cfloat>
 #include <climits>
