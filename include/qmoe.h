@@ -150,7 +150,12 @@ qmoe_status qmoe_workspace_size(const qmoe_layer* layer, int T, size_t* bytes);
 /* y[T, H] bf16 = MoE(x[T, H] bf16, logits[T, E] fp32).  With ws_bytes below
  * qmoe_workspace_size(T), tokens are processed in row tiles (halved until the
  * tile's workspace fits, explicit partial last tile); QMOE_ERR_SCRATCH when
- * one row does not fit.  ws must be 256-byte aligned. */
+ * one row does not fit.  ws must be 256-byte aligned.
+ * A decode batch (T <= 8, T*k <= 64) whose FC1 and FC2 share a format runs as
+ * one kernel with one block per SM and a grid-wide barrier: it needs every SM
+ * of the device at once.  Kernels of other streams that hold SMs only delay
+ * it; if the barrier waits longer than 2 s the call reports the timeout flag
+ * in the device status word (qmoe_get_stats) instead of hanging. */
 qmoe_status qmoe_forward(const qmoe_layer* layer, const uint16_t* x, const float* logits, int T,
                          uint16_t* y, void* ws, size_t ws_bytes, void* stream);
 
