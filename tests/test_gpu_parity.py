@@ -175,6 +175,20 @@ def test_decode_mixed_formats_and_ternary(qm):
         _close(y, ref, f"{cfg.name} decode T={T}")
 
 
+@pytest.mark.parametrize("E,k,n_shared", [(100, 8, 1), (128, 4, 0), (200, 8, 2), (256, 8, 1)])
+@pytest.mark.parametrize("T", [1, 3, 8])
+def test_decode_many_experts(qm, E, k, n_shared, T):
+    """Decode batches (one fused launch) over 65..256 experts: the routing's
+    4- and 8-experts-per-lane variants, ragged expert counts, shared experts."""
+    cfg = small_cfg(synth.TINY, E=E, k=k, n_shared=n_shared, H=256, I=256, fc1_fmt="int4", fc2_fmt="int4")
+    case = MoECase(cfg, seed=50 + E)
+    x = synth.tokens(cfg.H, 50 + E, T)
+    lg = synth.router_logits(cfg, 50 + E, T)
+    y = case.run(x, lg)
+    ref = Q.moe_forward(Q.bf16_bits_to_f64(x), lg, cfg.k, case.bank)
+    _close(y, ref, f"E={E} k={k} decode T={T}")
+
+
 @pytest.mark.parametrize("T", [1, 5, 8])
 def test_decode_routing_ties(qm, T):
     """Decode batches whose logits tie (a few distinct values, both signs of
