@@ -51,6 +51,8 @@ def parse():
     ap.add_argument("--quick", action="store_true", help="skip the sweeps")
     ap.add_argument("--profile", action="store_true",
                     help="a few eager layer forwards and linears only (for an ncu launch list or capture)")
+    ap.add_argument("--profile-prefill", action="store_true",
+                    help="two eager forwards of the prefill layer (T = 4096, one row tile) only, for an ncu capture")
     return ap.parse_args()
 
 
@@ -246,6 +248,25 @@ def run_profile(args):
         qmoe.linear(w, N, K, x, y, ws)
         torch.cuda.synchronize()
     print("profile run done", flush=True)
+
+
+def run_profile_prefill(args):
+    """Two eager forwards of the C5 prefill layer with a full workspace (one row tile)."""
+    import torch
+    from skinny_gemm_top_b200 import qmoe
+    cfg = synth.PREFILL
+    layer, keep = pack_cfg(qmoe, torch, cfg)
+    T = 4096
+    x = _to_dev(torch, synth.tokens(cfg.H, SEED, T))
+    lg = torch.from_numpy(np.ascontiguousarray(synth.router_logits(cfg, SEED, T, index=100))).cuda()
+    ws = torch.empty(qmoe.workspace_size(layer, T), dtype=torch.uint8, device="cuda")
+    y = torch.empty((T, cfg.H), dtype=torch.int16, device="cuda")
+    for _ in range(2):
+        qmoe.forward(layer, x, lg, y, ws)
+        torch.cuda.synchronize()
+    assert qmoe.get_stats().device_status == 0
+    del keep
+    print("prefill profile run done", flush=True)
 
 
 def run_ours(args):
@@ -641,6 +662,8 @@ def main():
         run_reference(args)
     elif args.profile:
         run_profile(args)
+    elif args.profile_prefill:
+        run_profile_prefill(args)
     else:
         run_ours(args)
 
