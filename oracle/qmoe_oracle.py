@@ -21,7 +21,7 @@ FC2 and combine with the router weights.  Sources, by page and section:
 * "The QMoE sub-1-bit expert kernel is a GEMV ..." note: top-k routed tokens,
   several tokens sharing one expert.
 
-Readings where the pages are silent (each is listed in the design doc):
+Readings where the pages are silent:
 
 * INT scale: s = bf16_rne(max|w| / 2^(bits-1)); codes c = clamp(rne(w/s),
   -2^(bits-1), 2^(bits-1)-1) in float64; s == 0 gives c = 0.
