@@ -251,7 +251,7 @@ def run_profile(args):
 
 
 def run_profile_prefill(args):
-    """Two eager forwards of the C5 prefill layer with a full workspace (one row tile)."""
+    """Two eager forwards of the prefill layer (T = 4096, 128 experts top-8) with a full workspace (one row tile)."""
     import torch
     from skinny_gemm_top_b200 import qmoe
     cfg = synth.PREFILL
@@ -343,8 +343,8 @@ def run_ours(args):
                                  "tokens_per_s": round(M / (r["ms_per_step"] * 1e-3), 1)})
     linear = [] if args.quick else linear_sweep(qmoe, torch, dist, args)
     lmhead = [] if args.quick else lmhead_sweep(qmoe, torch, dist, args)
-    # ternary layer (C4 per-expert shapes, 32 experts: one top-1 expert per token) and the
-    # prefill layer (C5, T = 4096, tcgen05 grouped path, 256 MiB workspace with row tiling)
+    # ternary layer (H=2048, I=6144 experts, 32 of them: one top-1 expert per token) and the
+    # prefill layer (T = 4096, 128 experts top-8, tcgen05 grouped path, 256 MiB workspace with row tiling)
     ternary = [] if args.quick else cfg_sweep(qmoe, torch, dist, args,
                                               dataclasses.replace(synth.TERNARY, E=32), (1, 8, 32), rotate=32)
     prefill = [] if args.quick else cfg_sweep(qmoe, torch, dist, args, synth.PREFILL, (4096,), rotate=1,
