@@ -125,11 +125,22 @@ qmoe_status qmoe_dequant(const qmoe_weights* w, int row_order, int rows, int K, 
                          float* out_f32, uint16_t* out_bf16, void* stream);
 
 /* Routing (device): logits fp32 [T, E] -> ids int32 [T, k] (descending logit,
- * ties to the lower index), weights fp32 [T, k] (softmax over the k selected
- * logits), perm int32 [T*k] (flat index t*k+s at each expert-sorted
- * position; stable), offsets int32 [E+1].  E <= 256, 1 <= k <= min(E, 32). */
+ * ties to the lower index, -0 equal to +0), weights fp32 [T, k] (softmax over
+ * the k selected logits), perm int32 [T*k] (flat index t*k+s at each
+ * expert-sorted position; stable), offsets int32 [E+1].  E <= 256,
+ * 1 <= k <= min(E, 32).  Logits must be finite.
+ * Top-k routing, then "expert maps" and rows expanded by expert: onnxruntime
+ * PR "Enable SM80+ FP16/BF16 mixed INT2/INT4 QMoE prefill by default",
+ * Description.
+ * The routing kernels are the ones qmoe_forward runs: for a decode batch
+ * (T <= 8 and T*k <= 64) one CTA with the in-kernel routing of the decode
+ * layer kernel; otherwise the two-launch general routing (per-chunk top-k and
+ * counts, then the stable scatter), whose per-chunk counts live in ws.
+ * ws: device scratch of at least qmoe_route_workspace_size() bytes, 16-byte
+ * aligned (NULL allowed when that size is 0); QMOE_ERR_SCRATCH if smaller. */
+qmoe_status qmoe_route_workspace_size(int T, int E, int k, size_t* bytes);
 qmoe_status qmoe_route(const float* logits, int T, int E, int k, int32_t* ids, float* weights,
-                       int32_t* perm, int32_t* offsets, void* stream);
+                       int32_t* perm, int32_t* offsets, void* ws, size_t ws_bytes, void* stream);
 
 /* One MoE layer.  fc1: E + n_shared matrices [2I, H] packed with
  * QMOE_ROWS_GATE_UP (shared experts after the routed ones); bias [.][2I].

@@ -39,19 +39,34 @@ def _stale() -> bool:
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and not _stale():
-        return LIB
-    tmp = LIB + ".tmp"
-    cmd = [_nvcc(), *ARCH, "-O3", "-std=c++17", "-lineinfo", "-shared", "-Xcompiler", "-fPIC,-fopenmp",
-           "-I", INCLUDE, "-I", CSRC, "-o", tmp, *sources(), "-lgomp"]
-    if verbose:
-        cmd.insert(1, "-Xptxas=-v")
+def _run(cmd):
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError("nvcc failed:\n" + " ".join(cmd) + "\n" + r.stdout + r.stderr)
+    return r.stdout + r.stderr
+
+
+def build(force: bool = False, verbose: bool = False) -> str:
+    """Compile every source to an object in parallel, then link the library."""
+    if not force and not _stale():
+        return LIB
+    from concurrent.futures import ThreadPoolExecutor
+    objdir = os.path.join(PKG, "_build")
+    os.makedirs(objdir, exist_ok=True)
+    flags = [*ARCH, "-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC,-fopenmp", "-I", INCLUDE, "-I", CSRC]
     if verbose:
-        sys.stderr.write(r.stdout + r.stderr)
+        flags.insert(0, "-Xptxas=-v")
+    objs, cmds = [], []
+    for src in sources():
+        obj = os.path.join(objdir, os.path.basename(src) + ".o")
+        objs.append(obj)
+        cmds.append([_nvcc(), *flags, "-c", src, "-o", obj])
+    with ThreadPoolExecutor(max_workers=min(len(cmds), os.cpu_count() or 1)) as ex:
+        logs = list(ex.map(_run, cmds))
+    if verbose:
+        sys.stderr.write("".join(logs))
+    tmp = LIB + ".tmp"
+    _run([_nvcc(), *ARCH, "-shared", "-o", tmp, *objs, "-lgomp"])
     os.replace(tmp, LIB)
     return LIB
 

@@ -10,8 +10,6 @@
 
 namespace qmoe {
 
-constexpr int kRouteThreads = 1024;
-
 struct RouteOut {
   int* ids;          // [T*k]
   float* w;          // [T*k]
@@ -32,159 +30,34 @@ struct RouteOut {
   int* chunk_counts; // [nchunks][E] (two-kernel routing)
 };
 
-// One CTA: warp top-k per token, then a stable counting sort by expert (ranks
-// from warp match masks, offsets from a prefix over warps in warp order), then
-// the (expert, chunk of <= 16 tokens) segment table.  Deterministic.
-__global__ void __launch_bounds__(kRouteThreads, 1)
-    route_kernel(const float* __restrict__ logits, int T, int E, int k, int n_shared, RouteOut o) {
-  __shared__ int counts[kMaxExperts];
-  __shared__ int running[kMaxExperts];
-  __shared__ int warp_cnt[32][kMaxExperts];
-  __shared__ float selv[32][32];
-  __shared__ int seg_base[kMaxExperts + 64];
-  __shared__ int gseg_base[kMaxExperts + 64];
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int nwarps = blockDim.x >> 5;
-  // Writes below may alias buffers the previous launch still reads.
-  pdl_wait();
-  pdl_trigger();
-
-  for (int e = tid; e < kMaxExperts; e += blockDim.x) { counts[e] = 0; running[e] = 0; }
-
-  // ---- top-k per token (ties to the lower expert index) ----
-  for (int t = warp; t < T; t += nwarps) {
-    float v[kMaxExperts / 32];
-    unsigned taken = 0;
-#pragma unroll
-    for (int j = 0; j < kMaxExperts / 32; ++j) {
-      const int idx = lane + 32 * j;
-      v[j] = idx < E ? logits[(size_t)t * E + idx] : -FLT_MAX;
-    }
-    for (int s = 0; s < k; ++s) {
-      float bv = -FLT_MAX;
-      int bi = INT_MAX;
-#pragma unroll
-      for (int j = 0; j < kMaxExperts / 32; ++j) {
-        const int idx = lane + 32 * j;
-        if (idx < E && !((taken >> j) & 1u) && (bi == INT_MAX || v[j] > bv)) { bv = v[j]; bi = idx; }
-      }
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-        const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
-        if (oi != INT_MAX && (bi == INT_MAX || ov > bv || (ov == bv && oi < bi))) { bv = ov; bi = oi; }
-      }
-      if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
-      if (lane == 0) {
-        o.ids[(size_t)t * k + s] = bi;
-        selv[warp][s] = bv;
-      }
-    }
-    __syncwarp();
-    if (lane < k) {
-      const float lmax = selv[warp][0];
-      float sum = 0.f;
-      for (int s = 0; s < k; ++s) sum += expf(selv[warp][s] - lmax);
-      o.w[(size_t)t * k + lane] = expf(selv[warp][lane] - lmax) / sum;
-    }
-    __syncwarp();
-  }
-  __syncthreads();
-
-  // ---- counts and offsets ----
+// Routing of a decode batch (T <= kDecMaxT, T*k <= kDecMaxTK) as a
+// standalone launch: the in-kernel routing of the decode layer kernel
+// (decode_route), written out as ids, weights, the expert-sorted permutation
+// and the expert offsets.  One CTA of kDecMaxT warps.
+__global__ void __launch_bounds__(kDecMaxT * 32)
+    route_decode_kernel(const float* __restrict__ logits, int T, int E, int k, int* ids, float* w, int* perm,
+                        int* offsets) {
+  __shared__ DecodeRoute R;
+  SmallParams p{};
+  p.logits = logits;
+  p.T = T;
+  p.E = E;
+  p.k = k;
+  p.n_shared = 0;
+  decode_route(p, R);
   const int TK = T * k;
-  for (int i = tid; i < TK; i += blockDim.x) atomicAdd(&counts[o.ids[i]], 1);
-  __syncthreads();
-  if (tid == 0) {
-    int acc = 0;
-    for (int e = 0; e < E; ++e) { o.offsets[e] = acc; seg_base[e] = acc; acc += counts[e]; }
-    o.offsets[E] = acc;
+  for (int i = threadIdx.x; i < TK; i += blockDim.x) {
+    ids[i] = R.ids[i];
+    w[i] = R.w[i];
+    perm[R.pos[i]] = i;
   }
-  __syncthreads();
-
-  // ---- stable scatter ----
-  const unsigned lt_mask = (1u << lane) - 1u;
-  for (int base = 0; base < TK; base += blockDim.x) {
-    for (int j = tid; j < 32 * kMaxExperts; j += blockDim.x) (&warp_cnt[0][0])[j] = 0;
-    __syncthreads();
-    const int i = base + tid;
-    const bool valid = i < TK;
-    const int e = valid ? o.ids[i] : -1;
-    const unsigned peers = __match_any_sync(0xffffffffu, e);
-    const int rank = __popc(peers & lt_mask);
-    if (valid && rank == 0) warp_cnt[warp][e] = __popc(peers);
-    __syncthreads();
-    if (valid) {
-      int pre = running[e];
-      for (int w = 0; w < warp; ++w) pre += warp_cnt[w][e];
-      const int pos = seg_base[e] + pre + rank;
-      o.perm[pos] = i;
-      if (o.inv) o.inv[i] = pos;
-      if (o.slot_token) o.slot_token[pos] = i / k;
-    }
-    __syncthreads();
-    for (int ee = tid; ee < E; ee += blockDim.x) {
-      int sum = 0;
-      for (int w = 0; w < 32; ++w) sum += warp_cnt[w][ee];
-      running[ee] += sum;
-    }
-    __syncthreads();
+  // offsets[e]: entries routed to experts below e (segments are in expert order)
+  for (int e = threadIdx.x; e <= E; e += blockDim.x) {
+    int before = 0;
+    for (int r = 0; r < R.nseg; ++r)
+      if (R.segs[r].expert < e) before += R.segs[r].m;
+    offsets[e] = before;
   }
-  if (o.slot_token)
-    for (int i = tid; i < n_shared * T; i += blockDim.x) o.slot_token[TK + i] = i % T;
-
-  // ---- segment tables: small-M chunks of <= 16 tokens, grouped tiles of <= 256 ----
-  if (o.nseg) {
-    const int EX = E + n_shared;
-    __syncthreads();
-    if (tid == 0) {
-      int sb = 0, gb = 0;
-      for (int e = 0; e < EX; ++e) {
-        const int cnt = e < E ? counts[e] : T;
-        const bool grouped = o.ngseg && cnt > o.thresh;
-        seg_base[e] = sb;
-        gseg_base[e] = gb;
-        if (grouped) gb += (cnt + kGTok - 1) / kGTok;
-        else sb += (cnt + kChunkTokens - 1) / kChunkTokens;
-      }
-      if (sb > o.max_seg || (o.ngseg && gb > o.max_gseg)) {
-        atomicOr(o.status, kStatusBadSegment);
-        sb = 0;  // never index past the tables
-        gb = 0;
-      }
-      *o.nseg = sb;
-      if (o.ngseg) *o.ngseg = gb;
-    }
-    __syncthreads();
-    const bool ok = *o.nseg > 0 || (o.ngseg && *o.ngseg > 0);
-    for (int e = tid; e < EX && ok; e += blockDim.x) {
-      const int cnt = e < E ? counts[e] : T;
-      const int slot_base = e < E ? o.offsets[e] : TK + (e - E) * T;
-      if (o.ngseg && cnt > o.thresh) {
-        const int nch = (cnt + kGTok - 1) / kGTok;
-        for (int c = 0; c < nch; ++c) {
-          GSeg g;
-          g.expert = e;
-          g.slot0 = slot_base + kGTok * c;
-          g.ntok = min(kGTok, cnt - kGTok * c);
-          g.pad = 0;
-          o.gsegs[gseg_base[e] + c] = g;
-        }
-        continue;
-      }
-      const int nch = (cnt + kChunkTokens - 1) / kChunkTokens;
-      for (int c = 0; c < nch; ++c) {
-        Seg s;
-        s.expert = e;
-        s.m = min(kChunkTokens, cnt - kChunkTokens * c);
-        s.tg = (s.m + 7) / 8;
-        s.slot0 = slot_base + kChunkTokens * c;
-        o.segs[seg_base[e] + c] = s;
-      }
-    }
-  }
-  if (o.tickets)
-    for (int i = tid; i < o.n_tickets; i += blockDim.x) o.tickets[i] = 0;
 }
 
 // ---- Two-kernel routing of the general path (any T) ------------------------

@@ -1,6 +1,6 @@
 // Internal: the packed weight layout shared by the host packer and the device
 // unpack.  Each table below is the register order of the device unpack in
-// qmm_small.cu; the packer writes codes where that unpack reads them.
+// unpack.cuh; the packer writes codes where that unpack reads them.
 //
 // A 16-row tile's operand for one m16n8k16 MMA k-step is held by 32 lanes:
 // lane l = 4g + q owns rows g and g+8 and k columns 2q, 2q+1 (fragment

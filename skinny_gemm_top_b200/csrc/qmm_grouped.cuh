@@ -351,18 +351,19 @@ __global__ void __launch_bounds__(kGThreads, 1)
 #pragma unroll
         for (int tt = 0; tt < kGDeqTiles; ++tt) {
           const int tile = kGDeqTiles * d + tt;
-          const float s_row[2] = {bf16_lo(sw[tt]), bf16_hi(sw[tt])};
 #pragma unroll
           for (int f = 0; f < 4; ++f) {
-            const float beta = (f >= 2) ? (float)Tr::kBetaHi : 1.0f;
-            const uint32_t negc = (f >= 2) ? Tr::kConstHi : Tr::kConstLo;   // -(128 + bias * beta)
-            const uint32_t sb = pack_bf16x2(s_row[f & 1] / beta, s_row[f & 1] / beta);  // exact: power-of-2 scaling
+            // signed code c (exact small integer): c = (128 + beta*u) / beta - (128 / beta + bias)
+            const uint32_t mul = (f >= 2) ? Tr::kCodeMulHi : kBf16One;
+            const uint32_t sub = (f >= 2) ? Tr::kCodeSubHi : Tr::kConstLo;
+            // the row's bf16 scale in both halves, straight from its bits (no fp32 round trip)
+            const uint32_t sp = __byte_perm(sw[tt], 0u, (f & 1) ? 0x3232u : 0x1010u);
             const int pr = tile * 16 + g + 8 * (f & 1);
             uint8_t* rowp = as + (pr >> 3) * 1024 + (pr & 7) * 128;
 #pragma unroll
             for (int k2 = 0; k2 < 4; ++k2) {
-              const uint32_t t = fma_bf16x2(am[tt][k2][f], 0x3F803F80u, negc);  // beta * c, exact
-              const uint32_t wv = fma_bf16x2(t, sb, 0x80008000u);              // bf16_rne(c * s)
+              const uint32_t c = fma_bf16x2(am[tt][k2][f], mul, sub);
+              const uint32_t wv = fma_bf16x2(c, sp, kBf16NegZero);  // bf16_rne(c * s): one rounding
               const int chunk = 2 * k2 + (f >> 1);
               *reinterpret_cast<uint32_t*>(rowp + ((chunk ^ (pr & 7)) << 4) + 4 * q) = wv;
             }

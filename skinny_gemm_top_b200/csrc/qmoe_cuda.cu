@@ -468,22 +468,43 @@ qmoe_status qmoe_clear_status(void) {
   return cudaMemset(di->status, 0, sizeof(unsigned)) == cudaSuccess ? QMOE_OK : QMOE_ERR_CUDA;
 }
 
+qmoe_status qmoe_route_workspace_size(int T, int E, int k, size_t* bytes) {
+  if (!bytes || T <= 0 || E <= 0 || k <= 0) return QMOE_ERR_INVALID_ARG;
+  if (E > kMaxExperts || k > 32 || k > E) return QMOE_ERR_UNSUPPORTED;
+  *bytes = (T <= kDecMaxT && T * k <= kDecMaxTK) ? 0 : align_up((size_t)((T + kRouteChunk - 1) / kRouteChunk) * E * 4);
+  return QMOE_OK;
+}
+
 qmoe_status qmoe_route(const float* logits, int T, int E, int k, int32_t* ids, float* weights, int32_t* perm,
-                       int32_t* offsets, void* stream) {
+                       int32_t* offsets, void* ws, size_t ws_bytes, void* stream) {
   if (!logits || !ids || !weights || !perm || !offsets || T <= 0 || E <= 0 || k <= 0) return QMOE_ERR_INVALID_ARG;
   if (E > kMaxExperts || k > 32 || k > E) return QMOE_ERR_UNSUPPORTED;
+  size_t need = 0;
+  qmoe_route_workspace_size(T, E, k, &need);
+  if (need > ws_bytes || (need && !ws)) return QMOE_ERR_SCRATCH;
+  if (reinterpret_cast<uintptr_t>(ws) & 15) return QMOE_ERR_INVALID_ARG;
   DevInfo* di;
   qmoe_status s = dev_info(&di);
   if (s != QMOE_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  TraceScope ts(st, K_ROUTE);
+  if (need == 0) {  // decode batch: the decode layer kernel's routing, as one CTA
+    route_decode_kernel<<<1, kDecMaxT * 32, 0, st>>>(logits, T, E, k, ids, weights, perm, offsets);
+    return cudaGetLastError() == cudaSuccess ? QMOE_OK : QMOE_ERR_CUDA;
+  }
   RouteOut o{};
   o.ids = ids;
   o.w = weights;
   o.perm = perm;
   o.offsets = offsets;
   o.status = di->status;
-  TraceScope ts(static_cast<cudaStream_t>(stream), K_ROUTE);
-  route_kernel<<<1, kRouteThreads, 0, static_cast<cudaStream_t>(stream)>>>(logits, T, E, k, 0, o);
-  return cudaGetLastError() == cudaSuccess ? QMOE_OK : QMOE_ERR_CUDA;
+  o.chunk_counts = static_cast<int*>(ws);
+  const int nchunks = (T + kRouteChunk - 1) / kRouteChunk;
+  if (launch_pdl(route_topk_kernel, dim3(nchunks), dim3(kRouteWarps * 32), 0, st, logits, T, E, k, o) !=
+          cudaSuccess ||
+      launch_pdl(route_scatter_kernel, dim3(nchunks), dim3(kRouteWarps * 32), 0, st, T, E, k, 0, o) != cudaSuccess)
+    return QMOE_ERR_CUDA;
+  return QMOE_OK;
 }
 
 qmoe_status qmoe_workspace_size(const qmoe_layer* layer, int T, size_t* bytes) {

@@ -16,6 +16,8 @@ constexpr uint32_t kBf16Sixteenth = 0x3D803D80u;  // (1/16, 1/16)
 constexpr uint32_t kBf16Quarter = 0x3E803E80u;    // (1/4, 1/4)
 constexpr uint32_t kBf16_120 = 0x42F042F0u;       // (120, 120)
 constexpr uint32_t kBf16_96 = 0x42C042C0u;        // (96, 96)
+constexpr uint32_t kBf16One = 0x3F803F80u;        // (1, 1)
+constexpr uint32_t kBf16NegZero = 0x80008000u;    // (-0, -0): x + (-0) = x for every x
 
 template <int FMT> struct FmtTraits;
 template <> struct FmtTraits<2> {             // INT2: codes -2..1, u = c + 2
@@ -25,6 +27,8 @@ template <> struct FmtTraits<2> {             // INT2: codes -2..1, u = c + 2
   static constexpr int kBetaHi = 4;
   static constexpr uint32_t kConstLo = 0xC302C302u;  // -(128 + 2)     = -130
   static constexpr uint32_t kConstHi = 0xC308C308u;  // -(128 + 2 * 4) = -136
+  static constexpr uint32_t kCodeMulHi = 0x3E803E80u;  // 1/4: (128 + 4u) / 4 = 32 + u
+  static constexpr uint32_t kCodeSubHi = 0xC208C208u;  // -(32 + 2) = -34
 };
 template <> struct FmtTraits<4> {             // INT4: codes -8..7, u = c + 8
   static constexpr int kKUcols = 64;
@@ -33,6 +37,8 @@ template <> struct FmtTraits<4> {             // INT4: codes -8..7, u = c + 8
   static constexpr int kBetaHi = 1;
   static constexpr uint32_t kConstLo = 0xC308C308u;  // -(128 + 8) = -136
   static constexpr uint32_t kConstHi = 0xC308C308u;
+  static constexpr uint32_t kCodeMulHi = 0x3F803F80u;  // 1
+  static constexpr uint32_t kCodeSubHi = 0xC308C308u;  // -136
 };
 template <> struct FmtTraits<3> {             // ternary: t in {-1,0,1}, digit d = t + 1
   static constexpr int kKUcols = 128;
@@ -41,6 +47,8 @@ template <> struct FmtTraits<3> {             // ternary: t in {-1,0,1}, digit d
   static constexpr int kBetaHi = 4;
   static constexpr uint32_t kConstLo = 0xC301C301u;  // -(128 + 1)     = -129
   static constexpr uint32_t kConstHi = 0xC304C304u;  // -(128 + 1 * 4) = -132
+  static constexpr uint32_t kCodeMulHi = 0x3E803E80u;  // 1/4
+  static constexpr uint32_t kCodeSubHi = 0xC204C204u;  // -(32 + 1) = -33
 };
 
 // INT2: one lane word (16 codes) -> A registers of two consecutive k-steps.

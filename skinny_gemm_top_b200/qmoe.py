@@ -49,8 +49,9 @@ EXPORTS = {
     "qmoe_unpack_host": [C.c_int, C.c_int, C.c_void_p, C.c_void_p, C.c_int, C.c_int, C.c_int, C.c_void_p,
                          C.c_void_p],
     "qmoe_dequant": [C.POINTER(Weights), C.c_int, C.c_int, C.c_int, C.c_int, C.c_void_p, C.c_void_p, C.c_void_p],
+    "qmoe_route_workspace_size": [C.c_int, C.c_int, C.c_int, C.POINTER(C.c_size_t)],
     "qmoe_route": [C.c_void_p, C.c_int, C.c_int, C.c_int, C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p,
-                   C.c_void_p],
+                   C.c_void_p, C.c_size_t, C.c_void_p],
     "qmoe_workspace_size": [C.POINTER(Layer), C.c_int, C.POINTER(C.c_size_t)],
     "qmoe_forward": [C.POINTER(Layer), C.c_void_p, C.c_void_p, C.c_int, C.c_void_p, C.c_void_p, C.c_size_t,
                      C.c_void_p],
@@ -161,10 +162,17 @@ def dequant(w: Weights, row_order: int, rows: int, K: int, n_mats: int, out_f32=
                              _stream(stream)), "qmoe_dequant")
 
 
-def route(logits, k: int, ids, weights, perm, offsets, stream=None):
+def route_workspace_size(T: int, E: int, k: int) -> int:
+    b = C.c_size_t()
+    _check(_lib.qmoe_route_workspace_size(T, E, k, C.byref(b)), "qmoe_route_workspace_size")
+    return b.value
+
+
+def route(logits, k: int, ids, weights, perm, offsets, ws=None, ws_bytes: int | None = None, stream=None):
     T, E = logits.shape
-    _check(_lib.qmoe_route(_ptr(logits), T, E, k, _ptr(ids), _ptr(weights), _ptr(perm), _ptr(offsets),
-                           _stream(stream)), "qmoe_route")
+    nbytes = (0 if ws is None else ws.numel() * ws.element_size()) if ws_bytes is None else ws_bytes
+    _check(_lib.qmoe_route(_ptr(logits), T, E, k, _ptr(ids), _ptr(weights), _ptr(perm), _ptr(offsets), _ptr(ws),
+                           nbytes, _stream(stream)), "qmoe_route")
 
 
 def workspace_size(layer: Layer, T: int) -> int:

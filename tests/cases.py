@@ -17,6 +17,18 @@ REL_L2 = 5e-3
 MAX_ERR_RMS = 3e-2
 
 
+def block_scaled_weights(seed, rows, K, block, factors):
+    """N(0, 0.02) bf16 weights whose 64/128-column blocks are multiplied by
+    `factors` in turn: tiny blocks give tiny normal and subnormal bf16 scales."""
+    w = synth.bf16_bits_to_f32(synth.normal_bf16(seed, 60, 99, (rows, K), 0.02))
+    f = np.asarray(factors, dtype=np.float32)
+    per_col = np.repeat(f[np.arange(K // block) % len(f)], block)
+    return synth.f32_to_bf16_bits(w * per_col[None, :])
+
+
+TINY_FACTORS = (1.0, 1e-30, 1e-36, 2e-37, 1e-38, 1e-39, 3e-40)
+
+
 def to_dev(a: np.ndarray):
     import torch
     a = np.ascontiguousarray(a)

@@ -54,6 +54,21 @@ def test_pack_matches_oracle_quantizer(fmt, block, order):
     assert np.array_equal(Q.bf16_bits_to_f64(s), os_)
 
 
+@pytest.mark.parametrize("fmt,block", [(qmoe.INT2, 64), (qmoe.INT4, 128), (qmoe.TERNARY, 64)])
+def test_pack_matches_oracle_quantizer_tiny_and_subnormal(fmt, block):
+    """Blocks scaled down to tiny normal and subnormal bf16 values: both
+    quantizers give the same codes and scales (subnormal scales included)."""
+    from cases import TINY_FACTORS, block_scaled_weights
+    rows, K = 32, 896
+    w = block_scaled_weights(5, rows, K, block, TINY_FACTORS)
+    codes, scales = qmoe.pack(fmt, qmoe.ROWS_PLAIN, w, block)
+    c, s = qmoe.unpack_host(fmt, qmoe.ROWS_PLAIN, codes, scales, rows, K, block)
+    oc, os_ = _oracle_q(fmt, w, block)
+    assert np.any((os_ > 0) & (os_ < 2.0 ** -126))
+    assert np.array_equal(c, oc)
+    assert np.array_equal(Q.bf16_bits_to_f64(s), os_)
+
+
 def test_pack_sizes_are_the_format_densities():
     assert qmoe.pack_size(qmoe.INT2, 16, 5120, 128) == (16 * 5120 // 4, 16 * 40 * 2)
     assert qmoe.pack_size(qmoe.INT4, 16, 5120, 128) == (16 * 5120 // 2, 16 * 40 * 2)

@@ -8,7 +8,8 @@ import pytest
 from oracle import qmoe_oracle as Q
 from skinny_gemm_top_b200 import synth
 
-from cases import FMTS, MAX_ERR_RMS, REL_L2, MoECase, bf16_dev_to_f64, oracle_quant, small_cfg, to_dev
+from cases import (FMTS, MAX_ERR_RMS, REL_L2, TINY_FACTORS, MoECase, bf16_dev_to_f64, block_scaled_weights,
+                   oracle_quant, small_cfg, to_dev)
 
 pytestmark = pytest.mark.gpu
 
@@ -29,12 +30,17 @@ def _close(got, ref, what=""):
 
 # ------------------------------------------------------------------ dequant
 
-@pytest.mark.parametrize("fmt,block,order", [
-    ("int2", 64, 1), ("int2", 128, 0), ("int4", 64, 0), ("int4", 128, 1), ("ternary", 64, 1), ("ternary", 64, 0)])
-def test_dequant_bit_exact(qm, fmt, block, order):
+@pytest.mark.parametrize("fmt,block,order,tiny", [
+    ("int2", 64, 1, False), ("int2", 128, 0, False), ("int4", 64, 0, False), ("int4", 128, 1, False),
+    ("ternary", 64, 1, False), ("ternary", 64, 0, False),
+    ("int2", 64, 0, True), ("int4", 128, 0, True), ("ternary", 64, 0, True)])
+def test_dequant_bit_exact(qm, fmt, block, order, tiny):
     import torch
-    rows, K, n = 48, 384, 2
-    mats = [synth.normal_bf16(21, 60, i, (rows, K), 0.02) for i in range(n)]
+    rows, K, n = 48, 384 if not tiny else 896, 2
+    if tiny:  # blocks with tiny normal and subnormal scales
+        mats = [block_scaled_weights(21 + i, rows, K, block, TINY_FACTORS) for i in range(n)]
+    else:
+        mats = [synth.normal_bf16(21, 60, i, (rows, K), 0.02) for i in range(n)]
     c, s = qm.pack_stack(FMTS[fmt], order, mats, block)
     dc, ds = to_dev(c), to_dev(s)
     w = qm.make_weights(FMTS[fmt], block, dc, ds)
@@ -44,33 +50,109 @@ def test_dequant_bit_exact(qm, fmt, block, order):
     torch.cuda.synchronize()
     for i in range(n):
         codes, scales = oracle_quant(fmt, mats[i], block)
+        if tiny:
+            assert np.any((scales > 0) & (scales < 2.0 ** -126)), "no subnormal scale drawn"
         ref = Q.dequant(codes, scales, block)
         assert np.array_equal(o32[i].cpu().numpy().astype(np.float64), ref)
         ref16 = Q.dequant_bf16_operand(codes, scales, block)
         assert np.array_equal(Q.bf16_bits_to_f64(o16[i].cpu().numpy().view(np.uint16)), ref16)
 
 
+@pytest.mark.parametrize("fmt,block,tiny", [("int2", 64, False), ("int4", 64, False), ("int2", 128, True),
+                                            ("int4", 64, True), ("int4", 128, True)])
+def test_grouped_operand_bit_exact_one_hot(qm, fmt, block, tiny):
+    """The tcgen05 path's weight operand bf16_rne(c*s), through its own code:
+    128 one-hot token rows (row m = 2^64 e_{k_m}) through qmoe_linear, which
+    takes the grouped path from 48 rows on.  y[m, n] = bf16(2^64 W_op[n, k_m])
+    exactly (one nonzero product, accumulated in fp32, already on the bf16
+    grid), so y / 2^64 is the operand column k_m, bit for bit; the 2^64 keeps
+    products and outputs of subnormal operands normal."""
+    import torch
+    N, K, M = 256, 1024, 128
+    wb = block_scaled_weights(31, N, K, block, TINY_FACTORS) if tiny else synth.linear_weight(31, N, K)
+    c, s = qm.pack(FMTS[fmt], 0, wb, block)
+    dc, ds = to_dev(c), to_dev(s)
+    w = qm.make_weights(FMTS[fmt], block, dc, ds)
+    km = (np.arange(M) * 37 + 5) % K          # every k-step column class, every block
+    x = np.zeros((M, K), dtype=np.uint16)
+    x[np.arange(M), km] = synth.f32_to_bf16_bits(np.float32(2.0 ** 64))
+    y = torch.empty((M, N), dtype=torch.int16, device="cuda")
+    ws = torch.empty(qm.linear_workspace_size(N, K, M), dtype=torch.uint8, device="cuda")
+    qm.linear(w, N, K, to_dev(x), y, ws)
+    torch.cuda.synchronize()
+    st = qm.get_stats()
+    assert st.last_path == qm.PATH_GROUPED
+    got = bf16_dev_to_f64(y) * 2.0 ** -64
+    codes, scales = oracle_quant(fmt, wb, block)
+    if tiny:
+        assert np.any((scales > 0) & (scales < 2.0 ** -126)), "no subnormal scale drawn"
+    op = Q.dequant_bf16_operand(codes, scales, block)   # [N, K]
+    assert np.array_equal(got, op[:, km].T)
+
+
 # ------------------------------------------------------------------ routing
 
-@pytest.mark.parametrize("T,E,k,seed", [(1, 8, 2, 1), (37, 64, 6, 2), (300, 128, 8, 3), (129, 256, 1, 4),
-                                        (1100, 64, 6, 5)])
-def test_route_matches_oracle(qm, T, E, k, seed):
+def _route_case(qm, lg, k):
     import torch
-    g = np.random.default_rng(seed)
-    lg = g.standard_normal((T, E)).astype(np.float32)
-    lg[::3, :: 5] = 0.5          # ties
-    d = torch.from_numpy(lg).cuda()
-    ids = torch.empty((T, k), dtype=torch.int32, device="cuda")
-    w = torch.empty((T, k), dtype=torch.float32, device="cuda")
-    perm = torch.empty(T * k, dtype=torch.int32, device="cuda")
-    off = torch.empty(E + 1, dtype=torch.int32, device="cuda")
-    qm.route(d, k, ids, w, perm, off)
+    T, E = lg.shape
+    d = torch.from_numpy(np.ascontiguousarray(lg)).cuda()
+    ids = torch.full((T, k), -1, dtype=torch.int32, device="cuda")
+    w = torch.full((T, k), -1.0, dtype=torch.float32, device="cuda")
+    perm = torch.full((T * k,), -1, dtype=torch.int32, device="cuda")
+    off = torch.full((E + 1,), -1, dtype=torch.int32, device="cuda")
+    nb = qm.route_workspace_size(T, E, k)
+    ws = torch.empty(max(nb, 16), dtype=torch.uint8, device="cuda") if nb else None
+    qm.route(d, k, ids, w, perm, off, ws)
     torch.cuda.synchronize()
     rids, rw, rperm, roff = Q.route(lg, k)
     assert np.array_equal(ids.cpu().numpy(), rids)
     assert np.array_equal(perm.cpu().numpy(), rperm)
     assert np.array_equal(off.cpu().numpy(), roff)
     assert np.allclose(w.cpu().numpy(), rw, rtol=1e-6, atol=0)
+    return nb
+
+
+def _tied_logits(g, T, E):
+    """Few distinct values, both signs of zero: many exact ties."""
+    lg = (np.round(g.standard_normal((T, E)) * 2.0) / 2.0).astype(np.float32)
+    lg[:, 1::5] = -0.0
+    lg[:, 3::5] = 0.0
+    lg[::2, 7::9] = 0.5
+    return lg
+
+
+# Decode routing (T <= 8, T*k <= 64): the routing the fused decode layer kernel runs in its prologue.
+@pytest.mark.parametrize("E,k", [(8, 2), (64, 6), (100, 7), (128, 8), (256, 8), (256, 1), (64, 32)])
+@pytest.mark.parametrize("T", [1, 3, 8])
+@pytest.mark.parametrize("tied", [False, True])
+def test_route_decode_matches_oracle(qm, T, E, k, tied):
+    if T * k > 64:
+        pytest.skip("not a decode batch")
+    g = np.random.default_rng(1000 * T + E + k)
+    lg = _tied_logits(g, T, E) if tied else g.standard_normal((T, E)).astype(np.float32)
+    assert _route_case(qm, lg, k) == 0  # no workspace: the decode routing ran
+
+
+# General routing (two launches: per-chunk top-k and counts, stable scatter), as qmoe_forward runs it above 8 tokens.
+@pytest.mark.parametrize("T,E,k", [(9, 64, 6), (37, 8, 2), (300, 128, 8), (1100, 64, 6), (4096, 128, 8),
+                                   (4096, 256, 8), (129, 256, 1), (3, 64, 32)])
+@pytest.mark.parametrize("tied", [False, True])
+def test_route_general_matches_oracle(qm, T, E, k, tied):
+    g = np.random.default_rng(7 * T + E + k)
+    lg = _tied_logits(g, T, E) if tied else g.standard_normal((T, E)).astype(np.float32)
+    assert _route_case(qm, lg, k) > 0  # workspace needed: the general routing ran
+
+
+def test_route_rejects_small_workspace(qm):
+    import torch
+    T, E, k = 100, 64, 6
+    lg = torch.zeros((T, E), dtype=torch.float32, device="cuda")
+    out = [torch.empty(T * k, dtype=torch.int32, device="cuda"), torch.empty(T * k, dtype=torch.float32, device="cuda"),
+           torch.empty(T * k, dtype=torch.int32, device="cuda"), torch.empty(E + 1, dtype=torch.int32, device="cuda")]
+    ws = torch.empty(16, dtype=torch.uint8, device="cuda")
+    with pytest.raises(qm.QmoeError) as e:
+        qm.route(lg, k, *out, ws)
+    assert e.value.status == qm.ERR_SCRATCH
 
 
 # ------------------------------------------------------------------ single linear

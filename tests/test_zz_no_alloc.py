@@ -1,5 +1,6 @@
 """qmoe_forward_static (library-owned scratch, no allocation) against the
-workspace entry point qmoe_forward, through the C ABI.
+workspace entry point qmoe_forward and against the fp64 oracle, through the
+C ABI.
 
 Collected after the other test files on purpose: the static scratch is
 resolved on its first use, and these tests must pass both alone and after
@@ -47,13 +48,17 @@ def test_static_matches_workspace_forward_twice(qm, name, T):
     torch.cuda.synchronize()
     ref = bf16_dev_to_f64(y_ref)
     assert np.all(np.isfinite(ref))
+    x_bits = synth.tokens(cfg.H, 11, T)
+    oracle = Q.moe_forward(Q.bf16_bits_to_f64(x_bits), synth.router_logits(cfg, 11, T), cfg.k, case.bank)
+    assert Q.rel_l2(ref, oracle) <= REL_L2 and Q.max_err_over_rms(ref, oracle) <= MAX_ERR_RMS, (name, T)
     for call in range(2):  # two calls in a row on the same static scratch
         y = torch.full((T, cfg.H), -1, dtype=torch.int16, device="cuda")
         qm.forward_static(layer, x, lg, y)
         torch.cuda.synchronize()
         got = bf16_dev_to_f64(y)
-        assert Q.rel_l2(got, ref) <= REL_L2, (name, T, call)
-        assert Q.max_err_over_rms(got, ref) <= MAX_ERR_RMS, (name, T, call)
+        for what, want in (("workspace forward", ref), ("oracle", oracle)):
+            assert Q.rel_l2(got, want) <= REL_L2, (name, T, call, what)
+            assert Q.max_err_over_rms(got, want) <= MAX_ERR_RMS, (name, T, call, what)
     assert qm.get_stats().device_status == 0
 
 
