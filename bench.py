@@ -144,14 +144,14 @@ def pack_moe(qmoe, torch, rotate: int):
     n = CFG.E + CFG.n_shared
     f1, f2 = qmoe.FMT[CFG.fc1_fmt], qmoe.FMT[CFG.fc2_fmt]
     c1, s1 = qmoe.pack_stack(f1, qmoe.ROWS_GATE_UP, (synth.expert_fc1(CFG, SEED, e) for e in range(n)), CFG.block)
-    c2, s2 = qmoe.pack_stack(f2, qmoe.ROWS_PLAIN, (synth.expert_fc2(CFG, SEED, e) for e in range(n)), CFG.block)
+    c2, s2 = qmoe.pack_stack(f2, qmoe.ROWS_KSPLIT, (synth.expert_fc2(CFG, SEED, e) for e in range(n)), CFG.block)
     dev = [_to_dev(torch, a) for a in (c1, s1, c2, s2)]
     layers, keep = [], []
     for r in range(rotate):
         copies = dev if r == 0 else [t.clone() for t in dev]
         keep.append(copies)
-        w1 = qmoe.make_weights(f1, CFG.block, copies[0], copies[1])
-        w2 = qmoe.make_weights(f2, CFG.block, copies[2], copies[3])
+        w1 = qmoe.make_weights(f1, CFG.block, copies[0], copies[1], None, qmoe.ROWS_GATE_UP)
+        w2 = qmoe.make_weights(f2, CFG.block, copies[2], copies[3], None, qmoe.ROWS_KSPLIT)
         layers.append(qmoe.make_layer(CFG.H, CFG.I, CFG.E, CFG.k, CFG.n_shared, w1, w2))
     return layers, keep
 
@@ -503,15 +503,15 @@ def pack_cfg(qmoe, torch, cfg):
     n = cfg.E + cfg.n_shared
     f1, f2 = qmoe.FMT[cfg.fc1_fmt], qmoe.FMT[cfg.fc2_fmt]
     c1, s1 = qmoe.pack_stack(f1, qmoe.ROWS_GATE_UP, (synth.expert_fc1(cfg, SEED, e) for e in range(n)), cfg.block)
-    c2, s2 = qmoe.pack_stack(f2, qmoe.ROWS_PLAIN, (synth.expert_fc2(cfg, SEED, e) for e in range(n)), cfg.block)
+    c2, s2 = qmoe.pack_stack(f2, qmoe.ROWS_KSPLIT, (synth.expert_fc2(cfg, SEED, e) for e in range(n)), cfg.block)
     keep = [_to_dev(torch, a) for a in (c1, s1, c2, s2)]
     b1 = b2 = None
     if cfg.bias:
         b1 = _to_dev(torch, np.stack([synth.expert_b1(cfg, SEED, e) for e in range(n)]))
         b2 = _to_dev(torch, np.stack([synth.expert_b2(cfg, SEED, e) for e in range(n)]))
         keep += [b1, b2]
-    w1 = qmoe.make_weights(f1, cfg.block, keep[0], keep[1], b1)
-    w2 = qmoe.make_weights(f2, cfg.block, keep[2], keep[3], b2)
+    w1 = qmoe.make_weights(f1, cfg.block, keep[0], keep[1], b1, qmoe.ROWS_GATE_UP)
+    w2 = qmoe.make_weights(f2, cfg.block, keep[2], keep[3], b2, qmoe.ROWS_KSPLIT)
     return qmoe.make_layer(cfg.H, cfg.I, cfg.E, cfg.k, cfg.n_shared, w1, w2), keep
 
 

@@ -58,10 +58,15 @@ typedef enum {
   QMOE_INT4 = 4               /* symmetric, codes -8..7, 8 codes per u32            */
 } qmoe_fmt;
 
-/* Row order of a packed matrix.  GATE_UP is for FC1 whose logical rows
- * interleave gate and up (row 2j = gate j, row 2j+1 = up j, the fused SwiGLU
- * layout of the onnxruntime PR, Current Scope "swiglu_fusion=1"). */
-typedef enum { QMOE_ROWS_PLAIN = 0, QMOE_ROWS_GATE_UP = 1 } qmoe_row_order;
+/* Row order (and code layout) of a packed matrix.
+ *   GATE_UP: FC1, whose logical rows interleave gate and up (row 2j = gate j,
+ *     row 2j+1 = up j: the fused SwiGLU layout of the onnxruntime PR, Current
+ *     Scope "swiglu_fusion=1").
+ *   PLAIN:   rows in order (the single linear).
+ *   KSPLIT:  rows in order, codes laid out so that a narrow range of K columns
+ *     of all rows is one contiguous run (FC2 of a MoE layer, whose K = I is
+ *     split across blocks by the decode kernel; see the layout below). */
+typedef enum { QMOE_ROWS_PLAIN = 0, QMOE_ROWS_GATE_UP = 1, QMOE_ROWS_KSPLIT = 2 } qmoe_row_order;
 
 /* Expert-compute path selection; AUTO picks per expert by its token count. */
 typedef enum { QMOE_PATH_AUTO = 0, QMOE_PATH_SMALL_M = 1, QMOE_PATH_GROUPED = 2 } qmoe_path;
@@ -83,10 +88,17 @@ typedef enum { QMOE_PATH_AUTO = 0, QMOE_PATH_SMALL_M = 1, QMOE_PATH_GROUPED = 2 
  * Each lane l (g = l/4, q = l%4) of a 32-lane warp owns the operand
  * fragment of an m16n8k16 MMA: rows g and g+8, k = 16ks + 2q + {0,1} and
  * 16ks + 2q + 8 + {0,1}.
- *   INT2/INT4 codes: [K/64][NT][32 lanes][W u32], W = 2 (INT2) or 4 (INT4);
- *     bytes = rows*K*bits/8.  Bit positions inside a lane's words follow the
- *     register order of the kernels' unpack; qmoe_unpack_host() inverts it.
- *   TERNARY codes: [K/128][NT][32 lanes][13 bytes]; bytes = rows*K*13/64 (1.625 bits per weight).
+ *   INT2/INT4 codes (GATE_UP, PLAIN): [K/64][NT][32 lanes][W u32], W = 2
+ *     (INT2) or 4 (INT4); word w of a lane covers k-steps 2w, 2w+1 (INT2) or
+ *     k-step w (INT4) of the 64 columns.  bytes = rows*K*bits/8.  Bit
+ *     positions inside a lane's words follow the register order of the
+ *     kernels' unpack; qmoe_unpack_host() inverts it.
+ *   INT2/INT4 codes (KSPLIT): the same words, slab-major:
+ *     [K/64][W][NT][32 lanes][1 u32] = one slab of 32 (INT2) or 16 (INT4)
+ *     columns of all rows per (K/64, w), contiguous.
+ *   TERNARY codes: [K/128][NT][32 lanes][13 bytes] for every row order (a
+ *     lane record is already one slab of 128 columns); bytes = rows*K*13/64
+ *     (1.625 bits per weight).
  *   Scales: [K/B][NT][8 u32], u32 g = s(row g) | s(row g+8) << 16 (bf16 bits);
  *     bytes = rows*(K/B)*2.
  * A layer's experts are packed one after another with the same strides.
@@ -108,21 +120,24 @@ qmoe_status qmoe_unpack_host(int fmt, int row_order, const void* codes, const vo
                              int rows, int K, int block, int8_t* codes_out, uint16_t* scales_out);
 
 /* One quantized weight set: n matrices of the same shape packed back to back
- * (matrix e at codes + e*codes_bytes, scales + e*scales_bytes), optional bf16
- * bias [n][rows] in logical row order (NULL = none).  Device pointers. */
+ * (matrix e at codes + e*codes_bytes, scales + e*scales_bytes) with the row
+ * order they were packed with, optional bf16 bias [n][rows] in logical row
+ * order (NULL = none).  Device pointers. */
 typedef struct {
   int fmt;
   int block;
+  int row_order;
   const void* codes;
   const void* scales;
   const uint16_t* bias;
 } qmoe_weights;
 
 /* Dequantize n_mats packed matrices (device): out_f32[e][rows][K] = c*s
- * (exact) and/or out_bf16 = bf16_rne(c*s), logical row order.  Debug and
- * parity entry point; uses the hot kernels' unpack routines. */
-qmoe_status qmoe_dequant(const qmoe_weights* w, int row_order, int rows, int K, int n_mats,
-                         float* out_f32, uint16_t* out_bf16, void* stream);
+ * (exact) and/or out_bf16 = bf16_rne(c*s), logical row order (w->row_order
+ * gives the packing).  Debug and parity entry point; uses the hot kernels'
+ * unpack routines. */
+qmoe_status qmoe_dequant(const qmoe_weights* w, int rows, int K, int n_mats, float* out_f32,
+                         uint16_t* out_bf16, void* stream);
 
 /* Routing (device): logits fp32 [T, E] -> ids int32 [T, k] (descending logit,
  * ties to the lower index, -0 equal to +0), weights fp32 [T, k] (softmax over
@@ -144,7 +159,8 @@ qmoe_status qmoe_route(const float* logits, int T, int E, int k, int32_t* ids, f
 
 /* One MoE layer.  fc1: E + n_shared matrices [2I, H] packed with
  * QMOE_ROWS_GATE_UP (shared experts after the routed ones); bias [.][2I].
- * fc2: E + n_shared matrices [H, I] packed with QMOE_ROWS_PLAIN; bias [.][H].
+ * fc2: E + n_shared matrices [H, I] packed with QMOE_ROWS_KSPLIT; bias [.][H].
+ * Other row orders are rejected (QMOE_ERR_INVALID_ARG).
  * H % 64 == 0, I % 64 == 0; E <= 256; shared experts get every token with
  * weight 1.  max_row_tile bounds the tokens per row tile (0 = none). */
 typedef struct {
@@ -161,12 +177,15 @@ qmoe_status qmoe_workspace_size(const qmoe_layer* layer, int T, size_t* bytes);
 /* y[T, H] bf16 = MoE(x[T, H] bf16, logits[T, E] fp32).  With ws_bytes below
  * qmoe_workspace_size(T), tokens are processed in row tiles (halved until the
  * tile's workspace fits, explicit partial last tile); QMOE_ERR_SCRATCH when
- * one row does not fit.  ws must be 256-byte aligned.
- * A decode batch (T <= 8, T*k <= 64) whose FC1 and FC2 share a format runs as
- * one kernel with one block per SM and a grid-wide barrier: it needs every SM
- * of the device at once.  Kernels of other streams that hold SMs only delay
- * it; if the barrier waits longer than 2 s the call reports the timeout flag
- * in the device status word (qmoe_get_stats) instead of hanging. */
+ * one row does not fit.  ws must be 256-byte aligned, x 16-byte aligned, y
+ * 8-byte aligned.
+ * A decode batch (T <= 8, T*k <= 64, H <= 2112) runs as one kernel that
+ * routes in its prologue and splits every selected expert's intermediate
+ * dimension across the SMs; its blocks never wait for one another.  Their
+ * partial outputs are summed with fp32 atomic adds, so the summation order,
+ * and with it the last bit of an output, can differ between runs.  Larger
+ * batches run routing, expert and combine kernels in sequence; their results
+ * do not depend on scheduling.  No part of ws needs any initial contents. */
 qmoe_status qmoe_forward(const qmoe_layer* layer, const uint16_t* x, const float* logits, int T,
                          uint16_t* y, void* ws, size_t ws_bytes, void* stream);
 
@@ -181,15 +200,15 @@ qmoe_status qmoe_forward(const qmoe_layer* layer, const uint16_t* x, const float
  * exceeds the array (no row tiling; nothing is launched).  The first call on
  * a device resolves the array's address (cudaGetSymbolAddress with that
  * device current) and can load the library's device code: make it before any
- * stream capture.  No scratch value must start at zero (the per-tile tickets
- * are cleared inside each call).  Calls that overlap in time on one device
- * share the array and race: serialise them. */
+ * stream capture.  No scratch value needs to start at any particular value:
+ * each call clears what it reads before writing it.  Calls that overlap in
+ * time on one device share the array and race: serialise them. */
 #define QMOE_STATIC_SCRATCH_BYTES (8u << 20)
 qmoe_status qmoe_forward_static(const qmoe_layer* layer, const uint16_t* x, const float* logits, int T,
                                 uint16_t* y, void* stream);
 
 /* Single quantized linear y[M, N] bf16 = x[M, K] bf16 @ dequant(W)[N, K]^T,
- * W packed PLAIN.  M >= 1. */
+ * W packed PLAIN (other row orders: QMOE_ERR_INVALID_ARG).  M >= 1. */
 qmoe_status qmoe_linear_workspace_size(int N, int K, int M, size_t* bytes);
 qmoe_status qmoe_linear(const qmoe_weights* w, int N, int K, const uint16_t* x, int M,
                         uint16_t* y, void* ws, size_t ws_bytes, void* stream);

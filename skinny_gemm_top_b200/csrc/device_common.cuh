@@ -57,6 +57,33 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// try_wait with a suspend-time hint: the thread sleeps until the phase
+// completes or about hint_ns elapse, instead of returning at once.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_addr(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
+// mbar_wait_bounded without busy polling: sleeps in try_wait between checks of the clock.
+__device__ __forceinline__ bool mbar_wait_sleep_bounded(uint64_t* bar, uint32_t parity, unsigned* status) {
+  if (mbar_try_wait_sleep(bar, parity, 100000u)) return true;
+  const unsigned long long t0 = global_timer_ns();
+  for (;;) {
+    if (mbar_try_wait_sleep(bar, parity, 100000u)) return true;
+    if (global_timer_ns() - t0 > kWaitLimitNs) {
+      if (status) atomicOr(status, kStatusTimeout);
+      return false;
+    }
+  }
+}
+
 // Waits for the phase with the given parity to complete.  Gives up after
 // kWaitLimitNs, ORs kStatusTimeout into *status and returns false.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, unsigned* status) {
@@ -101,49 +128,6 @@ __device__ __forceinline__ int atomic_add_acq_rel_gpu(int* p, int v) {
   int old;
   asm volatile("atom.add.acq_rel.gpu.global.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
   return old;
-}
-
-__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
-  int v;
-  asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
-
-__device__ __forceinline__ void red_add_release_gpu(int* p, int v) {
-  asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-
-// Split barrier over all CTAs of a launch whose CTAs are all resident at once
-// (one per SM).  *count starts the launch at 0 (cleared by the launch before)
-// and is used once.  grid_arrive (every thread, after a CTA barrier that
-// follows the CTA's writes) publishes them; grid_wait (every thread) returns
-// once every CTA has arrived, with all arrived CTAs' writes visible.  Work
-// that needs no other CTA's writes goes between the two.  grid_wait gives up
-// after kWaitLimitNs (status flag) and returns false then, in every thread.
-__device__ __forceinline__ void grid_arrive(int* count) {
-  if (threadIdx.x == 0) red_add_release_gpu(count, 1);  // cumulative: covers the writes the CTA barrier ordered
-}
-
-__device__ __forceinline__ bool grid_wait(const int* count, unsigned* status, int* s_ok) {
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    int ok = 1;
-    const int n = (int)gridDim.x;
-    if (ld_acquire_gpu(count) < n) {
-      const unsigned long long t0 = global_timer_ns();
-      for (uint32_t it = 1;; ++it) {
-        if (ld_acquire_gpu(count) >= n) break;
-        if ((it & 63) == 0 && global_timer_ns() - t0 > kWaitLimitNs) {
-          atomicOr(status, kStatusTimeout);
-          ok = 0;
-          break;
-        }
-      }
-    }
-    *s_ok = ok;
-  }
-  __syncthreads();
-  return *s_ok != 0;
 }
 
 // D (+)= A * B, m16n8k16, bf16 inputs, fp32 accumulators.

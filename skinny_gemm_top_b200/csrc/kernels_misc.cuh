@@ -38,13 +38,7 @@ __global__ void __launch_bounds__(kDecMaxT * 32)
     route_decode_kernel(const float* __restrict__ logits, int T, int E, int k, int* ids, float* w, int* perm,
                         int* offsets) {
   __shared__ DecodeRoute R;
-  SmallParams p{};
-  p.logits = logits;
-  p.T = T;
-  p.E = E;
-  p.k = k;
-  p.n_shared = 0;
-  decode_route(p, R);
+  decode_route(logits, T, E, k, R);
   const int TK = T * k;
   for (int i = threadIdx.x; i < TK; i += blockDim.x) {
     ids[i] = R.ids[i];
@@ -267,17 +261,6 @@ __global__ void __launch_bounds__(kRouteWarps * 32)
 // Token rows of the grouped tiles, in expert-sorted slot order: xrows[slot] =
 // x[token(slot)].  One warp per row (grid-stride over gseg x 256 row slots):
 // each lane moves K/256 16-byte pieces with its loads issued before its stores.
-// Clears the grid-barrier count and the combine tickets of the fused decode
-// launch that follows.  It lets that launch start at once (its CTAs wait for
-// this kernel's completion at their first instruction, so they see the
-// cleared words), then waits for the launch before, which may still use them.
-__global__ void decode_reset_kernel(int* gbar, int* ctick, int n) {
-  pdl_trigger();
-  pdl_wait();
-  for (int i = threadIdx.x; i < n; i += blockDim.x) ctick[i] = 0;
-  if (threadIdx.x == 0) *gbar = 0;
-}
-
 __global__ void gather_rows_kernel(const uint16_t* __restrict__ x, int K, const int* __restrict__ slot_token,
                                    const int* __restrict__ ngseg, const GSeg* __restrict__ gsegs, uint16_t* xrows) {
   pdl_wait();
@@ -377,19 +360,25 @@ __global__ void dequant_kernel(const uint8_t* __restrict__ codes, unsigned long 
     const int ku = r / NT, t = r % NT;
     const uint8_t* cp = codes + (unsigned long long)e * cstride + ((unsigned long long)ku * NT + t) * Tr::kCodeBytes;
     constexpr int NKS = Tr::kKUcols / 16;
+    // lane word w of this (k-unit, tile): [ku][tile][lane][W] (PLAIN, GATE_UP) or [ku][W][tile][lane] (KSPLIT)
+    constexpr int W = FMT == 2 ? 2 : 4;
+    auto word = [&](int w) -> uint32_t {
+      if (row_order == 2)
+        return *reinterpret_cast<const uint32_t*>(
+            codes + (unsigned long long)e * cstride + ((((unsigned long long)ku * W + w) * NT + t) * 32 + lane) * 4);
+      return *reinterpret_cast<const uint32_t*>(cp + (lane * W + w) * 4);
+    };
     uint32_t am[NKS][4];
     if constexpr (FMT == 2) {
-      const uint2 w = *reinterpret_cast<const uint2*>(cp + lane * 8);
       uint32_t (&a0)[4] = am[0]; uint32_t (&a1)[4] = am[1];
       uint32_t (&a2)[4] = am[2 % NKS]; uint32_t (&a3)[4] = am[3 % NKS];
-      unpack_int2_word(w.x, a0, a1);
-      unpack_int2_word(w.y, a2, a3);
+      unpack_int2_word(word(0), a0, a1);
+      unpack_int2_word(word(1), a2, a3);
     } else if constexpr (FMT == 4) {
-      const uint4 w = *reinterpret_cast<const uint4*>(cp + lane * 16);
-      unpack_int4_word(w.x, am[0]);
-      unpack_int4_word(w.y, am[1 % NKS]);
-      unpack_int4_word(w.z, am[2 % NKS]);
-      unpack_int4_word(w.w, am[3 % NKS]);
+      unpack_int4_word(word(0), am[0]);
+      unpack_int4_word(word(1), am[1 % NKS]);
+      unpack_int4_word(word(2), am[2 % NKS]);
+      unpack_int4_word(word(3), am[3 % NKS]);
     } else {
       uint8_t rec[13];
       for (int i = 0; i < 13; ++i) rec[i] = cp[lane * 13 + i];

@@ -37,6 +37,7 @@ uint16_t double_to_bf16(double v) {
 }
 
 bool fmt_ok(int fmt) { return fmt == QMOE_INT2 || fmt == QMOE_INT4 || fmt == QMOE_TERNARY; }
+bool row_order_ok(int r) { return r == QMOE_ROWS_PLAIN || r == QMOE_ROWS_GATE_UP || r == QMOE_ROWS_KSPLIT; }
 
 qmoe_status check_shape(int fmt, int rows, int K, int block) {
   if (!fmt_ok(fmt)) return QMOE_ERR_INVALID_ARG;
@@ -94,7 +95,7 @@ uint16_t quantize_block(int fmt, const uint16_t* w, int B, int8_t* c) {
 
 // Physical position of logical element (tile row tr of tile t, column k) for INT formats:
 // returns (word index within the whole codes array, bit shift).
-inline void int_position(int fmt, int NT, int t, int tr, int k, size_t* word, int* shift) {
+inline void int_position(int fmt, int row_order, int NT, int t, int tr, int k, size_t* word, int* shift) {
   const int kb = k / 64, kk = k % 64;
   const int ks = kk / 16, kc = kk % 16;
   const int hi8 = kc >= 8;                  // f >> 1
@@ -114,7 +115,8 @@ inline void int_position(int fmt, int NT, int t, int tr, int k, size_t* word, in
     wi = ks;
     slot = 4 * f + 16 * h;
   }
-  *word = (((size_t)kb * NT + t) * 32 + lane) * W + wi;
+  *word = row_order == QMOE_ROWS_KSPLIT ? (((size_t)kb * W + wi) * NT + t) * 32 + lane
+                                        : (((size_t)kb * NT + t) * 32 + lane) * W + wi;
   *shift = slot;
 }
 
@@ -149,7 +151,7 @@ struct PosTable {
         for (int k = 0; k < 64; ++k) {
           size_t w;
           int s;
-          int_position(which == 0 ? QMOE_INT2 : QMOE_INT4, 1, 0, tr, k, &w, &s);
+          int_position(which == 0 ? QMOE_INT2 : QMOE_INT4, QMOE_ROWS_PLAIN, 1, 0, tr, k, &w, &s);
           off[which][tr][k] = (int)w;
           sh[which][tr][k] = s;
         }
@@ -189,7 +191,7 @@ qmoe_status qmoe_pack(int fmt, int row_order, const uint16_t* w, int rows, int K
                       void* codes, void* scales) {
   qmoe_status st = check_shape(fmt, rows, K, block);
   if (st != QMOE_OK) return st;
-  if (row_order != QMOE_ROWS_PLAIN && row_order != QMOE_ROWS_GATE_UP) return QMOE_ERR_INVALID_ARG;
+  if (!row_order_ok(row_order)) return QMOE_ERR_INVALID_ARG;
   if (!w || !codes || !scales) return QMOE_ERR_INVALID_ARG;
   const int NT = rows / 16, SB = K / block;
   const size_t cbytes = codes_bytes_of(fmt, rows, K);
@@ -241,8 +243,11 @@ qmoe_status qmoe_pack(int fmt, int row_order, const uint16_t* w, int rows, int K
         if (tr < 8) slot = (slot & 0xFFFF0000u) | s; else slot = (slot & 0xFFFFu) | ((uint32_t)s << 16);
         for (int i = 0; i < block; ++i) {
           const int k = b * block + i;
-          const size_t unit = ((size_t)(k / 64) * NT + t) * 32 * W;
-          cw[unit + pt.off[which][tr][k % 64]] |= (uint32_t)(c[i] + bias) << pt.sh[which][tr][k % 64];
+          const int off = pt.off[which][tr][k % 64];  // lane * W + word within the 64-column unit
+          const size_t idx = row_order == QMOE_ROWS_KSPLIT
+                                 ? (((size_t)(k / 64) * W + off % W) * NT + t) * 32 + off / W
+                                 : ((size_t)(k / 64) * NT + t) * 32 * W + off;
+          cw[idx] |= (uint32_t)(c[i] + bias) << pt.sh[which][tr][k % 64];
         }
       }
     }
@@ -254,7 +259,7 @@ qmoe_status qmoe_unpack_host(int fmt, int row_order, const void* codes, const vo
                              int K, int block, int8_t* codes_out, uint16_t* scales_out) {
   qmoe_status st = check_shape(fmt, rows, K, block);
   if (st != QMOE_OK) return st;
-  if (row_order != QMOE_ROWS_PLAIN && row_order != QMOE_ROWS_GATE_UP) return QMOE_ERR_INVALID_ARG;
+  if (!row_order_ok(row_order)) return QMOE_ERR_INVALID_ARG;
   if ((codes_out && !codes) || (scales_out && !scales)) return QMOE_ERR_INVALID_ARG;
   const int NT = rows / 16, SB = K / block;
   for (int t = 0; t < NT; ++t)
@@ -279,7 +284,7 @@ qmoe_status qmoe_unpack_host(int fmt, int row_order, const void* codes, const vo
         } else {
           size_t word;
           int shift;
-          int_position(fmt, NT, t, tr, k, &word, &shift);
+          int_position(fmt, row_order, NT, t, tr, k, &word, &shift);
           uint32_t v = static_cast<const uint32_t*>(codes)[word];
           c = (int8_t)((int)((v >> shift) & ((1u << fmt) - 1)) - (1 << (fmt - 1)));
         }

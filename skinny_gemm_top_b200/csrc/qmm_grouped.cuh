@@ -183,6 +183,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
     qmm_grouped_kernel(const __grid_constant__ CUtensorMap tmap, const GroupedParams p) {
   using Tr = FmtTraits<FMT>;
   using GG = GGeom<FMT, BT, CS>;
+  constexpr bool kKS = EPI == EPI_FC2;  // FC2 weights are packed QMOE_ROWS_KSPLIT
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024 - (smem_addr(smem_raw) & 1023)) & 1023);
   uint8_t* sA = smem;                                        // [kGStages][16 KB]
@@ -250,11 +251,15 @@ __global__ void __launch_bounds__(kGThreads, 1)
         uint8_t* cdst = sC + s * GG::kCStage;
         if (lane == 0) mbar_arrive_expect_tx(&full_c[s], GG::kCStage);
         __syncwarp();
-        if (lane == 0)
-          bulk_copy_g2s(cdst, p.codes + (unsigned long long)sg.expert * p.codes_stride +
-                                  ((unsigned long long)ks * p.NT + rt * 8) * Tr::kCodeBytes,
-                        GG::kCodeBytes, &full_c[s]);
-        if (lane == 1) {
+        constexpr int kSlabs = kKS ? (FMT == 2 ? 2 : 4) : 1;  // FC2 (KSPLIT): one 8-tile copy per slab
+        if (lane < kSlabs) {
+          const unsigned long long off =
+              kKS ? (((unsigned long long)ks * kSlabs + lane) * p.NT + rt * 8) * 128
+                  : ((unsigned long long)ks * p.NT + rt * 8) * Tr::kCodeBytes;
+          bulk_copy_g2s(cdst + lane * (GG::kCodeBytes / kSlabs), p.codes + (unsigned long long)sg.expert * p.codes_stride + off,
+                        GG::kCodeBytes / kSlabs, &full_c[s]);
+        }
+        if (lane == kSlabs) {
           const int sb = ks * 64 / p.block;
           bulk_copy_g2s(cdst + GG::kCodeBytes, p.scales + (unsigned long long)sg.expert * p.scales_stride +
                                                    ((unsigned long long)sb * p.NT + rt * 8) * 32,
@@ -331,16 +336,20 @@ __global__ void __launch_bounds__(kGThreads, 1)
 #pragma unroll
         for (int tt = 0; tt < kGDeqTiles; ++tt) {
           const int tile = kGDeqTiles * d + tt;
+          // lane word w: [tile][lane][w] (PLAIN, GATE_UP) or [w][tile][lane] (KSPLIT: FC2)
+          auto word = [&](int w) -> uint32_t {
+            constexpr int W = FMT == 2 ? 2 : 4;
+            return kKS ? *reinterpret_cast<const uint32_t*>(cs + w * (8 * 128) + tile * 128 + lane * 4)
+                       : *reinterpret_cast<const uint32_t*>(cs + tile * Tr::kCodeBytes + (lane * W + w) * 4);
+          };
           if constexpr (FMT == 2) {
-            const uint2 w = *reinterpret_cast<const uint2*>(cs + tile * Tr::kCodeBytes + lane * 8);
-            unpack_int2_word(w.x, am[tt][0], am[tt][1]);
-            unpack_int2_word(w.y, am[tt][2], am[tt][3]);
+            unpack_int2_word(word(0), am[tt][0], am[tt][1]);
+            unpack_int2_word(word(1), am[tt][2], am[tt][3]);
           } else {
-            const uint4 w = *reinterpret_cast<const uint4*>(cs + tile * Tr::kCodeBytes + lane * 16);
-            unpack_int4_word(w.x, am[tt][0]);
-            unpack_int4_word(w.y, am[tt][1]);
-            unpack_int4_word(w.z, am[tt][2]);
-            unpack_int4_word(w.w, am[tt][3]);
+            unpack_int4_word(word(0), am[tt][0]);
+            unpack_int4_word(word(1), am[tt][1]);
+            unpack_int4_word(word(2), am[tt][2]);
+            unpack_int4_word(word(3), am[tt][3]);
           }
           sw[tt] = *reinterpret_cast<const uint32_t*>(cs + GG::kCodeBytes + tile * 32 + g * 4);
         }

@@ -26,19 +26,13 @@
 //    token at HBM rate.  The per-block scale multiplies the fp32 partial
 //    product of each 64-column block, so the dequantized weight c*s is never
 //    rounded.
-//  * Segment sources: a table written by an earlier routing launch; routing
-//    computed in the kernel's prologue by every CTA for a decode batch of up
-//    to 8 tokens (identical, deterministic results in all CTAs; no routing
-//    launch); or fixed chunks of the rows of a single linear.
+//  * Segment sources: a table written by an earlier routing launch, or fixed
+//    chunks of the rows of a single linear.
 //  * Programmatic dependent launch: the weights of the first stages are
 //    requested before griddepcontrol.wait (they depend only on the routing),
 //    the activations after it.
-//  * Decode FC2 fuses the router-weighted combine: the last CTA to finish a
-//    16-row output tile (atomic counter, no spin-wait) sums that tile's slot
-//    rows in slot order and writes y.
-//  * A decode layer whose FC1 and FC2 share a format runs as one launch
-//    (qmm_decode_kernel): routing, the FC1 phase, a split grid barrier and the
-//    FC2 phase with the combine, on the same stage rings.
+//  * The decode routing (decode_route) used by the decode layer kernel
+//    (qmm_slice.cuh) and by qmoe_route lives here too.
 #pragma once
 #include <cfloat>
 #include <climits>
@@ -49,7 +43,7 @@
 namespace qmoe {
 
 enum Epi { EPI_LINEAR = 0, EPI_SWIGLU = 1, EPI_FC2 = 2 };
-enum SegSrc { SRC_TABLE = 0, SRC_DECODE = 1, SRC_LINEAR = 2 };
+enum SegSrc { SRC_TABLE = 0, SRC_LINEAR = 2 };
 
 // Warps per CTA: 12 for one token group (three warps per SM sub-partition
 // hide the unpack/MMA latency better than two), 8 for two token groups, whose
@@ -67,13 +61,9 @@ constexpr int kMaxStages = 6;     // stages per consumer warp (barriers: 1024 by
 constexpr int kChunkTokens = 16;  // tokens per segment (<= 2 token groups of 8)
 
 
-// Decode batches routed inside the kernels: up to 8 tokens, T*k <= 64,
-// at most 8 shared experts.
+// Decode batches, routed inside the decode layer kernel: up to 8 tokens, T*k <= 64.
 constexpr int kDecMaxT = 8;
 constexpr int kDecMaxTK = 64;
-constexpr int kDecMaxShared = 8;
-constexpr int kDecMaxSegs = kDecMaxTK + kDecMaxShared;
-constexpr int kDecMaxSlots = kDecMaxTK + kDecMaxShared * kDecMaxT;
 constexpr int kMaxExperts = 256;
 
 // One (expert, token chunk) work item.
@@ -86,16 +76,13 @@ struct Seg {
 
 // Routing of a decode batch, computed in shared memory.
 struct DecodeRoute {
-  int nseg;
-  Seg segs[kDecMaxSegs];
-  int slot_token[kDecMaxSlots];  // slot -> token
-  int pos[kDecMaxTK];            // flat index t*k+s -> slot
+  int nseg;                      // selected (distinct) experts
+  Seg segs[kDecMaxTK];           // one per selected expert, in expert order
+  int pos[kDecMaxTK];            // flat index t*k+s -> position in the expert-sorted order
   float w[kDecMaxTK];            // router weight of flat index
   int ids[kDecMaxTK];            // expert of flat index
   int hist[kMaxExperts];         // scratch: entries per expert, then their exclusive prefix
 };
-// The part of DecodeRoute that FC2 reads (the scratch at the end is not copied).
-constexpr int kDecodeRouteWords = (int)(offsetof(DecodeRoute, hist) / 4);
 
 struct SmallParams {
   const uint8_t* codes;
@@ -113,11 +100,9 @@ struct SmallParams {
   // activation rows [*, K] bf16: row of slot s is act_index[s] (or s when null)
   const uint16_t* act;
   const int* act_index;
-  // routing inputs (SRC_DECODE) / row count (SRC_LINEAR)
-  const float* logits;
-  int T, E, k, n_shared;
+  int T;                             // SRC_LINEAR: rows
   // epilogues
-  uint16_t* y;                       // LINEAR: y[token][N]; decode FC2: combined y[token][H]
+  uint16_t* y;                       // LINEAR: y[token][N]
   int N;
   const uint16_t* bias;              // SWIGLU/FC2: bias + expert * bias_rows (logical rows)
   int bias_rows;
@@ -125,8 +110,6 @@ struct SmallParams {
   int I;
   float* yslot;                      // FC2: yslot[slot][H]
   int H;
-  int* ctick;                        // decode: per 16-row output tile counters (H/16)
-  DecodeRoute* route_tab;            // decode: routing tables, written by FC1's CTA 0, read by FC2
   int early;                         // 1: segments and weights may be read before griddepcontrol.wait
   unsigned* status;
 };
@@ -148,8 +131,7 @@ struct StageGeom {
 
 template <int SRC>
 struct SmemHead {
-  static constexpr int kRouteBytes = SRC == SRC_DECODE ? ((int)sizeof(DecodeRoute) + 127) / 128 * 128 : 0;
-  static constexpr int kFixed = 2048 + kRouteBytes;  // barriers + ternary LUT + routing
+  static constexpr int kFixed = 2048;  // barriers + ternary LUT
 };
 
 // ---------------------------------------------------------------------------
@@ -298,13 +280,26 @@ __device__ __forceinline__ void iter_begin(ItemIter& it, const SmallParams& p, c
 // (lane 0's expect-tx arrival and 32 cp.async arrivals).
 
 // Codes (TMA) and scales (cp.async) of the sub-panel's nt tiles at k-unit ku.
-template <int FMT, int TG, int SRC>
+// KS: the matrix is packed QMOE_ROWS_KSPLIT (FC2): an INT2/INT4 k-unit of nt
+// tiles is W slabs of nt x 128 bytes, copied by per-lane cp.async into
+// [slab][tile][lane] order (ternary records are laid out as in PLAIN).
+template <int FMT, int TG, int SRC, bool KS>
 __device__ __forceinline__ void issue_weights(const SmallParams& p, const ItemIter& it, uint8_t* stage, uint64_t* bar,
                                               int lane) {
   using G = StageGeom<FMT, TG, SRC>;
   using Tr = FmtTraits<FMT>;
   const int tile = it.sp.rt0, n = it.sp.nt;
-  if (lane == 0) {
+  if constexpr (KS && FMT != 3) {
+    constexpr int W = FMT == 2 ? 2 : 4;
+    const int per = n * 8;  // 16-byte pieces per slab
+    const uint8_t* base = p.codes + (unsigned long long)it.sg.expert * p.codes_stride;
+    for (int c = lane; c < W * per; c += 32) {
+      const int w = c / per, j = c - w * per;
+      cp_async16(stage + w * (G::kMT * 128) + 16 * j,
+                 base + (((unsigned long long)it.ku * W + w) * p.NT + tile) * 128 + 16 * j);
+    }
+    if (lane == 0) mbar_arrive(bar);  // the arrival a bulk copy's expect-tx would make
+  } else if (lane == 0) {
     const uint8_t* csrc = p.codes + (unsigned long long)it.sg.expert * p.codes_stride +
                           ((unsigned long long)it.ku * p.NT + tile) * Tr::kCodeBytes;
     const uint32_t bytes = (uint32_t)(n * Tr::kCodeBytes);
@@ -353,10 +348,12 @@ __device__ __forceinline__ void ldmatrix_x4(uint32_t (&r)[4], const void* p) {
 }
 
 // ---------------------------------------------------------------------------
-// Routing of a decode batch (T <= 8) in shared memory, identical in every CTA:
-// top-k with ties to the lower index, softmax over the selected logits, slot
-// order = stable sort of t*k+s by expert, shared experts after the routed
-// slots; one segment per active expert, experts in increasing order.
+// Routing of a decode batch (T <= 8, T*k <= 64) in shared memory, identical in
+// every CTA: top-k with ties to the lower index (-0 equal to +0), softmax over
+// the selected logits, positions = stable sort of t*k+s by expert; one
+// segment per selected expert, experts in increasing order.  Top-k routing
+// and the rows expanded by expert: onnxruntime PR "Enable SM80+ FP16/BF16
+// mixed INT2/INT4 QMoE prefill by default", Description.
 
 // Order-preserving key of a logit: a larger key is a larger value; -0 and +0
 // are equal; NaN is below every number.
@@ -377,27 +374,27 @@ __device__ __forceinline__ float logit_of_key(uint32_t key) {
 //  1. warp t < T: k rounds of a warp arg-max over token t's logits; lane s
 //     keeps selection s; softmax over the selected logits in selection order.
 //  2. T = 1 (warp 0 goes on without a CTA barrier): the k experts are
-//     distinct; the slot and the segment of selection s are the rank of its
-//     expert among them.
+//     distinct; the position and the segment of selection s are the rank of
+//     its expert among them.
 //     T > 1 (warp 0, after a CTA barrier): per expert, the mask of the tokens
 //     that selected it (shared-memory atomic OR: the same result in every CTA
 //     whatever the order); an entry's rank within its expert is the count of
 //     earlier tokens in the mask; a warp scan over the experts gives each
-//     entry the entries at lower experts (its slot base) and its expert's
-//     rank among the selected ones (its segment).
+//     entry the entries at lower experts (its position base) and its
+//     expert's rank among the selected ones (its segment).
 // V = experts per lane (E <= 32 V); decode_route picks the smallest.
+// Needs blockDim.x >= 32 T; ends with a CTA barrier.
 template <int V>
-__device__ void decode_route_v(const SmallParams& p, DecodeRoute& R) {
+__device__ void decode_route_v(const float* logits, int T, int E, int k, DecodeRoute& R) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int T = p.T, E = p.E, k = p.k, TK = T * k;
-  int nsel = k;  // selected experts (warp 0)
+  const int TK = T * k;
   if (warp < T) {
     uint32_t key[V];  // lane holds experts lane + 32j
     unsigned live = 0;
 #pragma unroll
     for (int j = 0; j < V; ++j) {
       const int idx = lane + 32 * j;
-      key[j] = idx < E ? logit_key(p.logits[(size_t)warp * E + idx]) : 0u;
+      key[j] = idx < E ? logit_key(logits[(size_t)warp * E + idx]) : 0u;
       if (idx < E) live |= 1u << j;
     }
     int my_id = 0;
@@ -428,7 +425,6 @@ __device__ void decode_route_v(const SmallParams& p, DecodeRoute& R) {
       for (int j = 0; j < k; ++j) rank += __shfl_sync(0xffffffffu, my_id, j) < my_id;
       if (lane < k) {
         R.pos[lane] = rank;
-        R.slot_token[rank] = 0;
         Seg sg;
         sg.expert = my_id;
         sg.m = 1;
@@ -436,6 +432,7 @@ __device__ void decode_route_v(const SmallParams& p, DecodeRoute& R) {
         sg.slot0 = rank;
         R.segs[rank] = sg;
       }
+      if (lane == 0) R.nseg = k;
     }
   }
   if (T > 1) {
@@ -483,9 +480,7 @@ __device__ void decode_route_v(const SmallParams& p, DecodeRoute& R) {
       for (int h = 0; h < 2; ++h) {
         if (is[h] >= TK) continue;
         const int pre = hist[es[h]], less = pre & 0xFFFF;
-        const int pos = less + bs[h];
-        R.pos[is[h]] = pos;
-        R.slot_token[pos] = is[h] / k;
+        R.pos[is[h]] = less + bs[h];
         if (bs[h] == 0) {
           Seg sg;
           sg.expert = es[h];
@@ -495,30 +490,19 @@ __device__ void decode_route_v(const SmallParams& p, DecodeRoute& R) {
           R.segs[pre >> 16] = sg;
         }
       }
-      nsel = __shfl_sync(0xffffffffu, inc, 31) >> 16;
+      const int nsel = __shfl_sync(0xffffffffu, inc, 31) >> 16;
+      if (lane == 0) R.nseg = nsel;
     }
-  }
-  if (warp == 0) {  // shared experts: one segment each (all T tokens), after the routed slots
-    if (lane < p.n_shared) {
-      Seg sg;
-      sg.expert = E + lane;
-      sg.m = T;
-      sg.tg = (T + 7) / 8;
-      sg.slot0 = TK + lane * T;
-      R.segs[nsel + lane] = sg;
-    }
-    for (int i = lane; i < p.n_shared * T; i += 32) R.slot_token[TK + i] = i % T;
-    if (lane == 0) R.nseg = nsel + p.n_shared;
   }
   __syncthreads();
 }
 
 // (A lane holding 8 experts where 2 would do made the routing of a 64-expert
 // layer about 1.5k cycles slower: measured in isolation.)
-__device__ __forceinline__ void decode_route(const SmallParams& p, DecodeRoute& R) {
-  if (p.E <= 64) decode_route_v<2>(p, R);
-  else if (p.E <= 128) decode_route_v<4>(p, R);
-  else decode_route_v<8>(p, R);
+__device__ __forceinline__ void decode_route(const float* logits, int T, int E, int k, DecodeRoute& R) {
+  if (E <= 64) decode_route_v<2>(logits, T, E, k, R);
+  else if (E <= 128) decode_route_v<4>(logits, T, E, k, R);
+  else decode_route_v<8>(logits, T, E, k, R);
 }
 
 // Epilogue of one reduced fragment: rows g / g+8 of tile rt, tokens n0, n0+1.
@@ -578,7 +562,7 @@ __device__ __forceinline__ void epilogue(const SmallParams& p, const Seg& sg, in
 // at or past nt contribute with scale 0 (their codes are stale but finite),
 // so all NTL tiles run the same straight-line code and the MMAs of a k-step
 // for every tile issue back to back.
-template <int FMT, int TG, int SRC, int NTL>
+template <int FMT, int TG, int SRC, bool KS, int NTL>
 __device__ __forceinline__ void compute_item(const uint8_t* st, bool tg2, int lane, int nt, const uint32_t* lut,
                                              float (&acc)[kTiles<FMT, TG, SRC>][TG][4]) {
   using Tr = FmtTraits<FMT>;
@@ -658,7 +642,11 @@ __device__ __forceinline__ void compute_item(const uint8_t* st, bool tg2, int la
     uint32_t wd[NTL][W];
 #pragma unroll
     for (int i = 0; i < NTL; ++i) {
-      if constexpr (FMT == 2) {
+      if constexpr (KS) {  // [slab][tile][lane]
+#pragma unroll
+        for (int w = 0; w < W; ++w)
+          wd[i][w] = *reinterpret_cast<const uint32_t*>(cbuf + w * (G::kMT * 128) + i * 128 + lane * 4);
+      } else if constexpr (FMT == 2) {
         const uint2 w = *reinterpret_cast<const uint2*>(cbuf + (size_t)i * Tr::kCodeBytes + lane * 8);
         wd[i][0] = w.x; wd[i][1] = w.y;
       } else {
@@ -709,39 +697,6 @@ __device__ __forceinline__ void compute_item(const uint8_t* st, bool tg2, int la
   }
 }
 
-// Router-weighted combine of the output tiles flagged in comb[0..nt) (tiles
-// rt0 + i): y[t][r] = sum_s w[t][s] * yslot[pos(t,s)][r] + sum_j yslot[shared j, t][r],
-// routed slots first, in slot order.  The k + n_shared slot rows of an output
-// are read in batches of 8 (one batch for k + n_shared <= 8), so that the
-// loads overlap.
-template <int NTHR>
-__device__ __forceinline__ void combine_tiles(const SmallParams& p, const DecodeRoute& R, int rt0, int nt,
-                                              const int* comb) {
-  const int k = p.k, TK = p.T * k, per = p.T * 16, ns = k + p.n_shared;
-  for (int e = threadIdx.x; e < nt * per; e += NTHR) {
-    const int i = e / per;
-    if (!comb[i]) continue;
-    const int t = (e - i * per) >> 4, r = (rt0 + i) * 16 + (e & 15);
-    float acc = 0.f;
-    for (int s0 = 0; s0 < ns; s0 += 8) {
-      float v[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int sl = s0 + u;
-        const int row = sl < k ? R.pos[t * k + sl] : TK + (sl - k) * p.T + t;
-        v[u] = sl < ns ? __ldcg(p.yslot + (size_t)row * p.H + r) : 0.f;
-      }
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int sl = s0 + u;
-        if (sl < k) acc = fmaf(R.w[t * k + sl], v[u], acc);
-        else if (sl < ns) acc += v[u];
-      }
-    }
-    p.y[(size_t)t * p.H + r] = __bfloat16_as_ushort(__float2bfloat16_rn(acc));
-  }
-}
-
 // ---------------------------------------------------------------------------
 // One matmul phase of a small-M kernel on the warps' stage rings.  The rings
 // (barriers, stage buffers, item counters) are kept in a context that could
@@ -759,9 +714,7 @@ struct PhaseCtx {
   bool aborted;     // this warp gave up waiting
   float4* red;
   const uint32_t* lut;
-  DecodeRoute* R;
   int* s_abort;
-  int* s_comb;
 };
 
 // Partition, prime (weights, then hook(), then activation rows), stream the
@@ -793,7 +746,7 @@ __device__ __forceinline__ void run_phase(const SmallParams& p, const SegSource&
     ItemIter it = prod;
     for (int i = 0; i < NST && it.valid && !cx.aborted; ++i, ++primed) {  // (a warp that gave up issues nothing)
       const int s = (cx.issued + i) % NST;
-      issue_weights<FMT, TG, SRC>(p, it, cx.wstage + s * cx.stride, &cx.wfull[s], lane);
+      issue_weights<FMT, TG, SRC, EPI == EPI_FC2>(p, it, cx.wstage + s * cx.stride, &cx.wfull[s], lane);
       iter_advance<TG>(it, p, segs, act_index, warp, lane);
     }
   }
@@ -846,16 +799,16 @@ __device__ __forceinline__ void run_phase(const SmallParams& p, const SegSource&
       }
       if (!cx.aborted) {
         const uint8_t* st = cx.wstage + s * cx.stride;
-        if (G::kMT > 8 && sp.nt > 8) compute_item<FMT, TG, SRC, G::kMT>(st, tg2, lane, sp.nt, cx.lut, acc);
-        else if (sp.nt > 4) compute_item<FMT, TG, SRC, 8>(st, tg2, lane, sp.nt, cx.lut, acc);
-        else if (sp.nt > 2) compute_item<FMT, TG, SRC, 4>(st, tg2, lane, sp.nt, cx.lut, acc);
-        else if (sp.nt > 1) compute_item<FMT, TG, SRC, 2>(st, tg2, lane, sp.nt, cx.lut, acc);
-        else compute_item<FMT, TG, SRC, 1>(st, tg2, lane, sp.nt, cx.lut, acc);
+        if (G::kMT > 8 && sp.nt > 8) compute_item<FMT, TG, SRC, EPI == EPI_FC2, G::kMT>(st, tg2, lane, sp.nt, cx.lut, acc);
+        else if (sp.nt > 4) compute_item<FMT, TG, SRC, EPI == EPI_FC2, 8>(st, tg2, lane, sp.nt, cx.lut, acc);
+        else if (sp.nt > 2) compute_item<FMT, TG, SRC, EPI == EPI_FC2, 4>(st, tg2, lane, sp.nt, cx.lut, acc);
+        else if (sp.nt > 1) compute_item<FMT, TG, SRC, EPI == EPI_FC2, 2>(st, tg2, lane, sp.nt, cx.lut, acc);
+        else compute_item<FMT, TG, SRC, EPI == EPI_FC2, 1>(st, tg2, lane, sp.nt, cx.lut, acc);
       }
       __syncwarp();
       if (prod.valid && !cx.aborted) {
         uint8_t* st = cx.wstage + s * cx.stride;
-        issue_weights<FMT, TG, SRC>(p, prod, st, &cx.wfull[s], lane);
+        issue_weights<FMT, TG, SRC, EPI == EPI_FC2>(p, prod, st, &cx.wfull[s], lane);
         issue_acts<FMT, TG, SRC>(p, prod, st, lane);
         cp_async_arrive(&cx.wfull[s]);
         ++cx.issued;
@@ -890,19 +843,6 @@ __device__ __forceinline__ void run_phase(const SmallParams& p, const SegSource&
       if (t == 1 && !tg2) continue;
       epilogue<EPI>(p, sg, sp.rt0 + i, t, ln, v);
     }
-    if constexpr (SRC == SRC_DECODE && EPI == EPI_FC2) {
-      // fused combine: the CTA that adds an output tile's last segment combines
-      // it.  After the barrier, one acquire-release ticket per tile publishes
-      // this CTA's slot rows and acquires the other CTAs' ones.
-      __syncthreads();
-      if (tid < sp.nt) {
-        const int old = ab ? -1 : atomic_add_acq_rel_gpu(&p.ctick[sp.rt0 + tid], 1);
-        cx.s_comb[tid] = old == nseg - 1;
-        if (old == nseg - 1) p.ctick[sp.rt0 + tid] = 0;  // ready for the next launch
-      }
-      __syncthreads();
-      combine_tiles<kCT>(p, *cx.R, sp.rt0, sp.nt, cx.s_comb);
-    }
     __syncthreads();
     pos = sp.next;
   }
@@ -922,13 +862,11 @@ template <int FMT, int TG, int SRC>
 struct SmallSmem {
   uint64_t* bars;  // [kNW][NST] full barriers
   uint32_t* lut;   // 243 entries (ternary)
-  DecodeRoute* R;  // SRC_DECODE only
   float4* red;     // [kNW][kMT][TG][32]
   uint8_t* stages; // [kNW][NST][stage]
   __device__ __forceinline__ explicit SmallSmem(uint8_t* smem) {
     bars = reinterpret_cast<uint64_t*>(smem);
     lut = reinterpret_cast<uint32_t*>(smem + 1024);
-    R = reinterpret_cast<DecodeRoute*>(smem + 2048);
     red = reinterpret_cast<float4*>(smem + SmemHead<SRC>::kFixed);
     stages = smem + SmemHead<SRC>::kFixed + StageGeom<FMT, TG, SRC>::kRedBytes;
   }
@@ -936,8 +874,7 @@ struct SmallSmem {
 
 // Ternary table, ring barriers and the phase context (ends with a CTA barrier).
 template <int FMT, int TG, int SRC>
-__device__ __forceinline__ void init_rings(const SmallSmem<FMT, TG, SRC>& sm, int NST, int* s_abort, int* s_comb,
-                                           PhaseCtx& cx) {
+__device__ __forceinline__ void init_rings(const SmallSmem<FMT, TG, SRC>& sm, int NST, int* s_abort, PhaseCtx& cx) {
   using G = StageGeom<FMT, TG, SRC>;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (tid == 0) *s_abort = 0;
@@ -950,9 +887,7 @@ __device__ __forceinline__ void init_rings(const SmallSmem<FMT, TG, SRC>& sm, in
   cx.NST = NST;
   cx.red = sm.red;
   cx.lut = sm.lut;
-  cx.R = sm.R;
   cx.s_abort = s_abort;
-  cx.s_comb = s_comb;
   if (lane == 0)
     for (int s = 0; s < NST; ++s) mbar_init(&cx.wfull[s], 33);
   fence_mbar_init();
@@ -962,11 +897,9 @@ __device__ __forceinline__ void init_rings(const SmallSmem<FMT, TG, SRC>& sm, in
 template <int FMT, int TG, int EPI, int SRC>
 __global__ void __launch_bounds__(kWarps<TG> * 32, 1) qmm_small_kernel(const SmallParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
-  const int tid = threadIdx.x, lane = tid & 31;
+  const int lane = threadIdx.x & 31;
   const SmallSmem<FMT, TG, SRC> sm(smem);
-  DecodeRoute& R = *sm.R;
   __shared__ int s_abort;
-  __shared__ int s_comb[kMaxT];
 
   // ---- segments ----
   // With p.early the segment source was written at least two launches back
@@ -977,26 +910,7 @@ __global__ void __launch_bounds__(kWarps<TG> * 32, 1) qmm_small_kernel(const Sma
   SegSource segs;
   segs.table = nullptr;
   segs.rows = p.T;
-  const int* act_index = p.act_index;
-  if constexpr (SRC == SRC_DECODE) {
-    if constexpr (EPI == EPI_FC2) {
-      // the routing of this call, from the FC1 launch just before (after the wait)
-      const uint32_t* src = reinterpret_cast<const uint32_t*>(p.route_tab);
-      uint32_t* dst = reinterpret_cast<uint32_t*>(&R);
-      for (int i = tid; i < kDecodeRouteWords; i += blockDim.x) dst[i] = __ldcg(src + i);
-      __syncthreads();
-    } else {
-      decode_route(p, R);
-      if (blockIdx.x == 0) {  // for the FC2 launch of this call
-        const uint32_t* src = reinterpret_cast<const uint32_t*>(&R);
-        uint32_t* dst = reinterpret_cast<uint32_t*>(p.route_tab);
-        for (int i = tid; i < kDecodeRouteWords; i += blockDim.x) dst[i] = src[i];
-      }
-    }
-    nseg = R.nseg;
-    segs.table = R.segs;
-    if (EPI == EPI_SWIGLU) act_index = R.slot_token;
-  } else if constexpr (SRC == SRC_LINEAR) {
+  if constexpr (SRC == SRC_LINEAR) {
     nseg = (p.T + kChunkTokens - 1) / kChunkTokens;
   } else {
     nseg = *p.nseg;
@@ -1004,49 +918,11 @@ __global__ void __launch_bounds__(kWarps<TG> * 32, 1) qmm_small_kernel(const Sma
   }
 
   PhaseCtx cx;
-  init_rings<FMT, TG, SRC>(sm, p.nstages, &s_abort, s_comb, cx);
+  init_rings<FMT, TG, SRC>(sm, p.nstages, &s_abort, cx);
 
-  run_phase<FMT, TG, EPI, SRC>(p, segs, nseg, act_index, cx, [&] {
+  run_phase<FMT, TG, EPI, SRC>(p, segs, nseg, p.act_index, cx, [&] {
     pdl_wait();
     pdl_trigger();
-    if (SRC == SRC_DECODE && EPI == EPI_SWIGLU && blockIdx.x == 0)
-      for (int i = tid; i < p.H / 16; i += blockDim.x) p.ctick[i] = 0;  // for the FC2 launch that follows
-  });
-  drain_ring(cx, lane);
-}
-
-// ---------------------------------------------------------------------------
-// A whole decode layer (T <= 8, FC1 and FC2 in one format) in one launch of
-// one CTA per SM: routing in the prologue, the FC1 phase, then the FC2 phase
-// on the same rings with the fused combine.  A split grid barrier (every CTA
-// resident) orders all of h before FC2's activation copies: a CTA arrives as
-// soon as its rows of h are written, requests FC2's first stages of weights,
-// and only then waits.  The launch before (decode_reset_kernel) cleared the
-// barrier count and the combine tickets.
-template <int FMT>
-__global__ void __launch_bounds__(kWarps<1> * 32, 1)
-    qmm_decode_kernel(const SmallParams p1, const SmallParams p2, int* gbar) {
-  extern __shared__ __align__(128) uint8_t smem[];
-  const int lane = threadIdx.x & 31;
-  const SmallSmem<FMT, 1, SRC_DECODE> sm(smem);
-  DecodeRoute& R = *sm.R;
-  __shared__ int s_abort;
-  __shared__ int s_comb[kMaxT];
-  __shared__ int s_bar_ok;
-
-  pdl_wait();  // logits and x from the launches before; cleared barrier and tickets
-  decode_route(p1, R);
-  const int nseg = R.nseg;
-  SegSource segs;
-  segs.table = R.segs;
-  segs.rows = p1.T;
-  PhaseCtx cx;
-  init_rings<FMT, 1, SRC_DECODE>(sm, p1.nstages, &s_abort, s_comb, cx);
-
-  run_phase<FMT, 1, EPI_SWIGLU, SRC_DECODE>(p1, segs, nseg, R.slot_token, cx, [] { pdl_trigger(); });
-  grid_arrive(gbar);  // this CTA's rows of h are written (run_phase ends with a CTA barrier)
-  run_phase<FMT, 1, EPI_FC2, SRC_DECODE>(p2, segs, nseg, nullptr, cx, [&] {
-    if (!grid_wait(gbar, p2.status, &s_bar_ok) && threadIdx.x == 0) s_abort = 1;  // h incomplete: no epilogue
   });
   drain_ring(cx, lane);
 }

@@ -19,6 +19,7 @@
 #include "qmm_small.cuh"
 #include "qmm_grouped.cuh"
 #include "kernels_misc.cuh"
+#include "slice.h"
 
 #include <cudaTypedefs.h>
 
@@ -60,6 +61,7 @@ qmoe_status dev_info(DevInfo** out) {
 // ---- tracing: CUDA events around each kernel launch ----
 enum KernelId { K_ROUTE = 0, K_GATHER, K_FC1_SMALL, K_FC2_SMALL, K_COMBINE, K_LINEAR_SMALL, K_LINEAR_SETUP,
                 K_DEQUANT, K_FC1_GROUPED, K_FC2_GROUPED, K_DECODE_RESET, K_DECODE_LAYER, K_LINEAR_GROUPED, K_COUNT };
+// K_DECODE_RESET / K_DECODE_LAYER: slice_reset_kernel / qmm_slice_kernel (the decode layer)
 const char* const kKernelNames[K_COUNT] = {"route",        "gather",      "fc1_small",    "fc2_small",
                                            "combine",      "linear_small", "linear_setup", "dequant",
                                            "fc1_grouped",  "fc2_grouped", "decode_reset", "decode_layer",
@@ -118,6 +120,7 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 inline size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 
 bool fmt_ok(int f) { return f == QMOE_INT2 || f == QMOE_INT4 || f == QMOE_TERNARY; }
+bool row_order_ok(int r) { return r == QMOE_ROWS_PLAIN || r == QMOE_ROWS_GATE_UP || r == QMOE_ROWS_KSPLIT; }
 int ku_cols(int fmt) { return fmt == QMOE_TERNARY ? 128 : 64; }
 int beta_hi(int fmt) { return fmt == QMOE_INT4 ? 1 : 4; }
 size_t codes_bytes(int fmt, int rows, int K) {
@@ -126,7 +129,7 @@ size_t codes_bytes(int fmt, int rows, int K) {
 size_t scales_bytes(int rows, int K, int block) { return (size_t)rows * (K / block) * 2; }
 
 qmoe_status check_weights(const qmoe_weights& w, int rows, int K) {
-  if (!fmt_ok(w.fmt) || !w.codes || !w.scales) return QMOE_ERR_INVALID_ARG;
+  if (!fmt_ok(w.fmt) || !row_order_ok(w.row_order) || !w.codes || !w.scales) return QMOE_ERR_INVALID_ARG;
   if (w.block != 64 && w.block != 128) return QMOE_ERR_UNSUPPORTED;
   if (rows % 16 || K % 64 || K % w.block) return QMOE_ERR_INVALID_ARG;
   if (w.fmt == QMOE_TERNARY && (w.block != 64 || K % 128)) return QMOE_ERR_UNSUPPORTED;
@@ -138,8 +141,9 @@ qmoe_status check_weights(const qmoe_weights& w, int rows, int K) {
 struct MoEPlan {
   int T, S, TK, max_seg, n_tickets, max_gseg;
   bool grouped, decode;
-  size_t ids, w, perm, inv, offsets, slot_token, nseg, segs, chunk_counts, yslot, hrows, ctick, route, gbar, ngseg,
-      gsegs, xrows, total;
+  SlicePlan slice;  // decode batches
+  size_t ids, w, perm, inv, offsets, slot_token, nseg, segs, chunk_counts, yslot, hrows, yacc, ticket, ngseg, gsegs,
+      xrows, total;
 };
 
 constexpr int kGroupedThreshold = 32;  // AUTO: experts with more tokens take the tcgen05 path
@@ -155,32 +159,38 @@ int grouped_threshold(const qmoe_layer& L) {
   return L.path == QMOE_PATH_GROUPED ? 0 : kGroupedThreshold;
 }
 
-// Decode batches route inside the expert kernels: one fused launch per layer
-// (after a tiny reset launch), or two expert launches when FC1 and FC2 differ
-// in format.
-bool decode_eligible(const qmoe_layer& L, int T) {
-  return T <= kDecMaxT && T * L.k <= kDecMaxTK && L.n_shared <= kDecMaxShared && T <= grouped_threshold(L);
+// Decode batches (T <= 8, T*k <= 64, H <= 2112) run as one launch of the
+// kernel split along the expert intermediate dimension, which routes in its
+// prologue (after a tiny reset launch of its accumulator).
+bool decode_eligible(const qmoe_layer& L, int T, int grid, SlicePlan* plan) {
+  if (T > kDecMaxT || T * L.k > kDecMaxTK || L.path == QMOE_PATH_GROUPED || L.H > kSMaxH) return false;
+  const SlicePlan pl = slice_plan(L.fc1.fmt, L.fc2.fmt, T, L.H);
+  if (!pl.ok || L.I % pl.gran_cols) return false;
+  const int gpe = L.I / pl.gran_cols;
+  if (slice_max_chunks(L.fc2.fmt, gpe, L.n_shared, std::min(L.E, T * L.k), grid) > kSMaxChunks) return false;
+  if (plan) *plan = pl;
+  return true;
 }
 
 MoEPlan plan_moe(const qmoe_layer& L, int T, int grid) {
-  (void)grid;
   MoEPlan p{};
   p.T = T;
   p.TK = T * L.k;
   p.S = T * (L.k + L.n_shared);
-  p.decode = decode_eligible(L, T);
+  p.decode = decode_eligible(L, T, grid, &p.slice);
   p.grouped = !p.decode && T > grouped_threshold(L);
   p.max_seg = std::min(L.E, p.TK) + p.TK / kChunkTokens + L.n_shared * ((T + kChunkTokens - 1) / kChunkTokens);
   size_t o = 0;
   auto take = [&](size_t bytes) { size_t at = o; o = align_up(o + bytes); return at; };
+  if (p.decode) {  // the fp32 output accumulator and the last-CTA ticket
+    p.yacc = take((size_t)T * L.H * 4);
+    p.ticket = take(16);
+    p.total = o;
+    return p;
+  }
   p.yslot = take((size_t)p.S * L.H * 4);
   p.hrows = take((size_t)p.S * L.I * 2 + 16);
-  p.ctick = take((size_t)(L.H / 16) * 4);
-  if (p.decode) {
-    p.route = take(sizeof(DecodeRoute));
-    p.gbar = take(16);
-  }
-  if (!p.decode) {
+  {
     p.ids = take((size_t)p.TK * 4);
     p.w = take((size_t)p.TK * 4);
     p.perm = take((size_t)p.TK * 4);
@@ -258,58 +268,13 @@ qmoe_status launch_small_t(SmallParams prm, int grid, cudaStream_t st) {
              : QMOE_ERR_CUDA;
 }
 
-// Fused decode layer: decode_reset_kernel, then qmm_decode_kernel (one CTA per SM).
-template <int FMT>
-qmoe_status launch_decode_t(SmallParams p1, SmallParams p2, int* gbar, int grid, cudaStream_t st) {
-  int nst = 0;
-  const int smem = small_smem<FMT, 1, SRC_DECODE>(&nst);
-  if (smem < 0) return QMOE_ERR_UNSUPPORTED;
-  p1.nstages = p2.nstages = nst;
-  // 0: not checked, 1: one CTA fits per SM (the grid barrier needs all CTAs resident), -1: it does not
-  static int resident[kMaxDevices] = {};
-  int d = 0;
-  cudaGetDevice(&d);
-  if (!resident[d]) {
-    int per_sm = 0;
-    if (cudaFuncSetAttribute(qmm_decode_kernel<FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
-            cudaSuccess ||
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, qmm_decode_kernel<FMT>, kWarps<1> * 32, smem) !=
-            cudaSuccess)
-      return QMOE_ERR_CUDA;
-    resident[d] = per_sm >= 1 ? 1 : -1;
-  }
-  if (resident[d] < 0) return QMOE_ERR_UNSUPPORTED;
-  {
-    TraceScope ts(st, K_DECODE_RESET);
-    if (launch_pdl(decode_reset_kernel, dim3(1), dim3(128), 0, st, gbar, p2.ctick, p2.H / 16) != cudaSuccess)
-      return QMOE_ERR_CUDA;
-  }
-  TraceScope ts(st, K_DECODE_LAYER);
-  return launch_pdl(qmm_decode_kernel<FMT>, dim3(grid), dim3(kWarps<1> * 32), smem, st, p1, p2, gbar) == cudaSuccess
-             ? QMOE_OK
-             : QMOE_ERR_CUDA;
-}
-
-qmoe_status launch_decode(int fmt, const SmallParams& p1, const SmallParams& p2, int* gbar, int grid,
-                          cudaStream_t st) {
-  if (fmt == QMOE_INT2) return launch_decode_t<2>(p1, p2, gbar, grid, st);
-  if (fmt == QMOE_INT4) return launch_decode_t<4>(p1, p2, gbar, grid, st);
-  return launch_decode_t<3>(p1, p2, gbar, grid, st);
-}
-
 template <int EPI, int SRC>
 qmoe_status launch_small(int fmt, int tg, const SmallParams& prm, int grid, cudaStream_t st) {
-  if constexpr (SRC == SRC_DECODE) {  // decode batches have at most 8 tokens: one token group
-    if (fmt == QMOE_INT2) return launch_small_t<2, 1, EPI, SRC>(prm, grid, st);
-    if (fmt == QMOE_INT4) return launch_small_t<4, 1, EPI, SRC>(prm, grid, st);
-    return launch_small_t<3, 1, EPI, SRC>(prm, grid, st);
-  } else {
-    if (fmt == QMOE_INT2)
-      return tg == 1 ? launch_small_t<2, 1, EPI, SRC>(prm, grid, st) : launch_small_t<2, 2, EPI, SRC>(prm, grid, st);
-    if (fmt == QMOE_INT4)
-      return tg == 1 ? launch_small_t<4, 1, EPI, SRC>(prm, grid, st) : launch_small_t<4, 2, EPI, SRC>(prm, grid, st);
-    return tg == 1 ? launch_small_t<3, 1, EPI, SRC>(prm, grid, st) : launch_small_t<3, 2, EPI, SRC>(prm, grid, st);
-  }
+  if (fmt == QMOE_INT2)
+    return tg == 1 ? launch_small_t<2, 1, EPI, SRC>(prm, grid, st) : launch_small_t<2, 2, EPI, SRC>(prm, grid, st);
+  if (fmt == QMOE_INT4)
+    return tg == 1 ? launch_small_t<4, 1, EPI, SRC>(prm, grid, st) : launch_small_t<4, 2, EPI, SRC>(prm, grid, st);
+  return tg == 1 ? launch_small_t<3, 1, EPI, SRC>(prm, grid, st) : launch_small_t<3, 2, EPI, SRC>(prm, grid, st);
 }
 
 template <int FMT, int EPI, int BT, int CS>
@@ -382,6 +347,7 @@ qmoe_status check_layer(const qmoe_layer* L) {
   if (L->H % 64 || L->I % 64) return QMOE_ERR_INVALID_ARG;
   if (L->path < QMOE_PATH_AUTO || L->path > QMOE_PATH_GROUPED) return QMOE_ERR_INVALID_ARG;
   if (L->max_row_tile < 0) return QMOE_ERR_INVALID_ARG;
+  if (L->fc1.row_order != QMOE_ROWS_GATE_UP || L->fc2.row_order != QMOE_ROWS_KSPLIT) return QMOE_ERR_INVALID_ARG;
   qmoe_status s = check_weights(L->fc1, 2 * L->I, L->H);
   if (s != QMOE_OK) return s;
   return check_weights(L->fc2, L->H, L->I);
@@ -550,6 +516,53 @@ qmoe_status qmoe_forward(const qmoe_layer* layer, const uint16_t* x, const float
     const uint16_t* xt = x + (size_t)t0 * L.H;
     const float* lt = logits + (size_t)t0 * L.E;
     uint16_t* yt = y + (size_t)t0 * L.H;
+    if (p.decode) {
+      // Decode batch: one launch, split along the experts' intermediate dimension.
+      SliceParams sp{};
+      sp.c1 = static_cast<const uint8_t*>(L.fc1.codes);
+      sp.c1_stride = codes_bytes(L.fc1.fmt, 2 * L.I, L.H);
+      sp.s1 = static_cast<const uint8_t*>(L.fc1.scales);
+      sp.s1_stride = scales_bytes(2 * L.I, L.H, L.fc1.block);
+      sp.b1 = L.fc1.bias;
+      sp.c2 = static_cast<const uint8_t*>(L.fc2.codes);
+      sp.c2_stride = codes_bytes(L.fc2.fmt, L.H, L.I);
+      sp.s2 = static_cast<const uint8_t*>(L.fc2.scales);
+      sp.s2_stride = scales_bytes(L.H, L.I, L.fc2.block);
+      sp.b2 = L.fc2.bias;
+      sp.NT1 = 2 * L.I / 16;
+      sp.KU1 = L.H / ku_cols(L.fc1.fmt);
+      sp.block1 = L.fc1.block;
+      sp.NT2 = L.H / 16;
+      sp.block2 = L.fc2.block;
+      sp.H = L.H;
+      sp.I = L.I;
+      sp.E = L.E;
+      sp.k = L.k;
+      sp.n_shared = L.n_shared;
+      sp.T = tt;
+      sp.gpe = L.I / p.slice.gran_cols;
+      sp.ring_bytes = p.slice.ring_bytes;
+      sp.ngm = p.slice.ngm;
+      sp.xrows = p.slice.xrows;
+      sp.x = xt;
+      sp.logits = lt;
+      sp.y = yt;
+      sp.yacc = reinterpret_cast<float*>(base + p.yacc);
+      sp.ticket = reinterpret_cast<int*>(base + p.ticket);
+      sp.status = di->status;
+      {
+        TraceScope ts(st, K_DECODE_RESET);
+        if (slice_reset_launch(sp.yacc, tt * L.H / 4, sp.ticket, st) != cudaSuccess) return QMOE_ERR_CUDA;
+      }
+      {
+        TraceScope ts(st, K_DECODE_LAYER);
+        if (slice_launch(L.fc1.fmt, L.fc2.fmt, sp, grid, p.slice.smem, st) != cudaSuccess) return QMOE_ERR_CUDA;
+      }
+      ++tiles;
+      ++small;
+      ++decode;
+      continue;
+    }
     float* yslot = reinterpret_cast<float*>(base + p.yslot);
     uint16_t* hrows = reinterpret_cast<uint16_t*>(base + p.hrows);
     SmallParams p1 = small_params(L.fc1, 2 * L.I, L.H, di->status);
@@ -567,36 +580,6 @@ qmoe_status qmoe_forward(const qmoe_layer* layer, const uint16_t* x, const float
     p2.yslot = yslot;
     p2.H = L.H;
     p2.I = L.I;
-    if (p.decode) {
-      // Decode batch: both expert kernels route in their prologue; FC2 fuses the combine.
-      for (SmallParams* q : {&p1, &p2}) {
-        q->logits = lt;
-        q->T = tt;
-        q->E = L.E;
-        q->k = L.k;
-        q->n_shared = L.n_shared;
-        q->ctick = reinterpret_cast<int*>(base + p.ctick);
-        q->route_tab = reinterpret_cast<DecodeRoute*>(base + p.route);
-      }
-      p1.early = 0;  // the logits may come from the previous launch
-      p2.early = 0;  // FC2 reads FC1's routing tables after its wait
-      p2.y = yt;
-      s = QMOE_ERR_UNSUPPORTED;
-      if (L.fc1.fmt == L.fc2.fmt)  // one launch for the layer (after the reset launch)
-        s = launch_decode(L.fc1.fmt, p1, p2, reinterpret_cast<int*>(base + p.gbar), grid, st);
-      if (s != QMOE_OK && s != QMOE_ERR_UNSUPPORTED) return s;
-      const bool fused = s == QMOE_OK;
-      if (!fused) {
-        s = launch_small<EPI_SWIGLU, SRC_DECODE>(L.fc1.fmt, 1, p1, grid, st);
-        if (s != QMOE_OK) return s;
-        s = launch_small<EPI_FC2, SRC_DECODE>(L.fc2.fmt, 1, p2, grid, st);
-        if (s != QMOE_OK) return s;
-      }
-      ++tiles;
-      small += fused ? 1 : 2;
-      ++decode;
-      continue;
-    }
     RouteOut o{};
     o.ids = reinterpret_cast<int*>(base + p.ids);
     o.w = reinterpret_cast<float*>(base + p.w);
@@ -700,6 +683,7 @@ qmoe_status qmoe_linear_workspace_size(int N, int K, int M, size_t* bytes) {
 qmoe_status qmoe_linear(const qmoe_weights* w, int N, int K, const uint16_t* x, int M, uint16_t* y, void* ws,
                         size_t ws_bytes, void* stream) {
   if (!w || !x || !y || M <= 0) return QMOE_ERR_INVALID_ARG;
+  if (w->row_order != QMOE_ROWS_PLAIN) return QMOE_ERR_INVALID_ARG;
   qmoe_status s = check_weights(*w, N, K);
   if (s != QMOE_OK) return s;
   (void)ws;
@@ -742,10 +726,10 @@ qmoe_status qmoe_linear(const qmoe_weights* w, int N, int K, const uint16_t* x, 
   return QMOE_OK;
 }
 
-qmoe_status qmoe_dequant(const qmoe_weights* w, int row_order, int rows, int K, int n_mats, float* out_f32,
-                         uint16_t* out_bf16, void* stream) {
+qmoe_status qmoe_dequant(const qmoe_weights* w, int rows, int K, int n_mats, float* out_f32, uint16_t* out_bf16,
+                         void* stream) {
   if (!w || n_mats <= 0 || (!out_f32 && !out_bf16)) return QMOE_ERR_INVALID_ARG;
-  if (row_order != QMOE_ROWS_PLAIN && row_order != QMOE_ROWS_GATE_UP) return QMOE_ERR_INVALID_ARG;
+  const int row_order = w->row_order;
   qmoe_status s = check_weights(*w, rows, K);
   if (s != QMOE_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);

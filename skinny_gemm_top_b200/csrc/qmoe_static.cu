@@ -18,10 +18,11 @@
 //    with cudaGetSymbolAddress, with that device current, and caches it; that
 //    call can load this library's device code, so it should come before any
 //    stream capture.
-//  * Zero state: the only scratch values read before being written in a call
-//    are the FC2 per-tile tickets; the FC1 launch of the same call sets them
-//    to zero before FC2 reads them, so the array needs no clearing between
-//    calls.
+//  * Zero state: no scratch value needs to start at any particular value.
+//    The only values a call reads before writing them are the decode
+//    kernel's fp32 accumulator and its last-block ticket, and the reset launch
+//    of the same call clears both first; so the array needs no clearing
+//    between calls.
 //  * One array per device: calls that overlap in time on the same device
 //    (other streams, other host threads) race on it.  Serialise them.
 #include <cstdint>

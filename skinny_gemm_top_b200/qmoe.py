@@ -16,7 +16,7 @@ _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libqmoe.so
 
 INT2, TERNARY, INT4 = 2, 3, 4
 FMT = {"int2": INT2, "int4": INT4, "ternary": TERNARY}
-ROWS_PLAIN, ROWS_GATE_UP = 0, 1
+ROWS_PLAIN, ROWS_GATE_UP, ROWS_KSPLIT = 0, 1, 2
 PATH_AUTO, PATH_SMALL_M, PATH_GROUPED = 0, 1, 2
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_SCRATCH, ERR_CUDA, ERR_TIMEOUT, ERR_STATIC_SCRATCH = range(7)
 STATIC_SCRATCH_BYTES = 8 << 20  # QMOE_STATIC_SCRATCH_BYTES
@@ -29,8 +29,8 @@ class QmoeError(RuntimeError):
 
 
 class Weights(C.Structure):
-    _fields_ = [("fmt", C.c_int), ("block", C.c_int), ("codes", C.c_void_p), ("scales", C.c_void_p),
-                ("bias", C.c_void_p)]
+    _fields_ = [("fmt", C.c_int), ("block", C.c_int), ("row_order", C.c_int), ("codes", C.c_void_p),
+                ("scales", C.c_void_p), ("bias", C.c_void_p)]
 
 
 class Layer(C.Structure):
@@ -48,7 +48,7 @@ EXPORTS = {
     "qmoe_pack": [C.c_int, C.c_int, C.c_void_p, C.c_int, C.c_int, C.c_int, C.c_void_p, C.c_void_p],
     "qmoe_unpack_host": [C.c_int, C.c_int, C.c_void_p, C.c_void_p, C.c_int, C.c_int, C.c_int, C.c_void_p,
                          C.c_void_p],
-    "qmoe_dequant": [C.POINTER(Weights), C.c_int, C.c_int, C.c_int, C.c_int, C.c_void_p, C.c_void_p, C.c_void_p],
+    "qmoe_dequant": [C.POINTER(Weights), C.c_int, C.c_int, C.c_int, C.c_void_p, C.c_void_p, C.c_void_p],
     "qmoe_route_workspace_size": [C.c_int, C.c_int, C.c_int, C.POINTER(C.c_size_t)],
     "qmoe_route": [C.c_void_p, C.c_int, C.c_int, C.c_int, C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p,
                    C.c_void_p, C.c_size_t, C.c_void_p],
@@ -149,17 +149,19 @@ def unpack_host(fmt: int, row_order: int, codes: np.ndarray, scales: np.ndarray,
 
 # ---------------------------------------------------------------- device entry points
 
-def make_weights(fmt: int, block: int, codes, scales, bias=None) -> Weights:
-    return Weights(fmt, block, _ptr(codes), _ptr(scales), _ptr(bias))
+def make_weights(fmt: int, block: int, codes, scales, bias=None, row_order: int = ROWS_PLAIN) -> Weights:
+    """Device weight set; row_order is the one the codes were packed with
+    (GATE_UP for a layer's FC1, KSPLIT for its FC2, PLAIN for a single linear)."""
+    return Weights(fmt, block, row_order, _ptr(codes), _ptr(scales), _ptr(bias))
 
 
 def make_layer(H, I, E, k, n_shared, fc1: Weights, fc2: Weights, path=PATH_AUTO, max_row_tile=0) -> Layer:
     return Layer(H, I, E, k, n_shared, fc1, fc2, path, max_row_tile)
 
 
-def dequant(w: Weights, row_order: int, rows: int, K: int, n_mats: int, out_f32=None, out_bf16=None, stream=None):
-    _check(_lib.qmoe_dequant(C.byref(w), row_order, rows, K, n_mats, _ptr(out_f32), _ptr(out_bf16),
-                             _stream(stream)), "qmoe_dequant")
+def dequant(w: Weights, rows: int, K: int, n_mats: int, out_f32=None, out_bf16=None, stream=None):
+    _check(_lib.qmoe_dequant(C.byref(w), rows, K, n_mats, _ptr(out_f32), _ptr(out_bf16), _stream(stream)),
+           "qmoe_dequant")
 
 
 def route_workspace_size(T: int, E: int, k: int) -> int:

@@ -58,14 +58,14 @@ class MoECase:
         n = cfg.E + cfg.n_shared
         f1, f2 = FMTS[cfg.fc1_fmt], FMTS[cfg.fc2_fmt]
         c1, s1 = qmoe.pack_stack(f1, qmoe.ROWS_GATE_UP, (synth.expert_fc1(cfg, seed, e) for e in range(n)), cfg.block)
-        c2, s2 = qmoe.pack_stack(f2, qmoe.ROWS_PLAIN, (synth.expert_fc2(cfg, seed, e) for e in range(n)), cfg.block)
+        c2, s2 = qmoe.pack_stack(f2, qmoe.ROWS_KSPLIT, (synth.expert_fc2(cfg, seed, e) for e in range(n)), cfg.block)
         self.dev = {"c1": to_dev(c1), "s1": to_dev(s1), "c2": to_dev(c2), "s2": to_dev(s2)}
         self.b1 = self.b2 = None
         if cfg.bias:
             self.dev["b1"] = to_dev(np.stack([synth.expert_b1(cfg, seed, e) for e in range(n)]))
             self.dev["b2"] = to_dev(np.stack([synth.expert_b2(cfg, seed, e) for e in range(n)]))
-        self.w1 = qmoe.make_weights(f1, cfg.block, self.dev["c1"], self.dev["s1"], self.dev.get("b1"))
-        self.w2 = qmoe.make_weights(f2, cfg.block, self.dev["c2"], self.dev["s2"], self.dev.get("b2"))
+        self.w1 = qmoe.make_weights(f1, cfg.block, self.dev["c1"], self.dev["s1"], self.dev.get("b1"), qmoe.ROWS_GATE_UP)
+        self.w2 = qmoe.make_weights(f2, cfg.block, self.dev["c2"], self.dev["s2"], self.dev.get("b2"), qmoe.ROWS_KSPLIT)
         self.bank = Q.QuantExpertBank(
             cfg.H, cfg.I, cfg.E, cfg.n_shared, cfg.block,
             lambda e: oracle_quant(cfg.fc1_fmt, synth.expert_fc1(cfg, seed, e), cfg.block),

@@ -41,7 +41,9 @@ def _oracle_q(fmt, w_bits, block):
 
 @pytest.mark.parametrize("fmt,block,order", [
     (qmoe.INT2, 64, qmoe.ROWS_GATE_UP), (qmoe.INT4, 64, qmoe.ROWS_PLAIN), (qmoe.INT2, 128, qmoe.ROWS_PLAIN),
-    (qmoe.INT4, 128, qmoe.ROWS_PLAIN), (qmoe.TERNARY, 64, qmoe.ROWS_GATE_UP), (qmoe.TERNARY, 64, qmoe.ROWS_PLAIN)])
+    (qmoe.INT4, 128, qmoe.ROWS_PLAIN), (qmoe.TERNARY, 64, qmoe.ROWS_GATE_UP), (qmoe.TERNARY, 64, qmoe.ROWS_PLAIN),
+    (qmoe.INT2, 64, qmoe.ROWS_KSPLIT), (qmoe.INT4, 64, qmoe.ROWS_KSPLIT), (qmoe.INT4, 128, qmoe.ROWS_KSPLIT),
+    (qmoe.TERNARY, 64, qmoe.ROWS_KSPLIT)])
 def test_pack_matches_oracle_quantizer(fmt, block, order):
     rows, K = 48, 256
     w = synth.normal_bf16(9, 50, fmt * 10 + block, (rows, K), 0.02)
@@ -86,7 +88,7 @@ def test_pack_every_code_at_every_position():
         c[:, 0] = qmin
         c[:, 64] = qmin
         w = synth.f32_to_bf16_bits((c * 2.0 ** -7).astype(np.float32))
-        for order in (qmoe.ROWS_PLAIN, qmoe.ROWS_GATE_UP):
+        for order in (qmoe.ROWS_PLAIN, qmoe.ROWS_GATE_UP, qmoe.ROWS_KSPLIT):
             codes, scales = qmoe.pack(fmt, order, w, 64)
             cc, ss = qmoe.unpack_host(fmt, order, codes, scales, rows, K, 64)
             assert np.array_equal(cc, c)
@@ -104,7 +106,7 @@ def test_pack_every_code_at_every_position():
     ((qmoe.INT2, 0, 16, 64, 32), qmoe.ERR_UNSUPPORTED),      # block
     ((qmoe.TERNARY, 0, 16, 64, 64), qmoe.ERR_UNSUPPORTED),   # ternary needs K % 128
     ((7, 0, 16, 64, 64), qmoe.ERR_INVALID_ARG),              # format
-    ((qmoe.INT4, 2, 16, 64, 64), qmoe.ERR_INVALID_ARG),      # row order
+    ((qmoe.INT4, 3, 16, 64, 64), qmoe.ERR_INVALID_ARG),      # row order
 ])
 def test_pack_rejects_bad_arguments(args, status):
     fmt, order, rows, K, block = args

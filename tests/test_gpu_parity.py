@@ -32,8 +32,9 @@ def _close(got, ref, what=""):
 
 @pytest.mark.parametrize("fmt,block,order,tiny", [
     ("int2", 64, 1, False), ("int2", 128, 0, False), ("int4", 64, 0, False), ("int4", 128, 1, False),
-    ("ternary", 64, 1, False), ("ternary", 64, 0, False),
-    ("int2", 64, 0, True), ("int4", 128, 0, True), ("ternary", 64, 0, True)])
+    ("ternary", 64, 1, False), ("ternary", 64, 0, False), ("int2", 64, 2, False), ("int4", 64, 2, False),
+    ("int4", 128, 2, False), ("ternary", 64, 2, False),
+    ("int2", 64, 0, True), ("int4", 128, 0, True), ("ternary", 64, 0, True), ("int4", 64, 2, True)])
 def test_dequant_bit_exact(qm, fmt, block, order, tiny):
     import torch
     rows, K, n = 48, 384 if not tiny else 896, 2
@@ -43,10 +44,10 @@ def test_dequant_bit_exact(qm, fmt, block, order, tiny):
         mats = [synth.normal_bf16(21, 60, i, (rows, K), 0.02) for i in range(n)]
     c, s = qm.pack_stack(FMTS[fmt], order, mats, block)
     dc, ds = to_dev(c), to_dev(s)
-    w = qm.make_weights(FMTS[fmt], block, dc, ds)
+    w = qm.make_weights(FMTS[fmt], block, dc, ds, None, order)
     o32 = torch.empty((n, rows, K), dtype=torch.float32, device="cuda")
     o16 = torch.empty((n, rows, K), dtype=torch.int16, device="cuda")
-    qm.dequant(w, order, rows, K, n, o32, o16)
+    qm.dequant(w, rows, K, n, o32, o16)
     torch.cuda.synchronize()
     for i in range(n):
         codes, scales = oracle_quant(fmt, mats[i], block)
@@ -286,6 +287,87 @@ def test_decode_routing_ties(qm, T):
     _close(y, ref, f"tiny ties T={T}")
 
 
+# ------------------------------------------------------------------ decode layer kernel (one launch, split along I)
+
+PAIRS = [(a, b) for a in ("int2", "int4", "ternary") for b in ("int2", "int4", "ternary")]
+
+
+@pytest.mark.parametrize("f1,f2", PAIRS)
+@pytest.mark.parametrize("T", [1, 5, 8])
+def test_decode_format_pairs_bias_shared(qm, f1, f2, T):
+    """Every FC1/FC2 format pair on the one-launch decode kernel, with routed
+    and shared experts and both biases (the FC2 bias is added once per expert
+    by the block holding its first granule)."""
+    cfg = small_cfg(synth.TINY, E=12, k=3, n_shared=1, H=384, I=384, fc1_fmt=f1, fc2_fmt=f2, bias=True)
+    case = MoECase(cfg, seed=70 + T)
+    x = synth.tokens(cfg.H, 70 + T, T)
+    lg = synth.router_logits(cfg, 70 + T, T)
+    y = case.run(x, lg)
+    st = qm.get_stats()
+    assert st.small_launches == 1 and st.grouped_launches == 0  # the one-launch decode layer
+    ref = Q.moe_forward(Q.bf16_bits_to_f64(x), lg, cfg.k, case.bank)
+    _close(y, ref, f"{f1}/{f2} T={T}")
+
+
+@pytest.mark.parametrize("H,I,E,k,n_shared,T", [
+    (320, 448, 64, 6, 2, 3),     # 20 output tiles over 12 warps; 28 granules per expert
+    (64, 128, 4, 2, 0, 2),       # fewer output tiles than warps
+    (2112, 192, 16, 4, 1, 8),    # the largest H of the decode kernel
+    (256, 1024, 256, 8, 1, 8),   # 64 selected experts: many sub-panels per block
+    (512, 64, 200, 1, 3, 1),     # one granule per routed expert, several shared experts
+])
+def test_decode_ragged_shapes(qm, H, I, E, k, n_shared, T):
+    cfg = small_cfg(synth.TINY, E=E, k=k, n_shared=n_shared, H=H, I=I, fc1_fmt="int4", fc2_fmt="int4", bias=True)
+    case = MoECase(cfg, seed=H + I + E)
+    x = synth.tokens(cfg.H, 3, T)
+    lg = synth.router_logits(cfg, 3, T)
+    y = case.run(x, lg)
+    assert qm.get_stats().small_launches == 1
+    ref = Q.moe_forward(Q.bf16_bits_to_f64(x), lg, cfg.k, case.bank)
+    _close(y, ref, f"H={H} I={I} E={E} k={k} T={T}")
+
+
+def test_decode_wide_hidden_takes_general_path(qm):
+    """H above 2112: a decode batch runs the routing / expert / combine launches."""
+    cfg = small_cfg(synth.TINY, E=8, k=2, n_shared=1, H=2176, I=128, fc1_fmt="int4", fc2_fmt="int4")
+    case = MoECase(cfg, seed=5)
+    x = synth.tokens(cfg.H, 5, 2)
+    lg = synth.router_logits(cfg, 5, 2)
+    y = case.run(x, lg)
+    assert qm.get_stats().small_launches == 2
+    ref = Q.moe_forward(Q.bf16_bits_to_f64(x), lg, cfg.k, case.bank)
+    _close(y, ref, "H=2176")
+
+
+def test_decode_v2lite_with_biases(qm):
+    cfg = small_cfg(synth.V2LITE, bias=True)
+    case = MoECase(cfg, seed=21)
+    for T in (1, 4):
+        x = synth.tokens(cfg.H, 21, T)
+        lg = synth.router_logits(cfg, 21, T)
+        y = case.run(x, lg)
+        ref = Q.moe_forward(Q.bf16_bits_to_f64(x), lg, cfg.k, case.bank)
+        _close(y, ref, f"v2lite+bias T={T}")
+
+
+@pytest.fixture(scope="module")
+def ternary_full(qm):
+    """The ternary Switch-style workload at full size: d=2048, d_ff=6144, 128 experts, top-1."""
+    return MoECase(synth.TERNARY, seed=4)
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("T", [1, 8, 32, 128])
+def test_forward_ternary_full_size(qm, ternary_full, T):
+    cfg = synth.TERNARY
+    x = synth.tokens(cfg.H, 4, T)
+    lg = synth.router_logits(cfg, 4, T)
+    y = ternary_full.run(x, lg)
+    pick = np.arange(T) if T <= 8 else np.random.default_rng(T).choice(T, 4, replace=False)
+    ref = np.stack([Q.moe_token(Q.bf16_bits_to_f64(x[t]), lg[t], cfg.k, ternary_full.bank) for t in pick])
+    _close(y[pick], ref, f"ternary full size T={T}")
+
+
 @pytest.mark.parametrize("M", [1, 5, 16, 32])
 def test_forward_v2lite_tokens_per_expert(qm, v2lite, M):
     """M tokens with identical router logits: every selected expert gets exactly M tokens."""
@@ -338,8 +420,9 @@ def test_forward_scratch_error_and_invalid_args(qm):
     lg = torch.from_numpy(synth.router_logits(synth.TINY, 3, 2)).cuda()
     y = torch.empty((2, synth.TINY.H), dtype=torch.int16, device="cuda")
     ws = torch.empty(4096, dtype=torch.uint8, device="cuda")
+    need1 = qmoe.workspace_size(case.layer(), 1)  # one token row of the decode layer
     with pytest.raises(qmoe.QmoeError) as e:
-        qmoe.forward(case.layer(), x, lg, y, ws)
+        qmoe.forward(case.layer(), x, lg, y, ws, ws_bytes=need1 - 256)
     assert e.value.status == qmoe.ERR_SCRATCH
     bad = case.layer()
     bad.k = 0
