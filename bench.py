@@ -18,7 +18,6 @@ linear K=5120 -> N=17408 (group 128, INT2 and INT4) at M = 1..32.
 from __future__ import annotations
 
 import argparse
-import dataclasses
 import json
 import os
 import statistics
@@ -343,10 +342,15 @@ def run_ours(args):
                                  "tokens_per_s": round(M / (r["ms_per_step"] * 1e-3), 1)})
     linear = [] if args.quick else linear_sweep(qmoe, torch, dist, args)
     lmhead = [] if args.quick else lmhead_sweep(qmoe, torch, dist, args)
-    # ternary layer (H=2048, I=6144 experts, 32 of them: one top-1 expert per token) and the
-    # prefill layer (T = 4096, 128 experts top-8, tcgen05 grouped path, 256 MiB workspace with row tiling)
-    ternary = [] if args.quick else cfg_sweep(qmoe, torch, dist, args,
-                                              dataclasses.replace(synth.TERNARY, E=32), (1, 8, 32), rotate=32)
+    # tiny layer (T = 1; 64 weight copies, 4 MB each, rotated past L2); the V2-Lite layer at
+    # its own batches T = 1, 2, 4, 8 with hot-expert routing; the ternary layer (H=2048,
+    # I=6144, 128 experts top-1; 8 distinct experts' bytes tiled over the 128) at
+    # T = 1, 8, 32, 128; the prefill layer (T = 4096, 128 experts top-8, tcgen05 grouped
+    # path, 256 MiB workspace with row tiling)
+    tiny = [] if args.quick else cfg_sweep(qmoe, torch, dist, args, synth.TINY, (1,), rotate=8, copies=64)
+    v2lite_batches = [] if args.quick else cfg_sweep(qmoe, torch, dist, args, synth.V2LITE, (1, 2, 4, 8), rotate=8)
+    ternary = [] if args.quick else cfg_sweep(qmoe, torch, dist, args, synth.TERNARY, (1, 8, 32, 128), rotate=32,
+                                              distinct=8)
     prefill = [] if args.quick else cfg_sweep(qmoe, torch, dist, args, synth.PREFILL, (4096,), rotate=1,
                                               ws_cap=256 << 20)
     e2e = measure_e2e(qmoe, torch, dist, layers[0], args.steps, args.warmup)
@@ -363,7 +367,12 @@ def run_ours(args):
     else:
         dom, dom_bytes = "fc1_small", head["fc1_bytes"]
         dom_desc = "fc1_small (dequant + gate/up MMA + SwiGLU)"
-    dom_ms = head["kernels"][dom]
+    # Kernel time for the roofline: in the clean graph the layer is the decode
+    # kernel plus an 8-CTA reset launch that runs under the previous layer's
+    # tail (programmatic dependent launch), so the step time bounds the decode
+    # kernel's time from above; events around each launch (a traced graph)
+    # break that overlap and are kept only as a breakdown.
+    dom_ms = min(head["kernels"][dom], head["ms_per_step"]) if dom != "decode_layer" else head["ms_per_step"]
     dom_gbps = dom_bytes / (dom_ms * 1e6)
     traffic = None
     tpath = os.path.join(ROOT, "profiles", "traffic.json")
@@ -401,10 +410,14 @@ def run_ours(args):
                      "achieved": round(dom_gbps, 1), "peak": hbm_peak, "peak_source": peak_src,
                      "unit": "GB/s", "frac": round(dom_gbps / hbm_peak, 3), "traffic": traffic,
                      "bytes_per_launch": int(dom_bytes), "launch_us": round(dom_ms * 1e3, 3),
-                     "kernels_us": {k: round(v * 1e3, 3) for k, v in head["kernels"].items()}},
+                     "launch_us_source": "ms_per_step (bounds the kernel; the reset launch overlaps the previous "
+                                         "layer)" if dom == "decode_layer" else "traced launch, capped at ms_per_step",
+                     "kernels_us_traced": {k: round(v * 1e3, 3) for k, v in head["kernels"].items()}},
         "sweep_tokens_per_expert": result_sweep,
         "linear_5120x17408_g128": linear,
         "linear_5120x248320_g128": lmhead,
+        "tiny_layer": tiny,
+        "v2lite_decode_batches": v2lite_batches,
         "ternary_layer": ternary,
         "prefill_layer": prefill,
         "e2e": e2e,
@@ -499,11 +512,18 @@ def cfg_layer_bytes(cfg, logits: np.ndarray) -> tuple[int, int]:
     return n * (f1 + f2) + T * cfg.H * 2 * 2 + T * cfg.E * 4, n
 
 
-def pack_cfg(qmoe, torch, cfg):
+def pack_cfg(qmoe, torch, cfg, distinct: int | None = None):
+    """Device layer for `cfg`.  With `distinct`, only that many experts are
+    drawn and quantized; expert e holds the packed bytes of expert e % distinct
+    (same sizes and layout, for timing a layer whose weights take minutes to draw)."""
     n = cfg.E + cfg.n_shared
+    d = n if distinct is None else min(n, distinct)
     f1, f2 = qmoe.FMT[cfg.fc1_fmt], qmoe.FMT[cfg.fc2_fmt]
-    c1, s1 = qmoe.pack_stack(f1, qmoe.ROWS_GATE_UP, (synth.expert_fc1(cfg, SEED, e) for e in range(n)), cfg.block)
-    c2, s2 = qmoe.pack_stack(f2, qmoe.ROWS_KSPLIT, (synth.expert_fc2(cfg, SEED, e) for e in range(n)), cfg.block)
+    c1, s1 = qmoe.pack_stack(f1, qmoe.ROWS_GATE_UP, (synth.expert_fc1(cfg, SEED, e) for e in range(d)), cfg.block)
+    c2, s2 = qmoe.pack_stack(f2, qmoe.ROWS_KSPLIT, (synth.expert_fc2(cfg, SEED, e) for e in range(d)), cfg.block)
+    if d < n:
+        reps = -(-n // d)
+        c1, s1, c2, s2 = (np.tile(a.reshape(d, -1), (reps, 1))[:n].reshape(-1) for a in (c1, s1, c2, s2))
     keep = [_to_dev(torch, a) for a in (c1, s1, c2, s2)]
     b1 = b2 = None
     if cfg.bias:
@@ -515,10 +535,22 @@ def pack_cfg(qmoe, torch, cfg):
     return qmoe.make_layer(cfg.H, cfg.I, cfg.E, cfg.k, cfg.n_shared, w1, w2), keep
 
 
-def cfg_sweep(qmoe, torch, dist, args, cfg, Ts, rotate: int, ws_cap: int | None = None) -> dict:
+def cfg_sweep(qmoe, torch, dist, args, cfg, Ts, rotate: int, ws_cap: int | None = None, copies: int = 1,
+              distinct: int | None = None) -> dict:
     """One layer forward per step on `cfg` for each T; router rows rotate over
-    `rotate` seeded draws so that consecutive steps touch different experts."""
-    layer, keep = pack_cfg(qmoe, torch, cfg)
+    `rotate` seeded draws so that consecutive steps touch different experts,
+    and over `copies` device copies of the weights (a layer smaller than L2)."""
+    layer0, keep = pack_cfg(qmoe, torch, cfg, distinct)
+    layers = [layer0]
+    base = list(keep)  # codes, scales of FC1 and FC2 (and the biases)
+    for _ in range(copies - 1):
+        cp = [a.clone() for a in base]
+        keep += cp
+        b1, b2 = (cp[4], cp[5]) if cfg.bias else (None, None)
+        w1 = qmoe.make_weights(qmoe.FMT[cfg.fc1_fmt], cfg.block, cp[0], cp[1], b1, qmoe.ROWS_GATE_UP)
+        w2 = qmoe.make_weights(qmoe.FMT[cfg.fc2_fmt], cfg.block, cp[2], cp[3], b2, qmoe.ROWS_KSPLIT)
+        layers.append(qmoe.make_layer(cfg.H, cfg.I, cfg.E, cfg.k, cfg.n_shared, w1, w2))
+    layer = layer0
     out = {"config": f"{cfg.name}: H={cfg.H} I={cfg.I} E={cfg.E} top-{cfg.k}"
                      f"{' + %d shared' % cfg.n_shared if cfg.n_shared else ''}, "
                      f"FC1 {cfg.fc1_fmt} / FC2 {cfg.fc2_fmt}, block {cfg.block}", "T": []}
@@ -530,12 +562,14 @@ def cfg_sweep(qmoe, torch, dist, args, cfg, Ts, rotate: int, ws_cap: int | None 
         ws = torch.empty(min(need, ws_cap) if ws_cap else need, dtype=torch.uint8, device="cuda")
         ys = [torch.empty((T, cfg.H), dtype=torch.int16, device="cuda") for _ in range(rotate)]
 
+        nrot = max(rotate, copies)
+
         def fn(i, n, xs=xs, lgs=lgs, ys=ys, ws=ws):
             r = i % rotate
-            qmoe.forward(layer, xs[r], lgs[r], ys[r], ws)
+            qmoe.forward(layers[i % copies], xs[r], lgs[r], ys[r], ws)
 
-        steps = Steps(torch, fn, rotate)
-        k = max(rotate, (args.steps // rotate) * rotate) if T <= 64 else rotate * 2
+        steps = Steps(torch, fn, nrot)
+        k = max(nrot, (args.steps // nrot) * nrot) if T <= 64 else nrot * 2
         steps.prepare(k, args.warmup)
         steps.run(max(args.warmup, 3))
         ms = reduce_ranks(torch, dist, time_steps(torch, dist, steps, k), 0.0)[0] / k
@@ -546,7 +580,11 @@ def cfg_sweep(qmoe, torch, dist, args, cfg, Ts, rotate: int, ws_cap: int | None 
                          "active_experts": round(statistics.mean(a for _, a in per), 1),
                          "GBps": round(nbytes / (ms * 1e6), 1), "TFLOPs": round(flops / (ms * 1e9), 2),
                          "workspace_bytes": ws.numel(), "row_tiles": qmoe.get_stats().row_tiles})
-    del keep
+    if copies > 1:
+        out["weight_copies_rotated"] = copies
+    if distinct is not None:
+        out["distinct_experts"] = f"{distinct} drawn and quantized; expert e holds the bytes of expert e % {distinct}"
+    del keep, layers
     return out
 
 
@@ -562,7 +600,7 @@ def lmhead_sweep(qmoe, torch, dist, args) -> list:
         del c, s
         w = qmoe.make_weights(qmoe.FMT[fmt], block, dc, ds)
         row = {"fmt": fmt, "bytes_M1": nbytes + K * 2 + N * 2, "M": []}
-        for M in (1, 2, 4, 8):
+        for M in range(1, 9):
             x = _to_dev(torch, synth.tokens(K, SEED, M))
             y = torch.empty((M, N), dtype=torch.int16, device="cuda")
             ws = torch.empty(qmoe.linear_workspace_size(N, K, M), dtype=torch.uint8, device="cuda")

@@ -71,17 +71,25 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t pari
   return ok != 0;
 }
 
-// mbar_wait_bounded without busy polling: sleeps in try_wait between checks of the clock.
-__device__ __forceinline__ bool mbar_wait_sleep_bounded(uint64_t* bar, uint32_t parity, unsigned* status) {
-  if (mbar_try_wait_sleep(bar, parity, 100000u)) return true;
+// mbar_wait_bounded without busy polling: sleeps in try_wait between checks
+// of the clock; gives up after limit_ns.
+static __device__ __noinline__ bool mbar_wait_sleep_slow(uint64_t* bar, uint32_t parity, unsigned* status,
+                                                         unsigned long long limit_ns) {
   const unsigned long long t0 = global_timer_ns();
+  const uint32_t hint = limit_ns < 100000ull ? (uint32_t)limit_ns : 100000u;
   for (;;) {
-    if (mbar_try_wait_sleep(bar, parity, 100000u)) return true;
-    if (global_timer_ns() - t0 > kWaitLimitNs) {
+    if (mbar_try_wait_sleep(bar, parity, hint)) return true;
+    if (global_timer_ns() - t0 > limit_ns) {
       if (status) atomicOr(status, kStatusTimeout);
       return false;
     }
   }
+}
+
+__device__ __forceinline__ bool mbar_wait_sleep_bounded(uint64_t* bar, uint32_t parity, unsigned* status,
+                                                        unsigned long long limit_ns = kWaitLimitNs) {
+  if (mbar_try_wait_sleep(bar, parity, limit_ns < 100000ull ? (uint32_t)limit_ns : 100000u)) return true;
+  return mbar_wait_sleep_slow(bar, parity, status, limit_ns);
 }
 
 // Waits for the phase with the given parity to complete.  Gives up after
@@ -132,11 +140,21 @@ __device__ __forceinline__ int atomic_add_acq_rel_gpu(int* p, int v) {
 
 // D (+)= A * B, m16n8k16, bf16 inputs, fp32 accumulators.
 __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-  asm volatile(
+  asm(
       "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
       "{%0,%1,%2,%3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// D = A * B + C, m16n8k16, bf16 inputs, fp32 accumulators, C kept.
+__device__ __forceinline__ void mma_bf16_16816_c(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1,
+                                                 const float (&c)[4]) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%10,%11,%12,%13};"
+      : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(c[0]), "f"(c[1]), "f"(c[2]),
+        "f"(c[3]));
 }
 
 // (x & mask) | magic in one LOP3.

@@ -72,6 +72,7 @@ constexpr int round128c(int v) { return (v + 127) / 128 * 128; }
 struct SliceSmemLayout {
   static constexpr int kBars = 0;                                       // [kSW][kSNB] u64
   static constexpr int kXBar = kBars + kSW * kSNB * 8;                  // x bulk-copy barrier
+  static constexpr int kDBar = kXBar + 8;                               // barrier nothing arrives at (fault injection)
   static constexpr int kMisc = kXBar + 16;                              // 16 ints
   static constexpr int kVst = kMisc + 64;                               // [kSW][kSNB] int: item virtual offsets
   static constexpr int kPst = kVst + kSW * kSNB * 4;                    // [kSW][kSNB] int: item ring offsets
@@ -380,6 +381,7 @@ __global__ void __launch_bounds__(kSThreads, 1) qmm_slice_kernel(const SlicePara
   extern __shared__ __align__(128) uint8_t smem[];
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBars);
   uint64_t* xbar = reinterpret_cast<uint64_t*>(smem + L::kXBar);
+  uint64_t* dbar = reinterpret_cast<uint64_t*>(smem + L::kDBar);
   int* misc = reinterpret_cast<int*>(smem + L::kMisc);
   DecodeRoute& R = *reinterpret_cast<DecodeRoute*>(smem + L::kRoute);
   float* wmat = reinterpret_cast<float*>(smem + L::kWmat);
@@ -407,6 +409,7 @@ __global__ void __launch_bounds__(kSThreads, 1) qmm_slice_kernel(const SlicePara
     for (int s = 0; s < kSNB; ++s) mbar_init(&wbar[s], 33);  // lane 0's arrival + 32 cp.async arrivals
   if (tid == 0) {
     mbar_init(xbar, 1);
+    mbar_init(dbar, 1);
     misc[kMiscAbort] = 0;
     misc[kMiscChunks] = 0;
     misc[kMiscEarly] = 0;
@@ -505,7 +508,7 @@ __global__ void __launch_bounds__(kSThreads, 1) qmm_slice_kernel(const SlicePara
 
   // ---- after the previous launches: x rows, routing ----
   pdl_wait();
-  if (warp == 0) {
+  if (warp == kSW - 1) {  // the first T warps route
     if (lane == 0) mbar_arrive_expect_tx(xbar, (uint32_t)(T * p.H * 2));
     __syncwarp();
     if (lane < T) bulk_copy_g2s(xs + lane * xpitch, p.x + (size_t)lane * p.H, (uint32_t)(p.H * 2), xbar);
@@ -534,7 +537,8 @@ __global__ void __launch_bounds__(kSThreads, 1) qmm_slice_kernel(const SlicePara
   refill();
 
   // x landed (bounded wait), then the hi columns divided by the code multiplier
-  if (!mbar_wait_sleep_bounded(xbar, 0, p.status)) misc[kMiscAbort] = 1;
+  if (!mbar_wait_sleep_bounded(xbar, 0, p.status, p.wait_ns)) misc[kMiscAbort] = 1;
+  if (p.inject == 1 && tid == 0 && !mbar_wait_sleep_bounded(dbar, 0, p.status, p.wait_ns)) misc[kMiscAbort] = 1;
   __syncthreads();
   if constexpr (T1::kBetaHi == 4) {
     for (int i = tid; i < T * p.H / 16; i += kSThreads) {  // one 8-column high half per item
@@ -579,7 +583,7 @@ __global__ void __launch_bounds__(kSThreads, 1) qmm_slice_kernel(const SlicePara
   uint32_t cpar = 0;  // phase parity of the consumed slot
   int drain = ok ? INT_MAX : 0;  // first item that may still be in flight after a wait gave up
   auto wait_item = [&]() -> const uint8_t* {
-    if (ok && __any_sync(0xffffffffu, !mbar_wait_sleep_bounded(&wbar[cslot], cpar, p.status))) {
+    if (ok && __any_sync(0xffffffffu, !mbar_wait_sleep_bounded(&wbar[cslot], cpar, p.status, p.wait_ns))) {
       ok = false;
       drain = cons;
       misc[kMiscAbort] = 1;
@@ -654,8 +658,8 @@ __global__ void __launch_bounds__(kSThreads, 1) qmm_slice_kernel(const SlicePara
   }
   // Nothing may land in shared memory past this point: after a wait gave up,
   // wait (bounded again) for the items issued from then on, and for x.
-  for (int i = drain; i < issued; ++i) mbar_wait_sleep_bounded(&wbar[i % kSNB], (i / kSNB) & 1, p.status);
-  if (misc[kMiscAbort] && tid == 0) mbar_wait_sleep_bounded(xbar, 0, p.status);
+  for (int i = drain; i < issued; ++i) mbar_wait_sleep_bounded(&wbar[i % kSNB], (i / kSNB) & 1, p.status, p.wait_ns);
+  if (misc[kMiscAbort] && tid == 0) mbar_wait_sleep_bounded(xbar, 0, p.status, p.wait_ns);
   cp_async_wait_all();
   __syncthreads();
 
@@ -693,7 +697,12 @@ __global__ void __launch_bounds__(kSThreads, 1) qmm_slice_kernel(const SlicePara
         red_add_v4_f32(p.yacc + 4 * i, reinterpret_cast<const float4*>(ys)[i]);
   }
   __syncthreads();
-  if (tid == 0) misc[kMiscLast] = atomic_add_acq_rel_gpu(p.ticket, 1) == G - 1;
+  if (tid == 0) {
+    if (misc[kMiscAbort]) atomicAdd(p.ticket + 1, 1);  // counted before this CTA's ticket
+    misc[kMiscLast] = atomic_add_acq_rel_gpu(p.ticket, 1) == G - 1;
+    // after a CTA gave up a wait the sum is incomplete: y stays as it was
+    if (misc[kMiscLast] && *(volatile int*)(p.ticket + 1) != 0) misc[kMiscLast] = 0;
+  }
   __syncthreads();
   if (misc[kMiscLast]) {
     for (int i = tid; i < T * p.H / 4; i += kSThreads) {
@@ -706,7 +715,7 @@ __global__ void __launch_bounds__(kSThreads, 1) qmm_slice_kernel(const SlicePara
   }
 }
 
-// Clears the fp32 accumulator and the ticket of the decode kernel launched
+// Clears the fp32 accumulator and the tickets of the decode kernel launched
 // after it.  It lets that launch start at once (its CTAs wait for this
 // kernel's completion before their first access to either), then waits for
 // the launch before it, which may still read them.
@@ -715,7 +724,7 @@ __global__ void slice_reset_kernel(float* yacc, int n4, int* ticket) {
   pdl_wait();
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += gridDim.x * blockDim.x)
     reinterpret_cast<float4*>(yacc)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-  if (blockIdx.x == 0 && threadIdx.x == 0) *ticket = 0;
+  if (blockIdx.x == 0 && threadIdx.x == 0) ticket[0] = ticket[1] = 0;
 }
 
 }  // namespace qmoe

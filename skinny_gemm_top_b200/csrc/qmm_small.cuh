@@ -384,8 +384,16 @@ __device__ __forceinline__ float logit_of_key(uint32_t key) {
 //     expert's rank among the selected ones (its segment).
 // V = experts per lane (E <= 32 V); decode_route picks the smallest.
 // Needs blockDim.x >= 32 T; ends with a CTA barrier.
-template <int V>
-__device__ void decode_route_v(const float* logits, int T, int E, int k, DecodeRoute& R) {
+// Barrier of the threads that route: the whole CTA (NB == 0), else the first
+// NB threads on named barrier 1.
+template <int NB>
+__device__ __forceinline__ void route_sync() {
+  if constexpr (NB == 0) __syncthreads();
+  else asm volatile("bar.sync 1, %0;" ::"n"(NB) : "memory");
+}
+
+template <int V, int NB>
+__device__ __noinline__ void decode_route_v(const float* logits, int T, int E, int k, DecodeRoute& R) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int TK = T * k;
   if (warp < T) {
@@ -436,7 +444,7 @@ __device__ void decode_route_v(const float* logits, int T, int E, int k, DecodeR
     }
   }
   if (T > 1) {
-    __syncthreads();
+    route_sync<NB>();
     if (warp == 0) {
       int* hist = R.hist;  // per expert: the mask of the tokens that selected it
       const int nb = (E + 31) / 32;  // experts per lane in the scan
@@ -494,15 +502,16 @@ __device__ void decode_route_v(const float* logits, int T, int E, int k, DecodeR
       if (lane == 0) R.nseg = nsel;
     }
   }
-  __syncthreads();
+  route_sync<NB>();
 }
 
 // (A lane holding 8 experts where 2 would do made the routing of a 64-expert
 // layer about 1.5k cycles slower: measured in isolation.)
+template <int NB = 0>
 __device__ __forceinline__ void decode_route(const float* logits, int T, int E, int k, DecodeRoute& R) {
-  if (E <= 64) decode_route_v<2>(logits, T, E, k, R);
-  else if (E <= 128) decode_route_v<4>(logits, T, E, k, R);
-  else decode_route_v<8>(logits, T, E, k, R);
+  if (E <= 64) decode_route_v<2, NB>(logits, T, E, k, R);
+  else if (E <= 128) decode_route_v<4, NB>(logits, T, E, k, R);
+  else decode_route_v<8, NB>(logits, T, E, k, R);
 }
 
 // Epilogue of one reduced fragment: rows g / g+8 of tile rt, tokens n0, n0+1.

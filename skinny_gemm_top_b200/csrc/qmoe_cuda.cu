@@ -159,6 +159,11 @@ int grouped_threshold(const qmoe_layer& L) {
   return L.path == QMOE_PATH_GROUPED ? 0 : kGroupedThreshold;
 }
 
+// Fault injection for tests (qmoe_test_set_fault): the decode kernel's wait
+// limit and what to inject.
+unsigned long long g_fault_wait_ns = kWaitLimitNs;
+int g_fault_inject = 0;
+
 // Decode batches (T <= 8, T*k <= 64, H <= 2112) run as one launch of the
 // kernel split along the expert intermediate dimension, which routes in its
 // prologue (after a tiny reset launch of its accumulator).
@@ -414,6 +419,13 @@ qmoe_status qmoe_trace_read(int cap, int* n, int* kernel_ids, float* ms) {
   return QMOE_OK;
 }
 
+qmoe_status qmoe_test_set_fault(int inject, unsigned long long wait_limit_ns) {
+  if (inject < 0 || inject > 1) return QMOE_ERR_INVALID_ARG;
+  qmoe::g_fault_inject = inject;
+  qmoe::g_fault_wait_ns = wait_limit_ns ? wait_limit_ns : qmoe::kWaitLimitNs;
+  return QMOE_OK;
+}
+
 qmoe_status qmoe_get_stats(qmoe_stats* out) {
   if (!out) return QMOE_ERR_INVALID_ARG;
   DevInfo* di;
@@ -550,6 +562,8 @@ qmoe_status qmoe_forward(const qmoe_layer* layer, const uint16_t* x, const float
       sp.yacc = reinterpret_cast<float*>(base + p.yacc);
       sp.ticket = reinterpret_cast<int*>(base + p.ticket);
       sp.status = di->status;
+      sp.wait_ns = g_fault_wait_ns;
+      sp.inject = g_fault_inject;
       {
         TraceScope ts(st, K_DECODE_RESET);
         if (slice_reset_launch(sp.yacc, tt * L.H / 4, sp.ticket, st) != cudaSuccess) return QMOE_ERR_CUDA;

@@ -63,8 +63,10 @@ struct SliceParams {
   const float* logits;  // [T][E]
   uint16_t* y;          // [T][H] bf16
   float* yacc;          // [T][H] fp32, zero at launch
-  int* ticket;          // zero at launch
+  int* ticket;          // [0]: CTAs done, [1]: CTAs that gave up a wait; zero at launch
   unsigned* status;
+  unsigned long long wait_ns;  // limit of every wait in the kernel
+  int inject;                  // fault injection (tests): 1 = one wait on a barrier nothing arrives at
 };
 
 // Geometry of one launch: ring stages and shared memory for (FC1 format,

@@ -61,6 +61,7 @@ EXPORTS = {
                     C.c_size_t, C.c_void_p],
     "qmoe_get_stats": [C.POINTER(Stats)],
     "qmoe_clear_status": [],
+    "qmoe_test_set_fault": [C.c_int, C.c_ulonglong],
     "qmoe_status_str": [C.c_int],
     "qmoe_trace_start": [C.c_int],
     "qmoe_trace_stop": [],
@@ -217,6 +218,14 @@ def get_stats() -> Stats:
 
 def clear_status():
     _check(_lib.qmoe_clear_status(), "qmoe_clear_status")
+
+
+DEVICE_TIMEOUT, DEVICE_BAD_SEGMENT = 1, 2
+
+
+def test_set_fault(inject: int, wait_limit_ns: int = 0):
+    """Test hook: fault injection for the decode-layer kernel (qmoe.h)."""
+    _check(_lib.qmoe_test_set_fault(inject, wait_limit_ns), "qmoe_test_set_fault")
 
 
 # ---------------------------------------------------------------- tracing

@@ -114,3 +114,11 @@ def test_pack_rejects_bad_arguments(args, status):
     codes = np.zeros(1 << 16, dtype=np.uint8)
     st = qmoe.lib().qmoe_pack(fmt, order, w.ctypes.data, rows, K, block, codes.ctypes.data, codes.ctypes.data)
     assert st == status
+
+
+def test_fault_hook_validates_host_side():
+    """The fault-injection hook only sets host state: no GPU needed."""
+    from skinny_gemm_top_b200 import qmoe
+    with pytest.raises(qmoe.QmoeError):
+        qmoe.test_set_fault(5, 0)
+    qmoe.test_set_fault(0, 0)

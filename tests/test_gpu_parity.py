@@ -231,6 +231,43 @@ def test_forward_tiny(qm, T):
     _close(y, ref, f"tiny T={T}")
 
 
+def test_decode_wait_expiry_leaves_y_and_recovers(qm):
+    """A bounded device wait driven to expiry: with the test hook, every CTA of
+    the decode kernel waits 1 ms on a barrier nothing arrives at.  The timeout
+    flag is set, y keeps its previous contents, and the next call (hook off)
+    is correct."""
+    import torch
+    cfg = synth.TINY
+    case = MoECase(cfg, seed=3)
+    x_bits = synth.tokens(cfg.H, 3, 1)
+    lg_np = synth.router_logits(cfg, 3, 1)
+    ref = Q.moe_forward(Q.bf16_bits_to_f64(x_bits), lg_np, cfg.k, case.bank)
+    layer = case.layer()
+    ws = torch.empty(qm.workspace_size(layer, 1), dtype=torch.uint8, device="cuda")
+    x = torch.from_numpy(x_bits.view(np.int16)).cuda()
+    lg = torch.from_numpy(np.ascontiguousarray(lg_np, dtype=np.float32)).cuda()
+    y = torch.full((1, cfg.H), 0x3F80, dtype=torch.int16, device="cuda")  # bf16 1.0 everywhere
+    try:
+        qm.test_set_fault(1, 1_000_000)
+        qm.clear_status()
+        qm.forward(layer, x, lg, y, ws)
+        torch.cuda.synchronize()
+        assert qm.get_stats().device_status & qm.DEVICE_TIMEOUT
+        assert bool((y == 0x3F80).all()), "y was written although a CTA gave up"
+    finally:
+        qm.test_set_fault(0, 0)
+        qm.clear_status()
+    qm.forward(layer, x, lg, y, ws)
+    torch.cuda.synchronize()
+    assert qm.get_stats().device_status == 0
+    _close(bf16_dev_to_f64(y), ref, "tiny after an expired wait")
+
+
+def test_fault_hook_rejects_unknown_injection(qm):
+    with pytest.raises(qm.QmoeError):
+        qm.test_set_fault(2, 0)
+
+
 @pytest.fixture(scope="module")
 def v2lite(qm):
     return MoECase(synth.V2LITE, seed=5)
