@@ -52,6 +52,8 @@ def parse():
                     help="a few eager layer forwards and linears only (for an ncu launch list or capture)")
     ap.add_argument("--profile-prefill", action="store_true",
                     help="two eager forwards of the prefill layer (T = 4096, one row tile) only, for an ncu capture")
+    ap.add_argument("--profile-ternary", action="store_true",
+                    help="a few eager forwards of the ternary layer (128 experts, T = 1) only, for an ncu capture")
     return ap.parse_args()
 
 
@@ -266,6 +268,24 @@ def run_profile_prefill(args):
     assert qmoe.get_stats().device_status == 0
     del keep
     print("prefill profile run done", flush=True)
+
+
+def run_profile_ternary(args):
+    """A few eager forwards of the ternary layer (H=2048, I=6144, 128 experts top-1) at T = 1."""
+    import torch
+    from skinny_gemm_top_b200 import qmoe
+    cfg = synth.TERNARY
+    layer, keep = pack_cfg(qmoe, torch, cfg, distinct=8)
+    x = _to_dev(torch, synth.tokens(cfg.H, SEED, 1))
+    ws = torch.empty(qmoe.workspace_size(layer, 1), dtype=torch.uint8, device="cuda")
+    y = torch.empty((1, cfg.H), dtype=torch.int16, device="cuda")
+    for r in range(max(args.steps, 1)):
+        lg = torch.from_numpy(np.ascontiguousarray(synth.router_logits(cfg, SEED, 1, index=100 + r))).cuda()
+        qmoe.forward(layer, x, lg, y, ws)
+        torch.cuda.synchronize()
+    assert qmoe.get_stats().device_status == 0
+    del keep
+    print("ternary profile run done", flush=True)
 
 
 def run_ours(args):
@@ -702,6 +722,8 @@ def main():
         run_profile(args)
     elif args.profile_prefill:
         run_profile_prefill(args)
+    elif args.profile_ternary:
+        run_profile_ternary(args)
     else:
         run_ours(args)
 

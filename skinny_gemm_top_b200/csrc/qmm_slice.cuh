@@ -7,8 +7,9 @@
 // shared experts of the layer get every token with weight 1.
 //
 // Work split (B200 design): every active expert's intermediate dimension I is
-// cut into granules of kCols columns of h (16 for an INT4 FC2, 32 INT2, 128
-// ternary: the K width of one slab of the QMOE_ROWS_KSPLIT FC2 layout).  Each
+// cut into granules of kCols columns of h (16 for an INT4 FC2, 32 INT2: the K
+// width of one slab of the QMOE_ROWS_KSPLIT FC2 layout; 64 ternary, half of
+// one 128-column record).  Each
 // CTA gets a contiguous range of granules: with at least two CTAs per active
 // expert, every expert (shared ones first, then the selected ones in expert
 // order) gets its own group of CTAs, so a CTA's range lies inside one expert;
@@ -26,7 +27,7 @@
 // accumulator with vector atomics; the last CTA (ticket) rounds it to bf16.
 //
 // Inside a CTA the range's FC1 tiles form chunks of up to 10 tiles of one
-// expert (8 for INT2 or ternary FC2).  Each of the 12 warps streams, through
+// expert (8 for INT2 or ternary FC2: whole granules).  Each of the 12 warps streams, through
 // its own ring of item buffers, the chunk's k-units w, w+12, ... (all the
 // chunk's tiles: one contiguous run of codes, one TMA bulk copy) and then,
 // after a cross-warp reduction (fixed warp order) has produced the chunk's h,
@@ -52,11 +53,15 @@ namespace qmoe {
 
 constexpr int kSThreads = kSW * 32;
 
-// FC2 granule of the K-split layout.
+// FC2 granule of the K-split layout: kCols columns of h; kRowBytes code bytes
+// loaded per 16-row tile.  A ternary granule is half of a 128-column record:
+// its CTA loads the whole record and uses its own four k-steps (the record's
+// other half, read by the neighbouring granule's CTA at about the same time,
+// is mostly served by L2), so that twice as many CTAs share a ternary layer.
 template <int F> struct KsTr;
-template <> struct KsTr<4> { static constexpr int kCols = 16, kRowBytes = 128, kKsteps = 1, kBlocks = 1; };
-template <> struct KsTr<2> { static constexpr int kCols = 32, kRowBytes = 128, kKsteps = 2, kBlocks = 1; };
-template <> struct KsTr<3> { static constexpr int kCols = 128, kRowBytes = 416, kKsteps = 8, kBlocks = 2; };
+template <> struct KsTr<4> { static constexpr int kCols = 16, kRowBytes = 128, kKsteps = 1, kBlocks = 1, kPerRec = 1; };
+template <> struct KsTr<2> { static constexpr int kCols = 32, kRowBytes = 128, kKsteps = 2, kBlocks = 1, kPerRec = 1; };
+template <> struct KsTr<3> { static constexpr int kCols = 64, kRowBytes = 416, kKsteps = 4, kBlocks = 1, kPerRec = 2; };
 
 // FC1 tiles per chunk at most: whole granules up to 10 tiles; a ternary
 // granule (16 tiles) is two chunks of 8.
@@ -125,16 +130,12 @@ __device__ void slice_add_piece(SChunk* tab, int* n, int expert, int wsel, int g
     C.pad = 0;
     tab[(*n)++] = C;
   };
-  if constexpr (TPG <= kSChunk) {
-    constexpr int gmax = CG::kMT / TPG;
-    const int ng = gb - ga, nch = (ng + gmax - 1) / gmax;
-    for (int i = 0; i < nch; ++i) {  // near-equal granule counts
-      const int g0 = ga + ng * i / nch, g1 = ga + ng * (i + 1) / nch;
-      push(g0 * TPG, (g1 - g0) * TPG, g0, g1 - g0, 0);
-    }
-  } else {
-    for (int g = ga; g < gb; ++g)
-      for (int h = 0; h < TPG / 8; ++h) push(g * TPG + 8 * h, 8, g, h == TPG / 8 - 1 ? 1 : 0, 8 * h);
+  static_assert(TPG <= kSChunk, "a granule fits in one chunk");
+  constexpr int gmax = CG::kMT / TPG;
+  const int ng = gb - ga, nch = (ng + gmax - 1) / gmax;
+  for (int i = 0; i < nch; ++i) {  // near-equal granule counts
+    const int g0 = ga + ng * i / nch, g1 = ga + ng * (i + 1) / nch;
+    push(g0 * TPG, (g1 - g0) * TPG, g0, g1 - g0, 0);
   }
 }
 
@@ -273,7 +274,7 @@ __device__ __forceinline__ void slice_fc1(const uint8_t* st, int nt, int ku, con
 // FC2 item: ng granules of this warp's nr row tiles, accumulated into acc2.
 // B fragments are the h window's k-steps from window granule wg0 on.
 template <int F2>
-__device__ __forceinline__ void slice_fc2(const uint8_t* st, int ng, int nr, int wg0, const uint2* hfrag,
+__device__ __forceinline__ void slice_fc2(const uint8_t* st, int ng, int nr, int wg0, int g_abs, const uint2* hfrag,
                                           const uint32_t* lut, int lane, float (&acc2)[kSRT][4]) {
   using K2 = KsTr<F2>;
   using Tr2 = FmtTraits<F2>;
@@ -299,20 +300,23 @@ __device__ __forceinline__ void slice_fc2(const uint8_t* st, int ng, int nr, int
     for (int i = 0; i < kSRT; ++i) {
       if (i >= nr) break;
       if constexpr (F2 == 3) {
+        // this granule's half of the record (the other half's unpack is dead code)
         uint32_t am[8][4];
         unpack_tern_record(cbase + i * 416 + lane * 13, lut, am);
+        float tmp[4] = {cr[0][0], cr[0][1], cr[0][2], cr[0][3]};
+        if ((g_abs + gi) & 1) {
 #pragma unroll
-        for (int bl = 0; bl < 2; ++bl) {
-          float tmp[4] = {cr[bl][0], cr[bl][1], cr[bl][2], cr[bl][3]};
+          for (int s = 0; s < 4; ++s) mma_bf16_16816(tmp, am[4 + s], b[s].x, b[s].y);
+        } else {
 #pragma unroll
-          for (int s = 0; s < 4; ++s) mma_bf16_16816(tmp, am[bl * 4 + s], b[bl * 4 + s].x, b[bl * 4 + s].y);
-          const uint32_t sc = sbuf[((gi * 2 + bl) * nr + i) * 8 + g];
-          const float slo = bf16_lo(sc), shi = bf16_hi(sc);
-          acc2[i][0] = fmaf(slo, tmp[0], acc2[i][0]);
-          acc2[i][1] = fmaf(slo, tmp[1], acc2[i][1]);
-          acc2[i][2] = fmaf(shi, tmp[2], acc2[i][2]);
-          acc2[i][3] = fmaf(shi, tmp[3], acc2[i][3]);
+          for (int s = 0; s < 4; ++s) mma_bf16_16816(tmp, am[s], b[s].x, b[s].y);
         }
+        const uint32_t sc = sbuf[(gi * nr + i) * 8 + g];
+        const float slo = bf16_lo(sc), shi = bf16_hi(sc);
+        acc2[i][0] = fmaf(slo, tmp[0], acc2[i][0]);
+        acc2[i][1] = fmaf(slo, tmp[1], acc2[i][1]);
+        acc2[i][2] = fmaf(shi, tmp[2], acc2[i][2]);
+        acc2[i][3] = fmaf(shi, tmp[3], acc2[i][3]);
       } else {
         const uint32_t w = *reinterpret_cast<const uint32_t*>(cbase + i * 128 + lane * 4);
         float tmp[4] = {cr[0][0], cr[0][1], cr[0][2], cr[0][3]};
@@ -479,9 +483,9 @@ __global__ void __launch_bounds__(kSThreads, 1) qmm_slice_kernel(const SlicePara
         if (lane == 0) mbar_arrive(bar);
         const int per = nr * (K2::kRowBytes / 16);
         for (int gi = 0; gi < ngi; ++gi) {
-          const int slab = C.g0 + prod.a + gi;  // granule of the expert = K-split slab
+          const int slab = C.g0 + prod.a + gi;  // granule of the expert = K-split slab (ternary: half a record)
           const uint8_t* src = p.c2 + (unsigned long long)C.expert * p.c2_stride +
-                               ((unsigned long long)slab * p.NT2 + r0) * K2::kRowBytes;
+                               ((unsigned long long)(slab / K2::kPerRec) * p.NT2 + r0) * K2::kRowBytes;
           uint8_t* dst = st + gi * nr * K2::kRowBytes;
           for (int i = lane; i < per; i += 32) cp_async16(dst + 16 * i, src + 16 * i);
 #pragma unroll
@@ -652,7 +656,7 @@ __global__ void __launch_bounds__(kSThreads, 1) qmm_slice_kernel(const SlicePara
     if (nr > 0)
       for (int a = 0; a < C.ngc; a += p.ngm) {  // window granule a: the chunk's completed granule a
         const uint8_t* st = wait_item();
-        if (ok) slice_fc2<F2>(st, min(p.ngm, C.ngc - a), nr, a, hfrag, lut, lane, acc2);
+        if (ok) slice_fc2<F2>(st, min(p.ngm, C.ngc - a), nr, a, C.g0 + a, hfrag, lut, lane, acc2);
         next_item();
       }
   }

@@ -15,8 +15,8 @@ constexpr int kSmemLimit = 227 * 1024;
 int fc1_code_bytes(int f) { return f == 2 ? 256 : f == 4 ? 512 : 416; }  // per tile and k-unit
 int fc1_blocks_per_ku(int f) { return f == 3 ? 2 : 1; }
 int fc2_row_bytes(int f) { return f == 3 ? 416 : 128; }                  // per row tile and granule
-int fc2_blocks(int f) { return f == 3 ? 2 : 1; }
-int fc2_cols(int f) { return f == 4 ? 16 : f == 2 ? 32 : 128; }         // granule width (h columns)
+int fc2_blocks(int) { return 1; }                                        // scale rows per granule
+int fc2_cols(int f) { return f == 4 ? 16 : f == 2 ? 32 : 64; }          // granule width (h columns)
 int round128(int v) { return (v + 127) / 128 * 128; }
 int chunk_tiles(int f2) { return f2 == 4 ? 10 : 8; }                    // SChunkGeom<f2>::kMT
 
