@@ -728,8 +728,7 @@ struct PhaseCtx {
 
 // Partition, prime (weights, then hook(), then activation rows), stream the
 // items, reduce and run the epilogue.  hook() is called by every thread of
-// the CTA exactly once (also by CTAs without work): the dependency wait, or a
-// grid barrier.
+// the CTA exactly once (also by CTAs without work): the dependency wait.
 template <int FMT, int TG, int EPI, int SRC, class Hook>
 __device__ __forceinline__ void run_phase(const SmallParams& p, const SegSource& segs, int nseg, const int* act_index,
                                           PhaseCtx& cx, Hook&& hook) {
