@@ -362,6 +362,7 @@ def run_ours(args):
                                  "tokens_per_s": round(M / (r["ms_per_step"] * 1e-3), 1)})
     linear = [] if args.quick else linear_sweep(qmoe, torch, dist, args)
     lmhead = [] if args.quick else lmhead_sweep(qmoe, torch, dist, args)
+    decoder_layer = [] if args.quick else model_layer_sweep(qmoe, torch, dist, args)
     # tiny layer (T = 1; 64 weight copies, 4 MB each, rotated past L2); the V2-Lite layer at
     # its own batches T = 1, 2, 4, 8 with hot-expert routing; the ternary layer (H=2048,
     # I=6144, 128 experts top-1; 8 distinct experts' bytes tiled over the 128) at
@@ -436,6 +437,11 @@ def run_ours(args):
         "sweep_tokens_per_expert": result_sweep,
         "linear_5120x17408_g128": linear,
         "linear_5120x248320_g128": lmhead,
+        "decoder_layer_linears_g128": {"shapes": [{"name": n, "N": N, "K": K, "count": c}
+                                                  for n, N, K, c in DECODER_LINEARS],
+                                       "note": "q, k, v, o taken as 5120x5120 (the pages give no attention shapes); "
+                                               "per-forward bill = layers x layer_us + lm_head",
+                                       "rows": decoder_layer},
         "tiny_layer": tiny,
         "v2lite_decode_batches": v2lite_batches,
         "ternary_layer": ternary,
@@ -605,6 +611,51 @@ def cfg_sweep(qmoe, torch, dist, args, cfg, Ts, rotate: int, ws_cap: int | None 
     if distinct is not None:
         out["distinct_experts"] = f"{distinct} drawn and quantized; expert e holds the bytes of expert e % {distinct}"
     del keep, layers
+    return out
+
+
+# One decoder layer of the model the MLX issue bills per forward (hidden 5120, MLP
+# intermediate 17408, vocabulary 248320).  The pages give no attention shapes; the
+# plainest reading, full multi-head attention with q, k, v and o all 5120 x 5120, is
+# taken here.  (N, K, count) per layer.
+DECODER_LINEARS = (("q_k_v_o", 5120, 5120, 4), ("gate_up", 17408, 5120, 2), ("down", 5120, 17408, 1))
+
+
+def model_layer_sweep(qmoe, torch, dist, args) -> list:
+    """Every linear of one decoder layer at widths M = 1..6 (the speculative-verify
+    window), group 128, INT2 and INT4: the per-layer bill of the MLX issue's per-forward
+    sum.  Each shape's weights rotate over copies past L2."""
+    out = []
+    for fmt in ("int2", "int4"):
+        per_shape = {}
+        for name, N, K, count in DECODER_LINEARS:
+            wb = synth.linear_weight(SEED, N, K)
+            c, s = qmoe.pack(qmoe.FMT[fmt], qmoe.ROWS_PLAIN, wb, 128)
+            nbytes = c.nbytes + s.nbytes
+            rot = max(2, int(np.ceil(2 * 126e6 / nbytes)) + 1)
+            dc, ds = _to_dev(torch, c), _to_dev(torch, s)
+            copies = [(dc, ds)] + [(dc.clone(), ds.clone()) for _ in range(rot - 1)]
+            wl = [qmoe.make_weights(qmoe.FMT[fmt], 128, a, b) for a, b in copies]
+            per_shape[name] = []
+            for M in range(1, 7):
+                x = _to_dev(torch, synth.tokens(K, SEED, M))
+                y = torch.empty((M, N), dtype=torch.int16, device="cuda")
+                ws = torch.empty(qmoe.linear_workspace_size(N, K, M), dtype=torch.uint8, device="cuda")
+
+                def fn(i, n, x=x, y=y, ws=ws, N=N, K=K):
+                    qmoe.linear(wl[i % rot], N, K, x, y, ws)
+
+                steps = Steps(torch, fn, rot)
+                k = max(args.steps, 64)
+                steps.prepare(k, args.warmup)
+                steps.run(args.warmup)
+                per_shape[name].append(reduce_ranks(torch, dist, time_steps(torch, dist, steps, k), 0.0)[0] / k)
+            del copies, wl, dc, ds
+        layer_us = [sum(per_shape[n][m] * cnt for n, _, _, cnt in DECODER_LINEARS) * 1e3 for m in range(6)]
+        out.append({"fmt": fmt, "M": list(range(1, 7)),
+                    "per_linear_us": {n: [round(v * 1e3, 3) for v in per_shape[n]] for n, _, _, _ in DECODER_LINEARS},
+                    "layer_us": [round(v, 2) for v in layer_us],
+                    "layer_slope_vs_M1": [round(v / layer_us[0], 3) for v in layer_us]})
     return out
 
 

@@ -25,6 +25,9 @@ Readings where the pages are silent:
 
 * INT scale: s = bf16_rne(max|w| / 2^(bits-1)); codes c = clamp(rne(w/s),
   -2^(bits-1), 2^(bits-1)-1) in float64; s == 0 gives c = 0.
+* Affine codes (scale and zero point per block, MLX-style): z = bf16_rne(min
+  w), s = bf16_rne((max w - min w) / (2^bits - 1)), u = clamp(rne((w - z) / s),
+  0, 2^bits - 1); w_hat = s * u + z.
 * Ternary: delta = 0.7 * (sum|w| / block); t = sign(w) where |w| > delta
   (strict), else 0; s = bf16_rne(mean of |w| over |w| > delta), 0 if none.
   Sums run sequentially in K order in float64.
@@ -98,6 +101,46 @@ def quantize_sym(w, bits: int, block: int):
     q = np.where(s[..., None] > 0, q, 0.0)
     c = np.clip(q, qmin, qmax).astype(np.int8)
     return c.reshape(rows, K), s
+
+
+def quantize_affine(w, bits: int, block: int):
+    """Affine (asymmetric) block quantization: one bf16 scale and one bf16 zero
+    point (bias) per block, unsigned codes (MLX issue "2-bit quantized_matmul
+    loses its size advantage over 4-bit at M >= 3", repro: ``mx.quantize``
+    returns (wq, scales, biases); its "2.25 effective" bits per weight at
+    group 128).
+
+    Reading (the pages give no formula): z = bf16_rne(min w), s =
+    bf16_rne((max w - min w) / (2^bits - 1)), u = clamp(rne((w - z) / s), 0,
+    2^bits - 1) in float64; s == 0 gives u = 0.  w_hat = s * u + z.
+    Returns (codes uint8 [rows, K], scales, zeros float64 [rows, K // block]).
+    """
+    w = np.asarray(w, dtype=np.float64)
+    rows, K = w.shape
+    assert K % block == 0
+    umax = (1 << bits) - 1
+    wb = w.reshape(rows, K // block, block)
+    lo, hi = wb.min(axis=2), wb.max(axis=2)
+    z = round_to_bf16(lo)
+    s = round_to_bf16((hi - lo) / float(umax))
+    safe = np.where(s > 0, s, 1.0)
+    q = np.round((wb - z[..., None]) / safe[..., None])   # half to even
+    q = np.where(s[..., None] > 0, q, 0.0)
+    u = np.clip(q, 0, umax).astype(np.uint8)
+    return u.reshape(rows, K), s, z
+
+
+def dequant_affine(codes, scales, zeros, block: int) -> np.ndarray:
+    """w_hat = s * u + z, exact in float64."""
+    u = np.asarray(codes, dtype=np.float64)
+    s = np.repeat(np.asarray(scales, dtype=np.float64), block, axis=1)
+    z = np.repeat(np.asarray(zeros, dtype=np.float64), block, axis=1)
+    return s * u + z
+
+
+def dequant_affine_bf16_operand(codes, scales, zeros, block: int) -> np.ndarray:
+    """bf16_rne(s * u + z): the affine weight operand of the bf16 tensor-core path."""
+    return round_to_bf16(dequant_affine(codes, scales, zeros, block))
 
 
 def quantize_ternary(w, block: int = 64):
@@ -237,8 +280,8 @@ def expert_ffn(x, w1, w2, b1=None, b2=None) -> np.ndarray:
 
 class QuantExpertBank:
     """Quantized experts, dequantized to float64 on demand (one cache entry per
-    expert).  ``fc1_q(e)`` / ``fc2_q(e)`` return (codes, scales); biases may be
-    None."""
+    expert).  ``fc1_q(e)`` / ``fc2_q(e)`` return (codes, scales), or (codes,
+    scales, zeros) for affine codes; biases may be None."""
 
     def __init__(self, H, I, E, n_shared, block, fc1_q, fc2_q, b1=None, b2=None, cache=8):
         self.H, self.I, self.E, self.n_shared, self.block = H, I, E, n_shared, block
@@ -246,14 +289,16 @@ class QuantExpertBank:
         self._cache = {}
         self._cache_max = cache
 
+    def _dq(self, q):
+        """(codes, scales): symmetric; (codes, scales, zeros): affine."""
+        return dequant(q[0], q[1], self.block) if len(q) == 2 else dequant_affine(q[0], q[1], q[2], self.block)
+
     def weights(self, e: int):
         if e not in self._cache:
             if len(self._cache) >= self._cache_max:
                 self._cache.pop(next(iter(self._cache)))
-            c1, s1 = self._fc1_q(e)
-            c2, s2 = self._fc2_q(e)
-            w1 = dequant(c1, s1, self.block)
-            w2 = dequant(c2, s2, self.block)
+            w1 = self._dq(self._fc1_q(e))
+            w2 = self._dq(self._fc2_q(e))
             b1 = None if self._b1 is None else self._b1(e)
             b2 = None if self._b2 is None else self._b2(e)
             self._cache[e] = (w1, w2, b1, b2)

@@ -219,6 +219,17 @@ def test_linear_full_size_sampled_rows(qm, fmt, M):
     _close(y[:, rows], ref, f"{fmt} M={M}")
 
 
+@pytest.mark.parametrize("fmt", ["int2", "int4"])
+@pytest.mark.parametrize("N,K,M", [(5120, 17408, 1), (5120, 17408, 6), (5120, 5120, 3)])
+def test_linear_decoder_layer_shapes_sampled_rows(qm, fmt, N, K, M):
+    """The decoder-layer shapes of the model-level sweep (down 17408 -> 5120, attention 5120 -> 5120), g128."""
+    wb, x, y, _ = _linear_case(qm, fmt, 128, N, K, M, seed=11)
+    rows = np.random.default_rng(1).choice(N, 256, replace=False)
+    codes, scales = oracle_quant(fmt, wb[rows], 128)
+    ref = Q.linear(Q.bf16_bits_to_f64(x), Q.dequant(codes, scales, 128))
+    _close(y[:, rows], ref, f"{fmt} {N}x{K} M={M}")
+
+
 # ------------------------------------------------------------------ MoE layer
 
 @pytest.mark.parametrize("T", [1, 3, 8, 13])

@@ -81,6 +81,21 @@ def test_linear_exact_rational_brute_force(bits, N, M):
             assert abs(Fraction(float(y[m, n])) - exact) <= abs(exact) * Fraction(1, 2 ** 48) + Fraction(1, 2 ** 80)
 
 
+@pytest.mark.parametrize("bits,N,M", [(2, 1, 1), (2, 4, 3), (4, 3, 2)])
+def test_linear_affine_exact_rational_brute_force(bits, N, M):
+    """K = 64, affine codes: the oracle's float64 result equals the exact
+    rational sum of (s*u + z)*x to within float64 rounding."""
+    w = _bf16((N, 64), bits * 10 + N + 5, 0.02)
+    x = _bf16((M, 64), 200 + M, 1.0)
+    codes, s, z = Q.quantize_affine(w, bits, 64)
+    y = Q.linear(x, Q.dequant_affine(codes, s, z, 64))
+    for m in range(M):
+        for n in range(N):
+            exact = sum((Fraction(int(codes[n, k])) * Fraction(float(s[n, 0])) + Fraction(float(z[n, 0])))
+                        * Fraction(float(x[m, k])) for k in range(64))
+            assert abs(Fraction(float(y[m, n])) - exact) <= abs(exact) * Fraction(1, 2 ** 48) + Fraction(1, 2 ** 80)
+
+
 def test_linear_reduces_to_integer_matmul_with_unit_scale():
     g = np.random.default_rng(4)
     c = g.integers(-8, 8, size=(6, 256))

@@ -123,6 +123,68 @@ def test_dequant_is_code_times_scale_and_bf16_operand():
     assert op[0, 0] == 7 + 2.0 ** -4                 # 7 + 7*2^-7 = 7.0546875 -> 7.0625 in bf16
 
 
+# ---------------------------------------------------------------- affine quantizer (scale and zero point)
+
+@pytest.mark.parametrize("bits", [2, 4])
+def test_affine_exact_grid_round_trips(bits):
+    """w = z0 + s0 * u0 with both code extremes in every block gives z = z0,
+    s = s0 and codes exactly u0 (all values exact in bf16)."""
+    umax = (1 << bits) - 1
+    g = np.random.default_rng(10 + bits)
+    s0, z0 = 2.0 ** -6, -0.25
+    u0 = g.integers(0, umax + 1, size=(4, 128))
+    u0[:, 0] = 0
+    u0[:, 1] = umax
+    u0[:, 64] = umax
+    u0[:, 65] = 0
+    w = z0 + s0 * u0
+    assert np.array_equal(Q.round_to_bf16(w), w)
+    codes, s, z = Q.quantize_affine(w, bits, 64)
+    assert np.all(s == s0) and np.all(z == z0)
+    assert np.array_equal(codes, u0)
+    assert np.array_equal(Q.dequant_affine(codes, s, z, 64), w)
+
+
+@pytest.mark.parametrize("bits", [2, 4])
+@pytest.mark.parametrize("block", [64, 128])
+def test_affine_codes_minimise_error_over_the_code_range(bits, block):
+    """Brute force: each code is a nearest point of {s*u + z : 0 <= u < 2^bits}."""
+    umax = (1 << bits) - 1
+    w = synth.bf16_bits_to_f32(synth.normal_bf16(5, 98, bits, (16, 256), 0.02)).astype(np.float64)
+    codes, s, z = Q.quantize_affine(w, bits, block)
+    sf, zf = np.repeat(s, block, axis=1), np.repeat(z, block, axis=1)
+    cand = np.arange(0, umax + 1, dtype=np.float64)
+    err = np.abs(w[..., None] - (cand[None, None, :] * sf[..., None] + zf[..., None]))
+    mine = np.abs(w - (codes * sf + zf))
+    assert np.all(mine <= err.min(axis=2) + 1e-18)
+    wb = w.reshape(16, 256 // block, block)
+    assert np.array_equal(z, Q.round_to_bf16(wb.min(axis=2)))
+    assert np.array_equal(s, Q.round_to_bf16((wb.max(axis=2) - wb.min(axis=2)) / umax))
+
+
+def test_affine_constant_block_ties_and_clip():
+    w = np.full((2, 64), 0.375)
+    codes, s, z = Q.quantize_affine(w, 4, 64)
+    assert np.all(s == 0) and np.all(z == 0.375) and not codes.any()
+    assert np.array_equal(Q.dequant_affine(codes, s, z, 64), w)
+    # INT2, min 0, max 3/64: s = 1/64; 0.5 s -> 0 and 1.5 s -> 2 (ties to even), 2.5 s -> 2
+    w2 = np.zeros((1, 64))
+    w2[0, :4] = np.array([0.5, 1.5, 2.5, 3.0]) / 64
+    codes2, s2, z2 = Q.quantize_affine(w2, 2, 64)
+    assert s2[0, 0] == 1 / 64 and z2[0, 0] == 0
+    assert list(codes2[0, :4]) == [0, 2, 2, 3]
+
+
+def test_affine_dequant_and_bf16_operand():
+    codes = np.array([[0, 1, 2, 3] * 16], dtype=np.uint8)
+    s, z = np.array([[0.01171875]]), np.array([[-0.0234375]])
+    wh = Q.dequant_affine(codes, s, z, 64)
+    assert np.array_equal(wh[0, :4], np.array([0, 1, 2, 3]) * 0.01171875 - 0.0234375)
+    # 15 * (1 + 2^-7) + 2^-9 needs more than 8 significant bits: the operand rounds once
+    op = Q.dequant_affine_bf16_operand(np.full((1, 64), 15), np.array([[1 + 2.0 ** -7]]), np.array([[2.0 ** -9]]), 64)
+    assert op[0, 0] == Q.round_to_bf16(15 * (1 + 2.0 ** -7) + 2.0 ** -9) == 15.125
+
+
 # ---------------------------------------------------------------- ternary quantizer
 
 def test_ternary_closed_form():
