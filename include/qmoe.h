@@ -114,15 +114,31 @@ qmoe_status qmoe_pack_size(int fmt, int rows, int K, int block,
 qmoe_status qmoe_pack(int fmt, int row_order, const uint16_t* w, int rows, int K, int block,
                       void* codes, void* scales);
 
+/* Affine (asymmetric) variant, INT2 / INT4 only: one bf16 scale s and one
+ * bf16 zero point z per block, unsigned codes u in [0, 2^bits), w_hat = s*u
+ * + z (the (scales, biases) format of the MLX issue "2-bit
+ * quantized_matmul loses its size advantage over 4-bit at M >= 3", repro).
+ * z = bf16_rne(min w), s = bf16_rne((max w - min w) / (2^bits - 1)), u =
+ * clamp(rne((w - z) / s)), all per block in float64 (s == 0 gives u = 0).
+ * The codes use the layout and bit positions of qmoe_pack (the stored field
+ * is u); zeros use the layout of the scales (sizes from qmoe_pack_size).
+ * QMOE_ERR_UNSUPPORTED for ternary. */
+qmoe_status qmoe_pack_affine(int fmt, int row_order, const uint16_t* w, int rows, int K, int block,
+                             void* codes, void* scales, void* zeros);
+
 /* Inverse of the layout (host): logical signed codes [rows, K] (int8) and
- * bf16 scales [rows, K/block].  Either output may be NULL. */
+ * bf16 scales [rows, K/block].  Either output may be NULL.  For affine codes
+ * codes_out holds u - 2^(bits-1); zeros unpack like scales (pass them as
+ * `scales`). */
 qmoe_status qmoe_unpack_host(int fmt, int row_order, const void* codes, const void* scales,
                              int rows, int K, int block, int8_t* codes_out, uint16_t* scales_out);
 
 /* One quantized weight set: n matrices of the same shape packed back to back
  * (matrix e at codes + e*codes_bytes, scales + e*scales_bytes) with the row
  * order they were packed with, optional bf16 bias [n][rows] in logical row
- * order (NULL = none).  Device pointers. */
+ * order (NULL = none), and for affine codes (qmoe_pack_affine) the zero
+ * points (NULL = symmetric codes; same layout and strides as the scales).
+ * Device pointers, 16-byte aligned. */
 typedef struct {
   int fmt;
   int block;
@@ -130,12 +146,14 @@ typedef struct {
   const void* codes;
   const void* scales;
   const uint16_t* bias;
+  const void* zeros;
 } qmoe_weights;
 
 /* Dequantize n_mats packed matrices (device): out_f32[e][rows][K] = c*s
- * (exact) and/or out_bf16 = bf16_rne(c*s), logical row order (w->row_order
- * gives the packing).  Debug and parity entry point; uses the hot kernels'
- * unpack routines. */
+ * (exact; affine: f32_rne(s*u + z)) and/or out_bf16 = bf16_rne(c*s) (affine:
+ * bf16_rne(s*u + z), one rounding), logical row order (w->row_order gives
+ * the packing).  Debug and parity entry point; uses the hot kernels' unpack
+ * routines. */
 qmoe_status qmoe_dequant(const qmoe_weights* w, int rows, int K, int n_mats, float* out_f32,
                          uint16_t* out_bf16, void* stream);
 

@@ -338,10 +338,13 @@ __global__ void combine_kernel(const float* __restrict__ yslot, const float* __r
 }
 
 // Dequantize through the hot kernels' unpack: one warp per (matrix, k-unit, tile).
+// Affine codes (zeros != NULL): w = s*u + z, fp32 by one fused multiply-add,
+// bf16 by one bf16 fused multiply-add (a single rounding of the exact value).
 template <int FMT>
 __global__ void dequant_kernel(const uint8_t* __restrict__ codes, unsigned long long cstride,
-                               const uint8_t* __restrict__ scales, unsigned long long sstride, int NT, int K,
-                               int block, int row_order, int nmat, float* o32, uint16_t* o16) {
+                               const uint8_t* __restrict__ scales, const uint8_t* __restrict__ zeros,
+                               unsigned long long sstride, int NT, int K, int block, int row_order, int nmat,
+                               float* o32, uint16_t* o16) {
   using Tr = FmtTraits<FMT>;
   __shared__ uint32_t lut[243];
   if constexpr (FMT == 3)
@@ -352,7 +355,7 @@ __global__ void dequant_kernel(const uint8_t* __restrict__ codes, unsigned long 
   const long long items = (long long)nmat * KU * NT;
   const long long wid = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const long long nwt = ((long long)gridDim.x * blockDim.x) >> 5;
-  const int bias = FMT == 3 ? 1 : (1 << (FMT - 1));
+  const int bias = FMT == 3 ? 1 : zeros ? 0 : (1 << (FMT - 1));  // code = stored field - bias
   const int rows = NT * 16;
   for (long long itm = wid; itm < items; itm += nwt) {
     const int e = (int)(itm / ((long long)KU * NT));
@@ -401,13 +404,22 @@ __global__ void dequant_kernel(const uint8_t* __restrict__ codes, unsigned long 
           const float c = (raw - 128.0f) / beta - (float)bias;
           const int pr = g + 8 * (f & 1);
           const int k = ku * Tr::kKUcols + 16 * ks + 2 * q + 8 * (f >> 1) + h;
-          const uint32_t sw = *reinterpret_cast<const uint32_t*>(sp + (((size_t)(k / block) * NT + t) * 8 + (pr & 7)) * 4);
+          const size_t so = (((size_t)(k / block) * NT + t) * 8 + (pr & 7)) * 4;
+          const uint32_t sw = *reinterpret_cast<const uint32_t*>(sp + so);
           const float s = pr < 8 ? bf16_lo(sw) : bf16_hi(sw);
           const int lr = row_order == 1 ? 16 * t + (pr < 8 ? 2 * pr : 2 * (pr - 8) + 1) : 16 * t + pr;
           const size_t o = ((size_t)e * rows + lr) * K + k;
-          const float val = c * s;
-          if (o32) o32[o] = val;
-          if (o16) o16[o] = __bfloat16_as_ushort(__float2bfloat16_rn(val));
+          if (zeros) {
+            const uint32_t zw = *reinterpret_cast<const uint32_t*>(zeros + (unsigned long long)e * sstride + so);
+            const float z = pr < 8 ? bf16_lo(zw) : bf16_hi(zw);
+            if (o32) o32[o] = fmaf(c, s, z);
+            if (o16)
+              o16[o] = __bfloat16_as_ushort(__hfma(__float2bfloat16_rn(c), __float2bfloat16_rn(s), __float2bfloat16_rn(z)));
+          } else {
+            const float val = c * s;
+            if (o32) o32[o] = val;
+            if (o16) o16[o] = __bfloat16_as_ushort(__float2bfloat16_rn(val));
+          }
         }
   }
 }

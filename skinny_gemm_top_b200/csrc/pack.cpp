@@ -53,6 +53,33 @@ size_t codes_bytes_of(int fmt, int rows, int K) {
   return (size_t)rows * K * fmt / 8;
 }
 
+// Affine: one row-block of INT codes u in [0, 2^bits) (written to c as
+// small non-negative values), returns the bf16 scale bits, *z the zero point.
+uint16_t quantize_block_affine(int fmt, const uint16_t* w, int B, int8_t* c, uint16_t* z) {
+  const int umax = (1 << fmt) - 1;
+  double lo = bf16_to_double(w[0]), hi = lo;
+  for (int i = 1; i < B; ++i) {
+    const double v = bf16_to_double(w[i]);
+    lo = std::fmin(lo, v);
+    hi = std::fmax(hi, v);
+  }
+  *z = double_to_bf16(lo);
+  const double zd = bf16_to_double(*z);
+  const uint16_t sb = double_to_bf16((hi - lo) / (double)umax);
+  const double s = bf16_to_double(sb);
+  for (int i = 0; i < B; ++i) {
+    if (s > 0) {
+      double q = std::nearbyint((bf16_to_double(w[i]) - zd) / s);
+      if (q < 0) q = 0;
+      if (q > umax) q = umax;
+      c[i] = (int8_t)q;
+    } else {
+      c[i] = 0;
+    }
+  }
+  return sb;
+}
+
 // Quantize one row-block; writes signed codes c[0..B) and returns the bf16 scale bits.
 uint16_t quantize_block(int fmt, const uint16_t* w, int B, int8_t* c) {
   if (fmt == QMOE_TERNARY) {
@@ -187,8 +214,23 @@ qmoe_status qmoe_pack_size(int fmt, int rows, int K, int block, size_t* codes_by
   return QMOE_OK;
 }
 
+static qmoe_status pack_impl(int fmt, int row_order, const uint16_t* w, int rows, int K, int block, void* codes,
+                      void* scales, void* zeros);
+
 qmoe_status qmoe_pack(int fmt, int row_order, const uint16_t* w, int rows, int K, int block,
                       void* codes, void* scales) {
+  return pack_impl(fmt, row_order, w, rows, K, block, codes, scales, nullptr);
+}
+
+qmoe_status qmoe_pack_affine(int fmt, int row_order, const uint16_t* w, int rows, int K, int block,
+                             void* codes, void* scales, void* zeros) {
+  if (fmt == QMOE_TERNARY) return QMOE_ERR_UNSUPPORTED;
+  if (!zeros) return QMOE_ERR_INVALID_ARG;
+  return pack_impl(fmt, row_order, w, rows, K, block, codes, scales, zeros);
+}
+
+static qmoe_status pack_impl(int fmt, int row_order, const uint16_t* w, int rows, int K, int block,
+                      void* codes, void* scales, void* zeros) {
   qmoe_status st = check_shape(fmt, rows, K, block);
   if (st != QMOE_OK) return st;
   if (!row_order_ok(row_order)) return QMOE_ERR_INVALID_ARG;
@@ -228,7 +270,8 @@ qmoe_status qmoe_pack(int fmt, int row_order, const uint16_t* w, int rows, int K
   }
   std::memset(codes, 0, cbytes);
   uint32_t* cw = static_cast<uint32_t*>(codes);
-  const int bias = 1 << (fmt - 1);
+  uint32_t* zc = static_cast<uint32_t*>(zeros);
+  const int bias = zeros ? 0 : 1 << (fmt - 1);  // stored field: u (affine) or c + 2^(bits-1)
   const PosTable& pt = pos_table();
   const int which = fmt == QMOE_INT2 ? 0 : 1;
   const int W = fmt == QMOE_INT2 ? 2 : 4;
@@ -238,9 +281,15 @@ qmoe_status qmoe_pack(int fmt, int row_order, const uint16_t* w, int rows, int K
     for (int tr = 0; tr < 16; ++tr) {
       const int lr = qmoe::logical_row(row_order, t, tr);
       for (int b = 0; b < SB; ++b) {
-        uint16_t s = quantize_block(fmt, w + (size_t)lr * K + (size_t)b * block, block, c.data());
+        uint16_t z = 0;
+        uint16_t s = zeros ? quantize_block_affine(fmt, w + (size_t)lr * K + (size_t)b * block, block, c.data(), &z)
+                           : quantize_block(fmt, w + (size_t)lr * K + (size_t)b * block, block, c.data());
         uint32_t& slot = sc[((size_t)b * NT + t) * 8 + (tr % 8)];
         if (tr < 8) slot = (slot & 0xFFFF0000u) | s; else slot = (slot & 0xFFFFu) | ((uint32_t)s << 16);
+        if (zeros) {
+          uint32_t& zs = zc[((size_t)b * NT + t) * 8 + (tr % 8)];
+          if (tr < 8) zs = (zs & 0xFFFF0000u) | z; else zs = (zs & 0xFFFFu) | ((uint32_t)z << 16);
+        }
         for (int i = 0; i < block; ++i) {
           const int k = b * block + i;
           const int off = pt.off[which][tr][k % 64];  // lane * W + word within the 64-column unit

@@ -65,6 +65,7 @@ struct GroupedParams {
   unsigned long long codes_stride;
   const uint8_t* scales;
   unsigned long long scales_stride;
+  const uint8_t* zeros;  // affine codes: zero points, laid out like the scales; NULL: symmetric
   int NT;       // 16-row tiles per matrix
   int K;
   int block;
@@ -102,7 +103,7 @@ __device__ __forceinline__ GSeg g_seg(const GroupedParams& p, int i) {
 template <int FMT, int BT, int CS>
 struct GGeom {
   static constexpr int kCodeBytes = 8 * FmtTraits<FMT>::kCodeBytes;  // 8 tiles of 16 rows, 64 columns
-  static constexpr int kCStage = kCodeBytes + 8 * 32;
+  static constexpr int kCStage = kCodeBytes + 2 * 8 * 32;  // codes, scales, zero points (affine)
   static constexpr int kBBytes = BT * 64 * 2;                         // token tile per k-stage
   static constexpr int kCRing = ((CS * kCStage + 127) / 128) * 128;
   static constexpr int kBars = (((2 * CS + 4 * kGStages + 5) * 8 + 16 + 127) / 128) * 128;
@@ -249,7 +250,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
         const int w_ok = lane == 0 ? (int)gwait(&empty_c[s], ph ^ 1u, p.status, abort_flag) : 0;
         if (!__shfl_sync(0xffffffffu, w_ok, 0)) { ok = false; break; }
         uint8_t* cdst = sC + s * GG::kCStage;
-        if (lane == 0) mbar_arrive_expect_tx(&full_c[s], GG::kCStage);
+        if (lane == 0) mbar_arrive_expect_tx(&full_c[s], GG::kCodeBytes + (p.zeros ? 2 : 1) * 8 * 32);
         __syncwarp();
         constexpr int kSlabs = kKS ? (FMT == 2 ? 2 : 4) : 1;  // FC2 (KSPLIT): one 8-tile copy per slab
         if (lane < kSlabs) {
@@ -263,6 +264,12 @@ __global__ void __launch_bounds__(kGThreads, 1)
           const int sb = ks * 64 / p.block;
           bulk_copy_g2s(cdst + GG::kCodeBytes, p.scales + (unsigned long long)sg.expert * p.scales_stride +
                                                    ((unsigned long long)sb * p.NT + rt * 8) * 32,
+                        8 * 32, &full_c[s]);
+        }
+        if (lane == kSlabs + 1 && p.zeros) {
+          const int sb = ks * 64 / p.block;
+          bulk_copy_g2s(cdst + GG::kCodeBytes + 8 * 32, p.zeros + (unsigned long long)sg.expert * p.scales_stride +
+                                                            ((unsigned long long)sb * p.NT + rt * 8) * 32,
                         8 * 32, &full_c[s]);
         }
       }
@@ -322,6 +329,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
   } else if (warp < 2 + kGDeqWarps) {
     // ---------------- dequantize ----------------
     const int d = warp - 2, g = lane >> 2, q = lane & 3;
+    const bool aff = p.zeros != nullptr;
     uint32_t it = 0;
     for (int u = blockIdx.x; u < n_units && !*abort_flag; u += gridDim.x) {
       for (int ks = 0; ks < KS; ++ks, ++it) {
@@ -332,7 +340,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
         if (!gwait(&full_c[sc], phc, p.status, abort_flag)) break;
         const uint8_t* cs = sC + sc * GG::kCStage;
         uint32_t am[kGDeqTiles][4][4];
-        uint32_t sw[kGDeqTiles];
+        uint32_t sw[kGDeqTiles], zw[kGDeqTiles];
 #pragma unroll
         for (int tt = 0; tt < kGDeqTiles; ++tt) {
           const int tile = kGDeqTiles * d + tt;
@@ -352,6 +360,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
             unpack_int4_word(word(3), am[tt][3]);
           }
           sw[tt] = *reinterpret_cast<const uint32_t*>(cs + GG::kCodeBytes + tile * 32 + g * 4);
+          zw[tt] = aff ? *reinterpret_cast<const uint32_t*>(cs + GG::kCodeBytes + 8 * 32 + tile * 32 + g * 4) : 0u;
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty_c[sc]);
@@ -362,17 +371,20 @@ __global__ void __launch_bounds__(kGThreads, 1)
           const int tile = kGDeqTiles * d + tt;
 #pragma unroll
           for (int f = 0; f < 4; ++f) {
-            // signed code c (exact small integer): c = (128 + beta*u) / beta - (128 / beta + bias)
+            // signed code c (exact small integer): c = (128 + beta*u) / beta - (128 / beta + bias);
+            // affine codes: u = (128 + beta*u) / beta - 128 / beta
             const uint32_t mul = (f >= 2) ? Tr::kCodeMulHi : kBf16One;
-            const uint32_t sub = (f >= 2) ? Tr::kCodeSubHi : Tr::kConstLo;
-            // the row's bf16 scale in both halves, straight from its bits (no fp32 round trip)
+            const uint32_t sub = aff ? ((f >= 2) ? aff_sub_hi<FMT>() : kAffConst)
+                                     : ((f >= 2) ? Tr::kCodeSubHi : Tr::kConstLo);
+            // the row's bf16 scale (and zero point) in both halves, straight from its bits (no fp32 round trip)
             const uint32_t sp = __byte_perm(sw[tt], 0u, (f & 1) ? 0x3232u : 0x1010u);
+            const uint32_t zp = aff ? __byte_perm(zw[tt], 0u, (f & 1) ? 0x3232u : 0x1010u) : kBf16NegZero;
             const int pr = tile * 16 + g + 8 * (f & 1);
             uint8_t* rowp = as + (pr >> 3) * 1024 + (pr & 7) * 128;
 #pragma unroll
             for (int k2 = 0; k2 < 4; ++k2) {
               const uint32_t c = fma_bf16x2(am[tt][k2][f], mul, sub);
-              const uint32_t wv = fma_bf16x2(c, sp, kBf16NegZero);  // bf16_rne(c * s): one rounding
+              const uint32_t wv = fma_bf16x2(c, sp, zp);  // bf16_rne(c * s) or bf16_rne(s * u + z): one rounding
               const int chunk = 2 * k2 + (f >> 1);
               *reinterpret_cast<uint32_t*>(rowp + ((chunk ^ (pr & 7)) << 4) + 4 * q) = wv;
             }

@@ -134,6 +134,10 @@ qmoe_status check_weights(const qmoe_weights& w, int rows, int K) {
   if (rows % 16 || K % 64 || K % w.block) return QMOE_ERR_INVALID_ARG;
   if (w.fmt == QMOE_TERNARY && (w.block != 64 || K % 128)) return QMOE_ERR_UNSUPPORTED;
   if ((reinterpret_cast<uintptr_t>(w.codes) | reinterpret_cast<uintptr_t>(w.scales)) & 15) return QMOE_ERR_INVALID_ARG;
+  if (w.zeros) {  // affine codes: INT2 / INT4 only
+    if (w.fmt == QMOE_TERNARY) return QMOE_ERR_UNSUPPORTED;
+    if (reinterpret_cast<uintptr_t>(w.zeros) & 15) return QMOE_ERR_INVALID_ARG;
+  }
   return QMOE_OK;
 }
 
@@ -153,10 +157,15 @@ bool grouped_eligible(const qmoe_layer& L) {
   return L.fc1.fmt != QMOE_TERNARY && L.fc2.fmt != QMOE_TERNARY && (2 * L.I) % kGRows == 0 && L.H % kGRows == 0;
 }
 
+// Affine codes (zero points): the decode kernel and the grouped (tcgen05)
+// kernel take them; the small-M expert kernel does not, so outside the decode
+// kernel every expert of an affine layer runs on the grouped path.
+bool affine(const qmoe_layer& L) { return L.fc1.zeros || L.fc2.zeros; }
+
 // Token-count threshold above which an expert runs on the grouped path.
 int grouped_threshold(const qmoe_layer& L) {
   if (L.path == QMOE_PATH_SMALL_M || !grouped_eligible(L)) return INT_MAX;
-  return L.path == QMOE_PATH_GROUPED ? 0 : kGroupedThreshold;
+  return L.path == QMOE_PATH_GROUPED || affine(L) ? 0 : kGroupedThreshold;
 }
 
 // Fault injection for tests (qmoe_test_set_fault): the decode kernel's wait
@@ -169,6 +178,7 @@ int g_fault_inject = 0;
 // prologue (after a tiny reset launch of its accumulator).
 bool decode_eligible(const qmoe_layer& L, int T, int grid, SlicePlan* plan) {
   if (T > kDecMaxT || T * L.k > kDecMaxTK || L.path == QMOE_PATH_GROUPED || L.H > kSMaxH) return false;
+  if (affine(L)) return false;  // the decode kernel takes symmetric codes (for now)
   const SlicePlan pl = slice_plan(L.fc1.fmt, L.fc2.fmt, T, L.H);
   if (!pl.ok || L.I % pl.gran_cols) return false;
   const int gpe = L.I / pl.gran_cols;
@@ -323,6 +333,7 @@ GroupedParams grouped_params(const qmoe_weights& w, int rows, int K, unsigned* s
   p.codes_stride = codes_bytes(w.fmt, rows, K);
   p.scales = static_cast<const uint8_t*>(w.scales);
   p.scales_stride = scales_bytes(rows, K, w.block);
+  p.zeros = static_cast<const uint8_t*>(w.zeros);
   p.NT = rows / 16;
   p.K = K;
   p.block = w.block;
@@ -355,7 +366,10 @@ qmoe_status check_layer(const qmoe_layer* L) {
   if (L->fc1.row_order != QMOE_ROWS_GATE_UP || L->fc2.row_order != QMOE_ROWS_KSPLIT) return QMOE_ERR_INVALID_ARG;
   qmoe_status s = check_weights(L->fc1, 2 * L->I, L->H);
   if (s != QMOE_OK) return s;
-  return check_weights(L->fc2, L->H, L->I);
+  s = check_weights(L->fc2, L->H, L->I);
+  if (s != QMOE_OK) return s;
+  if (affine(*L) && (L->path == QMOE_PATH_SMALL_M || !grouped_eligible(*L))) return QMOE_ERR_UNSUPPORTED;
+  return QMOE_OK;
 }
 
 }  // namespace
@@ -716,7 +730,9 @@ qmoe_status qmoe_linear(const qmoe_weights* w, int N, int K, const uint16_t* x, 
   // More than one token group: the tcgen05 path, whose cost barely depends on
   // M (the dequantized tile serves up to 256 tokens; the small-M kernel's
   // mma.sync work grows with every group of 8 tokens).
-  const bool grouped = M >= kLinearGroupedMinM && N % kGRows == 0 && w->fmt != QMOE_TERNARY;
+  // Affine codes: the tcgen05 path at every M (the small-M kernel takes symmetric codes only).
+  const bool grouped = (M >= kLinearGroupedMinM || w->zeros) && N % kGRows == 0 && w->fmt != QMOE_TERNARY;
+  if (w->zeros && !grouped) return QMOE_ERR_UNSUPPORTED;
   if (grouped) {
     CUtensorMap map;
     s = encode_rows_map(&map, x, K, M);
@@ -750,15 +766,19 @@ qmoe_status qmoe_dequant(const qmoe_weights* w, int rows, int K, int n_mats, flo
   const unsigned long long cs = codes_bytes(w->fmt, rows, K), ss = scales_bytes(rows, K, w->block);
   const uint8_t* c = static_cast<const uint8_t*>(w->codes);
   const uint8_t* sc = static_cast<const uint8_t*>(w->scales);
+  const uint8_t* zc = static_cast<const uint8_t*>(w->zeros);
   const long long items = (long long)n_mats * (K / ku_cols(w->fmt)) * (rows / 16);
   const int grid = (int)std::min<long long>((items + 7) / 8, 65535);
   TraceScope ts(st, K_DEQUANT);
   if (w->fmt == QMOE_INT2)
-    dequant_kernel<2><<<grid, 256, 0, st>>>(c, cs, sc, ss, rows / 16, K, w->block, row_order, n_mats, out_f32, out_bf16);
+    dequant_kernel<2><<<grid, 256, 0, st>>>(c, cs, sc, zc, ss, rows / 16, K, w->block, row_order, n_mats, out_f32,
+                                            out_bf16);
   else if (w->fmt == QMOE_INT4)
-    dequant_kernel<4><<<grid, 256, 0, st>>>(c, cs, sc, ss, rows / 16, K, w->block, row_order, n_mats, out_f32, out_bf16);
+    dequant_kernel<4><<<grid, 256, 0, st>>>(c, cs, sc, zc, ss, rows / 16, K, w->block, row_order, n_mats, out_f32,
+                                            out_bf16);
   else
-    dequant_kernel<3><<<grid, 256, 0, st>>>(c, cs, sc, ss, rows / 16, K, w->block, row_order, n_mats, out_f32, out_bf16);
+    dequant_kernel<3><<<grid, 256, 0, st>>>(c, cs, sc, nullptr, ss, rows / 16, K, w->block, row_order, n_mats,
+                                            out_f32, out_bf16);
   return cudaGetLastError() == cudaSuccess ? QMOE_OK : QMOE_ERR_CUDA;
 }
 

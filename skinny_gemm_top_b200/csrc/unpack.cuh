@@ -51,6 +51,22 @@ template <> struct FmtTraits<3> {             // ternary: t in {-1,0,1}, digit d
   static constexpr uint32_t kCodeSubHi = 0xC204C204u;  // -(32 + 1) = -33
 };
 
+// Affine codes (zero point per block): the stored field is u itself, so the
+// constant parts to remove are 128 (lo columns) and 128 / beta (hi columns
+// after the 1/beta multiplier); as a constant MMA operand on beta-divided
+// activations both read -128.
+constexpr uint32_t kAffConst = 0xC300C300u;  // -128
+template <int FMT>
+__host__ __device__ constexpr uint32_t aff_sub_hi() {
+  return FmtTraits<FMT>::kBetaHi == 4 ? 0xC200C200u /* -32 */ : 0xC300C300u /* -128 */;
+}
+// Sum of the activations from the beta-divided ones: a constant operand of 1
+// (lo columns) and beta (hi columns).
+template <int FMT>
+__host__ __device__ constexpr uint32_t sum_const_hi() {
+  return FmtTraits<FMT>::kBetaHi == 4 ? 0x40804080u /* 4 */ : kBf16One;
+}
+
 // INT2: one lane word (16 codes) -> A registers of two consecutive k-steps.
 __device__ __forceinline__ void unpack_int2_word(uint32_t w, uint32_t (&a0)[4], uint32_t (&a1)[4]) {
   const uint32_t v1 = w >> 6, v2 = w >> 12;

@@ -30,7 +30,7 @@ class QmoeError(RuntimeError):
 
 class Weights(C.Structure):
     _fields_ = [("fmt", C.c_int), ("block", C.c_int), ("row_order", C.c_int), ("codes", C.c_void_p),
-                ("scales", C.c_void_p), ("bias", C.c_void_p)]
+                ("scales", C.c_void_p), ("bias", C.c_void_p), ("zeros", C.c_void_p)]
 
 
 class Layer(C.Structure):
@@ -46,6 +46,8 @@ class Stats(C.Structure):
 EXPORTS = {
     "qmoe_pack_size": [C.c_int, C.c_int, C.c_int, C.c_int, C.POINTER(C.c_size_t), C.POINTER(C.c_size_t)],
     "qmoe_pack": [C.c_int, C.c_int, C.c_void_p, C.c_int, C.c_int, C.c_int, C.c_void_p, C.c_void_p],
+    "qmoe_pack_affine": [C.c_int, C.c_int, C.c_void_p, C.c_int, C.c_int, C.c_int, C.c_void_p, C.c_void_p,
+                         C.c_void_p],
     "qmoe_unpack_host": [C.c_int, C.c_int, C.c_void_p, C.c_void_p, C.c_int, C.c_int, C.c_int, C.c_void_p,
                          C.c_void_p],
     "qmoe_dequant": [C.POINTER(Weights), C.c_int, C.c_int, C.c_int, C.c_void_p, C.c_void_p, C.c_void_p],
@@ -129,6 +131,30 @@ def pack(fmt: int, row_order: int, w_bits: np.ndarray, block: int):
     return codes, scales
 
 
+def pack_affine(fmt: int, row_order: int, w_bits: np.ndarray, block: int):
+    """Affine quantize + pack one bf16 matrix -> (codes u8, scales u8, zeros u8)."""
+    w = np.ascontiguousarray(w_bits, dtype=np.uint16)
+    rows, K = w.shape
+    cb, sb = pack_size(fmt, rows, K, block)
+    codes = np.empty(cb, dtype=np.uint8)
+    scales = np.empty(sb, dtype=np.uint8)
+    zeros = np.empty(sb, dtype=np.uint8)
+    _check(_lib.qmoe_pack_affine(fmt, row_order, _ptr(w), rows, K, block, _ptr(codes), _ptr(scales), _ptr(zeros)),
+           "qmoe_pack_affine")
+    return codes, scales, zeros
+
+
+def pack_stack_affine(fmt: int, row_order: int, mats, block: int):
+    """pack_affine for matrices back to back."""
+    cs, ss, zs = [], [], []
+    for m in mats:
+        c, s, z = pack_affine(fmt, row_order, m, block)
+        cs.append(c)
+        ss.append(s)
+        zs.append(z)
+    return np.concatenate(cs), np.concatenate(ss), np.concatenate(zs)
+
+
 def pack_stack(fmt: int, row_order: int, mats, block: int):
     """Pack matrices back to back (matrix e at e * codes_bytes)."""
     cs, ss = [], []
@@ -150,10 +176,11 @@ def unpack_host(fmt: int, row_order: int, codes: np.ndarray, scales: np.ndarray,
 
 # ---------------------------------------------------------------- device entry points
 
-def make_weights(fmt: int, block: int, codes, scales, bias=None, row_order: int = ROWS_PLAIN) -> Weights:
+def make_weights(fmt: int, block: int, codes, scales, bias=None, row_order: int = ROWS_PLAIN, zeros=None) -> Weights:
     """Device weight set; row_order is the one the codes were packed with
-    (GATE_UP for a layer's FC1, KSPLIT for its FC2, PLAIN for a single linear)."""
-    return Weights(fmt, block, row_order, _ptr(codes), _ptr(scales), _ptr(bias))
+    (GATE_UP for a layer's FC1, KSPLIT for its FC2, PLAIN for a single linear);
+    zeros for affine codes (pack_affine)."""
+    return Weights(fmt, block, row_order, _ptr(codes), _ptr(scales), _ptr(bias), _ptr(zeros))
 
 
 def make_layer(H, I, E, k, n_shared, fc1: Weights, fc2: Weights, path=PATH_AUTO, max_row_tile=0) -> Layer:

@@ -48,28 +48,46 @@ def oracle_quant(fmt: str, w_bits: np.ndarray, block: int):
     return Q.quantize_sym(w, FMTS[fmt], block)
 
 
+def oracle_quant_affine(fmt: str, w_bits: np.ndarray, block: int):
+    return Q.quantize_affine(Q.bf16_bits_to_f64(w_bits), FMTS[fmt], block)
+
+
 class MoECase:
     """A MoE layer: packed on the device for the library, quantized lazily by
     the oracle for reference values."""
 
-    def __init__(self, cfg: synth.MoEConfig, seed: int = 1):
+    def __init__(self, cfg: synth.MoEConfig, seed: int = 1, affine: bool = False):
         from skinny_gemm_top_b200 import qmoe
         self.cfg, self.seed = cfg, seed
         n = cfg.E + cfg.n_shared
         f1, f2 = FMTS[cfg.fc1_fmt], FMTS[cfg.fc2_fmt]
-        c1, s1 = qmoe.pack_stack(f1, qmoe.ROWS_GATE_UP, (synth.expert_fc1(cfg, seed, e) for e in range(n)), cfg.block)
-        c2, s2 = qmoe.pack_stack(f2, qmoe.ROWS_KSPLIT, (synth.expert_fc2(cfg, seed, e) for e in range(n)), cfg.block)
+        z1 = z2 = None
+        if affine:  # scale and zero point per block (INT2 / INT4)
+            c1, s1, z1 = qmoe.pack_stack_affine(f1, qmoe.ROWS_GATE_UP,
+                                                (synth.expert_fc1(cfg, seed, e) for e in range(n)), cfg.block)
+            c2, s2, z2 = qmoe.pack_stack_affine(f2, qmoe.ROWS_KSPLIT,
+                                                (synth.expert_fc2(cfg, seed, e) for e in range(n)), cfg.block)
+        else:
+            c1, s1 = qmoe.pack_stack(f1, qmoe.ROWS_GATE_UP, (synth.expert_fc1(cfg, seed, e) for e in range(n)),
+                                     cfg.block)
+            c2, s2 = qmoe.pack_stack(f2, qmoe.ROWS_KSPLIT, (synth.expert_fc2(cfg, seed, e) for e in range(n)),
+                                     cfg.block)
         self.dev = {"c1": to_dev(c1), "s1": to_dev(s1), "c2": to_dev(c2), "s2": to_dev(s2)}
+        if affine:
+            self.dev["z1"], self.dev["z2"] = to_dev(z1), to_dev(z2)
         self.b1 = self.b2 = None
         if cfg.bias:
             self.dev["b1"] = to_dev(np.stack([synth.expert_b1(cfg, seed, e) for e in range(n)]))
             self.dev["b2"] = to_dev(np.stack([synth.expert_b2(cfg, seed, e) for e in range(n)]))
-        self.w1 = qmoe.make_weights(f1, cfg.block, self.dev["c1"], self.dev["s1"], self.dev.get("b1"), qmoe.ROWS_GATE_UP)
-        self.w2 = qmoe.make_weights(f2, cfg.block, self.dev["c2"], self.dev["s2"], self.dev.get("b2"), qmoe.ROWS_KSPLIT)
+        self.w1 = qmoe.make_weights(f1, cfg.block, self.dev["c1"], self.dev["s1"], self.dev.get("b1"), qmoe.ROWS_GATE_UP,
+                                    self.dev.get("z1"))
+        self.w2 = qmoe.make_weights(f2, cfg.block, self.dev["c2"], self.dev["s2"], self.dev.get("b2"), qmoe.ROWS_KSPLIT,
+                                    self.dev.get("z2"))
+        quant = oracle_quant_affine if affine else oracle_quant
         self.bank = Q.QuantExpertBank(
             cfg.H, cfg.I, cfg.E, cfg.n_shared, cfg.block,
-            lambda e: oracle_quant(cfg.fc1_fmt, synth.expert_fc1(cfg, seed, e), cfg.block),
-            lambda e: oracle_quant(cfg.fc2_fmt, synth.expert_fc2(cfg, seed, e), cfg.block),
+            lambda e: quant(cfg.fc1_fmt, synth.expert_fc1(cfg, seed, e), cfg.block),
+            lambda e: quant(cfg.fc2_fmt, synth.expert_fc2(cfg, seed, e), cfg.block),
             (lambda e: Q.bf16_bits_to_f64(synth.expert_b1(cfg, seed, e))) if cfg.bias else None,
             (lambda e: Q.bf16_bits_to_f64(synth.expert_b2(cfg, seed, e))) if cfg.bias else None,
             cache=16)

@@ -56,6 +56,29 @@ def test_pack_matches_oracle_quantizer(fmt, block, order):
     assert np.array_equal(Q.bf16_bits_to_f64(s), os_)
 
 
+@pytest.mark.parametrize("fmt,block,order", [
+    (qmoe.INT2, 64, qmoe.ROWS_GATE_UP), (qmoe.INT4, 64, qmoe.ROWS_PLAIN), (qmoe.INT2, 128, qmoe.ROWS_PLAIN),
+    (qmoe.INT4, 128, qmoe.ROWS_KSPLIT), (qmoe.INT2, 64, qmoe.ROWS_KSPLIT)])
+def test_pack_affine_matches_oracle_quantizer(fmt, block, order):
+    rows, K = 48, 256
+    w = synth.normal_bf16(9, 51, fmt * 10 + block, (rows, K), 0.02)
+    codes, scales, zeros = qmoe.pack_affine(fmt, order, w, block)
+    cb, sb = qmoe.pack_size(fmt, rows, K, block)
+    assert codes.nbytes == cb and scales.nbytes == sb and zeros.nbytes == sb
+    c, s = qmoe.unpack_host(fmt, order, codes, scales, rows, K, block)
+    _, z = qmoe.unpack_host(fmt, order, codes, zeros, rows, K, block)
+    ou, os_, oz = Q.quantize_affine(Q.bf16_bits_to_f64(w), fmt, block)
+    assert np.array_equal(c.astype(np.int64) + (1 << (fmt - 1)), ou.astype(np.int64))
+    assert np.array_equal(Q.bf16_bits_to_f64(s), os_)
+    assert np.array_equal(Q.bf16_bits_to_f64(z), oz)
+
+
+def test_pack_affine_rejects_ternary():
+    w = synth.normal_bf16(9, 52, 0, (16, 128), 0.02)
+    with pytest.raises(qmoe.QmoeError):
+        qmoe.pack_affine(qmoe.TERNARY, qmoe.ROWS_PLAIN, w, 64)
+
+
 @pytest.mark.parametrize("fmt,block", [(qmoe.INT2, 64), (qmoe.INT4, 128), (qmoe.TERNARY, 64)])
 def test_pack_matches_oracle_quantizer_tiny_and_subnormal(fmt, block):
     """Blocks scaled down to tiny normal and subnormal bf16 values: both

@@ -9,6 +9,7 @@ from oracle import qmoe_oracle as Q
 from skinny_gemm_top_b200 import synth
 
 from cases import (FMTS, MAX_ERR_RMS, REL_L2, TINY_FACTORS, MoECase, bf16_dev_to_f64, block_scaled_weights,
+                   oracle_quant_affine,
                    oracle_quant, small_cfg, to_dev)
 
 pytestmark = pytest.mark.gpu
@@ -89,6 +90,104 @@ def test_grouped_operand_bit_exact_one_hot(qm, fmt, block, tiny):
         assert np.any((scales > 0) & (scales < 2.0 ** -126)), "no subnormal scale drawn"
     op = Q.dequant_bf16_operand(codes, scales, block)   # [N, K]
     assert np.array_equal(got, op[:, km].T)
+
+
+# ------------------------------------------------------------------ affine codes (scale and zero point)
+
+@pytest.mark.parametrize("fmt,block,order,tiny", [
+    ("int2", 64, 1, False), ("int4", 128, 0, False), ("int4", 64, 2, False), ("int2", 128, 2, False),
+    ("int2", 64, 0, True), ("int4", 128, 0, True)])
+def test_dequant_affine_bit_exact(qm, fmt, block, order, tiny):
+    """fp32: f32_rne(s*u + z); bf16: bf16_rne(s*u + z), one rounding each."""
+    import torch
+    rows, K, n = 48, 384 if not tiny else 896, 2
+    if tiny:
+        mats = [block_scaled_weights(41 + i, rows, K, block, TINY_FACTORS) for i in range(n)]
+    else:
+        mats = [synth.normal_bf16(41, 61, i, (rows, K), 0.02) for i in range(n)]
+    c, s, z = qm.pack_stack_affine(FMTS[fmt], order, mats, block)
+    keep = [to_dev(a) for a in (c, s, z)]  # the weight set holds raw pointers
+    w = qm.make_weights(FMTS[fmt], block, keep[0], keep[1], None, order, keep[2])
+    o32 = torch.empty((n, rows, K), dtype=torch.float32, device="cuda")
+    o16 = torch.empty((n, rows, K), dtype=torch.int16, device="cuda")
+    qm.dequant(w, rows, K, n, o32, o16)
+    torch.cuda.synchronize()
+    for i in range(n):
+        codes, scales, zeros = oracle_quant_affine(fmt, mats[i], block)
+        if tiny:
+            assert np.any((scales > 0) & (scales < 2.0 ** -126)), "no subnormal scale drawn"
+        exact = Q.dequant_affine(codes, scales, zeros, block)
+        assert np.array_equal(o32[i].cpu().numpy(), exact.astype(np.float32))
+        ref16 = Q.dequant_affine_bf16_operand(codes, scales, zeros, block)
+        assert np.array_equal(Q.bf16_bits_to_f64(o16[i].cpu().numpy().view(np.uint16)), ref16)
+
+
+@pytest.mark.parametrize("fmt,block,tiny", [("int2", 64, False), ("int4", 128, False), ("int4", 64, True)])
+def test_grouped_operand_affine_bit_exact_one_hot(qm, fmt, block, tiny):
+    """The tcgen05 path's affine operand bf16_rne(s*u + z) through qmoe_linear
+    (one-hot token rows as in the symmetric test above)."""
+    import torch
+    N, K, M = 256, 1024, 128
+    wb = block_scaled_weights(33, N, K, block, TINY_FACTORS) if tiny else synth.linear_weight(33, N, K)
+    c, s, z = qm.pack_affine(FMTS[fmt], 0, wb, block)
+    keep = [to_dev(a) for a in (c, s, z)]
+    w = qm.make_weights(FMTS[fmt], block, keep[0], keep[1], None, 0, keep[2])
+    km = (np.arange(M) * 37 + 5) % K
+    x = np.zeros((M, K), dtype=np.uint16)
+    x[np.arange(M), km] = synth.f32_to_bf16_bits(np.float32(2.0 ** 64))
+    y = torch.empty((M, N), dtype=torch.int16, device="cuda")
+    ws = torch.empty(qm.linear_workspace_size(N, K, M), dtype=torch.uint8, device="cuda")
+    qm.linear(w, N, K, to_dev(x), y, ws)
+    torch.cuda.synchronize()
+    assert qm.get_stats().last_path == qm.PATH_GROUPED
+    got = bf16_dev_to_f64(y) * 2.0 ** -64
+    codes, scales, zeros = oracle_quant_affine(fmt, wb, block)
+    op = Q.dequant_affine_bf16_operand(codes, scales, zeros, block)
+    assert np.array_equal(got, op[:, km].T)
+
+
+@pytest.mark.parametrize("fmt,block", [("int2", 128), ("int4", 128), ("int4", 64)])
+@pytest.mark.parametrize("M", [1, 5, 8, 32])
+def test_linear_affine(qm, fmt, block, M):
+    import torch
+    N, K = 384, 1024
+    wb = synth.linear_weight(50 + M, N, K)
+    c, s, z = qm.pack_affine(FMTS[fmt], 0, wb, block)
+    keep = [to_dev(a) for a in (c, s, z)]
+    w = qm.make_weights(FMTS[fmt], block, keep[0], keep[1], None, 0, keep[2])
+    x = synth.tokens(K, 50 + M, M)
+    y = torch.empty((M, N), dtype=torch.int16, device="cuda")
+    ws = torch.empty(qm.linear_workspace_size(N, K, M), dtype=torch.uint8, device="cuda")
+    qm.linear(w, N, K, to_dev(x), y, ws)
+    torch.cuda.synchronize()
+    codes, scales, zeros = oracle_quant_affine(fmt, wb, block)
+    ref = Q.linear(Q.bf16_bits_to_f64(x), Q.dequant_affine(codes, scales, zeros, block))
+    _close(bf16_dev_to_f64(y), ref, f"affine {fmt} g{block} M={M}")
+
+
+@pytest.mark.parametrize("T", [1, 3, 8, 13, 40])
+def test_forward_affine_layer(qm, T):
+    """A MoE layer with affine codes (tiny shapes, INT2 FC1 / INT4 FC2, plus a shared expert and biases)."""
+    cfg = small_cfg(synth.TINY, n_shared=1, bias=True)
+    case = MoECase(cfg, seed=7, affine=True)
+    x = synth.tokens(cfg.H, 7, T)
+    lg = synth.router_logits(cfg, 7, T)
+    y = case.run(x, lg)
+    ref = Q.moe_forward(Q.bf16_bits_to_f64(x), lg, cfg.k, case.bank)
+    _close(y, ref, f"affine layer T={T}")
+
+
+def test_affine_rejected_where_unsupported(qm):
+    import torch
+    cfg = synth.TINY
+    case = MoECase(cfg, seed=7, affine=True)
+    layer = case.layer(path=qm.PATH_SMALL_M)
+    ws = torch.empty(1 << 20, dtype=torch.uint8, device="cuda")
+    x = to_dev(synth.tokens(cfg.H, 7, 2))
+    lg = torch.from_numpy(np.ascontiguousarray(synth.router_logits(cfg, 7, 2))).cuda()
+    y = torch.empty((2, cfg.H), dtype=torch.int16, device="cuda")
+    with pytest.raises(qm.QmoeError):
+        qm.forward(layer, x, lg, y, ws)
 
 
 # ------------------------------------------------------------------ routing
