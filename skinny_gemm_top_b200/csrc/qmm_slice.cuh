@@ -86,7 +86,8 @@ struct SliceSmemLayout {
   static constexpr int kChunks = kWmat + kDecMaxTK * 8 * 4;            // [kSMaxChunks] SChunk
   static constexpr int kLut = kChunks + kSMaxChunks * (int)sizeof(SChunk);  // 243 u32 (ternary)
   static constexpr int kCorr = kLut + 1024;                             // [kSMaxH / 64][8] f32
-  static constexpr int kH = kCorr + round128c((kSMaxH / 64) * 8 * 4);   // [kSHWin][32] uint2
+  static constexpr int kSx = kCorr + round128c((kSMaxH / 64) * 8 * 4);  // [kSMaxH / 64][8] f32 (affine codes)
+  static constexpr int kH = kSx + round128c((kSMaxH / 64) * 8 * 4);     // [kSHWin][32] uint2
   static constexpr int kRed = kH + kSHWin * 32 * 8;                     // [kSW][kSRed][32] float4
   static constexpr int kFixed = kRed + kSW * kSRed * 32 * 16;           // x rows start here
 };
@@ -171,10 +172,13 @@ __device__ __forceinline__ bool slice_fix(SIt& it, const SChunk* tab, int nch, i
 // buffer), accumulated into acc1.  B fragments come from the x rows in shared
 // memory (columns k % 16 >= 8 already divided by the code multiplier); the
 // constant-operand correction of each 64-column block is the precomputed
-// corr1.  Tiles go four at a time so that their MMA chains overlap.
+// corr1.  Tiles go four at a time so that their MMA chains overlap.  Affine
+// codes (aff): the zero points follow the scales in the buffer, and each
+// block adds z * (sum of its activations), sx1.
 template <int F1, int MT>
 __device__ __forceinline__ void slice_fc1(const uint8_t* st, int nt, int ku, const uint8_t* xrow, const float* corr1,
-                                          const uint32_t* lut, int lane, float (&acc1)[MT][4]) {
+                                          const float* sx1, bool aff, const uint32_t* lut, int lane,
+                                          float (&acc1)[MT][4]) {
   using T1 = FmtTraits<F1>;
   constexpr int BPK = T1::kKUcols / 64;
   const int g = lane >> 2, n0 = 2 * (lane & 3);
@@ -257,6 +261,20 @@ __device__ __forceinline__ void slice_fc1(const uint8_t* st, int nt, int ku, con
             mma_bf16_16816(tmp[i], a, bfr[0][w][0], bfr[0][w][1]);
           }
       }
+      if (aff) {  // z * (sum of the block's activations), per row and token
+        const float sxa = sx1[ku * 8 + n0], sxb = sx1[ku * 8 + n0 + 1];
+        const uint8_t* zeros = scales + nt * 32;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          if (i0 + i >= MT || i0 + i >= nt) break;
+          const uint32_t zc = *reinterpret_cast<const uint32_t*>(zeros + (i0 + i) * 32 + g * 4);
+          const float zlo = bf16_lo(zc), zhi = bf16_hi(zc);
+          acc1[i0 + i][0] = fmaf(zlo, sxa, acc1[i0 + i][0]);
+          acc1[i0 + i][1] = fmaf(zlo, sxb, acc1[i0 + i][1]);
+          acc1[i0 + i][2] = fmaf(zhi, sxa, acc1[i0 + i][2]);
+          acc1[i0 + i][3] = fmaf(zhi, sxb, acc1[i0 + i][3]);
+        }
+      }
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         if (i0 + i >= MT || i0 + i >= nt) break;
@@ -274,13 +292,17 @@ __device__ __forceinline__ void slice_fc1(const uint8_t* st, int nt, int ku, con
 // FC2 item: ng granules of this warp's nr row tiles, accumulated into acc2.
 // B fragments are the h window's k-steps from window granule wg0 on.
 template <int F2>
-__device__ __forceinline__ void slice_fc2(const uint8_t* st, int ng, int nr, int wg0, int g_abs, const uint2* hfrag,
-                                          const uint32_t* lut, int lane, float (&acc2)[kSRT][4]) {
+__device__ __forceinline__ void slice_fc2(const uint8_t* st, int ng, int nr, int wg0, int g_abs, bool aff,
+                                          const uint2* hfrag, const uint32_t* lut, int lane,
+                                          float (&acc2)[kSRT][4]) {
   using K2 = KsTr<F2>;
   using Tr2 = FmtTraits<F2>;
   const int g = lane >> 2;
-  const uint32_t aconst[4] = {Tr2::kConstLo, Tr2::kConstLo, Tr2::kConstHi, Tr2::kConstHi};
+  const uint32_t aconst[4] = {aff ? kAffConst : Tr2::kConstLo, aff ? kAffConst : Tr2::kConstLo,
+                              aff ? kAffConst : Tr2::kConstHi, aff ? kAffConst : Tr2::kConstHi};
   const uint32_t* sbuf = reinterpret_cast<const uint32_t*>(st + ng * nr * K2::kRowBytes);
+  // affine codes: zero points after the scales
+  const uint32_t* zbuf = sbuf + ng * K2::kBlocks * nr * 8;
   for (int gi = 0; gi < ng; ++gi) {
     uint2 b[K2::kKsteps];
 #pragma unroll
@@ -293,6 +315,14 @@ __device__ __forceinline__ void slice_fc2(const uint8_t* st, int ng, int nr, int
       for (int s = 0; s < K2::kKsteps / K2::kBlocks; ++s) {
         const uint2 bb = b[bl * (K2::kKsteps / K2::kBlocks) + s];
         mma_bf16_16816(cr[bl], aconst, bb.x, bb.y);
+      }
+    }
+    float sx[4] = {0.f, 0.f, 0.f, 0.f};  // affine: the granule's sum of h per token
+    if constexpr (F2 != 3) {
+      if (aff) {
+        const uint32_t asum[4] = {kBf16One, kBf16One, sum_const_hi<F2>(), sum_const_hi<F2>()};
+#pragma unroll
+        for (int s = 0; s < K2::kKsteps; ++s) mma_bf16_16816(sx, asum, b[s].x, b[s].y);
       }
     }
     const uint8_t* cbase = st + gi * nr * K2::kRowBytes;
@@ -329,6 +359,14 @@ __device__ __forceinline__ void slice_fc2(const uint8_t* st, int ng, int nr, int
           uint32_t a[4];
           unpack_int4_word(w, a);
           mma_bf16_16816(tmp, a, b[0].x, b[0].y);
+        }
+        if (aff) {
+          const uint32_t zc = zbuf[(gi * nr + i) * 8 + g];
+          const float zlo = bf16_lo(zc), zhi = bf16_hi(zc);
+          acc2[i][0] = fmaf(zlo, sx[0], acc2[i][0]);
+          acc2[i][1] = fmaf(zlo, sx[1], acc2[i][1]);
+          acc2[i][2] = fmaf(zhi, sx[2], acc2[i][2]);
+          acc2[i][3] = fmaf(zhi, sx[3], acc2[i][3]);
         }
         const uint32_t sc = sbuf[(gi * nr + i) * 8 + g];
         const float slo = bf16_lo(sc), shi = bf16_hi(sc);
@@ -374,7 +412,7 @@ __device__ void slice_partition(SChunk* tab, int* n, int c, int G, int nslots, i
   }
 }
 
-template <int F1, int F2>
+template <int F1, int F2, bool AFF>
 __global__ void __launch_bounds__(kSThreads, 1) qmm_slice_kernel(const SliceParams p) {
   using T1 = FmtTraits<F1>;
   using K2 = KsTr<F2>;
@@ -392,6 +430,8 @@ __global__ void __launch_bounds__(kSThreads, 1) qmm_slice_kernel(const SlicePara
   SChunk* tab = reinterpret_cast<SChunk*>(smem + L::kChunks);
   uint32_t* lut = reinterpret_cast<uint32_t*>(smem + L::kLut);
   float* corr1 = reinterpret_cast<float*>(smem + L::kCorr);
+  float* sx1 = reinterpret_cast<float*>(smem + L::kSx);
+  constexpr bool aff = AFF;  // affine codes (zero points): a separate instantiation
   uint2* hfrag = reinterpret_cast<uint2*>(smem + L::kH);
   uint16_t* hbits = reinterpret_cast<uint16_t*>(smem + L::kH);
   float4* red = reinterpret_cast<float4*>(smem + L::kRed);
@@ -448,8 +488,9 @@ __global__ void __launch_bounds__(kSThreads, 1) qmm_slice_kernel(const SlicePara
       __syncwarp();
       const SChunk& C = tab[prod.c];
       const int ngi = min(p.ngm, C.ngc - prod.a);
-      const int bytes = prod.kind == 0 ? C.nt * (T1::kCodeBytes + BPK * 32)
-                                       : ngi * nr * (K2::kRowBytes + K2::kBlocks * 32);
+      constexpr int zb = aff ? 1 : 0;  // affine codes: zero points after the scales
+      const int bytes = prod.kind == 0 ? C.nt * (T1::kCodeBytes + (1 + zb) * BPK * 32)
+                                       : ngi * nr * (K2::kRowBytes + (1 + zb) * K2::kBlocks * 32);
       int v = head, ph = hp;
       if (ph + bytes > RB) {  // items never wrap around the ring's end
         v += RB - ph;
@@ -478,6 +519,9 @@ __global__ void __launch_bounds__(kSThreads, 1) qmm_slice_kernel(const SlicePara
           const uint8_t* ss =
               p.s1 + (unsigned long long)C.expert * p.s1_stride + ((unsigned long long)sb * p.NT1 + C.etile0) * 32;
           if (lane < 2 * C.nt) cp_async16(st + C.nt * T1::kCodeBytes + bl * C.nt * 32 + 16 * lane, ss + 16 * lane);
+          if (zb && lane < 2 * C.nt)
+            cp_async16(st + C.nt * T1::kCodeBytes + (BPK + bl) * C.nt * 32 + 16 * lane,
+                       p.z1 + (ss - p.s1) + 16 * lane);
         }
       } else {  // FC2: granules [a, a + ngi) of the chunk, this warp's rows of each slab, and their scales
         if (lane == 0) mbar_arrive(bar);
@@ -495,6 +539,9 @@ __global__ void __launch_bounds__(kSThreads, 1) qmm_slice_kernel(const SlicePara
                 p.s2 + (unsigned long long)C.expert * p.s2_stride + ((unsigned long long)sb * p.NT2 + r0) * 32;
             if (lane < 2 * nr) cp_async16(st + ngi * nr * K2::kRowBytes + (gi * K2::kBlocks + bl) * nr * 32 + 16 * lane,
                                           ss + 16 * lane);
+            if (zb && lane < 2 * nr)
+              cp_async16(st + ngi * nr * K2::kRowBytes + ((ngi + gi) * K2::kBlocks + bl) * nr * 32 + 16 * lane,
+                         p.z2 + (ss - p.s2) + 16 * lane);
           }
         }
       }
@@ -559,21 +606,32 @@ __global__ void __launch_bounds__(kSThreads, 1) qmm_slice_kernel(const SlicePara
   }
   // per-lane x row for ldmatrix: token lane & 7, or the zero row past the batch
   const uint8_t* xrow = xs + min(lane & 7, p.xrows - 1) * xpitch;
-  // constant-operand correction of FC1 per 64-column block and token
+  // constant-operand correction of FC1 per 64-column block and token (and,
+  // for affine codes, the block's sum of the activations)
   {
-    const uint32_t aconst[4] = {T1::kConstLo, T1::kConstLo, T1::kConstHi, T1::kConstHi};
+    const uint32_t aconst[4] = {aff ? kAffConst : T1::kConstLo, aff ? kAffConst : T1::kConstLo,
+                                aff ? kAffConst : T1::kConstHi, aff ? kAffConst : T1::kConstHi};
+    const uint32_t asum[4] = {kBf16One, kBf16One, sum_const_hi<F1>(), sum_const_hi<F1>()};
     for (int b = warp; b < p.H / 64; b += kSW) {
-      float cr[4] = {0.f, 0.f, 0.f, 0.f};
+      float cr[4] = {0.f, 0.f, 0.f, 0.f}, sx[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         uint32_t r[4];
         ldmatrix_x4(r, xrow + (b * 64 + h * 32 + (lane >> 3) * 8) * 2);
         mma_bf16_16816(cr, aconst, r[0], r[1]);
         mma_bf16_16816(cr, aconst, r[2], r[3]);
+        if (aff) {
+          mma_bf16_16816(sx, asum, r[0], r[1]);
+          mma_bf16_16816(sx, asum, r[2], r[3]);
+        }
       }
       if (lane < 4) {
         corr1[b * 8 + 2 * lane] = cr[0];
         corr1[b * 8 + 2 * lane + 1] = cr[1];
+        if (aff) {
+          sx1[b * 8 + 2 * lane] = sx[0];
+          sx1[b * 8 + 2 * lane + 1] = sx[1];
+        }
       }
     }
   }
@@ -610,7 +668,7 @@ __global__ void __launch_bounds__(kSThreads, 1) qmm_slice_kernel(const SlicePara
     for (int i = 0; i < MT; ++i) acc1[i][0] = acc1[i][1] = acc1[i][2] = acc1[i][3] = 0.f;
     for (int ku = warp; ku < p.KU1; ku += kSW) {
       const uint8_t* st = wait_item();
-      if (ok) slice_fc1<F1, MT>(st, C.nt, ku, xrow, corr1, lut, lane, acc1);
+      if (ok) slice_fc1<F1, MT>(st, C.nt, ku, xrow, corr1, sx1, aff, lut, lane, acc1);
       next_item();
     }
     // cross-warp reduction (fixed warp order) -> w * SwiGLU -> h window (bf16,
@@ -656,7 +714,7 @@ __global__ void __launch_bounds__(kSThreads, 1) qmm_slice_kernel(const SlicePara
     if (nr > 0)
       for (int a = 0; a < C.ngc; a += p.ngm) {  // window granule a: the chunk's completed granule a
         const uint8_t* st = wait_item();
-        if (ok) slice_fc2<F2>(st, min(p.ngm, C.ngc - a), nr, a, C.g0 + a, hfrag, lut, lane, acc2);
+        if (ok) slice_fc2<F2>(st, min(p.ngm, C.ngc - a), nr, a, C.g0 + a, aff, hfrag, lut, lane, acc2);
         next_item();
       }
   }

@@ -178,8 +178,7 @@ int g_fault_inject = 0;
 // prologue (after a tiny reset launch of its accumulator).
 bool decode_eligible(const qmoe_layer& L, int T, int grid, SlicePlan* plan) {
   if (T > kDecMaxT || T * L.k > kDecMaxTK || L.path == QMOE_PATH_GROUPED || L.H > kSMaxH) return false;
-  if (affine(L)) return false;  // the decode kernel takes symmetric codes (for now)
-  const SlicePlan pl = slice_plan(L.fc1.fmt, L.fc2.fmt, T, L.H);
+  const SlicePlan pl = slice_plan(L.fc1.fmt, L.fc2.fmt, T, L.H, affine(L));
   if (!pl.ok || L.I % pl.gran_cols) return false;
   const int gpe = L.I / pl.gran_cols;
   if (slice_max_chunks(L.fc2.fmt, gpe, L.n_shared, std::min(L.E, T * L.k), grid) > kSMaxChunks) return false;
@@ -555,6 +554,9 @@ qmoe_status qmoe_forward(const qmoe_layer* layer, const uint16_t* x, const float
       sp.s2 = static_cast<const uint8_t*>(L.fc2.scales);
       sp.s2_stride = scales_bytes(L.H, L.I, L.fc2.block);
       sp.b2 = L.fc2.bias;
+      sp.aff = affine(L) ? 1 : 0;
+      sp.z1 = static_cast<const uint8_t*>(L.fc1.zeros);
+      sp.z2 = static_cast<const uint8_t*>(L.fc2.zeros);
       sp.NT1 = 2 * L.I / 16;
       sp.KU1 = L.H / ku_cols(L.fc1.fmt);
       sp.block1 = L.fc1.block;

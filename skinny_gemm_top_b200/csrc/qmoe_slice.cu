@@ -20,7 +20,7 @@ int fc2_cols(int f) { return f == 4 ? 16 : f == 2 ? 32 : 64; }          // granu
 int round128(int v) { return (v + 127) / 128 * 128; }
 int chunk_tiles(int f2) { return f2 == 4 ? 10 : 8; }                    // SChunkGeom<f2>::kMT
 
-template <int F1, int F2>
+template <int F1, int F2, bool AFF>
 cudaError_t launch_t(const SliceParams& p, int grid, size_t smem, cudaStream_t st) {
   static bool attr_set[64] = {};
   int d = 0;
@@ -28,7 +28,7 @@ cudaError_t launch_t(const SliceParams& p, int grid, size_t smem, cudaStream_t s
   if (d < 0 || d >= 64) return cudaErrorInvalidDevice;
   if (!attr_set[d]) {
     const cudaError_t e =
-        cudaFuncSetAttribute(qmm_slice_kernel<F1, F2>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
+        cudaFuncSetAttribute(qmm_slice_kernel<F1, F2, AFF>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
     if (e != cudaSuccess) return e;
     attr_set[d] = true;
   }
@@ -42,18 +42,19 @@ cudaError_t launch_t(const SliceParams& p, int grid, size_t smem, cudaStream_t s
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, qmm_slice_kernel<F1, F2>, p);
+  return cudaLaunchKernelEx(&cfg, qmm_slice_kernel<F1, F2, AFF>, p);
 }
 
 }  // namespace
 
-SlicePlan slice_plan(int f1, int f2, int T, int H) {
+SlicePlan slice_plan(int f1, int f2, int T, int H, bool aff) {
   SlicePlan pl{};
   pl.ok = false;
   if (T < 1 || T > 8 || H > kSMaxH || H % 64) return pl;
-  const int fc1_item = chunk_tiles(f2) * (fc1_code_bytes(f1) + fc1_blocks_per_ku(f1) * 32);
+  const int zb = aff ? 2 : 1;  // scale (and zero point) bytes per 16 rows and block
+  const int fc1_item = chunk_tiles(f2) * (fc1_code_bytes(f1) + zb * fc1_blocks_per_ku(f1) * 32);
   const int nr_max = (H / 16 + kSW - 1) / kSW;
-  const int per_granule = nr_max * (fc2_row_bytes(f2) + fc2_blocks(f2) * 32);
+  const int per_granule = nr_max * (fc2_row_bytes(f2) + zb * fc2_blocks(f2) * 32);
   pl.ngm = std::max(1, std::min(3, 4096 / per_granule));  // FC2 items of about 4 KB
   pl.xrows = T < 8 ? T + 1 : 8;
   pl.gran_cols = fc2_cols(f2);
@@ -89,17 +90,20 @@ int slice_max_chunks(int f2, int gpe, int n_shared, int max_routed, int grid) {
 
 cudaError_t slice_launch(int f1, int f2, const SliceParams& p, int grid, size_t smem, cudaStream_t st) {
 #define QMOE_SLICE_CASE(A, B) \
-  if (f1 == A && f2 == B) return launch_t<A, B>(p, grid, smem, st);
+  if (f1 == A && f2 == B) return p.aff ? launch_t<A, B, true>(p, grid, smem, st) : launch_t<A, B, false>(p, grid, smem, st);
+#define QMOE_SLICE_CASE_SYM(A, B) \
+  if (f1 == A && f2 == B) return p.aff ? cudaErrorInvalidValue : launch_t<A, B, false>(p, grid, smem, st);
   QMOE_SLICE_CASE(2, 2)
   QMOE_SLICE_CASE(2, 4)
-  QMOE_SLICE_CASE(2, 3)
+  QMOE_SLICE_CASE_SYM(2, 3)
   QMOE_SLICE_CASE(4, 2)
   QMOE_SLICE_CASE(4, 4)
-  QMOE_SLICE_CASE(4, 3)
-  QMOE_SLICE_CASE(3, 2)
-  QMOE_SLICE_CASE(3, 4)
-  QMOE_SLICE_CASE(3, 3)
+  QMOE_SLICE_CASE_SYM(4, 3)
+  QMOE_SLICE_CASE_SYM(3, 2)
+  QMOE_SLICE_CASE_SYM(3, 4)
+  QMOE_SLICE_CASE_SYM(3, 3)
 #undef QMOE_SLICE_CASE
+#undef QMOE_SLICE_CASE_SYM
   return cudaErrorInvalidValue;
 }
 

@@ -52,6 +52,9 @@ struct SliceParams {
   const uint8_t* s2;
   unsigned long long s2_stride;
   const uint16_t* b2;    // [E + n_shared][H] or null
+  const uint8_t* z1;     // affine codes: FC1 / FC2 zero points (scale layout and strides), else null
+  const uint8_t* z2;
+  int aff;               // 1: affine codes (INT2 / INT4)
   int NT1, KU1, block1;  // FC1: 16-row tiles, k-units along H, scale block
   int NT2, block2;       // FC2: 16-row tiles (H / 16), scale block
   int H, I, E, k, n_shared, T;
@@ -76,7 +79,7 @@ struct SlicePlan {
   int ring_bytes, ngm, xrows, gran_cols;
   size_t smem;
 };
-SlicePlan slice_plan(int f1, int f2, int T, int H);
+SlicePlan slice_plan(int f1, int f2, int T, int H, bool aff);
 
 // Upper bound of the chunks one CTA can get, over every count of selected
 // experts up to max_routed (host check against kSMaxChunks).

@@ -177,6 +177,19 @@ def test_forward_affine_layer(qm, T):
     _close(y, ref, f"affine layer T={T}")
 
 
+@pytest.mark.parametrize("f1,f2,T", [("int2", "int4", 1), ("int4", "int4", 4), ("int4", "int2", 8), ("int2", "int2", 2)])
+def test_decode_affine_layer(qm, f1, f2, T):
+    """Decode batches (the decode-layer kernel) with affine codes, shared experts and biases."""
+    cfg = small_cfg(synth.TINY, fc1_fmt=f1, fc2_fmt=f2, n_shared=1, bias=True, E=16, k=4)
+    case = MoECase(cfg, seed=8, affine=True)
+    x = synth.tokens(cfg.H, 8, T)
+    lg = synth.router_logits(cfg, 8, T)
+    y = case.run(x, lg)
+    assert qm.get_stats().last_path == qm.PATH_SMALL_M  # the decode kernel, not the grouped path
+    ref = Q.moe_forward(Q.bf16_bits_to_f64(x), lg, cfg.k, case.bank)
+    _close(y, ref, f"affine decode {f1}/{f2} T={T}")
+
+
 def test_affine_rejected_where_unsupported(qm):
     import torch
     cfg = synth.TINY
