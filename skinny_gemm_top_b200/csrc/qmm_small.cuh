@@ -89,6 +89,7 @@ struct SmallParams {
   unsigned long long codes_stride;   // bytes per matrix
   const uint8_t* scales;
   unsigned long long scales_stride;  // bytes per matrix
+  const uint8_t* zeros;              // affine codes: zero points (scale layout and strides), else null
   int NT;                            // 16-row tiles per matrix
   int K;
   int KU;                            // k-units per row
@@ -115,13 +116,13 @@ struct SmallParams {
 };
 
 // Stage geometry for a format and token-group count.
-template <int FMT, int TG, int SRC>
+template <int FMT, int TG, int SRC, bool AFF = false>
 struct StageGeom {
   using Tr = FmtTraits<FMT>;
   static constexpr int kBlocksPerKU = Tr::kKUcols / 64;                 // 64-col blocks per k-unit
   static constexpr int kMT = kTiles<FMT, TG, SRC>;
   static constexpr int kCodeBytes = kMT * Tr::kCodeBytes;
-  static constexpr int kScaleBytes = kBlocksPerKU * kMT * 32;
+  static constexpr int kScaleBytes = (AFF ? 2 : 1) * kBlocksPerKU * kMT * 32;  // scales (then zero points)
   static constexpr int kActPitch = Tr::kKUcols * 2 + 16;               // padded: conflict-free ldmatrix
   static constexpr int kActBytes = TG * 8 * kActPitch;
   static constexpr int kStageBytes = ((kCodeBytes + kScaleBytes + kActBytes) + 127) / 128 * 128;
@@ -283,10 +284,10 @@ __device__ __forceinline__ void iter_begin(ItemIter& it, const SmallParams& p, c
 // KS: the matrix is packed QMOE_ROWS_KSPLIT (FC2): an INT2/INT4 k-unit of nt
 // tiles is W slabs of nt x 128 bytes, copied by per-lane cp.async into
 // [slab][tile][lane] order (ternary records are laid out as in PLAIN).
-template <int FMT, int TG, int SRC, bool KS>
+template <int FMT, int TG, int SRC, bool KS, bool AFF>
 __device__ __forceinline__ void issue_weights(const SmallParams& p, const ItemIter& it, uint8_t* stage, uint64_t* bar,
                                               int lane) {
-  using G = StageGeom<FMT, TG, SRC>;
+  using G = StageGeom<FMT, TG, SRC, AFF>;
   using Tr = FmtTraits<FMT>;
   const int tile = it.sp.rt0, n = it.sp.nt;
   if constexpr (KS && FMT != 3) {
@@ -314,14 +315,17 @@ __device__ __forceinline__ void issue_weights(const SmallParams& p, const ItemIt
     const uint8_t* ssrc = p.scales + (unsigned long long)it.sg.expert * p.scales_stride +
                           ((unsigned long long)sb * p.NT + tile) * 32;
     if (lane < 2 * n) cp_async16(stage + G::kCodeBytes + bl * G::kMT * 32 + 16 * lane, ssrc + 16 * lane);
+    if (AFF && lane < 2 * n)
+      cp_async16(stage + G::kCodeBytes + (G::kBlocksPerKU + bl) * G::kMT * 32 + 16 * lane,
+                 p.zeros + (ssrc - p.scales) + 16 * lane);
   }
 }
 
 // Activation part of a stage: the k-unit slice of each of the segment's m
 // token rows (the row of token n is held by lane n of the iterator).
-template <int FMT, int TG, int SRC>
+template <int FMT, int TG, int SRC, bool AFF>
 __device__ __forceinline__ void issue_acts(const SmallParams& p, const ItemIter& it, uint8_t* stage, int lane) {
-  using G = StageGeom<FMT, TG, SRC>;
+  using G = StageGeom<FMT, TG, SRC, AFF>;
   constexpr int kChunks = FmtTraits<FMT>::kKUcols * 2 / 16;  // 16-byte pieces per row slice
   const int total = it.sg.m * kChunks;
   for (int base = 0; base < total; base += 32) {
@@ -571,22 +575,28 @@ __device__ __forceinline__ void epilogue(const SmallParams& p, const Seg& sg, in
 // at or past nt contribute with scale 0 (their codes are stale but finite),
 // so all NTL tiles run the same straight-line code and the MMAs of a k-step
 // for every tile issue back to back.
-template <int FMT, int TG, int SRC, bool KS, int NTL>
+template <int FMT, int TG, int SRC, bool KS, int NTL, bool AFF>
 __device__ __forceinline__ void compute_item(const uint8_t* st, bool tg2, int lane, int nt, const uint32_t* lut,
                                              float (&acc)[kTiles<FMT, TG, SRC>][TG][4]) {
   using Tr = FmtTraits<FMT>;
-  using G = StageGeom<FMT, TG, SRC>;
+  using G = StageGeom<FMT, TG, SRC, AFF>;
   constexpr int BPK = Tr::kKUcols / 64;
   const uint8_t* cbuf = st;
   const uint32_t* sbuf = reinterpret_cast<const uint32_t*>(st + G::kCodeBytes);
   const uint8_t* abuf = st + G::kCodeBytes + G::kScaleBytes;
-  const uint32_t aconst[4] = {Tr::kConstLo, Tr::kConstLo, Tr::kConstHi, Tr::kConstHi};
+  // affine codes: the stored field is u, so the constant operand is -128 in
+  // both column classes, and each block adds z * (sum of its activations)
+  const uint32_t aconst[4] = {AFF ? kAffConst : Tr::kConstLo, AFF ? kAffConst : Tr::kConstLo,
+                              AFF ? kAffConst : Tr::kConstHi, AFF ? kAffConst : Tr::kConstHi};
   const int g = lane >> 2;
   // B fragments from the token rows (ldmatrix: lanes 8j..8j+7 address the
   // rows of matrix j = columns 8j..8j+7 of a 32-column half), columns
   // k%16 >= 8 divided by the code multiplier, and the constant-operand products.
   uint32_t bfr[BPK][TG][4][2];
   float corr[BPK][TG][4];
+  float sx[TG][4];  // affine codes (INT2 / INT4: one block per k-unit): sum of the activations
+#pragma unroll
+  for (int t = 0; t < TG; ++t) sx[t][0] = sx[t][1] = sx[t][2] = sx[t][3] = 0.f;
 #pragma unroll
   for (int bl = 0; bl < BPK; ++bl)
 #pragma unroll
@@ -609,6 +619,13 @@ __device__ __forceinline__ void compute_item(const uint8_t* st, bool tg2, int la
         }
 #pragma unroll
         for (int k2 = 0; k2 < 4; ++k2) mma_bf16_16816(corr[bl][t], aconst, bfr[bl][t][k2][0], bfr[bl][t][k2][1]);
+        if constexpr (AFF) {
+          const uint32_t asum[4] = {kBf16One, kBf16One, sum_const_hi<FMT>(), sum_const_hi<FMT>()};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) sx[t][e] = 0.f;
+#pragma unroll
+          for (int k2 = 0; k2 < 4; ++k2) mma_bf16_16816(sx[t], asum, bfr[bl][t][k2][0], bfr[bl][t][k2][1]);
+        }
       } else {
 #pragma unroll
         for (int k2 = 0; k2 < 4; ++k2) bfr[bl][t][k2][0] = bfr[bl][t][k2][1] = 0u;
@@ -694,6 +711,22 @@ __device__ __forceinline__ void compute_item(const uint8_t* st, bool tg2, int la
         }
       }
     }
+    if constexpr (AFF) {
+      const uint32_t* zbuf = sbuf + G::kBlocksPerKU * G::kMT * 8;
+#pragma unroll
+      for (int i = 0; i < NTL; ++i) {
+        const uint32_t zc = zbuf[i * 8 + g];
+        const bool on = i < nt;
+        const float zlo = on ? bf16_lo(zc) : 0.f, zhi = on ? bf16_hi(zc) : 0.f;
+#pragma unroll
+        for (int t = 0; t < TG; ++t) {
+          acc[i][t][0] = fmaf(zlo, sx[t][0], acc[i][t][0]);
+          acc[i][t][1] = fmaf(zlo, sx[t][1], acc[i][t][1]);
+          acc[i][t][2] = fmaf(zhi, sx[t][2], acc[i][t][2]);
+          acc[i][t][3] = fmaf(zhi, sx[t][3], acc[i][t][3]);
+        }
+      }
+    }
 #pragma unroll
     for (int i = 0; i < NTL; ++i)
 #pragma unroll
@@ -729,10 +762,10 @@ struct PhaseCtx {
 // Partition, prime (weights, then hook(), then activation rows), stream the
 // items, reduce and run the epilogue.  hook() is called by every thread of
 // the CTA exactly once (also by CTAs without work): the dependency wait.
-template <int FMT, int TG, int EPI, int SRC, class Hook>
+template <int FMT, int TG, int EPI, int SRC, bool AFF, class Hook>
 __device__ __forceinline__ void run_phase(const SmallParams& p, const SegSource& segs, int nseg, const int* act_index,
                                           PhaseCtx& cx, Hook&& hook) {
-  using G = StageGeom<FMT, TG, SRC>;
+  using G = StageGeom<FMT, TG, SRC, AFF>;
   constexpr int kNW = kWarps<TG>;
   constexpr int kCT = kNW * 32;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -754,7 +787,7 @@ __device__ __forceinline__ void run_phase(const SmallParams& p, const SegSource&
     ItemIter it = prod;
     for (int i = 0; i < NST && it.valid && !cx.aborted; ++i, ++primed) {  // (a warp that gave up issues nothing)
       const int s = (cx.issued + i) % NST;
-      issue_weights<FMT, TG, SRC, EPI == EPI_FC2>(p, it, cx.wstage + s * cx.stride, &cx.wfull[s], lane);
+      issue_weights<FMT, TG, SRC, EPI == EPI_FC2, AFF>(p, it, cx.wstage + s * cx.stride, &cx.wfull[s], lane);
       iter_advance<TG>(it, p, segs, act_index, warp, lane);
     }
   }
@@ -762,7 +795,7 @@ __device__ __forceinline__ void run_phase(const SmallParams& p, const SegSource&
   __syncwarp();
   for (int i = 0; i < primed; ++i) {
     const int s = (cx.issued + i) % NST;
-    issue_acts<FMT, TG, SRC>(p, prod, cx.wstage + s * cx.stride, lane);
+    issue_acts<FMT, TG, SRC, AFF>(p, prod, cx.wstage + s * cx.stride, lane);
     cp_async_arrive(&cx.wfull[s]);
     iter_advance<TG>(prod, p, segs, act_index, warp, lane);
   }
@@ -807,17 +840,17 @@ __device__ __forceinline__ void run_phase(const SmallParams& p, const SegSource&
       }
       if (!cx.aborted) {
         const uint8_t* st = cx.wstage + s * cx.stride;
-        if (G::kMT > 8 && sp.nt > 8) compute_item<FMT, TG, SRC, EPI == EPI_FC2, G::kMT>(st, tg2, lane, sp.nt, cx.lut, acc);
-        else if (sp.nt > 4) compute_item<FMT, TG, SRC, EPI == EPI_FC2, 8>(st, tg2, lane, sp.nt, cx.lut, acc);
-        else if (sp.nt > 2) compute_item<FMT, TG, SRC, EPI == EPI_FC2, 4>(st, tg2, lane, sp.nt, cx.lut, acc);
-        else if (sp.nt > 1) compute_item<FMT, TG, SRC, EPI == EPI_FC2, 2>(st, tg2, lane, sp.nt, cx.lut, acc);
-        else compute_item<FMT, TG, SRC, EPI == EPI_FC2, 1>(st, tg2, lane, sp.nt, cx.lut, acc);
+        if (G::kMT > 8 && sp.nt > 8) compute_item<FMT, TG, SRC, EPI == EPI_FC2, G::kMT, AFF>(st, tg2, lane, sp.nt, cx.lut, acc);
+        else if (sp.nt > 4) compute_item<FMT, TG, SRC, EPI == EPI_FC2, 8, AFF>(st, tg2, lane, sp.nt, cx.lut, acc);
+        else if (sp.nt > 2) compute_item<FMT, TG, SRC, EPI == EPI_FC2, 4, AFF>(st, tg2, lane, sp.nt, cx.lut, acc);
+        else if (sp.nt > 1) compute_item<FMT, TG, SRC, EPI == EPI_FC2, 2, AFF>(st, tg2, lane, sp.nt, cx.lut, acc);
+        else compute_item<FMT, TG, SRC, EPI == EPI_FC2, 1, AFF>(st, tg2, lane, sp.nt, cx.lut, acc);
       }
       __syncwarp();
       if (prod.valid && !cx.aborted) {
         uint8_t* st = cx.wstage + s * cx.stride;
-        issue_weights<FMT, TG, SRC, EPI == EPI_FC2>(p, prod, st, &cx.wfull[s], lane);
-        issue_acts<FMT, TG, SRC>(p, prod, st, lane);
+        issue_weights<FMT, TG, SRC, EPI == EPI_FC2, AFF>(p, prod, st, &cx.wfull[s], lane);
+        issue_acts<FMT, TG, SRC, AFF>(p, prod, st, lane);
         cp_async_arrive(&cx.wfull[s]);
         ++cx.issued;
         iter_advance<TG>(prod, p, segs, act_index, warp, lane);
@@ -866,7 +899,7 @@ __device__ __forceinline__ void drain_ring(const PhaseCtx& cx, int lane) {
 }
 
 // Shared-memory layout of a small-M kernel and the rings' context.
-template <int FMT, int TG, int SRC>
+template <int FMT, int TG, int SRC, bool AFF>
 struct SmallSmem {
   uint64_t* bars;  // [kNW][NST] full barriers
   uint32_t* lut;   // 243 entries (ternary)
@@ -876,14 +909,15 @@ struct SmallSmem {
     bars = reinterpret_cast<uint64_t*>(smem);
     lut = reinterpret_cast<uint32_t*>(smem + 1024);
     red = reinterpret_cast<float4*>(smem + SmemHead<SRC>::kFixed);
-    stages = smem + SmemHead<SRC>::kFixed + StageGeom<FMT, TG, SRC>::kRedBytes;
+    stages = smem + SmemHead<SRC>::kFixed + StageGeom<FMT, TG, SRC, AFF>::kRedBytes;
   }
 };
 
 // Ternary table, ring barriers and the phase context (ends with a CTA barrier).
-template <int FMT, int TG, int SRC>
-__device__ __forceinline__ void init_rings(const SmallSmem<FMT, TG, SRC>& sm, int NST, int* s_abort, PhaseCtx& cx) {
-  using G = StageGeom<FMT, TG, SRC>;
+template <int FMT, int TG, int SRC, bool AFF>
+__device__ __forceinline__ void init_rings(const SmallSmem<FMT, TG, SRC, AFF>& sm, int NST, int* s_abort,
+                                           PhaseCtx& cx) {
+  using G = StageGeom<FMT, TG, SRC, AFF>;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (tid == 0) *s_abort = 0;
   if constexpr (FMT == 3)
@@ -902,11 +936,11 @@ __device__ __forceinline__ void init_rings(const SmallSmem<FMT, TG, SRC>& sm, in
   __syncthreads();
 }
 
-template <int FMT, int TG, int EPI, int SRC>
+template <int FMT, int TG, int EPI, int SRC, bool AFF>
 __global__ void __launch_bounds__(kWarps<TG> * 32, 1) qmm_small_kernel(const SmallParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
   const int lane = threadIdx.x & 31;
-  const SmallSmem<FMT, TG, SRC> sm(smem);
+  const SmallSmem<FMT, TG, SRC, AFF> sm(smem);
   __shared__ int s_abort;
 
   // ---- segments ----
@@ -926,9 +960,9 @@ __global__ void __launch_bounds__(kWarps<TG> * 32, 1) qmm_small_kernel(const Sma
   }
 
   PhaseCtx cx;
-  init_rings<FMT, TG, SRC>(sm, p.nstages, &s_abort, cx);
+  init_rings<FMT, TG, SRC, AFF>(sm, p.nstages, &s_abort, cx);
 
-  run_phase<FMT, TG, EPI, SRC>(p, segs, nseg, p.act_index, cx, [&] {
+  run_phase<FMT, TG, EPI, SRC, AFF>(p, segs, nseg, p.act_index, cx, [&] {
     pdl_wait();
     pdl_trigger();
   });

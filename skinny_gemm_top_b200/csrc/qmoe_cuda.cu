@@ -157,15 +157,13 @@ bool grouped_eligible(const qmoe_layer& L) {
   return L.fc1.fmt != QMOE_TERNARY && L.fc2.fmt != QMOE_TERNARY && (2 * L.I) % kGRows == 0 && L.H % kGRows == 0;
 }
 
-// Affine codes (zero points): the decode kernel and the grouped (tcgen05)
-// kernel take them; the small-M expert kernel does not, so outside the decode
-// kernel every expert of an affine layer runs on the grouped path.
+// Affine codes (zero points): every kernel takes them (INT2 / INT4).
 bool affine(const qmoe_layer& L) { return L.fc1.zeros || L.fc2.zeros; }
 
 // Token-count threshold above which an expert runs on the grouped path.
 int grouped_threshold(const qmoe_layer& L) {
   if (L.path == QMOE_PATH_SMALL_M || !grouped_eligible(L)) return INT_MAX;
-  return L.path == QMOE_PATH_GROUPED || affine(L) ? 0 : kGroupedThreshold;
+  return L.path == QMOE_PATH_GROUPED ? 0 : kGroupedThreshold;
 }
 
 // Fault injection for tests (qmoe_test_set_fault): the decode kernel's wait
@@ -250,9 +248,9 @@ qmoe_status encode_rows_map(CUtensorMap* map, const void* base, int K, int rows)
 // ---- small-M kernel launch ----
 // Dynamic shared memory of a small-M kernel: fixed head, reduction buffer and
 // as many ring stages per warp as fit (at most kMaxStages, at least 2).
-template <int FMT, int TG, int SRC>
+template <int FMT, int TG, int SRC, bool AFF>
 int small_smem(int* nstages) {
-  using G = StageGeom<FMT, TG, SRC>;
+  using G = StageGeom<FMT, TG, SRC, AFF>;
   constexpr int kNW = kWarps<TG>;
   const int fixed = SmemHead<SRC>::kFixed + G::kRedBytes;
   const int nst = std::min((kSmemLimit - fixed - 1024) / (kNW * G::kStageBytes), kMaxStages);
@@ -260,35 +258,44 @@ int small_smem(int* nstages) {
   return nst < 2 ? -1 : fixed + nst * kNW * G::kStageBytes;
 }
 
-template <int FMT, int TG, int EPI, int SRC>
+template <int FMT, int TG, int EPI, int SRC, bool AFF>
 qmoe_status launch_small_t(SmallParams prm, int grid, cudaStream_t st) {
   constexpr int kNW = kWarps<TG>;
   int nst = 0;
-  const int smem = small_smem<FMT, TG, SRC>(&nst);
+  const int smem = small_smem<FMT, TG, SRC, AFF>(&nst);
   if (smem < 0) return QMOE_ERR_UNSUPPORTED;
   prm.nstages = nst;
   static bool attr_set[kMaxDevices] = {};
   int d = 0;
   cudaGetDevice(&d);
   if (!attr_set[d]) {
-    if (cudaFuncSetAttribute(qmm_small_kernel<FMT, TG, EPI, SRC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(qmm_small_kernel<FMT, TG, EPI, SRC, AFF>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              smem) != cudaSuccess)
       return QMOE_ERR_CUDA;
     attr_set[d] = true;
   }
   TraceScope ts(st, EPI == EPI_SWIGLU ? K_FC1_SMALL : (EPI == EPI_FC2 ? K_FC2_SMALL : K_LINEAR_SMALL));
-  return launch_pdl(qmm_small_kernel<FMT, TG, EPI, SRC>, dim3(grid), dim3(kNW * 32), smem, st, prm) == cudaSuccess
+  return launch_pdl(qmm_small_kernel<FMT, TG, EPI, SRC, AFF>, dim3(grid), dim3(kNW * 32), smem, st, prm) == cudaSuccess
              ? QMOE_OK
              : QMOE_ERR_CUDA;
 }
 
+template <int FMT, int EPI, int SRC, bool AFF>
+qmoe_status launch_small_tg(int tg, const SmallParams& prm, int grid, cudaStream_t st) {
+  return tg == 1 ? launch_small_t<FMT, 1, EPI, SRC, AFF>(prm, grid, st)
+                 : launch_small_t<FMT, 2, EPI, SRC, AFF>(prm, grid, st);
+}
+
+// Affine codes (prm.zeros) take their own instantiations (INT2 / INT4).
 template <int EPI, int SRC>
 qmoe_status launch_small(int fmt, int tg, const SmallParams& prm, int grid, cudaStream_t st) {
+  const bool aff = prm.zeros != nullptr;
   if (fmt == QMOE_INT2)
-    return tg == 1 ? launch_small_t<2, 1, EPI, SRC>(prm, grid, st) : launch_small_t<2, 2, EPI, SRC>(prm, grid, st);
+    return aff ? launch_small_tg<2, EPI, SRC, true>(tg, prm, grid, st) : launch_small_tg<2, EPI, SRC, false>(tg, prm, grid, st);
   if (fmt == QMOE_INT4)
-    return tg == 1 ? launch_small_t<4, 1, EPI, SRC>(prm, grid, st) : launch_small_t<4, 2, EPI, SRC>(prm, grid, st);
-  return tg == 1 ? launch_small_t<3, 1, EPI, SRC>(prm, grid, st) : launch_small_t<3, 2, EPI, SRC>(prm, grid, st);
+    return aff ? launch_small_tg<4, EPI, SRC, true>(tg, prm, grid, st) : launch_small_tg<4, EPI, SRC, false>(tg, prm, grid, st);
+  if (aff) return QMOE_ERR_UNSUPPORTED;
+  return launch_small_tg<3, EPI, SRC, false>(tg, prm, grid, st);
 }
 
 template <int FMT, int EPI, int BT, int CS>
@@ -347,6 +354,7 @@ SmallParams small_params(const qmoe_weights& w, int rows, int K, unsigned* statu
   p.codes_stride = codes_bytes(w.fmt, rows, K);
   p.scales = static_cast<const uint8_t*>(w.scales);
   p.scales_stride = scales_bytes(rows, K, w.block);
+  p.zeros = static_cast<const uint8_t*>(w.zeros);
   p.NT = rows / 16;
   p.K = K;
   p.KU = K / ku_cols(w.fmt);
@@ -366,9 +374,7 @@ qmoe_status check_layer(const qmoe_layer* L) {
   qmoe_status s = check_weights(L->fc1, 2 * L->I, L->H);
   if (s != QMOE_OK) return s;
   s = check_weights(L->fc2, L->H, L->I);
-  if (s != QMOE_OK) return s;
-  if (affine(*L) && (L->path == QMOE_PATH_SMALL_M || !grouped_eligible(*L))) return QMOE_ERR_UNSUPPORTED;
-  return QMOE_OK;
+  return s;
 }
 
 }  // namespace
@@ -732,9 +738,7 @@ qmoe_status qmoe_linear(const qmoe_weights* w, int N, int K, const uint16_t* x, 
   // More than one token group: the tcgen05 path, whose cost barely depends on
   // M (the dequantized tile serves up to 256 tokens; the small-M kernel's
   // mma.sync work grows with every group of 8 tokens).
-  // Affine codes: the tcgen05 path at every M (the small-M kernel takes symmetric codes only).
-  const bool grouped = (M >= kLinearGroupedMinM || w->zeros) && N % kGRows == 0 && w->fmt != QMOE_TERNARY;
-  if (w->zeros && !grouped) return QMOE_ERR_UNSUPPORTED;
+  const bool grouped = M >= kLinearGroupedMinM && N % kGRows == 0 && w->fmt != QMOE_TERNARY;
   if (grouped) {
     CUtensorMap map;
     s = encode_rows_map(&map, x, K, M);

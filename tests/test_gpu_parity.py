@@ -146,8 +146,8 @@ def test_grouped_operand_affine_bit_exact_one_hot(qm, fmt, block, tiny):
     assert np.array_equal(got, op[:, km].T)
 
 
-@pytest.mark.parametrize("fmt,block", [("int2", 128), ("int4", 128), ("int4", 64)])
-@pytest.mark.parametrize("M", [1, 5, 8, 32])
+@pytest.mark.parametrize("fmt,block", [("int2", 128), ("int4", 128), ("int4", 64), ("int2", 64)])
+@pytest.mark.parametrize("M", [1, 5, 8, 16, 32, 64])
 def test_linear_affine(qm, fmt, block, M):
     import torch
     N, K = 384, 1024
@@ -190,17 +190,28 @@ def test_decode_affine_layer(qm, f1, f2, T):
     _close(y, ref, f"affine decode {f1}/{f2} T={T}")
 
 
-def test_affine_rejected_where_unsupported(qm):
+@pytest.mark.parametrize("path,T", [("small", 13), ("small", 40), ("grouped", 13)])
+def test_forward_affine_forced_paths(qm, path, T):
+    """Affine layers on the small-M expert kernel (forced) and on the tcgen05 path (forced)."""
+    cfg = small_cfg(synth.TINY, n_shared=1, bias=True)
+    case = MoECase(cfg, seed=9, affine=True)
+    x = synth.tokens(cfg.H, 9, T)
+    lg = synth.router_logits(cfg, 9, T)
+    y = case.run(x, lg, path=qm.PATH_SMALL_M if path == "small" else qm.PATH_GROUPED)
+    ref = Q.moe_forward(Q.bf16_bits_to_f64(x), lg, cfg.k, case.bank)
+    _close(y, ref, f"affine {path} T={T}")
+
+
+def test_affine_ternary_rejected(qm):
     import torch
-    cfg = synth.TINY
-    case = MoECase(cfg, seed=7, affine=True)
-    layer = case.layer(path=qm.PATH_SMALL_M)
-    ws = torch.empty(1 << 20, dtype=torch.uint8, device="cuda")
-    x = to_dev(synth.tokens(cfg.H, 7, 2))
-    lg = torch.from_numpy(np.ascontiguousarray(synth.router_logits(cfg, 7, 2))).cuda()
-    y = torch.empty((2, cfg.H), dtype=torch.int16, device="cuda")
+    c, s = qm.pack(qm.TERNARY, 0, synth.linear_weight(3, 64, 128), 64)
+    keep = [to_dev(c), to_dev(s), to_dev(s.copy())]
+    w = qm.make_weights(qm.TERNARY, 64, keep[0], keep[1], None, 0, keep[2])
+    x = to_dev(synth.tokens(128, 3, 1))
+    y = torch.empty((1, 64), dtype=torch.int16, device="cuda")
+    ws = torch.empty(qm.linear_workspace_size(64, 128, 1), dtype=torch.uint8, device="cuda")
     with pytest.raises(qm.QmoeError):
-        qm.forward(layer, x, lg, y, ws)
+        qm.linear(w, 64, 128, x, y, ws)
 
 
 # ------------------------------------------------------------------ routing
