@@ -226,7 +226,13 @@ qmoe_status qmoe_forward_static(const qmoe_layer* layer, const uint16_t* x, cons
                                 uint16_t* y, void* stream);
 
 /* Single quantized linear y[M, N] bf16 = x[M, K] bf16 @ dequant(W)[N, K]^T,
- * W packed PLAIN (other row orders: QMOE_ERR_INVALID_ARG).  M >= 1. */
+ * W packed PLAIN (other row orders: QMOE_ERR_INVALID_ARG).  M >= 1.
+ * ws (device, 256-byte aligned, contents irrelevant): with at least
+ * qmoe_linear_workspace_size() bytes, a shape with few 16-row tiles (such as
+ * N = 5120) is split along K over more SMs, its partial sums accumulated in ws
+ * in fp32 (their order varies from run to run); with less (or NULL) it runs
+ * unsplit.  The MLX issue "2-bit quantized_matmul loses its size advantage
+ * over 4-bit at M >= 3", table: K = 5120 -> N = 17408 / 248320, group 128. */
 qmoe_status qmoe_linear_workspace_size(int N, int K, int M, size_t* bytes);
 qmoe_status qmoe_linear(const qmoe_weights* w, int N, int K, const uint16_t* x, int M,
                         uint16_t* y, void* ws, size_t ws_bytes, void* stream);

@@ -337,6 +337,18 @@ __global__ void combine_kernel(const float* __restrict__ yslot, const float* __r
   }
 }
 
+// Clears an fp32 accumulator and a ticket array for the launch after it:
+// lets that launch start at once (it waits for this one before touching
+// either), then waits for the launch before, which may still use them.
+__global__ void accum_reset_kernel(float* acc, int n4, int* tickets, int nt) {
+  pdl_trigger();
+  pdl_wait();
+  const int stride = gridDim.x * blockDim.x;
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += stride)
+    reinterpret_cast<float4*>(acc)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < nt; i += stride) tickets[i] = 0;
+}
+
 // Dequantize through the hot kernels' unpack: one warp per (matrix, k-unit, tile).
 // Affine codes (zeros != NULL): w = s*u + z, fp32 by one fused multiply-add,
 // bf16 by one bf16 fused multiply-add (a single rounding of the exact value).

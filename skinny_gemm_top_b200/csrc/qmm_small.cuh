@@ -90,6 +90,10 @@ struct SmallParams {
   const uint8_t* scales;
   unsigned long long scales_stride;  // bytes per matrix
   const uint8_t* zeros;              // affine codes: zero points (scale layout and strides), else null
+  int ksplit;                        // single linear: k-unit slices per tile (1: none)
+  int KUs;                           // k-units per slice (KU / ksplit)
+  float* yacc;                       // ksplit > 1: fp32 output accumulator [T][N], zero at launch
+  int* tickets;                      // ksplit > 1: per (token chunk, tile) slice count, zero at launch
   int NT;                            // 16-row tiles per matrix
   int K;
   int KU;                            // k-units per row
@@ -229,13 +233,16 @@ struct ItemIter {
   int ku;
   int row;     // this lane's activation row (lane < sg.m)
   int cap;     // tiles per sub-panel
+  int slice;   // k-unit slice of the sub-panel (single linear split along K)
   bool valid;
 };
 
 template <int TG>
 __device__ __forceinline__ void iter_load_seg(ItemIter& it, const SmallParams& p, const SegSource& segs,
                                               const int* act_index, int lane) {
-  it.sg = segs.get(it.sp.seg);
+  // with a K split, "segment" sp.seg = token chunk * ksplit + slice
+  it.sg = segs.get(it.sp.seg / p.ksplit);
+  it.slice = it.sp.seg % p.ksplit;
   if (it.sg.tg > TG || it.sg.tg < 1) it.sg.tg = TG;  // never overrun the stage (flagged by the consumer)
   if (it.sg.m > 8 * it.sg.tg) it.sg.m = 8 * it.sg.tg;
   const int s = it.sg.slot0 + (lane < it.sg.m ? lane : 0);
@@ -246,14 +253,14 @@ template <int TG>
 __device__ __forceinline__ void iter_advance(ItemIter& it, const SmallParams& p, const SegSource& segs,
                                              const int* act_index, int warp, int lane) {
   it.ku += kWarps<TG>;
-  if (it.ku < p.KU) return;
+  if (it.ku < p.KUs) return;
   for (;;) {
     if (it.sp.next >= it.f1) { it.valid = false; return; }
     const int prev = it.sp.seg;
-    load_subpanel(it.sp, it.sp.next, it.f1, p.NT, p.KU, it.cap);
+    load_subpanel(it.sp, it.sp.next, it.f1, p.NT, p.KUs, it.cap);
     if (it.sp.seg != prev) iter_load_seg<TG>(it, p, segs, act_index, lane);
     it.ku = warp;
-    if (it.ku < p.KU) return;
+    if (it.ku < p.KUs) return;
   }
 }
 
@@ -264,11 +271,11 @@ __device__ __forceinline__ void iter_begin(ItemIter& it, const SmallParams& p, c
   it.cap = cap;
   it.valid = f0 < f1;
   if (!it.valid) return;
-  load_subpanel(it.sp, f0, f1, p.NT, p.KU, cap);
+  load_subpanel(it.sp, f0, f1, p.NT, p.KUs, cap);
   iter_load_seg<TG>(it, p, segs, act_index, lane);
   it.ku = warp;
-  if (it.ku >= p.KU) {
-    it.ku = p.KU - kWarps<TG>;  // so that the advance moves to the next sub-panel
+  if (it.ku >= p.KUs) {
+    it.ku = p.KUs - kWarps<TG>;  // so that the advance moves to the next sub-panel
     iter_advance<TG>(it, p, segs, act_index, warp, lane);
   }
 }
@@ -290,6 +297,7 @@ __device__ __forceinline__ void issue_weights(const SmallParams& p, const ItemIt
   using G = StageGeom<FMT, TG, SRC, AFF>;
   using Tr = FmtTraits<FMT>;
   const int tile = it.sp.rt0, n = it.sp.nt;
+  const int ku = it.slice * p.KUs + it.ku;  // k-unit of the matrix
   if constexpr (KS && FMT != 3) {
     constexpr int W = FMT == 2 ? 2 : 4;
     const int per = n * 8;  // 16-byte pieces per slab
@@ -297,12 +305,12 @@ __device__ __forceinline__ void issue_weights(const SmallParams& p, const ItemIt
     for (int c = lane; c < W * per; c += 32) {
       const int w = c / per, j = c - w * per;
       cp_async16(stage + w * (G::kMT * 128) + 16 * j,
-                 base + (((unsigned long long)it.ku * W + w) * p.NT + tile) * 128 + 16 * j);
+                 base + (((unsigned long long)ku * W + w) * p.NT + tile) * 128 + 16 * j);
     }
     if (lane == 0) mbar_arrive(bar);  // the arrival a bulk copy's expect-tx would make
   } else if (lane == 0) {
     const uint8_t* csrc = p.codes + (unsigned long long)it.sg.expert * p.codes_stride +
-                          ((unsigned long long)it.ku * p.NT + tile) * Tr::kCodeBytes;
+                          ((unsigned long long)ku * p.NT + tile) * Tr::kCodeBytes;
     const uint32_t bytes = (uint32_t)(n * Tr::kCodeBytes);
     // No proxy fence: the warp's reads of this stage were consumed by its MMAs
     // before the refill is issued.
@@ -311,7 +319,7 @@ __device__ __forceinline__ void issue_weights(const SmallParams& p, const ItemIt
   }
 #pragma unroll
   for (int bl = 0; bl < G::kBlocksPerKU; ++bl) {
-    const int sb = (it.ku * Tr::kKUcols + bl * 64) >> (p.block == 128 ? 7 : 6);  // block is 64 or 128
+    const int sb = (ku * Tr::kKUcols + bl * 64) >> (p.block == 128 ? 7 : 6);  // block is 64 or 128
     const uint8_t* ssrc = p.scales + (unsigned long long)it.sg.expert * p.scales_stride +
                           ((unsigned long long)sb * p.NT + tile) * 32;
     if (lane < 2 * n) cp_async16(stage + G::kCodeBytes + bl * G::kMT * 32 + 16 * lane, ssrc + 16 * lane);
@@ -334,7 +342,7 @@ __device__ __forceinline__ void issue_acts(const SmallParams& p, const ItemIter&
     const int row = __shfl_sync(0xffffffffu, it.row, n < 32 ? n : 0);
     if (c < total) {
       const uint8_t* src = reinterpret_cast<const uint8_t*>(p.act) + ((unsigned long long)row * p.K) * 2 +
-                           (unsigned long long)it.ku * kChunks * 16 + 16 * j;
+                           (unsigned long long)(it.slice * p.KUs + it.ku) * kChunks * 16 + 16 * j;
       cp_async16(stage + G::kCodeBytes + G::kScaleBytes + n * G::kActPitch + 16 * j, src);
     }
   }
@@ -743,6 +751,45 @@ __device__ __forceinline__ void compute_item(const uint8_t* st, bool tg2, int la
 // One matmul phase of a small-M kernel on the warps' stage rings.  The rings
 // (barriers, stage buffers, item counters) are kept in a context that could
 // persist across phases of one kernel.
+// Single linear split along K: this CTA's fp32 partial of one reduced
+// fragment (rows g / g+8 of tile rt, tokens n0, n0+1) added to the output
+// accumulator.
+__device__ __forceinline__ void linear_partial(const SmallParams& p, const Seg& sg, int rt, int tg, int lane, float4 v) {
+  const int g = lane >> 2, q = lane & 3;
+  const int n0 = tg * 8 + 2 * q;
+  const int r0 = rt * 16 + g, r1 = r0 + 8;
+  if (n0 < sg.m) {
+    float* yr = p.yacc + (size_t)(sg.slot0 + n0) * p.N;
+    atomicAdd(yr + r0, v.x);
+    atomicAdd(yr + r1, v.z);
+  }
+  if (n0 + 1 < sg.m) {
+    float* yr = p.yacc + (size_t)(sg.slot0 + n0 + 1) * p.N;
+    atomicAdd(yr + r0, v.y);
+    atomicAdd(yr + r1, v.w);
+  }
+}
+
+// After a sub-panel's partials: one ticket per tile; the CTA that adds a
+// tile's last slice rounds its rows to bf16.  Ends with a CTA barrier.
+__device__ __forceinline__ void linear_tickets(const SmallParams& p, const Seg& sg, int chunk, int rt0, int nt,
+                                               bool aborted, int* s_last) {
+  const int tid = threadIdx.x;
+  if (tid < nt) {
+    const int old = atomic_add_acq_rel_gpu(p.tickets + chunk * p.NT + rt0 + tid, 1);
+    s_last[tid] = (old == p.ksplit - 1 && !aborted) ? 1 : 0;
+  }
+  __syncthreads();
+  for (int e = tid; e < nt * 16 * sg.m; e += blockDim.x) {
+    const int i = e / (16 * sg.m), rem = e - i * 16 * sg.m, n = rem / 16, r = rem % 16;
+    if (!s_last[i]) continue;
+    const size_t o = (size_t)(sg.slot0 + n) * p.N + (rt0 + i) * 16 + r;
+    const float v = *reinterpret_cast<volatile const float*>(p.yacc + o);
+    p.y[o] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+  }
+  __syncthreads();
+}
+
 struct PhaseCtx {
   uint64_t* wfull;  // this warp's full barriers [NST]
   uint8_t* wstage;  // this warp's first stage
@@ -757,6 +804,7 @@ struct PhaseCtx {
   float4* red;
   const uint32_t* lut;
   int* s_abort;
+  int* s_last;     // [kMT] tiles whose last K slice this CTA added (single linear split along K)
 };
 
 // Partition, prime (weights, then hook(), then activation rows), stream the
@@ -772,7 +820,7 @@ __device__ __forceinline__ void run_phase(const SmallParams& p, const SegSource&
   const int NST = cx.NST;
 
   unsigned f0, f1;
-  cta_range(nseg, p.NT, p.KU, f0, f1);
+  cta_range(nseg * p.ksplit, p.NT, p.KUs, f0, f1);
   if (f0 >= f1) {  // whole CTA idle in this phase
     hook();
     return;
@@ -806,10 +854,10 @@ __device__ __forceinline__ void run_phase(const SmallParams& p, const SegSource&
   int cur_seg = -1;
   Seg sg;
   while (pos < f1) {
-    load_subpanel(sp, pos, f1, p.NT, p.KU, G::kMT);
+    load_subpanel(sp, pos, f1, p.NT, p.KUs, G::kMT);
     if (sp.seg != cur_seg) {
       cur_seg = sp.seg;
-      sg = segs.get(sp.seg);
+      sg = segs.get(sp.seg / p.ksplit);
       if (sg.tg > TG || sg.tg < 1 || sg.m > 8 * sg.tg) {
         if (tid == 0) atomicOr(p.status, kStatusBadSegment);
         sg.tg = TG;
@@ -825,7 +873,7 @@ __device__ __forceinline__ void run_phase(const SmallParams& p, const SegSource&
 #pragma unroll
         for (int e = 0; e < 4; ++e) acc[i][t][e] = 0.f;
 
-    for (int ku = warp; ku < p.KU; ku += kNW) {
+    for (int ku = warp; ku < p.KUs; ku += kNW) {
       const int s = cx.stage;
       const uint32_t par = cx.phase;
       ++cx.item;
@@ -882,9 +930,11 @@ __device__ __forceinline__ void run_phase(const SmallParams& p, const SegSource&
       }
       const int i = e / (TG * 32), t = (e / 32) % TG, ln = e % 32;
       if (t == 1 && !tg2) continue;
-      epilogue<EPI>(p, sg, sp.rt0 + i, t, ln, v);
+      if (EPI == EPI_LINEAR && p.ksplit > 1) linear_partial(p, sg, sp.rt0 + i, t, ln, v);
+      else epilogue<EPI>(p, sg, sp.rt0 + i, t, ln, v);
     }
     __syncthreads();
+    if (EPI == EPI_LINEAR && p.ksplit > 1) linear_tickets(p, sg, sp.seg / p.ksplit, sp.rt0, sp.nt, ab, cx.s_last);
     pos = sp.next;
   }
 }
@@ -942,6 +992,7 @@ __global__ void __launch_bounds__(kWarps<TG> * 32, 1) qmm_small_kernel(const Sma
   const int lane = threadIdx.x & 31;
   const SmallSmem<FMT, TG, SRC, AFF> sm(smem);
   __shared__ int s_abort;
+  __shared__ int s_last[kTiles<FMT, TG, SRC>];
 
   // ---- segments ----
   // With p.early the segment source was written at least two launches back
@@ -961,6 +1012,7 @@ __global__ void __launch_bounds__(kWarps<TG> * 32, 1) qmm_small_kernel(const Sma
 
   PhaseCtx cx;
   init_rings<FMT, TG, SRC, AFF>(sm, p.nstages, &s_abort, cx);
+  cx.s_last = s_last;
 
   run_phase<FMT, TG, EPI, SRC, AFF>(p, segs, nseg, p.act_index, cx, [&] {
     pdl_wait();

@@ -166,6 +166,24 @@ int grouped_threshold(const qmoe_layer& L) {
   return L.path == QMOE_PATH_GROUPED ? 0 : kGroupedThreshold;
 }
 
+// Single linear on the small-M kernel, split along K when it has fewer than
+// 4 16-row tiles per SM (N = 5120: 320 tiles for 148 SMs), into about 8 (tile,
+// k-slice) units per SM: slices of at least 12 k-units (one per warp), partial
+// sums added into an fp32 accumulator in the workspace, the last slice of a
+// tile rounds it to bf16.  (N = 17408, 7.4 tiles per SM, measured slower split.)
+constexpr int kLinSplitTiles = 8;
+int linear_ksplit(int N, int K, int fmt, int sms) {
+  const int NT = N / 16, KU = K / ku_cols(fmt);
+  if (2 * NT >= kLinSplitTiles * sms) return 1;
+  const int want = (kLinSplitTiles * sms + NT / 2) / NT;
+  for (int S = std::min(want, KU / 12); S > 1; --S)
+    if (KU % S == 0) return S;
+  return 1;
+}
+size_t linear_split_bytes(int N, int M) {
+  return align_up((size_t)M * N * 4) + align_up((size_t)((M + kChunkTokens - 1) / kChunkTokens) * (N / 16) * 4);
+}
+
 // Fault injection for tests (qmoe_test_set_fault): the decode kernel's wait
 // limit and what to inject.
 unsigned long long g_fault_wait_ns = kWaitLimitNs;
@@ -358,6 +376,8 @@ SmallParams small_params(const qmoe_weights& w, int rows, int K, unsigned* statu
   p.NT = rows / 16;
   p.K = K;
   p.KU = K / ku_cols(w.fmt);
+  p.ksplit = 1;
+  p.KUs = p.KU;
   p.block = w.block;
   p.status = status;
   return p;
@@ -712,7 +732,7 @@ qmoe_status qmoe_forward(const qmoe_layer* layer, const uint16_t* x, const float
 
 qmoe_status qmoe_linear_workspace_size(int N, int K, int M, size_t* bytes) {
   if (N <= 0 || K <= 0 || M <= 0 || N % 16 || K % 64 || !bytes) return QMOE_ERR_INVALID_ARG;
-  *bytes = kAlign;  // the single linear needs no scratch; a minimal workspace keeps the ABI stable
+  *bytes = linear_split_bytes(N, M);
   return QMOE_OK;
 }
 
@@ -722,8 +742,6 @@ qmoe_status qmoe_linear(const qmoe_weights* w, int N, int K, const uint16_t* x, 
   if (w->row_order != QMOE_ROWS_PLAIN) return QMOE_ERR_INVALID_ARG;
   qmoe_status s = check_weights(*w, N, K);
   if (s != QMOE_OK) return s;
-  (void)ws;
-  (void)ws_bytes;
   if (reinterpret_cast<uintptr_t>(x) & 15) return QMOE_ERR_INVALID_ARG;
   DevInfo* di;
   s = dev_info(&di);
@@ -750,6 +768,18 @@ qmoe_status qmoe_linear(const qmoe_weights* w, int N, int K, const uint16_t* x, 
     const int units = (M + kLinBT - 1) / kLinBT * g.rtiles;
     s = launch_grouped_linear(w->fmt, map, g, std::min(units, di->sms), st);
   } else {
+    const int S = linear_ksplit(N, K, w->fmt, di->sms);
+    if (S > 1 && ws && ws_bytes >= linear_split_bytes(N, M) && !(reinterpret_cast<uintptr_t>(ws) % kAlign)) {
+      p.ksplit = S;
+      p.KUs = p.KU / S;
+      p.yacc = static_cast<float*>(ws);
+      p.tickets = reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + align_up((size_t)M * N * 4));
+      const int n4 = M * N / 4, nt = (M + kChunkTokens - 1) / kChunkTokens * (N / 16);
+      TraceScope ts(st, K_DECODE_RESET);
+      if (launch_pdl(accum_reset_kernel, dim3(std::max(1, std::min(di->sms, (n4 + 255) / 256))), dim3(256), 0, st,
+                     p.yacc, n4, p.tickets, nt) != cudaSuccess)
+        return QMOE_ERR_CUDA;
+    }
     s = launch_small<EPI_LINEAR, SRC_LINEAR>(w->fmt, M <= 8 ? 1 : 2, p, di->sms, st);
   }
   if (s != QMOE_OK) return s;

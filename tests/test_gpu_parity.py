@@ -342,6 +342,27 @@ def test_linear_full_size_sampled_rows(qm, fmt, M):
     _close(y[:, rows], ref, f"{fmt} M={M}")
 
 
+@pytest.mark.parametrize("fmt,block", [("int2", 128), ("int4", 64)])
+@pytest.mark.parametrize("M", [1, 9, 16, 33])
+def test_linear_split_along_k(qm, fmt, block, M):
+    """N = 1024 (64 tiles) is split along K over the SMs; partial sums meet in the workspace.
+    A second call on the same workspace must give the same result (the accumulator is cleared per call)."""
+    import torch
+    N, K = 1024, 2048
+    wb, x, y, dev = _linear_case(qm, fmt, block, N, K, M, seed=60 + M)
+    codes, scales = oracle_quant(fmt, wb, block)
+    ref = Q.linear(Q.bf16_bits_to_f64(x), Q.dequant(codes, scales, block))
+    _close(y, ref, f"{fmt} split M={M}")
+    w = qm.make_weights(FMTS[fmt], block, dev[0], dev[1])
+    ws = torch.empty(qm.linear_workspace_size(N, K, M), dtype=torch.uint8, device="cuda")
+    y2 = torch.empty((M, N), dtype=torch.int16, device="cuda")
+    xd = to_dev(x)
+    for _ in range(2):
+        qm.linear(w, N, K, xd, y2, ws)
+    torch.cuda.synchronize()
+    _close(bf16_dev_to_f64(y2), ref, f"{fmt} split M={M}, repeated")
+
+
 @pytest.mark.parametrize("fmt", ["int2", "int4"])
 @pytest.mark.parametrize("N,K,M", [(5120, 17408, 1), (5120, 17408, 6), (5120, 5120, 3)])
 def test_linear_decoder_layer_shapes_sampled_rows(qm, fmt, N, K, M):
