@@ -26,7 +26,7 @@ from __future__ import annotations
 import dataclasses
 import numpy as np
 
-TAG_FC1, TAG_FC2, TAG_B1, TAG_B2, TAG_X, TAG_LOGITS, TAG_HOT, TAG_ZIPF, TAG_LINEAR = range(9)
+TAG_FC1, TAG_FC2, TAG_B1, TAG_B2, TAG_X, TAG_LOGITS, TAG_HOT, TAG_ZIPF, TAG_LINEAR, TAG_SIGNS = range(10)
 
 
 def f32_to_bf16_bits(a) -> np.ndarray:
@@ -136,3 +136,9 @@ def shared_logit_tokens(cfg: MoEConfig, seed: int, M: int) -> np.ndarray:
 def linear_weight(seed: int, N: int, K: int, std: float = 0.02, index: int = 0) -> np.ndarray:
     """Single quantized linear: bf16 bits [N, K]."""
     return normal_bf16(seed, TAG_LINEAR, index, (N, K), std)
+
+
+def rht_signs(seed: int, H: int) -> np.ndarray:
+    """The random signs d [H] (float32, +1 or -1) of the channel layer's
+    randomized Hadamard rotation: a draw the method makes once at load time."""
+    return np.where(_rng(seed, TAG_SIGNS).random(H) < 0.5, -1.0, 1.0).astype(np.float32)
