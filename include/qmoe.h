@@ -237,6 +237,82 @@ qmoe_status qmoe_linear_workspace_size(int N, int K, int M, size_t* bytes);
 qmoe_status qmoe_linear(const qmoe_weights* w, int N, int K, const uint16_t* x, int M,
                         uint16_t* y, void* ws, size_t ws_bytes, void* stream);
 
+/* ---- Top-k channel-selective MoE layer ----
+ * "Skip MoE channels for up to 2.69x faster MoE blocks - top-k channel
+ * selection" explainer: sketch paragraph (each gate and up row rotated by a
+ * randomized Hadamard transform, then three values plus one scale per block
+ * of 128 weights), scoring paragraph (score = router weight x down-column
+ * norm x |estimated activation|; channels of all routed experts compete in
+ * one top-k; the winners are read in full and computed exactly),
+ * choosing-k paragraph (a fixed number of channels per token).
+ *
+ * Channel record, one per expert channel j (record_bytes, a multiple of 16):
+ * gate row j (FC1 row 2j) codes, H * fmt1 / 8 bytes; up row j (FC1 row 2j+1)
+ * codes; down column j (W2[:, j]) codes, H * fmt2 / 8 bytes; then bf16
+ * scales: gate [H / block], up [H / block], down [H / block]; zero padding.
+ * Codes are symmetric INT2 / INT4 (stored c + 2^(bits-1)), code i of a row at
+ * bit i * bits of its little-endian bytes.  The down column is quantized in
+ * blocks of `block` rows (qmoe_pack's FC2 blocks run along I instead), so
+ * that one channel is one contiguous read.
+ * Sketch record, one per routed expert channel (sketch_bytes, a multiple of
+ * 16): the trits t of the rotated gate row, then of the rotated up row, 2 bits
+ * each (stored t + 2), same bit order; then bf16 scales, gate [H / 128] and
+ * up [H / 128].  Rotation: v' = Had_H (d * v) / sqrt(H), Had_H the Sylvester
+ * Hadamard matrix, d the caller's signs.  Ternary rule per block of 128:
+ * threshold 0.7 * mean|v'|, t = sign(v') where |v'| exceeds it, else 0;
+ * scale = bf16 of the mean |v'| above the threshold (0 if none).
+ * dn[j]: fp32 of the Euclidean norm of the dequantized down column j.
+ * fmt1, fmt2: QMOE_INT2 or QMOE_INT4 (else QMOE_ERR_INVALID_ARG); block 64 or
+ * 128, H a power of two in 512..4096 (else QMOE_ERR_UNSUPPORTED). */
+qmoe_status qmoe_chan_sizes(int fmt1, int fmt2, int H, int block, size_t* record_bytes,
+                            size_t* sketch_bytes);
+
+/* Host: quantize and pack the I channels of one expert.  w1 [2I, H] bf16 (row
+ * 2j gate j, row 2j+1 up j), w2 [H, I] bf16.  records: I * record_bytes.
+ * sketch (I * sketch_bytes) and dn (I floats) may be NULL: shared experts
+ * need neither.  signs [H]: +1.0f or -1.0f (else QMOE_ERR_INVALID_ARG),
+ * needed with a sketch.  QMOE_ERR_INVALID_ARG also for a non-finite norm. */
+qmoe_status qmoe_chan_pack(int fmt1, int fmt2, int H, int I, int block, const uint16_t* w1,
+                           const uint16_t* w2, const float* signs, void* records, void* sketch,
+                           float* dn);
+
+/* A channel layer on the device.  records: [E + n_shared][I] channel records
+ * (shared experts after the routed ones), 16-byte aligned; sketch: [E][I]
+ * sketch records, 16-byte aligned; dn: [E][I]; signs: [H], the signs the
+ * sketch was built with.  1 <= k <= 8, k <= E <= 256, k * I <= 32768. */
+typedef struct {
+  int H, I, E, k, n_shared;
+  int fmt1, fmt2, block;
+  const void* records;
+  const void* sketch;
+  const float* dn;
+  const float* signs;
+} qmoe_chan_layer;
+
+/* Workspace of qmoe_chan_forward for T tokens and n_keep channels per token. */
+qmoe_status qmoe_chan_workspace_size(const qmoe_chan_layer* layer, int T, int n_keep, size_t* bytes);
+
+/* y[T, H] bf16 = for each token, the sum over its n_keep best channels (among
+ * the k * I channels of its routed experts, flat index s * I + j with s the
+ * routing slot; score descending, ties to the lower index) of
+ * w_{t,s} * silu(g_j) * u_j * W2_e[:, j] with g_j, u_j the exact gate and up
+ * products, plus the shared experts in full (weight 1).  Routing as
+ * qmoe_route: top-k of the fp32 logits (finite), ties to the lower expert,
+ * softmax over the k.  1 <= T <= 8, 0 <= n_keep <= k * I; x 16-byte aligned.
+ * Scores are computed in fp32 and ranked on their fp32 values.
+ * Optional device outputs (NULL to skip, 4-byte aligned): sel[T][n_keep]
+ * int32, the selected flat indices in ascending order; scores[T][k * I]
+ * fp32.  ws: device, 256-byte aligned, at least qmoe_chan_workspace_size()
+ * bytes (else QMOE_ERR_SCRATCH); no initial contents needed.  Three kernels:
+ * scoring (routing, rotation, sketch products), selection (one block per
+ * token; skipped when n_keep = 0), exact read and combine.  Partial outputs
+ * are summed with fp32 atomic adds, so the last bit of y can vary between
+ * runs.  A bounded wait that runs out sets QMOE_DEVICE_TIMEOUT and leaves y
+ * unwritten. */
+qmoe_status qmoe_chan_forward(const qmoe_chan_layer* layer, const uint16_t* x, const float* logits,
+                              int T, int n_keep, uint16_t* y, int32_t* sel, float* scores, void* ws,
+                              size_t ws_bytes, void* stream);
+
 /* Per-launch GPU timing (tracing).  After qmoe_trace_start(cap) every kernel
  * the library launches - also while the stream is being captured into a CUDA
  * graph - is bracketed by CUDA events, up to cap launches; qmoe_trace_stop()

@@ -131,6 +131,11 @@ __device__ __forceinline__ void cp_async_arrive(uint64_t* bar) {
 // Waits until every cp.async this thread issued has landed.
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
+// Programmatic dependent launch: wait for the previous kernel in the stream
+// (and its memory), and let the next one start launching.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // Atomic add with acquire-release semantics at GPU scope; returns the old value.
 __device__ __forceinline__ int atomic_add_acq_rel_gpu(int* p, int v) {
   int old;

@@ -343,4 +343,131 @@ qmoe_status qmoe_unpack_host(int fmt, int row_order, const void* codes, const vo
   return QMOE_OK;
 }
 
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Channel layer (top-k channel-selective read): one record per channel holding
+// its gate row, up row and down column, and a 2-bit ternary sketch of the
+// rotated gate and up rows.  Layouts are stated in qmoe.h.
+namespace {
+
+bool chan_fmt_ok(int f) { return f == QMOE_INT2 || f == QMOE_INT4; }
+
+qmoe_status chan_check(int fmt1, int fmt2, int H, int block) {
+  if (!chan_fmt_ok(fmt1) || !chan_fmt_ok(fmt2)) return QMOE_ERR_INVALID_ARG;
+  if (block != 64 && block != 128) return QMOE_ERR_UNSUPPORTED;
+  if (H < 512 || H > 4096 || (H & (H - 1))) return QMOE_ERR_UNSUPPORTED;
+  return QMOE_OK;
+}
+
+size_t align16(size_t v) { return (v + 15) / 16 * 16; }
+
+// Ternary rule of quantize_block on float64 inputs (the rotated rows are not bf16).
+uint16_t ternary_block_f64(const double* w, int B, int8_t* c) {
+  double sum_abs = 0.0;
+  for (int i = 0; i < B; ++i) sum_abs += std::fabs(w[i]);
+  const double delta = 0.7 * (sum_abs / (double)B);
+  double sel = 0.0;
+  int cnt = 0;
+  for (int i = 0; i < B; ++i) {
+    const double a = std::fabs(w[i]);
+    if (a > delta) {
+      c[i] = w[i] > 0 ? 1 : -1;
+      sel += a;
+      ++cnt;
+    } else {
+      c[i] = 0;
+    }
+  }
+  return cnt ? double_to_bf16(sel / (double)cnt) : 0;
+}
+
+// In-place fast Walsh-Hadamard transform in Sylvester order, then one scaling
+// by 1/sqrt(n).  On bf16 inputs every partial sum is exact in float64.
+void fwht_scaled(double* v, int n) {
+  for (int len = 1; len < n; len <<= 1)
+    for (int i = 0; i < n; i += 2 * len)
+      for (int j = i; j < i + len; ++j) {
+        const double a = v[j], b = v[j + len];
+        v[j] = a + b;
+        v[j + len] = a - b;
+      }
+  const double r = 1.0 / std::sqrt((double)n);
+  for (int i = 0; i < n; ++i) v[i] *= r;
+}
+
+// Packs `n` codes (signed c, stored as c + bias) of `bits` bits little-endian into `out`.
+void put_codes(uint8_t* out, const int8_t* c, int n, int bits, int bias) {
+  uint32_t* wd = reinterpret_cast<uint32_t*>(out);
+  const int per = 32 / bits;
+  std::memset(out, 0, (size_t)n * bits / 8);
+  for (int i = 0; i < n; ++i) wd[i / per] |= (uint32_t)(c[i] + bias) << ((i % per) * bits);
+}
+
+}  // namespace
+
+extern "C" {
+
+qmoe_status qmoe_chan_sizes(int fmt1, int fmt2, int H, int block, size_t* record_bytes, size_t* sketch_bytes) {
+  qmoe_status st = chan_check(fmt1, fmt2, H, block);
+  if (st != QMOE_OK) return st;
+  if (record_bytes) *record_bytes = align16((size_t)2 * H * fmt1 / 8 + (size_t)H * fmt2 / 8 + 3 * (size_t)(H / block) * 2);
+  if (sketch_bytes) *sketch_bytes = align16((size_t)2 * H / 4 + 2 * (size_t)(H / 128) * 2);
+  return QMOE_OK;
+}
+
+qmoe_status qmoe_chan_pack(int fmt1, int fmt2, int H, int I, int block, const uint16_t* w1, const uint16_t* w2,
+                           const float* signs, void* records, void* sketch, float* dn) {
+  size_t R = 0, SK = 0;
+  qmoe_status st = qmoe_chan_sizes(fmt1, fmt2, H, block, &R, &SK);
+  if (st != QMOE_OK) return st;
+  if (I <= 0 || !w1 || !w2 || !records || (sketch && !signs)) return QMOE_ERR_INVALID_ARG;
+  if (sketch)
+    for (int i = 0; i < H; ++i)
+      if (signs[i] != 1.0f && signs[i] != -1.0f) return QMOE_ERR_INVALID_ARG;
+  const int SB = H / block, SKB = H / 128;
+  const size_t off_u = (size_t)H * fmt1 / 8, off_d = 2 * off_u, off_s = off_d + (size_t)H * fmt2 / 8;
+  uint8_t* rec = static_cast<uint8_t*>(records);
+  uint8_t* sk = static_cast<uint8_t*>(sketch);
+  bool bad = false;
+#pragma omp parallel for schedule(static)
+  for (int j = 0; j < I; ++j) {
+    std::vector<int8_t> c(H);
+    std::vector<uint16_t> col(H);
+    std::vector<double> rot(H);
+    uint8_t* r = rec + (size_t)j * R;
+    std::memset(r, 0, R);
+    uint16_t* sc = reinterpret_cast<uint16_t*>(r + off_s);  // gate, up, down scales
+    for (int which = 0; which < 2; ++which) {               // 0: gate row 2j, 1: up row 2j+1
+      const uint16_t* row = w1 + (size_t)(2 * j + which) * H;
+      for (int b = 0; b < SB; ++b) sc[which * SB + b] = quantize_block(fmt1, row + (size_t)b * block, block, &c[(size_t)b * block]);
+      put_codes(r + which * off_u, c.data(), H, fmt1, 1 << (fmt1 - 1));
+      if (sk) {
+        for (int i = 0; i < H; ++i) rot[i] = bf16_to_double(row[i]) * (double)signs[i];
+        fwht_scaled(rot.data(), H);
+        uint8_t* s = sk + (size_t)j * SK;
+        uint16_t* ss = reinterpret_cast<uint16_t*>(s + (size_t)H / 2);
+        for (int b = 0; b < SKB; ++b) ss[which * SKB + b] = ternary_block_f64(&rot[(size_t)b * 128], 128, &c[(size_t)b * 128]);
+        put_codes(s + which * (size_t)H / 4, c.data(), H, 2, 2);
+      }
+    }
+    for (int i = 0; i < H; ++i) col[i] = w2[(size_t)i * I + j];
+    double ss = 0.0;
+    for (int b = 0; b < SB; ++b) {
+      const uint16_t s = quantize_block(fmt2, &col[(size_t)b * block], block, &c[(size_t)b * block]);
+      sc[2 * SB + b] = s;
+      const double sd = bf16_to_double(s);
+      for (int i = 0; i < block; ++i) {
+        const double v = (double)c[(size_t)b * block + i] * sd;
+        ss += v * v;
+      }
+    }
+    put_codes(r + off_d, c.data(), H, fmt2, 1 << (fmt2 - 1));
+    if (dn) dn[j] = (float)std::sqrt(ss);
+    if (!std::isfinite(ss)) bad = true;
+  }
+  return bad ? QMOE_ERR_INVALID_ARG : QMOE_OK;
+}
+
 }  // extern "C"

@@ -19,6 +19,7 @@
 #include "qmm_small.cuh"
 #include "qmm_grouped.cuh"
 #include "kernels_misc.cuh"
+#include "chan.cuh"
 #include "slice.h"
 
 #include <cudaTypedefs.h>
@@ -60,12 +61,13 @@ qmoe_status dev_info(DevInfo** out) {
 
 // ---- tracing: CUDA events around each kernel launch ----
 enum KernelId { K_ROUTE = 0, K_GATHER, K_FC1_SMALL, K_FC2_SMALL, K_COMBINE, K_LINEAR_SMALL, K_LINEAR_SETUP,
-                K_DEQUANT, K_FC1_GROUPED, K_FC2_GROUPED, K_DECODE_RESET, K_DECODE_LAYER, K_LINEAR_GROUPED, K_COUNT };
+                K_DEQUANT, K_FC1_GROUPED, K_FC2_GROUPED, K_DECODE_RESET, K_DECODE_LAYER, K_LINEAR_GROUPED,
+                K_CHAN_SCORE, K_CHAN_SELECT, K_CHAN_EXACT, K_COUNT };
 // K_DECODE_RESET / K_DECODE_LAYER: slice_reset_kernel / qmm_slice_kernel (the decode layer)
 const char* const kKernelNames[K_COUNT] = {"route",        "gather",      "fc1_small",    "fc2_small",
                                            "combine",      "linear_small", "linear_setup", "dequant",
                                            "fc1_grouped",  "fc2_grouped", "decode_reset", "decode_layer",
-                                           "linear_grouped"};
+                                           "linear_grouped", "chan_score", "chan_select", "chan_exact"};
 struct Tracer {
   bool on = false;
   int cap = 0, n = 0;
@@ -395,6 +397,74 @@ qmoe_status check_layer(const qmoe_layer* L) {
   if (s != QMOE_OK) return s;
   s = check_weights(L->fc2, L->H, L->I);
   return s;
+}
+
+
+// ---- channel layer (top-k channel-selective read) ----
+struct ChanPlan {
+  size_t ids, wts, scores, sel, yacc, ticket, total;
+};
+
+ChanPlan chan_plan(const qmoe_chan_layer& L, int T, int n_keep) {
+  ChanPlan c;
+  size_t o = 0;
+  c.ids = o;
+  o += align_up((size_t)T * L.k * 4);
+  c.wts = o;
+  o += align_up((size_t)T * L.k * 4);
+  c.scores = o;
+  o += align_up((size_t)T * L.k * L.I * 4);
+  c.sel = o;
+  o += align_up((size_t)T * std::max(n_keep, 1) * 4);
+  c.yacc = o;
+  o += align_up((size_t)T * L.H * 4);
+  c.ticket = o;
+  o += align_up(2 * 4);
+  c.total = o;
+  return c;
+}
+
+qmoe_status chan_check(const qmoe_chan_layer* L, size_t* rec, size_t* sk) {
+  if (!L) return QMOE_ERR_INVALID_ARG;
+  if (L->k < 1 || L->k > kChanMaxK || L->E < L->k || L->E > 256 || L->I < 1 || L->n_shared < 0)
+    return QMOE_ERR_INVALID_ARG;
+  if ((size_t)L->k * L->I > (size_t)kChanMaxCand) return QMOE_ERR_UNSUPPORTED;
+  qmoe_status s = qmoe_chan_sizes(L->fmt1, L->fmt2, L->H, L->block, rec, sk);
+  if (s != QMOE_OK) return s;
+  if (!L->records || !L->sketch || !L->dn || !L->signs) return QMOE_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(L->records) | reinterpret_cast<uintptr_t>(L->sketch)) & 15)
+    return QMOE_ERR_INVALID_ARG;
+  return QMOE_OK;
+}
+
+size_t align_to(size_t v, size_t a) { return (v + a - 1) / a * a; }
+// Dynamic shared memory of the score and exact kernels (as laid out in chan.cuh), with
+// slack for aligning the wave buffer to 128 bytes.
+size_t chan_score_smem(int T, int H, int wave, int skb) {
+  return align_to(4 * ((size_t)T * H + (size_t)T * (H / 16)), 16) + 8 * (size_t)wave + 256 + (size_t)wave * skb;
+}
+int chan_tm(int T) { return T == 1 ? 1 : kChanMaxT; }
+size_t chan_exact_smem(int T, int H, int f1, int wave, int R) {
+  const size_t nc = (size_t)H / (128 / f1);
+  return align_to(4 * ((size_t)T * H + T * nc + (size_t)wave * chan_tm(T) + 2 * (size_t)wave), 16) +
+         8 * (size_t)wave + 256 + (size_t)wave * R;
+}
+constexpr size_t kChanSmemBudget = kSmemLimit - 8 * 1024;  // static shared memory of the kernels
+
+template <int TM>
+void (*chan_exact_of(int f1, int f2))(ChanParams) {
+  if (f1 == QMOE_INT4 && f2 == QMOE_INT4) return chan_exact_kernel<4, 4, TM>;
+  if (f1 == QMOE_INT4 && f2 == QMOE_INT2) return chan_exact_kernel<4, 2, TM>;
+  if (f1 == QMOE_INT2 && f2 == QMOE_INT4) return chan_exact_kernel<2, 4, TM>;
+  return chan_exact_kernel<2, 2, TM>;
+}
+
+qmoe_status launch_chan_exact(int f1, int f2, const ChanParams& p, int grid, size_t smem, cudaStream_t st) {
+  void (*k)(ChanParams) = chan_tm(p.T) == 1 ? chan_exact_of<1>(f1, f2) : chan_exact_of<kChanMaxT>(f1, f2);
+  if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return QMOE_ERR_CUDA;
+  TraceScope ts(st, K_CHAN_EXACT);
+  return launch_pdl(k, dim3(grid), dim3(kChanThreads), smem, st, p) == cudaSuccess ? QMOE_OK : QMOE_ERR_CUDA;
 }
 
 }  // namespace
@@ -816,6 +886,107 @@ qmoe_status qmoe_dequant(const qmoe_weights* w, int rows, int K, int n_mats, flo
     dequant_kernel<3><<<grid, 256, 0, st>>>(c, cs, sc, nullptr, ss, rows / 16, K, w->block, row_order, n_mats,
                                             out_f32, out_bf16);
   return cudaGetLastError() == cudaSuccess ? QMOE_OK : QMOE_ERR_CUDA;
+}
+
+qmoe_status qmoe_chan_workspace_size(const qmoe_chan_layer* layer, int T, int n_keep, size_t* bytes) {
+  size_t rec, sk;
+  qmoe_status s = chan_check(layer, &rec, &sk);
+  if (s != QMOE_OK) return s;
+  if (T < 1 || T > kChanMaxT || n_keep < 0 || n_keep > layer->k * layer->I || !bytes) return QMOE_ERR_INVALID_ARG;
+  *bytes = chan_plan(*layer, T, n_keep).total;
+  return QMOE_OK;
+}
+
+qmoe_status qmoe_chan_forward(const qmoe_chan_layer* layer, const uint16_t* x, const float* logits, int T,
+                              int n_keep, uint16_t* y, int32_t* sel, float* scores, void* ws, size_t ws_bytes,
+                              void* stream) {
+  size_t rec, sk;
+  qmoe_status s = chan_check(layer, &rec, &sk);
+  if (s != QMOE_OK) return s;
+  const qmoe_chan_layer& L = *layer;
+  if (!x || !logits || !y || !ws || T < 1 || T > kChanMaxT || n_keep < 0 || n_keep > L.k * L.I)
+    return QMOE_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(ws) % kAlign) || (reinterpret_cast<uintptr_t>(scores) & 3) ||
+      (reinterpret_cast<uintptr_t>(sel) & 3))
+    return QMOE_ERR_INVALID_ARG;
+  const ChanPlan plan = chan_plan(L, T, n_keep);
+  if (ws_bytes < plan.total) return QMOE_ERR_SCRATCH;
+  DevInfo* di;
+  s = dev_info(&di);
+  if (s != QMOE_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  ChanParams p = {};
+  p.H = L.H;
+  p.I = L.I;
+  p.E = L.E;
+  p.k = L.k;
+  p.S = L.n_shared;
+  p.T = T;
+  p.fmt1 = L.fmt1;
+  p.fmt2 = L.fmt2;
+  p.block = L.block;
+  p.rec_bytes = (int)rec;
+  p.sk_bytes = (int)sk;
+  p.rec = static_cast<const uint8_t*>(L.records);
+  p.sketch = static_cast<const uint8_t*>(L.sketch);
+  p.dn = L.dn;
+  p.signs = L.signs;
+  p.x = x;
+  p.logits = logits;
+  p.n_keep = n_keep;
+  p.ids = reinterpret_cast<int*>(w + plan.ids);
+  p.wts = reinterpret_cast<float*>(w + plan.wts);
+  p.scores = scores ? scores : reinterpret_cast<float*>(w + plan.scores);
+  p.sel = sel ? sel : reinterpret_cast<int*>(w + plan.sel);
+  p.yacc = reinterpret_cast<float*>(w + plan.yacc);
+  p.ticket = reinterpret_cast<int*>(w + plan.ticket);
+  p.y = y;
+  p.inv_sqrt_h = (float)(1.0 / std::sqrt((double)L.H));
+  p.wait_ns = g_fault_wait_ns;
+  p.status = di->status;
+
+  // scores: every block may hold up to ceil(units / grid) sketch records
+  const int g1 = di->sms;
+  const int units1 = std::min(L.E, T * L.k) * L.I;
+  const size_t fix1 = chan_score_smem(T, L.H, 0, (int)sk);
+  if (fix1 + 2 * sk + 8 > kChanSmemBudget) return QMOE_ERR_UNSUPPORTED;
+  p.wave_sk = (int)std::min<size_t>((units1 + g1 - 1) / g1, (kChanSmemBudget - fix1) / (sk + 8));
+  const size_t smem1 = chan_score_smem(T, L.H, p.wave_sk, (int)sk);
+  // exact: shared channels then the selected ones
+  const int units3 = L.n_shared * L.I + T * n_keep;
+  const int g3 = std::max(1, std::min(di->sms, (units3 + 3) / 4));
+  const size_t fix3 = chan_exact_smem(T, L.H, L.fmt1, 0, (int)rec);
+  const size_t per3 = rec + 8 + 4 * (chan_tm(T) + 2);
+  if (fix3 + 2 * per3 > kChanSmemBudget) return QMOE_ERR_UNSUPPORTED;
+  p.wave_rec = (int)std::max<size_t>(1, std::min<size_t>((units3 + g3 - 1) / g3, (kChanSmemBudget - fix3) / per3));
+  const size_t smem3 = chan_exact_smem(T, L.H, L.fmt1, p.wave_rec, (int)rec);
+  const size_t smem2 = (size_t)L.k * L.I * 4;
+
+  if (cudaFuncSetAttribute(chan_score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem1) !=
+          cudaSuccess ||
+      cudaFuncSetAttribute(chan_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem2) !=
+          cudaSuccess)
+    return QMOE_ERR_CUDA;
+  {
+    TraceScope ts(st, K_CHAN_SCORE);
+    if (launch_pdl(chan_score_kernel, dim3(g1), dim3(kChanThreads), smem1, st, p) != cudaSuccess)
+      return QMOE_ERR_CUDA;
+  }
+  if (n_keep > 0) {
+    TraceScope ts(st, K_CHAN_SELECT);
+    if (launch_pdl(chan_select_kernel, dim3(T), dim3(kSelThreads), smem2, st, p) != cudaSuccess)
+      return QMOE_ERR_CUDA;
+  }
+  s = launch_chan_exact(L.fmt1, L.fmt2, p, g3, smem3, st);
+  if (s != QMOE_OK) return s;
+  std::lock_guard<std::mutex> lk(g_mu);
+  g_stats.last_path = QMOE_PATH_SMALL_M;
+  g_stats.row_tiles = 1;
+  g_stats.row_tile_tokens = T;
+  g_stats.small_launches = n_keep > 0 ? 3 : 2;
+  g_stats.grouped_launches = 0;
+  return QMOE_OK;
 }
 
 }  // extern "C"

@@ -38,6 +38,12 @@ class Layer(C.Structure):
                 ("fc1", Weights), ("fc2", Weights), ("path", C.c_int), ("max_row_tile", C.c_int)]
 
 
+class ChanLayer(C.Structure):
+    _fields_ = [("H", C.c_int), ("I", C.c_int), ("E", C.c_int), ("k", C.c_int), ("n_shared", C.c_int),
+                ("fmt1", C.c_int), ("fmt2", C.c_int), ("block", C.c_int), ("records", C.c_void_p),
+                ("sketch", C.c_void_p), ("dn", C.c_void_p), ("signs", C.c_void_p)]
+
+
 class Stats(C.Structure):
     _fields_ = [("last_path", C.c_int), ("row_tiles", C.c_int), ("row_tile_tokens", C.c_int),
                 ("small_launches", C.c_int), ("grouped_launches", C.c_int), ("device_status", C.c_uint32)]
@@ -69,6 +75,12 @@ EXPORTS = {
     "qmoe_trace_stop": [],
     "qmoe_trace_read": [C.c_int, C.POINTER(C.c_int), C.c_void_p, C.c_void_p],
     "qmoe_kernel_name": [C.c_int],
+    "qmoe_chan_sizes": [C.c_int, C.c_int, C.c_int, C.c_int, C.POINTER(C.c_size_t), C.POINTER(C.c_size_t)],
+    "qmoe_chan_pack": [C.c_int, C.c_int, C.c_int, C.c_int, C.c_int, C.c_void_p, C.c_void_p, C.c_void_p,
+                       C.c_void_p, C.c_void_p, C.c_void_p],
+    "qmoe_chan_workspace_size": [C.POINTER(ChanLayer), C.c_int, C.c_int, C.POINTER(C.c_size_t)],
+    "qmoe_chan_forward": [C.POINTER(ChanLayer), C.c_void_p, C.c_void_p, C.c_int, C.c_int, C.c_void_p,
+                          C.c_void_p, C.c_void_p, C.c_void_p, C.c_size_t, C.c_void_p],
 }
 
 if not os.path.exists(_LIB_PATH):
@@ -174,6 +186,31 @@ def unpack_host(fmt: int, row_order: int, codes: np.ndarray, scales: np.ndarray,
     return c, s
 
 
+def chan_sizes(fmt1: int, fmt2: int, H: int, block: int):
+    """(record_bytes, sketch_bytes) of the channel layer."""
+    r, k = C.c_size_t(), C.c_size_t()
+    _check(_lib.qmoe_chan_sizes(fmt1, fmt2, H, block, C.byref(r), C.byref(k)), "qmoe_chan_sizes")
+    return r.value, k.value
+
+
+def chan_pack(fmt1: int, fmt2: int, w1_bits: np.ndarray, w2_bits: np.ndarray, block: int, signs=None,
+              sketch: bool = True):
+    """Channel records of one expert (w1 [2I, H], w2 [H, I] bf16 bits) -> (records u8 [I * R],
+    sketch u8 [I * SK] or None, dn float32 [I] or None)."""
+    w1 = np.ascontiguousarray(w1_bits, dtype=np.uint16)
+    w2 = np.ascontiguousarray(w2_bits, dtype=np.uint16)
+    two_i, H = w1.shape
+    I = two_i // 2
+    R, SK = chan_sizes(fmt1, fmt2, H, block)
+    rec = np.empty(I * R, dtype=np.uint8)
+    sk = np.empty(I * SK, dtype=np.uint8) if sketch else None
+    dn = np.empty(I, dtype=np.float32) if sketch else None
+    sg = None if signs is None else np.ascontiguousarray(signs, dtype=np.float32)
+    _check(_lib.qmoe_chan_pack(fmt1, fmt2, H, I, block, _ptr(w1), _ptr(w2), _ptr(sg), _ptr(rec), _ptr(sk), _ptr(dn)),
+           "qmoe_chan_pack")
+    return rec, sk, dn
+
+
 # ---------------------------------------------------------------- device entry points
 
 def make_weights(fmt: int, block: int, codes, scales, bias=None, row_order: int = ROWS_PLAIN, zeros=None) -> Weights:
@@ -235,6 +272,24 @@ def linear(w: Weights, N: int, K: int, x, y, ws, ws_bytes: int | None = None, st
     nbytes = ws.numel() * ws.element_size() if ws_bytes is None else ws_bytes
     _check(_lib.qmoe_linear(C.byref(w), N, K, _ptr(x), M, _ptr(y), _ptr(ws), nbytes, _stream(stream)),
            "qmoe_linear")
+
+
+def make_chan_layer(H, I, E, k, n_shared, fmt1, fmt2, block, records, sketch, dn, signs) -> ChanLayer:
+    return ChanLayer(H, I, E, k, n_shared, fmt1, fmt2, block, _ptr(records), _ptr(sketch), _ptr(dn), _ptr(signs))
+
+
+def chan_workspace_size(layer: ChanLayer, T: int, n_keep: int) -> int:
+    b = C.c_size_t()
+    _check(_lib.qmoe_chan_workspace_size(C.byref(layer), T, n_keep, C.byref(b)), "qmoe_chan_workspace_size")
+    return b.value
+
+
+def chan_forward(layer: ChanLayer, x, logits, n_keep: int, y, ws, sel=None, scores=None, ws_bytes: int | None = None,
+                 stream=None):
+    T = x.shape[0]
+    nbytes = ws.numel() * ws.element_size() if ws_bytes is None else ws_bytes
+    _check(_lib.qmoe_chan_forward(C.byref(layer), _ptr(x), _ptr(logits), T, n_keep, _ptr(y), _ptr(sel), _ptr(scores),
+                                  _ptr(ws), nbytes, _stream(stream)), "qmoe_chan_forward")
 
 
 def get_stats() -> Stats:

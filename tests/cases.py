@@ -115,3 +115,50 @@ class MoECase:
 
 def small_cfg(base: synth.MoEConfig, **kw) -> synth.MoEConfig:
     return dataclasses.replace(base, **kw)
+
+
+class ChanCase:
+    """A channel layer (top-k channel-selective read): channel records and
+    sketches packed by the library on the host, and, independently, the
+    oracle's bank built from the same bf16 weights and signs."""
+
+    def __init__(self, cfg: synth.MoEConfig, seed: int = 1):
+        import torch
+        from oracle import channel_select as CS
+        from skinny_gemm_top_b200 import qmoe
+        self.cfg, self.seed = cfg, seed
+        f1, f2 = FMTS[cfg.fc1_fmt], FMTS[cfg.fc2_fmt]
+        self.signs = synth.rht_signs(seed, cfg.H)
+        recs, sks, dns = [], [], []
+        for e in range(cfg.E + cfg.n_shared):
+            routed = e < cfg.E
+            r, s, d = qmoe.chan_pack(f1, f2, synth.expert_fc1(cfg, seed, e), synth.expert_fc2(cfg, seed, e),
+                                     cfg.block, self.signs if routed else None, sketch=routed)
+            recs.append(r)
+            if routed:
+                sks.append(s)
+                dns.append(d)
+        self.dev = {"rec": to_dev(np.concatenate(recs)), "sk": to_dev(np.concatenate(sks)),
+                    "dn": torch.from_numpy(np.concatenate(dns)).cuda(), "signs": torch.from_numpy(self.signs).cuda()}
+        self.layer = qmoe.make_chan_layer(cfg.H, cfg.I, cfg.E, cfg.k, cfg.n_shared, f1, f2, cfg.block,
+                                          self.dev["rec"], self.dev["sk"], self.dev["dn"], self.dev["signs"])
+        self.bank = CS.ChannelExpertBank(
+            cfg.H, cfg.I, cfg.E, cfg.n_shared, cfg.block, f1, f2,
+            lambda e: Q.bf16_bits_to_f64(synth.expert_fc1(cfg, seed, e)),
+            lambda e: Q.bf16_bits_to_f64(synth.expert_fc2(cfg, seed, e)), self.signs)
+
+    def run(self, x_bits: np.ndarray, logits: np.ndarray, n_keep: int, ws_bytes: int | None = None):
+        """(y float64 [T, H], sel [T, n_keep], scores float32 [T, k * I]) from the device."""
+        import torch
+        from skinny_gemm_top_b200 import qmoe
+        T, c = x_bits.shape[0], self.cfg
+        need = qmoe.chan_workspace_size(self.layer, T, n_keep)
+        ws = torch.empty(need if ws_bytes is None else ws_bytes, dtype=torch.uint8, device="cuda")
+        x = to_dev(x_bits)
+        lg = torch.from_numpy(np.ascontiguousarray(logits, dtype=np.float32)).cuda()
+        y = torch.empty((T, c.H), dtype=torch.int16, device="cuda")
+        sel = torch.full((T, max(n_keep, 1)), -1, dtype=torch.int32, device="cuda")
+        sc = torch.empty((T, c.k * c.I), dtype=torch.float32, device="cuda")
+        qmoe.chan_forward(self.layer, x, lg, n_keep, y, ws, sel=sel, scores=sc)
+        torch.cuda.synchronize()
+        return bf16_dev_to_f64(y), sel.cpu().numpy()[:, :n_keep], sc.cpu().numpy()

@@ -145,3 +145,66 @@ def test_fault_hook_validates_host_side():
     with pytest.raises(qmoe.QmoeError):
         qmoe.test_set_fault(5, 0)
     qmoe.test_set_fault(0, 0)
+
+
+# ---------------------------------------------------------------- channel layer packing
+
+def _codes_of(buf: np.ndarray, n: int, bits: int) -> np.ndarray:
+    """Signed codes of a little-endian bit-packed row (stored c + 2^(bits-1))."""
+    words = np.frombuffer(np.ascontiguousarray(buf).tobytes(), dtype="<u4")
+    per = 32 // bits
+    i = np.arange(n)
+    u = (words[i // per] >> ((i % per) * bits).astype(np.uint32)) & ((1 << bits) - 1)
+    return u.astype(np.int64) - (1 << (bits - 1))
+
+
+@pytest.mark.parametrize("f1,f2,block,H,I", [(4, 4, 128, 512, 12), (2, 4, 64, 1024, 5), (2, 2, 128, 512, 3)])
+def test_chan_pack_matches_oracle(f1, f2, block, H, I):
+    from oracle import channel_select as CS
+    w1 = synth.normal_bf16(21, 70, 0, (2 * I, H), 0.02)
+    w2 = synth.normal_bf16(21, 71, 0, (H, I), 0.02)
+    d = synth.rht_signs(21, H)
+    R, SK = qmoe.chan_sizes(f1, f2, H, block)
+    assert R % 16 == 0 and SK % 16 == 0
+    rec, sk, dn = qmoe.chan_pack(f1, f2, w1, w2, block, d)
+    w1d, w2d = Q.bf16_bits_to_f64(w1), Q.bf16_bits_to_f64(w2)
+    cg, sg = Q.quantize_sym(w1d[0::2], f1, block)
+    cu, su = Q.quantize_sym(w1d[1::2], f1, block)
+    cd, sd, w2_hat = CS.quantize_down_columns(w2d, f2, block)
+    tg, stg = CS.sketch_rows(w1d[0::2], d)
+    tu, stu = CS.sketch_rows(w1d[1::2], d)
+    SB, rb1, rb2 = H // block, H * f1 // 8, H * f2 // 8
+    for j in range(I):
+        r = rec[j * R:(j + 1) * R]
+        assert np.array_equal(_codes_of(r[:rb1], H, f1), cg[j])
+        assert np.array_equal(_codes_of(r[rb1:2 * rb1], H, f1), cu[j])
+        assert np.array_equal(_codes_of(r[2 * rb1:2 * rb1 + rb2], H, f2), cd[j])
+        sc = Q.bf16_bits_to_f64(np.frombuffer(r[2 * rb1 + rb2:2 * rb1 + rb2 + 6 * SB].tobytes(), dtype="<u2"))
+        assert np.array_equal(sc, np.concatenate([sg[j], su[j], sd[j]]))
+        assert not r[2 * rb1 + rb2 + 6 * SB:].any()
+        s = sk[j * SK:(j + 1) * SK]
+        assert np.array_equal(_codes_of(s[:H // 4], H, 2), tg[j])
+        assert np.array_equal(_codes_of(s[H // 4:H // 2], H, 2), tu[j])
+        ss = Q.bf16_bits_to_f64(np.frombuffer(s[H // 2:H // 2 + 4 * (H // 128)].tobytes(), dtype="<u2"))
+        assert np.array_equal(ss, np.concatenate([stg[j], stu[j]]))
+    want_dn = np.sqrt((w2_hat * w2_hat).sum(axis=0))
+    assert np.allclose(dn, want_dn, rtol=1e-7, atol=0)
+
+
+def test_chan_pack_without_sketch_and_bad_arguments():
+    H, I = 512, 4
+    w1 = synth.normal_bf16(3, 70, 1, (2 * I, H), 0.02)
+    w2 = synth.normal_bf16(3, 71, 1, (H, I), 0.02)
+    rec, sk, dn = qmoe.chan_pack(4, 4, w1, w2, 64, None, sketch=False)
+    assert sk is None and dn is None and rec.size == I * qmoe.chan_sizes(4, 4, H, 64)[0]
+    for args, st in (((3, 4, 512, 64), qmoe.ERR_INVALID_ARG), ((4, 4, 768, 64), qmoe.ERR_UNSUPPORTED),
+                     ((4, 4, 256, 64), qmoe.ERR_UNSUPPORTED), ((4, 4, 8192, 64), qmoe.ERR_UNSUPPORTED),
+                     ((4, 4, 512, 32), qmoe.ERR_UNSUPPORTED)):
+        with pytest.raises(qmoe.QmoeError) as ei:
+            qmoe.chan_sizes(*args)
+        assert ei.value.status == st
+    bad = np.ones(H, dtype=np.float32)
+    bad[5] = 0.5
+    with pytest.raises(qmoe.QmoeError) as ei:
+        qmoe.chan_pack(4, 4, w1, w2, 64, bad)
+    assert ei.value.status == qmoe.ERR_INVALID_ARG
