@@ -54,6 +54,8 @@ def parse():
                     help="two eager forwards of the prefill layer (T = 4096, one row tile) only, for an ncu capture")
     ap.add_argument("--profile-ternary", action="store_true",
                     help="a few eager forwards of the ternary layer (128 experts, T = 1) only, for an ncu capture")
+    ap.add_argument("--profile-chan", action="store_true",
+                    help="a few eager forwards of the channel-selective layer (V2-Lite, T = 1, 18%%) only, for ncu")
     return ap.parse_args()
 
 
@@ -288,6 +290,99 @@ def run_profile_ternary(args):
     print("ternary profile run done", flush=True)
 
 
+# ------------------------------------------------------------------ channel-selective layer
+
+CHAN_BUDGETS = (0.13, 0.18, 1.0)  # the explainer's 13% and 18% read budgets, and every channel
+
+
+def pack_chan(qmoe, torch, cfg, copies: int = 1):
+    """Channel layer of `cfg` (records, sketches, norms, signs) packed once on the
+    host, `copies` device copies (so that consecutive steps do not reuse L2)."""
+    f1, f2 = qmoe.FMT[cfg.fc1_fmt], qmoe.FMT[cfg.fc2_fmt]
+    signs = synth.rht_signs(SEED, cfg.H)
+    recs, sks, dns = [], [], []
+    for e in range(cfg.E + cfg.n_shared):
+        routed = e < cfg.E
+        r, s, d = qmoe.chan_pack(f1, f2, synth.expert_fc1(cfg, SEED, e), synth.expert_fc2(cfg, SEED, e), cfg.block,
+                                 signs if routed else None, sketch=routed)
+        recs.append(r)
+        if routed:
+            sks.append(s)
+            dns.append(d)
+    host = [np.concatenate(recs), np.concatenate(sks), np.concatenate(dns), signs]
+    layers, keep = [], []
+    for _ in range(copies):
+        dev = [_to_dev(torch, a) for a in host]
+        keep.append(dev)
+        layers.append(qmoe.make_chan_layer(cfg.H, cfg.I, cfg.E, cfg.k, cfg.n_shared, f1, f2, cfg.block, *dev))
+    R, SK = qmoe.chan_sizes(f1, f2, cfg.H, cfg.block)
+    return layers, keep, R, SK
+
+
+def chan_step_bytes(cfg, logits: np.ndarray, n_keep: int, R: int, SK: int) -> int:
+    """Algorithmic bytes of one channel-layer forward: the sketch records and
+    norms of the active routed experts, the selected and shared channel
+    records, x, y and the logits."""
+    T = logits.shape[0]
+    act = set()
+    for t in range(T):
+        act.update(int(e) for e in np.argsort(-logits[t].astype(np.float64), kind="stable")[:cfg.k])
+    return (len(act) * cfg.I * (SK + 4) + T * n_keep * R + cfg.n_shared * cfg.I * R
+            + 2 * T * cfg.H * 2 + T * cfg.E * 4)
+
+
+def chan_sweep(qmoe, torch, dist, args, cfg, Ts, rotate: int = 16, copies: int = 3) -> dict:
+    """The channel-selective layer on `cfg` for each T and read budget."""
+    layers, keep, R, SK = pack_chan(qmoe, torch, cfg, copies)
+    out = {"config": f"{cfg.name}: H={cfg.H} I={cfg.I} E={cfg.E} top-{cfg.k} + {cfg.n_shared} shared, "
+                     f"FC1 {cfg.fc1_fmt} / FC2 {cfg.fc2_fmt} (columns), block {cfg.block}; sketch 2-bit trits, "
+                     f"block 128; {copies} device copies rotated", "record_bytes": R, "sketch_bytes": SK, "runs": []}
+    for T in Ts:
+        xs = [_to_dev(torch, synth.tokens(cfg.H, SEED, T, index=r)) for r in range(rotate)]
+        lgs_np = [synth.router_logits(cfg, SEED, T, index=100 + r) for r in range(rotate)]
+        lgs = [torch.from_numpy(np.ascontiguousarray(l)).cuda() for l in lgs_np]
+        ys = [torch.empty((T, cfg.H), dtype=torch.int16, device="cuda") for _ in range(rotate)]
+        for b in CHAN_BUDGETS:
+            n_keep = int(round(b * cfg.k * cfg.I))
+            ws = torch.empty(qmoe.chan_workspace_size(layers[0], T, n_keep), dtype=torch.uint8, device="cuda")
+            nrot = max(rotate, copies)
+
+            def fn(i, n, xs=xs, lgs=lgs, ys=ys, ws=ws, n_keep=n_keep):
+                r = i % rotate
+                qmoe.chan_forward(layers[i % copies], xs[r], lgs[r], n_keep, ys[r], ws)
+
+            steps = Steps(torch, fn, nrot)
+            k = max(nrot, (args.steps // nrot) * nrot)
+            steps.prepare(k, args.warmup)
+            steps.run(max(args.warmup, 3))
+            ms = reduce_ranks(torch, dist, time_steps(torch, dist, steps, k), 0.0)[0] / k
+            nbytes = statistics.mean(chan_step_bytes(cfg, l, n_keep, R, SK) for l in lgs_np)
+            out["runs"].append({"T": T, "budget": b, "n_keep": n_keep, "us": round(ms * 1e3, 3),
+                                "GBps": round(nbytes / (ms * 1e6), 1), "bytes": int(nbytes)})
+    assert qmoe.get_stats().device_status == 0
+    del keep, layers
+    return out
+
+
+def run_profile_chan(args):
+    """A few eager forwards of the channel-selective layer (V2-Lite shapes, T = 1, 18% of the routed channels)."""
+    import torch
+    from skinny_gemm_top_b200 import qmoe
+    cfg = synth.V2LITE
+    layers, keep, _, _ = pack_chan(qmoe, torch, cfg, 1)
+    n_keep = int(round(0.18 * cfg.k * cfg.I))
+    x = _to_dev(torch, synth.tokens(cfg.H, SEED, 1))
+    ws = torch.empty(qmoe.chan_workspace_size(layers[0], 1, n_keep), dtype=torch.uint8, device="cuda")
+    y = torch.empty((1, cfg.H), dtype=torch.int16, device="cuda")
+    for r in range(max(args.steps, 1)):
+        lg = torch.from_numpy(np.ascontiguousarray(synth.router_logits(cfg, SEED, 1, index=100 + r))).cuda()
+        qmoe.chan_forward(layers[0], x, lg, n_keep, y, ws)
+        torch.cuda.synchronize()
+    assert qmoe.get_stats().device_status == 0
+    del keep
+    print("channel profile run done", flush=True)
+
+
 def run_ours(args):
     import torch
     from skinny_gemm_top_b200 import qmoe
@@ -374,6 +469,8 @@ def run_ours(args):
                                               distinct=8)
     prefill = [] if args.quick else cfg_sweep(qmoe, torch, dist, args, synth.PREFILL, (4096,), rotate=1,
                                               ws_cap=256 << 20)
+    # the channel-selective layer on the V2-Lite shapes (13% / 18% / all routed channels)
+    chan = [] if args.quick else chan_sweep(qmoe, torch, dist, args, synth.V2LITE, (1, 2, 4, 8))
     e2e = measure_e2e(qmoe, torch, dist, layers[0], args.steps, args.warmup)
 
     peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json"))) if os.path.exists(
@@ -446,6 +543,7 @@ def run_ours(args):
         "v2lite_decode_batches": v2lite_batches,
         "ternary_layer": ternary,
         "prefill_layer": prefill,
+        "channel_select_layer": chan,
         "e2e": e2e,
         "gpu_launches": head["launches_per_step"] * args.steps,
         "clocks": clocks,
@@ -775,6 +873,8 @@ def main():
         run_profile_prefill(args)
     elif args.profile_ternary:
         run_profile_ternary(args)
+    elif args.profile_chan:
+        run_profile_chan(args)
     else:
         run_ours(args)
 

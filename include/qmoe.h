@@ -263,7 +263,7 @@ qmoe_status qmoe_linear(const qmoe_weights* w, int N, int K, const uint16_t* x, 
  * scale = bf16 of the mean |v'| above the threshold (0 if none).
  * dn[j]: fp32 of the Euclidean norm of the dequantized down column j.
  * fmt1, fmt2: QMOE_INT2 or QMOE_INT4 (else QMOE_ERR_INVALID_ARG); block 64 or
- * 128, H a power of two in 512..4096 (else QMOE_ERR_UNSUPPORTED). */
+ * 128, H a power of two in 512..2048 (else QMOE_ERR_UNSUPPORTED). */
 qmoe_status qmoe_chan_sizes(int fmt1, int fmt2, int H, int block, size_t* record_bytes,
                             size_t* sketch_bytes);
 
@@ -278,8 +278,8 @@ qmoe_status qmoe_chan_pack(int fmt1, int fmt2, int H, int I, int block, const ui
 
 /* A channel layer on the device.  records: [E + n_shared][I] channel records
  * (shared experts after the routed ones), 16-byte aligned; sketch: [E][I]
- * sketch records, 16-byte aligned; dn: [E][I]; signs: [H], the signs the
- * sketch was built with.  1 <= k <= 8, k <= E <= 256, k * I <= 32768. */
+ * sketch records, 16-byte aligned; dn: [E][I]; signs: [H], 16-byte aligned,
+ * the signs the sketch was built with.  1 <= k <= 8, k <= E <= 256, k * I <= 32768. */
 typedef struct {
   int H, I, E, k, n_shared;
   int fmt1, fmt2, block;

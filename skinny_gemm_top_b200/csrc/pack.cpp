@@ -357,7 +357,7 @@ bool chan_fmt_ok(int f) { return f == QMOE_INT2 || f == QMOE_INT4; }
 qmoe_status chan_check(int fmt1, int fmt2, int H, int block) {
   if (!chan_fmt_ok(fmt1) || !chan_fmt_ok(fmt2)) return QMOE_ERR_INVALID_ARG;
   if (block != 64 && block != 128) return QMOE_ERR_UNSUPPORTED;
-  if (H < 512 || H > 4096 || (H & (H - 1))) return QMOE_ERR_UNSUPPORTED;
+  if (H < 512 || H > 2048 || (H & (H - 1))) return QMOE_ERR_UNSUPPORTED;
   return QMOE_OK;
 }
 

@@ -62,12 +62,13 @@ qmoe_status dev_info(DevInfo** out) {
 // ---- tracing: CUDA events around each kernel launch ----
 enum KernelId { K_ROUTE = 0, K_GATHER, K_FC1_SMALL, K_FC2_SMALL, K_COMBINE, K_LINEAR_SMALL, K_LINEAR_SETUP,
                 K_DEQUANT, K_FC1_GROUPED, K_FC2_GROUPED, K_DECODE_RESET, K_DECODE_LAYER, K_LINEAR_GROUPED,
-                K_CHAN_SCORE, K_CHAN_SELECT, K_CHAN_EXACT, K_COUNT };
+                K_CHAN_SCORE, K_CHAN_SELECT, K_CHAN_EXACT, K_CHAN_RESET, K_COUNT };
 // K_DECODE_RESET / K_DECODE_LAYER: slice_reset_kernel / qmm_slice_kernel (the decode layer)
 const char* const kKernelNames[K_COUNT] = {"route",        "gather",      "fc1_small",    "fc2_small",
                                            "combine",      "linear_small", "linear_setup", "dequant",
                                            "fc1_grouped",  "fc2_grouped", "decode_reset", "decode_layer",
-                                           "linear_grouped", "chan_score", "chan_select", "chan_exact"};
+                                           "linear_grouped", "chan_score", "chan_select", "chan_exact",
+                                           "chan_reset"};
 struct Tracer {
   bool on = false;
   int cap = 0, n = 0;
@@ -402,7 +403,7 @@ qmoe_status check_layer(const qmoe_layer* L) {
 
 // ---- channel layer (top-k channel-selective read) ----
 struct ChanPlan {
-  size_t ids, wts, scores, sel, yacc, ticket, total;
+  size_t ids, wts, scores, sel, hist, yacc, ticket, total;  // hist and yacc adjacent (one reset)
 };
 
 ChanPlan chan_plan(const qmoe_chan_layer& L, int T, int n_keep) {
@@ -416,6 +417,8 @@ ChanPlan chan_plan(const qmoe_chan_layer& L, int T, int n_keep) {
   o += align_up((size_t)T * L.k * L.I * 4);
   c.sel = o;
   o += align_up((size_t)T * std::max(n_keep, 1) * 4);
+  c.hist = o;
+  o += (size_t)T * kChanBins * 4;
   c.yacc = o;
   o += align_up((size_t)T * L.H * 4);
   c.ticket = o;
@@ -431,8 +434,10 @@ qmoe_status chan_check(const qmoe_chan_layer* L, size_t* rec, size_t* sk) {
   if ((size_t)L->k * L->I > (size_t)kChanMaxCand) return QMOE_ERR_UNSUPPORTED;
   qmoe_status s = qmoe_chan_sizes(L->fmt1, L->fmt2, L->H, L->block, rec, sk);
   if (s != QMOE_OK) return s;
+  if (L->H > kChanMaxH) return QMOE_ERR_UNSUPPORTED;
   if (!L->records || !L->sketch || !L->dn || !L->signs) return QMOE_ERR_INVALID_ARG;
-  if ((reinterpret_cast<uintptr_t>(L->records) | reinterpret_cast<uintptr_t>(L->sketch)) & 15)
+  if ((reinterpret_cast<uintptr_t>(L->records) | reinterpret_cast<uintptr_t>(L->sketch) |
+       reinterpret_cast<uintptr_t>(L->signs)) & 15)
     return QMOE_ERR_INVALID_ARG;
   return QMOE_OK;
 }
@@ -443,7 +448,7 @@ size_t align_to(size_t v, size_t a) { return (v + a - 1) / a * a; }
 size_t chan_score_smem(int T, int H, int wave, int skb) {
   return align_to(4 * ((size_t)T * H + (size_t)T * (H / 16)), 16) + 8 * (size_t)wave + 256 + (size_t)wave * skb;
 }
-int chan_tm(int T) { return T == 1 ? 1 : kChanMaxT; }
+int chan_tm(int T) { return T <= 1 ? 1 : T <= 2 ? 2 : T <= 4 ? 4 : 8; }
 size_t chan_exact_smem(int T, int H, int f1, int wave, int R) {
   const size_t nc = (size_t)H / (128 / f1);
   return align_to(4 * ((size_t)T * H + T * nc + (size_t)wave * chan_tm(T) + 2 * (size_t)wave), 16) +
@@ -460,7 +465,11 @@ void (*chan_exact_of(int f1, int f2))(ChanParams) {
 }
 
 qmoe_status launch_chan_exact(int f1, int f2, const ChanParams& p, int grid, size_t smem, cudaStream_t st) {
-  void (*k)(ChanParams) = chan_tm(p.T) == 1 ? chan_exact_of<1>(f1, f2) : chan_exact_of<kChanMaxT>(f1, f2);
+  const int tm = chan_tm(p.T);
+  void (*k)(ChanParams) = tm == 1   ? chan_exact_of<1>(f1, f2)
+                          : tm == 2 ? chan_exact_of<2>(f1, f2)
+                          : tm == 4 ? chan_exact_of<4>(f1, f2)
+                                    : chan_exact_of<8>(f1, f2);
   if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return QMOE_ERR_CUDA;
   TraceScope ts(st, K_CHAN_EXACT);
@@ -939,6 +948,7 @@ qmoe_status qmoe_chan_forward(const qmoe_chan_layer* layer, const uint16_t* x, c
   p.wts = reinterpret_cast<float*>(w + plan.wts);
   p.scores = scores ? scores : reinterpret_cast<float*>(w + plan.scores);
   p.sel = sel ? sel : reinterpret_cast<int*>(w + plan.sel);
+  p.hist = reinterpret_cast<int*>(w + plan.hist);
   p.yacc = reinterpret_cast<float*>(w + plan.yacc);
   p.ticket = reinterpret_cast<int*>(w + plan.ticket);
   p.y = y;
@@ -961,16 +971,27 @@ qmoe_status qmoe_chan_forward(const qmoe_chan_layer* layer, const uint16_t* x, c
   if (fix3 + 2 * per3 > kChanSmemBudget) return QMOE_ERR_UNSUPPORTED;
   p.wave_rec = (int)std::max<size_t>(1, std::min<size_t>((units3 + g3 - 1) / g3, (kChanSmemBudget - fix3) / per3));
   const size_t smem3 = chan_exact_smem(T, L.H, L.fmt1, p.wave_rec, (int)rec);
-  const size_t smem2 = (size_t)L.k * L.I * 4;
 
-  if (cudaFuncSetAttribute(chan_score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem1) !=
-          cudaSuccess ||
+  const int tm = chan_tm(T);
+  void (*score)(ChanParams) = tm == 1   ? chan_score_kernel<1>
+                              : tm == 2 ? chan_score_kernel<2>
+                              : tm == 4 ? chan_score_kernel<4>
+                                        : chan_score_kernel<8>;
+  const size_t smem2 = (size_t)L.k * L.I * 4;
+  if (cudaFuncSetAttribute(score, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem1) != cudaSuccess ||
       cudaFuncSetAttribute(chan_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem2) !=
           cudaSuccess)
     return QMOE_ERR_CUDA;
+  {  // the selection histogram, the output accumulator and the tickets start at zero
+    const int n4 = (int)(((size_t)T * kChanBins + (size_t)T * L.H) / 4);
+    TraceScope ts(st, K_CHAN_RESET);
+    if (launch_pdl(accum_reset_kernel, dim3(std::max(1, std::min(di->sms, (n4 + 255) / 256))), dim3(256), 0, st,
+                   reinterpret_cast<float*>(p.hist), n4, p.ticket, 2) != cudaSuccess)
+      return QMOE_ERR_CUDA;
+  }
   {
     TraceScope ts(st, K_CHAN_SCORE);
-    if (launch_pdl(chan_score_kernel, dim3(g1), dim3(kChanThreads), smem1, st, p) != cudaSuccess)
+    if (launch_pdl(score, dim3(g1), dim3(kChanThreads), smem1, st, p) != cudaSuccess)
       return QMOE_ERR_CUDA;
   }
   if (n_keep > 0) {
@@ -984,7 +1005,7 @@ qmoe_status qmoe_chan_forward(const qmoe_chan_layer* layer, const uint16_t* x, c
   g_stats.last_path = QMOE_PATH_SMALL_M;
   g_stats.row_tiles = 1;
   g_stats.row_tile_tokens = T;
-  g_stats.small_launches = n_keep > 0 ? 3 : 2;
+  g_stats.small_launches = n_keep > 0 ? 4 : 3;
   g_stats.grouped_launches = 0;
   return QMOE_OK;
 }

@@ -198,7 +198,7 @@ def test_chan_pack_without_sketch_and_bad_arguments():
     rec, sk, dn = qmoe.chan_pack(4, 4, w1, w2, 64, None, sketch=False)
     assert sk is None and dn is None and rec.size == I * qmoe.chan_sizes(4, 4, H, 64)[0]
     for args, st in (((3, 4, 512, 64), qmoe.ERR_INVALID_ARG), ((4, 4, 768, 64), qmoe.ERR_UNSUPPORTED),
-                     ((4, 4, 256, 64), qmoe.ERR_UNSUPPORTED), ((4, 4, 8192, 64), qmoe.ERR_UNSUPPORTED),
+                     ((4, 4, 256, 64), qmoe.ERR_UNSUPPORTED), ((4, 4, 4096, 64), qmoe.ERR_UNSUPPORTED),
                      ((4, 4, 512, 32), qmoe.ERR_UNSUPPORTED)):
         with pytest.raises(qmoe.QmoeError) as ei:
             qmoe.chan_sizes(*args)
