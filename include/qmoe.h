@@ -344,11 +344,11 @@ const char* qmoe_status_str(int status);
 #define QMOE_DEVICE_BAD_SEGMENT 2u /* a work table overflowed; its excess skipped */
 
 /* Test hook: fault injection for the decode-layer kernel (the qmoe_forward
- * path of T <= 8 tokens).  wait_limit_ns bounds every wait of that kernel (0:
- * the default, 2 s).  inject = 1 makes one thread of every CTA wait on a
- * barrier that nothing arrives at: the wait runs out, the CTA drops its part
- * of the output, sets QMOE_DEVICE_TIMEOUT and returns, and y is left as it
- * was.  The library stays usable: after qmoe_test_set_fault(0, 0) and
+ * path of T <= 8 tokens) and the exact-read kernel of qmoe_chan_forward.
+ * wait_limit_ns bounds every wait of those kernels (0: the default, 2 s).
+ * inject = 1 makes one thread of every CTA wait on a barrier that nothing
+ * arrives at: the wait runs out, the CTA drops its part of the output, sets
+ * QMOE_DEVICE_TIMEOUT and returns, and y is left as it was.  The library stays usable: after qmoe_test_set_fault(0, 0) and
  * qmoe_clear_status() the next call is correct.  Process-wide setting, read
  * at launch; not thread-safe.  QMOE_ERR_INVALID_ARG for another inject. */
 qmoe_status qmoe_test_set_fault(int inject, unsigned long long wait_limit_ns);

@@ -65,6 +65,7 @@ struct ChanParams {
   int wave_sk;            // sketch records per wave of the score kernel
   int wave_rec;           // channel records per wave of the exact kernel
   unsigned long long wait_ns;
+  int inject;             // test hook: 1 = every exact-kernel block waits on a barrier nothing arrives at
   unsigned* status;
 };
 
@@ -517,10 +518,14 @@ __global__ void __launch_bounds__(kSelThreads, 1) chan_select_kernel(ChanParams 
   pdl_wait();
   pdl_trigger();
   if (tid == 0) s_res[0] = s_res[1] = 0;
+  // scores and the level-1 histogram into shared memory, every element's copy in flight at once
   const float* sc = p.scores + (size_t)t * n;
-  for (int i = tid; i < n; i += kSelThreads) keys[i] = __float_as_uint(__ldcg(sc + i)) & 0x7FFFFFFFu;
+  for (int i = tid; i < n; i += kSelThreads) cp_async4(keys + i, sc + i);
   const int* h1 = p.hist + (size_t)t * kChanBins;
-  for (int i = tid; i < kChanBins; i += kSelThreads) hist[i] = __ldcg(h1 + i);
+  for (int i = tid; i < kChanBins / 4; i += kSelThreads) cp_async16(hist + 4 * i, h1 + 4 * i);
+  cp_async_wait_all();
+  __syncthreads();
+  for (int i = tid; i < n; i += kSelThreads) keys[i] &= 0x7FFFFFFFu;
   __syncthreads();
   const int per = (n + kSelThreads - 1) / kSelThreads;
   const int lo = min(n, tid * per), hi = min(n, lo + per);
@@ -580,7 +585,10 @@ __global__ void __launch_bounds__(kChanThreads, 1) chan_exact_kernel(ChanParams 
   constexpr float kB = F1 == 4 ? 24.f : 6.f;
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ uint64_t bar[2];  // per wave: [0] its shared-expert records, [1] its selected records
+  __shared__ uint64_t dbar;    // test hook: a barrier nothing arrives at
   __shared__ int s_last, s_abort;
+  __shared__ int s_ids[kChanMaxAct];
+  __shared__ float s_wts[kChanMaxAct];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int H = p.H, T = p.T, I = p.I, NC = H >> LCPC, R = p.rec_bytes, WR = p.wave_rec;
   const int SB = H / p.block;
@@ -597,6 +605,7 @@ __global__ void __launch_bounds__(kChanThreads, 1) chan_exact_kernel(ChanParams 
   if (tid == 0) {
     mbar_init(&bar[0], kChanThreads);
     mbar_init(&bar[1], kChanThreads);
+    mbar_init(&dbar, 1);
     fence_mbar_init();
     s_abort = 0;
   }
@@ -612,9 +621,9 @@ __global__ void __launch_bounds__(kChanThreads, 1) chan_exact_kernel(ChanParams 
     const int v = u - n_sh, t = v / p.n_keep;
     const int f = p.sel[v];
     const int s = f / I;
-    int e = (f >= 0 && s < p.k) ? p.ids[t * p.k + s] : -1;
+    int e = (f >= 0 && s < p.k) ? s_ids[t * p.k + s] : -1;
     int j = f - s * I;
-    float wt = e >= 0 ? p.wts[t * p.k + s] : 0.f;
+    float wt = e >= 0 ? s_wts[t * p.k + s] : 0.f;
     if (e < 0 || e >= p.E) {  // a corrupt selection: read record 0, add nothing
       atomicOr(p.status, kStatusBadSegment);
       e = 0;
@@ -625,6 +634,13 @@ __global__ void __launch_bounds__(kChanThreads, 1) chan_exact_kernel(ChanParams 
     utok[i] = t;
     uw[i] = wt;
   };
+  // routing of the score kernel: with a selection step in between, the score
+  // kernel has completed before this kernel launches (every kernel of the chain
+  // waits for its predecessor before it lets the next one start)
+  if (p.n_keep > 0 && tid < T * p.k) {
+    s_ids[tid] = p.ids[tid];
+    s_wts[tid] = p.wts[tid];
+  }
   // first wave's shared-expert records, before the wait
   const int nw0 = min(WR, u1 - u0), ns0 = max(0, min(nw0, n_sh - u0));
   for (int i = tid; i < ns0; i += kChanThreads) unit_shared(i, u0 + i);
@@ -782,10 +798,12 @@ __global__ void __launch_bounds__(kChanThreads, 1) chan_exact_kernel(ChanParams 
     }
     __syncthreads();  // the wave buffer and h are reused
   }
+  if (p.inject == 1 && tid == 0 && !mbar_wait_sleep_bounded(&dbar, 0, p.status, p.wait_ns)) s_abort = 1;
+  __syncthreads();
   if (s_abort) cp_async_wait_all();
 
-  // block rows -> yacc
-  if (has_rows) {
+  // block rows -> yacc (a block that gave up adds nothing; the last block then leaves y as it was)
+  if (has_rows && !s_abort) {
 #pragma unroll
     for (int t = 0; t < TM; ++t) {
       if (TM == 1 || t < T)

@@ -122,6 +122,11 @@ __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(dst)), "l"(src) : "memory");
 }
 
+// 4-byte asynchronous copy global -> shared (through L1).
+__device__ __forceinline__ void cp_async4(void* dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_addr(dst)), "l"(src) : "memory");
+}
+
 // Arrive on `bar` once every cp.async this thread issued so far has landed
 // (the arrival is counted in the barrier's initial count).
 __device__ __forceinline__ void cp_async_arrive(uint64_t* bar) {

@@ -954,6 +954,7 @@ qmoe_status qmoe_chan_forward(const qmoe_chan_layer* layer, const uint16_t* x, c
   p.y = y;
   p.inv_sqrt_h = (float)(1.0 / std::sqrt((double)L.H));
   p.wait_ns = g_fault_wait_ns;
+  p.inject = g_fault_inject;
   p.status = di->status;
 
   // scores: every block may hold up to ceil(units / grid) sketch records

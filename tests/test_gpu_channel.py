@@ -181,3 +181,38 @@ def test_channel_layer_rejects_bad_arguments(qm):
     with pytest.raises(qm.QmoeError) as ei:
         qm.chan_forward(case.layer, x9, lg, 10, y, ws)
     assert ei.value.status == qm.ERR_INVALID_ARG
+
+
+def test_channel_wait_expiry_leaves_y_and_recovers(qm):
+    """The exact-read kernel's bounded wait driven to expiry by the test hook
+    (every block waits 1 ms on a barrier nothing arrives at): the timeout flag
+    is set, y keeps its contents, and the next call (hook off) is correct."""
+    import torch
+    cfg = SMALL
+    case = _case(cfg)
+    x_bits = synth.tokens(cfg.H, 13, 1)
+    lg_np = synth.router_logits(cfg, 13, 1)
+    xd = Q.bf16_bits_to_f64(x_bits)
+    _, _, ref_scores = CS.channel_scores(xd, lg_np, cfg.k, case.bank)
+    n_keep, clear = _gap_n_keep(ref_scores, 150)
+    assert clear.all()
+    y_ref, _, _ = CS.channel_forward(xd, lg_np, cfg.k, case.bank, n_keep)
+    ws = torch.empty(qm.chan_workspace_size(case.layer, 1, n_keep), dtype=torch.uint8, device="cuda")
+    x = torch.from_numpy(x_bits.view(np.int16)).cuda()
+    lg = torch.from_numpy(np.ascontiguousarray(lg_np, dtype=np.float32)).cuda()
+    y = torch.full((1, cfg.H), 0x3F80, dtype=torch.int16, device="cuda")  # bf16 1.0 everywhere
+    try:
+        qm.test_set_fault(1, 1_000_000)
+        qm.clear_status()
+        qm.chan_forward(case.layer, x, lg, n_keep, y, ws)
+        torch.cuda.synchronize()
+        assert qm.get_stats().device_status & qm.DEVICE_TIMEOUT
+        assert bool((y == 0x3F80).all()), "y was written although a block gave up"
+    finally:
+        qm.test_set_fault(0, 0)
+        qm.clear_status()
+    qm.chan_forward(case.layer, x, lg, n_keep, y, ws)
+    torch.cuda.synchronize()
+    assert qm.get_stats().device_status == 0
+    from cases import bf16_dev_to_f64
+    _close(bf16_dev_to_f64(y), y_ref, "channel layer after an expired wait")
