@@ -241,8 +241,9 @@ __device__ __forceinline__ void fwht_rows(float* xs, int T, int lgh) {
   }
 }
 
-template <int TM>
+template <int TM, int NWL>  // NWL: sketch words per lane per row (H = 512 * NWL)
 __global__ void __launch_bounds__(kChanThreads, 1) chan_score_kernel(ChanParams p) {
+  constexpr int H = 512 * NWL, W16 = H / 16, SKB = H / kSketchBlock, LGH = NWL == 1 ? 9 : NWL == 2 ? 10 : 11;
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ uint64_t bar[kChanChunks];
   __shared__ int s_ids[kChanMaxAct];
@@ -250,14 +251,15 @@ __global__ void __launch_bounds__(kChanThreads, 1) chan_score_kernel(ChanParams 
   __shared__ int s_act_e[kChanMaxAct], s_act_n[kChanMaxAct], s_act_m[kChanMaxAct][kChanMaxT];
   __shared__ int s_nact, s_abort;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int H = p.H, W16 = H / 16, T = p.T, I = p.I, k = p.k;
-  const int lgh = 31 - __clz(H);
+  const int T = p.T, I = p.I, k = p.k;
+  constexpr int lgh = LGH;
+  // shared memory by offsets from the array (so every access stays a shared-memory access)
   float* xs = reinterpret_cast<float*>(smem);
-  float* sxw = xs + (size_t)T * H;
-  const uint8_t** src =
-      reinterpret_cast<const uint8_t**>((reinterpret_cast<uintptr_t>(sxw + (size_t)T * W16) + 15) & ~uintptr_t(15));
-  uint8_t* buf = reinterpret_cast<uint8_t*>(src + p.wave_sk);
-  buf = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(buf) + 127) & ~uintptr_t(127));
+  float* sxw = xs + T * H;
+  const int src_off = (4 * (T * H + T * W16) + 15) & ~15;
+  const uint8_t** src = reinterpret_cast<const uint8_t**>(smem + src_off);
+  const int buf_off = (src_off + 8 * p.wave_sk + 127) & ~127;
+  uint8_t* buf = smem + buf_off;
 
   if (tid == 0) {
     for (int c = 0; c < kChanChunks; ++c) mbar_init(&bar[c], kChanThreads);
@@ -349,7 +351,6 @@ __global__ void __launch_bounds__(kChanThreads, 1) chan_score_kernel(ChanParams 
   __syncthreads();
 
   const float4* x4 = reinterpret_cast<const float4*>(xs);
-  const int SKB = H / kSketchBlock;
   int wave = 0;
   for (int w0 = u0; w0 < u1; w0 += p.wave_sk, ++wave) {
     const int nw = min(p.wave_sk, u1 - w0);
@@ -364,9 +365,8 @@ __global__ void __launch_bounds__(kChanThreads, 1) chan_score_kernel(ChanParams 
       if (*reinterpret_cast<volatile int*>(&s_abort)) break;
       const int u = w0 + i, a = u / I, j = u - a * I;
       const int nm = s_act_n[a];
-      const uint8_t* r = buf + (size_t)i * skb;
-      const uint32_t* gw = reinterpret_cast<const uint32_t*>(r);
-      const uint32_t* uw = gw + W16;
+      const uint8_t* r = buf + i * p.sk_bytes;
+      const uint32_t* gw = reinterpret_cast<const uint32_t*>(r) + lane;
       const uint16_t* sc = reinterpret_cast<const uint16_t*>(r + H / 2);
       int tok[TM];
 #pragma unroll
@@ -374,8 +374,10 @@ __global__ void __launch_bounds__(kChanThreads, 1) chan_score_kernel(ChanParams 
       float ag[TM], au[TM];
 #pragma unroll
       for (int m = 0; m < TM; ++m) ag[m] = au[m] = 0.f;
-      for (int w = lane; w < W16; w += 32) {
-        const uint32_t g = gw[w], uu = uw[w];
+#pragma unroll
+      for (int n = 0; n < NWL; ++n) {
+        const int w = lane + 32 * n;
+        const uint32_t g = gw[32 * n], uu = gw[W16 + 32 * n];
         const float sg = bf16_to_f(sc[w >> 3]), su = bf16_to_f(sc[SKB + (w >> 3)]);
         float vg[16], vu[16];
         Unroll<16>::run([&](auto kk) {
@@ -388,7 +390,7 @@ __global__ void __launch_bounds__(kChanThreads, 1) chan_score_kernel(ChanParams 
           if (TM == 1 || m < nm) {
             const int t = tok[m];
             float dg0 = 0.f, dg1 = 0.f, du0 = 0.f, du1 = 0.f;
-            const float4* xr = x4 + (size_t)t * 4 * W16 + w;
+            const float4* xr = x4 + t * 4 * W16 + w;
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
               const float4 xv = xr[q * W16];
@@ -598,9 +600,10 @@ __global__ void __launch_bounds__(kChanThreads, 1) chan_exact_kernel(ChanParams 
   float* hc = sxc + (size_t)T * NC;                                 // [WR][TM]
   int* utok = reinterpret_cast<int*>(hc + (size_t)WR * TM);         // [WR]: token, or -1 for all
   float* uw = reinterpret_cast<float*>(utok + WR);                  // [WR]: weight
-  uintptr_t sp = reinterpret_cast<uintptr_t>(uw + WR);
-  const uint8_t** src = reinterpret_cast<const uint8_t**>((sp + 15) & ~uintptr_t(15));
-  uint8_t* buf = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(src + WR) + 127) & ~uintptr_t(127));
+  // by offsets from the array, so that every access stays a shared-memory access
+  const int src_off = (4 * (T * H + T * NC + WR * TM + 2 * WR) + 15) & ~15;
+  const uint8_t** src = reinterpret_cast<const uint8_t**>(smem + src_off);
+  uint8_t* buf = smem + ((src_off + 8 * WR + 127) & ~127);
 
   if (tid == 0) {
     mbar_init(&bar[0], kChanThreads);

@@ -456,6 +456,12 @@ size_t chan_exact_smem(int T, int H, int f1, int wave, int R) {
 }
 constexpr size_t kChanSmemBudget = kSmemLimit - 8 * 1024;  // static shared memory of the kernels
 
+template <int NWL>
+void (*chan_score_of(int tm))(ChanParams) {
+  return tm == 1 ? chan_score_kernel<1, NWL> : tm == 2 ? chan_score_kernel<2, NWL>
+         : tm == 4 ? chan_score_kernel<4, NWL> : chan_score_kernel<8, NWL>;
+}
+
 template <int TM>
 void (*chan_exact_of(int f1, int f2))(ChanParams) {
   if (f1 == QMOE_INT4 && f2 == QMOE_INT4) return chan_exact_kernel<4, 4, TM>;
@@ -973,11 +979,9 @@ qmoe_status qmoe_chan_forward(const qmoe_chan_layer* layer, const uint16_t* x, c
   p.wave_rec = (int)std::max<size_t>(1, std::min<size_t>((units3 + g3 - 1) / g3, (kChanSmemBudget - fix3) / per3));
   const size_t smem3 = chan_exact_smem(T, L.H, L.fmt1, p.wave_rec, (int)rec);
 
-  const int tm = chan_tm(T);
-  void (*score)(ChanParams) = tm == 1   ? chan_score_kernel<1>
-                              : tm == 2 ? chan_score_kernel<2>
-                              : tm == 4 ? chan_score_kernel<4>
-                                        : chan_score_kernel<8>;
+  void (*score)(ChanParams) = L.H == 512    ? chan_score_of<1>(chan_tm(T))
+                              : L.H == 1024 ? chan_score_of<2>(chan_tm(T))
+                                            : chan_score_of<4>(chan_tm(T));
   const size_t smem2 = (size_t)L.k * L.I * 4;
   if (cudaFuncSetAttribute(score, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem1) != cudaSuccess ||
       cudaFuncSetAttribute(chan_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem2) !=
