@@ -471,11 +471,6 @@ __device__ __forceinline__ void block_scan2(int a, int b, int* ea, int* eb, int*
   __syncthreads();
 }
 
-// Exclusive prefix sums over the block of (a, b), kSelThreads threads; sh: 2 * 32 ints.
-__device__ __forceinline__ void sel_scan2(int a, int b, int* ea, int* eb, int* sh) {
-  block_scan2(a, b, ea, eb, sh);
-}
-
 // The bin (of nb, counts in h, digit order = key order) holding the need-th
 // largest key: returns it, and in *above the count of keys in higher bins.
 // Each thread takes nb / kSelThreads consecutive bins, highest first.
@@ -484,7 +479,7 @@ __device__ __forceinline__ int sel_find_bin(const int* h, int nb, int need, int*
   int tot = 0;
   for (int m = 0; m < per; ++m) tot += h[hi - m];
   int excl, unused;
-  sel_scan2(tot, 0, &excl, &unused, sh);
+  block_scan2(tot, 0, &excl, &unused, sh);
   if (excl < need && need <= excl + tot) {
     int run = excl;
     for (int m = 0; m < per; ++m) {
@@ -556,7 +551,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) chan_select_kernel(ChanParams 
     eq += keys[i] == theta;
   }
   int gt0, eq0;
-  sel_scan2(gt, eq, &gt0, &eq0, sh);
+  block_scan2(gt, eq, &gt0, &eq0, sh);
   int pos = gt0 + min(eq0, need), eqs = eq0;
   int* out = p.sel + (size_t)t * p.n_keep;
   for (int i = lo; i < hi; ++i) {

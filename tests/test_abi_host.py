@@ -208,3 +208,33 @@ def test_chan_pack_without_sketch_and_bad_arguments():
     with pytest.raises(qmoe.QmoeError) as ei:
         qmoe.chan_pack(4, 4, w1, w2, 64, bad)
     assert ei.value.status == qmoe.ERR_INVALID_ARG
+
+
+def test_chan_workspace_size_validates_on_the_host():
+    """qmoe_chan_workspace_size runs on the host: shapes and limits are checked without a device."""
+    H, I, E, k = 2048, 1408, 64, 6
+    # fake, 16-byte aligned device addresses: the size query never dereferences them
+    layer = qmoe.make_chan_layer(H, I, E, k, 2, qmoe.INT4, qmoe.INT4, 128, None, None, None, None)
+    layer.records = layer.sketch = layer.dn = layer.signs = 0x10000
+    n = qmoe.chan_workspace_size(layer, 1, 1521)
+    R, _ = qmoe.chan_sizes(qmoe.INT4, qmoe.INT4, H, 128)
+    assert n >= 1 * k * I * 4 + 1521 * 4 + 4096 * 4 + H * 4 and n % 256 == 0
+    assert qmoe.chan_workspace_size(layer, 8, 1521) > n
+    for T, nk in ((0, 10), (9, 10), (1, k * I + 1), (1, -1)):
+        with pytest.raises(qmoe.QmoeError) as ei:
+            qmoe.chan_workspace_size(layer, T, nk)
+        assert ei.value.status == qmoe.ERR_INVALID_ARG
+    bad = qmoe.make_chan_layer(H, I, E, 9, 2, qmoe.INT4, qmoe.INT4, 128, None, None, None, None)  # k > 8
+    bad.records = bad.sketch = bad.dn = bad.signs = 0x10000
+    with pytest.raises(qmoe.QmoeError):
+        qmoe.chan_workspace_size(bad, 1, 10)
+    big = qmoe.make_chan_layer(H, 8192, E, k, 2, qmoe.INT4, qmoe.INT4, 128, None, None, None, None)  # k * I > 32768
+    big.records = big.sketch = big.dn = big.signs = 0x10000
+    with pytest.raises(qmoe.QmoeError) as ei:
+        qmoe.chan_workspace_size(big, 1, 10)
+    assert ei.value.status == qmoe.ERR_UNSUPPORTED
+    unaligned = qmoe.make_chan_layer(H, I, E, k, 2, qmoe.INT4, qmoe.INT4, 128, None, None, None, None)
+    unaligned.records, unaligned.sketch, unaligned.dn, unaligned.signs = 0x10008, 0x10000, 0x10000, 0x10000
+    with pytest.raises(qmoe.QmoeError) as ei:
+        qmoe.chan_workspace_size(unaligned, 1, 10)
+    assert ei.value.status == qmoe.ERR_INVALID_ARG
