@@ -93,11 +93,12 @@ def _close(got, ref, what=""):
     assert r <= REL_L2 and m <= MAX_ERR_RMS, f"{what}: rel_l2={r:.3g} max_err/rms={m:.3g}"
 
 
-@pytest.mark.parametrize("f1,f2,block,T,budget", [
-    ("int4", "int4", 64, 1, 0.18), ("int4", "int4", 64, 3, 0.13), ("int2", "int4", 128, 1, 0.18),
-    ("int2", "int2", 64, 8, 0.18), ("int4", "int2", 128, 2, 0.5)])
-def test_channel_layer_small(qm, f1, f2, block, T, budget):
-    cfg = small_cfg(SMALL, fc1_fmt=f1, fc2_fmt=f2, block=block)
+@pytest.mark.parametrize("f1,f2,block,T,budget,H", [
+    ("int4", "int4", 64, 1, 0.18, 512), ("int4", "int4", 64, 3, 0.13, 512), ("int2", "int4", 128, 1, 0.18, 512),
+    ("int2", "int2", 64, 8, 0.18, 512), ("int4", "int2", 128, 2, 0.5, 512), ("int4", "int4", 128, 5, 0.18, 1024),
+    ("int2", "int4", 64, 1, 0.13, 1024)])
+def test_channel_layer_small(qm, f1, f2, block, T, budget, H):
+    cfg = small_cfg(SMALL, fc1_fmt=f1, fc2_fmt=f2, block=block, H=H)
     case = _case(cfg)
     x = synth.tokens(cfg.H, 5, T)
     lg = synth.router_logits(cfg, 5, T)
