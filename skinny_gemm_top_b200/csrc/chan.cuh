@@ -8,17 +8,19 @@
 // full and computed exactly (scoring paragraph); the number of channels read
 // per token is fixed (choosing-k paragraph).  Shared experts are read in full.
 //
-// Three launches, chained by programmatic dependent launch:
-//   chan_score_kernel   routing, rotation of x, sketch products, scores
+// Launches, chained by programmatic dependent launch (after a reset of the
+// histogram, the accumulator and the tickets):
+//   chan_score_kernel   routing, rotation of x, sketch products, scores and a
+//                       histogram of their top bits
 //   chan_select_kernel  one block per token: radix select of the n_keep best
 //   chan_exact_kernel   the selected and shared channel records: gate/up dot
 //                       products, SwiGLU, down-column accumulation, combine
 //
 // A channel (and its sketch) is one contiguous record, so a block's work is a
 // list of records streamed into shared memory with 16-byte cp.async by every
-// thread, completing on one mbarrier per wave.  The dot products run on the
-// CUDA cores: a code u is turned into the float 1 + u / 2^bits' (one shift and
-// one LOP3 into the mantissa), multiplied with x, and the constant part is
+// thread, completing on mbarriers (a few per wave).  The dot products run on
+// the CUDA cores: a code u is turned into the float 1 + u / 2^bits (one shift
+// and one LOP3 into the mantissa), multiplied with x, and the constant part is
 // removed with the per-chunk sum of x.
 #pragma once
 #include <climits>
