@@ -512,18 +512,10 @@ def run_ours(args):
         "vs_baseline": None,
         "dtype": "int4-weights/bf16-act/fp32-acc",
         "data": "synthetic",
-        "config": {
-            "workload": "v2lite-decode-moe-layer: H=2048 I=1408 E=64 top-6 + 2 shared, INT4 FC1/FC2 block 64, "
-                        "M=1 token per expert",
-            "tokens_per_expert": 1,
-            "global_batch": world,
-            "parallelism": f"replicas x{world} (independent decode batches, no data-path collective)",
-            "l2": "8 weight copies (2.4 GB) rotated step by step: inputs larger than L2",
-            "graph": "CUDA graphs of forward calls",
-            "bytes_per_step": int(head["bytes"]),
-            "pct_of_hbm_peak": round(100 * value / world / hbm_peak, 1),
-            "pct_of_nominal_8TBps": round(100 * value / world / 8000, 1),
-        },
+        "config": headline_config(world),
+        "bytes_per_step": int(head["bytes"]),
+        "pct_of_hbm_peak": round(100 * value / world / hbm_peak, 1),
+        "pct_of_nominal_8TBps": round(100 * value / world / 8000, 1),
         "roofline": {"bound": "hbm", "kernel": dom_desc,
                      "achieved": round(dom_gbps, 1), "peak": hbm_peak, "peak_source": peak_src,
                      "unit": "GB/s", "frac": round(dom_gbps / hbm_peak, 3), "traffic": traffic,
@@ -814,8 +806,21 @@ def _cores() -> int:
         return os.cpu_count() or 1
 
 
-def cpu_baseline(gpu_bytes_per_step: float, budget_s: float = 12.0) -> dict:
-    """The oracle as it stands, one M=1 layer step at a time, for about budget_s seconds."""
+def cpu_baseline(gpu_bytes_per_step: float, budget_s: float = 12.0, single_s: float = 8.0) -> dict:
+    """The oracle as it stands, one M=1 layer step at a time, for about budget_s
+    seconds on all host threads, then for about single_s seconds on one thread."""
+    out = _cpu_baseline_run(budget_s)
+    out["cores"] = _cores()
+    if single_s > 0:
+        from threadpoolctl import threadpool_limits
+        with threadpool_limits(limits=1):
+            one = _cpu_baseline_run(single_s)
+        out["single_thread"] = {"value": one["value"], "unit": "GB/s", "cores": 1, "sample": one["sample"],
+                                "us_per_layer": one["us_per_layer"]}
+    return out
+
+
+def _cpu_baseline_run(budget_s: float) -> dict:
     Q, bank = _oracle_bank()
     rows = synth.router_logits(CFG, SEED, 64, index=7)
     x = Q.bf16_bits_to_f64(synth.tokens(CFG.H, SEED, 1))
@@ -827,9 +832,22 @@ def cpu_baseline(gpu_bytes_per_step: float, budget_s: float = 12.0) -> dict:
         nbytes += layer_bytes(rows[n % 64:n % 64 + 1])["total"]
         n += 1
     dt = time.perf_counter() - t0
-    return {"value": round(nbytes / (dt * 1e9), 4), "unit": "GB/s", "cores": _cores(), "kind": "oracle",
+    return {"value": round(nbytes / (dt * 1e9), 4), "unit": "GB/s", "kind": "oracle",
             "sample": f"{n} single-token layer steps (M=1, rotating router rows), {dt:.1f} s",
             "us_per_layer": round(dt / n * 1e6, 1)}
+
+
+def headline_config(world: int) -> dict:
+    """The workload the headline line (and the reference arm's line) is quoted on."""
+    return {
+        "workload": "v2lite-decode-moe-layer: H=2048 I=1408 E=64 top-6 + 2 shared, INT4 FC1/FC2 block 64, "
+                    "M=1 token per expert",
+        "tokens_per_expert": 1,
+        "global_batch": world,
+        "parallelism": f"replicas x{world} (independent decode batches, no data-path collective)",
+        "l2": "8 weight copies (2.4 GB) rotated step by step: inputs larger than L2",
+        "graph": "CUDA graphs of forward calls",
+    }
 
 
 def run_reference(args):
@@ -854,8 +872,7 @@ def run_reference(args):
         "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": "v2lite-decode-moe-layer: H=2048 I=1408 E=64 top-6 + 2 shared, INT4 FC1/FC2 "
-                               "block 64, M=1 token per expert", "tokens_per_expert": 1},
+        "config": headline_config(world),
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": _cores(), "kind": "oracle",
                          "sample": f"{args.steps} single-token layer steps after {args.warmup} warm-up steps"},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
