@@ -158,7 +158,8 @@ def _codes_of(buf: np.ndarray, n: int, bits: int) -> np.ndarray:
     return u.astype(np.int64) - (1 << (bits - 1))
 
 
-@pytest.mark.parametrize("f1,f2,block,H,I", [(4, 4, 128, 512, 12), (2, 4, 64, 1024, 5), (2, 2, 128, 512, 3)])
+@pytest.mark.parametrize("f1,f2,block,H,I", [(4, 4, 128, 512, 12), (2, 4, 64, 1024, 5), (2, 2, 128, 512, 3),
+                                             (4, 4, 64, 2048, 3)])
 def test_chan_pack_matches_oracle(f1, f2, block, H, I):
     from oracle import channel_select as CS
     w1 = synth.normal_bf16(21, 70, 0, (2 * I, H), 0.02)
